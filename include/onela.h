@@ -1,0 +1,179 @@
+/*
+ * onela.h -- C ABI of the shared-state Gated DeltaNet beam-decode library.
+ *
+ * One decode step of a Gated DeltaNet (GDN) layer for W beams that all grow
+ * out of one shared prompt-derived state S0 per (request, head), following
+ * "OneLA: Scaling Linear-Attention Decoding to Large Beams in Generative
+ * Recommendation" (abstract; evolve.pub review, Summary and key claims on
+ * section 3.2, equations 2-4).  Per head, with S_{t-1} the state of the beam's
+ * parent,
+ *
+ *     S_t     = alpha_t S_{t-1} + delta_t k_t^T
+ *     delta_t = beta_t (v_t - alpha_t S_{t-1} k_t),   alpha_t = exp(g_t)
+ *     o_t     = S_t q_t = alpha_t S_{t-1} q_t + delta_t (k_t . q_t)
+ *
+ * No per-beam state is ever formed.  Every beam is a chain of transition
+ * records (alpha, delta, k) reached through an ancestry index (review,
+ * Summary: "compact append-only GDN Transition Records"; abstract: "a
+ * lightweight ancestry index ... without moving or copying existing
+ * records").  S_{t-1} x for x in {k_t, q_t} is computed as
+ *     G (S0 x) + sum_j w_j (k_j . x) delta_j
+ * over the beam's ancestor records j (w_j: product of the gates of the
+ * records after j, G: product of all of them), with S0 read once per head and
+ * shared by every beam (abstract: "A fused GPU kernel further reuses the
+ * shared state across beams").
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers on the handle's device unless a
+ *     comment says otherwise; tensors are dense, row-major, no padding.
+ *   - Streams are CUDA streams passed as opaque pointers (NULL = the legacy
+ *     default stream).  Work is enqueued on the stream; no entry point on the
+ *     decode path synchronises the host, so the calls can be captured in a
+ *     CUDA graph.
+ *   - Inputs are borrowed for the stream-ordered duration of the call; the
+ *     library never keeps a pointer to caller memory.  The library owns its
+ *     copy of S0, the record store and the ancestry index and frees them in
+ *     onela_destroy.
+ *   - Return value: ONELA_OK or one of the ONELA_ERR_* codes below.  A call
+ *     that returns an error has enqueued no work.
+ */
+#ifndef ONELA_H
+#define ONELA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct onela_handle onela_handle;
+typedef void *onela_stream; /* a cudaStream_t */
+
+/* Element types. */
+enum { ONELA_F32 = 0, ONELA_BF16 = 1 };
+
+/* Return codes. */
+enum {
+  ONELA_OK = 0,
+  ONELA_ERR_ARG = 1,         /* null pointer, bad size or dtype, bad W_prev  */
+  ONELA_ERR_STATE = 2,       /* decode before onela_set_prompt_state         */
+  ONELA_ERR_CAPACITY = 3,    /* step beyond T_max, or W beyond W_max         */
+  ONELA_ERR_PARENT = 4,      /* the device saw a parent index outside
+                                [0, W_prev); reported by the next call or by
+                                onela_status                                 */
+  ONELA_ERR_CUDA = 5,        /* a CUDA call failed (allocation, launch ...)  */
+  ONELA_ERR_UNSUPPORTED = 6  /* the requested kernel cannot run this shape   */
+};
+
+/* Which decode kernel runs.  AUTO picks the tensor-core kernel when the
+ * shape allows it (bf16 q/k/v, d_k and d_v in {64, 128, 256}) and the SIMT
+ * kernel otherwise. */
+enum { ONELA_KERNEL_AUTO = 0, ONELA_KERNEL_SIMT = 1, ONELA_KERNEL_TC = 2 };
+
+/* Handle configuration.
+ *   R, H            requests and heads (each (request, head) pair has its own
+ *                   S0 and its own records).
+ *   d_k, d_v        key and value widths, 1 <= d <= 256.
+ *   W_max, T_max    most beams per step and most decode steps per decode.
+ *   s0_dtype        ONELA_F32 or ONELA_BF16: element type of S0.
+ *   qkv_dtype       ONELA_F32 or ONELA_BF16: element type of q, k, v (and of
+ *                   the k stored in the records).
+ *   kernel          ONELA_KERNEL_*.
+ *   s0_split        fp32 S0 on the tensor-core kernel only: number of bf16
+ *                   terms S0 is split into (2 or 3; 0 means 2).  Ignored
+ *                   otherwise.
+ *   device          CUDA device ordinal the handle lives on.
+ */
+typedef struct {
+  int32_t R, H, d_k, d_v, W_max, T_max;
+  int32_t s0_dtype;
+  int32_t qkv_dtype;
+  int32_t kernel;
+  int32_t s0_split;
+  int32_t device;
+} onela_config;
+
+/* Create a handle: validates cfg and allocates, on cfg->device, the S0 copy,
+ * the record store (alpha fp32 [T_max][R][H][W_max], delta fp32
+ * [T_max][R][H][W_max][d_v], k [T_max][R][H][W_max][d_k] in qkv_dtype), the
+ * ancestry index (int32 [T_max][R][W_max][T_max]) and a device error word.
+ * Host-side allocation only; no kernel runs.  *out receives the handle.
+ * Errors: ONELA_ERR_ARG (null pointer or invalid field), ONELA_ERR_CUDA. */
+int onela_create(const onela_config *cfg, onela_handle **out);
+
+/* Install the shared prompt-derived state (abstract: "a single shared
+ * prompt-derived state") and rewind the decode to step 0.
+ *   S0  device pointer, [R][H][d_v][d_k] in cfg.s0_dtype.  Copied on `stream`
+ *       (and, for the tensor-core kernel, converted once into the bf16
+ *       operand layout); S0 may be freed once the stream has passed the call.
+ * Errors: ONELA_ERR_ARG, ONELA_ERR_CUDA. */
+int onela_set_prompt_state(onela_handle *h, const void *S0, onela_stream stream);
+
+/* One decode step t = (number of previous steps since the last rewind) + 1.
+ *   W_prev      beams of the previous step; must be 1 at t = 1 (the prompt
+ *               root) and the previous call's W afterwards.
+ *   W           beams of this step, 1 <= W <= W_max.
+ *   q, k        [R][W][H][d_k] in qkv_dtype.
+ *   v           [R][W][H][d_v] in qkv_dtype.
+ *   g           [R][W][H] fp32, the log of the decay gate: alpha = exp(g).
+ *   beta        [R][W][H] fp32, the delta-rule write strength.
+ *   parent_idx  [R][W] int32, beam b's parent among the previous step's
+ *               beams, in [0, W_prev).  One array serves all heads.
+ *   o           [R][W][H][d_v] fp32, written: o_t = S_t q_t.
+ * Also appends the records (alpha_t, delta_t, k_t) of every (beam, head) at
+ * depth t and the ancestry rows of depth t; earlier records are never moved.
+ * A parent index outside [0, W_prev) is clamped to 0 on the device, recorded
+ * in the device error word and reported as ONELA_ERR_PARENT by the next call
+ * on the handle (or by onela_status); the outputs of that step are then
+ * meaningless.
+ * Errors: ONELA_ERR_ARG, ONELA_ERR_STATE, ONELA_ERR_CAPACITY,
+ * ONELA_ERR_PARENT, ONELA_ERR_UNSUPPORTED, ONELA_ERR_CUDA. */
+int onela_decode_step(onela_handle *h, int32_t W_prev, int32_t W,
+                      const void *q, const void *k, const void *v,
+                      const float *g, const float *beta,
+                      const int32_t *parent_idx, float *o,
+                      onela_stream stream);
+
+/* Rewind to step 0 keeping S0 (records are logically dropped, nothing is
+ * freed) and clear the device error word on `stream`.
+ * Errors: ONELA_ERR_ARG, ONELA_ERR_CUDA. */
+int onela_reset(onela_handle *h, onela_stream stream);
+
+/* Wait for the handle's device (cudaDeviceSynchronize on it) and report the
+ * device error word in *device_err (0: none; bit 0: a bad parent index).
+ * Returns ONELA_ERR_PARENT when bit 0 is set, ONELA_OK otherwise.
+ * Errors: ONELA_ERR_ARG, ONELA_ERR_CUDA. */
+int onela_status(onela_handle *h, int32_t *device_err);
+
+/* Free everything the handle owns (synchronises its device first).
+ * Errors: ONELA_ERR_ARG. */
+int onela_destroy(onela_handle *h);
+
+/* Copy the records of depth t (1 <= t <= steps done) into caller DEVICE
+ * buffers on `stream`: alpha fp32 [R][H][W_t], delta fp32 [R][H][W_t][d_v],
+ * k [R][H][W_t][d_k] in qkv_dtype.  Any of the three may be NULL.
+ * Errors: ONELA_ERR_ARG, ONELA_ERR_CUDA. */
+int onela_read_records(onela_handle *h, int32_t t, float *alpha, float *delta,
+                       void *k, onela_stream stream);
+
+/* Copy the ancestry rows of depth t (1 <= t <= steps done) into a caller
+ * DEVICE buffer on `stream`: int32 [R][W_t][t-1], entry [r][b][j] = index of
+ * the beam at depth j+1 on the path from the root to beam b of step t.
+ * Errors: ONELA_ERR_ARG, ONELA_ERR_CUDA. */
+int onela_read_ancestry(onela_handle *h, int32_t t, int32_t *anc,
+                        onela_stream stream);
+
+/* Query: number of decode steps done since the last rewind, and the kernel
+ * the handle runs (ONELA_KERNEL_SIMT or ONELA_KERNEL_TC). */
+int onela_steps_done(const onela_handle *h);
+int onela_kernel_kind(const onela_handle *h);
+
+/* Static description of a return code (never NULL). */
+const char *onela_error_string(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ONELA_H */
