@@ -1,0 +1,415 @@
+#!/usr/bin/env python
+"""Benchmark: shared-state GDN beam decode on B200.
+
+One benchmark step = one whole T-step beam decode of the workload (every
+decode step of the hot path: ancestry update, S0 [K; Q] products, replay,
+epilogue, record append), captured once in a CUDA graph and replayed.  L2 is
+flushed (a 512 MiB write) before every timed step, outside the timed events.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload long5k] [--kernel auto|simt|tc]
+
+Multi-GPU (launched by torchrun): every rank decodes its own request (its own
+S0 and inputs) with no collective on the data path; value = all ranks' beam.head
+steps / max-over-ranks device time ("weak" scaling).
+
+``--impl reference`` times the fp64 CPU oracle (the plain-C full-state beam
+tree) on the host cores for the same workload, metric and unit.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import glob
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "GDN beam·head decode steps/s at W=256,T=7; % of HBM/tensor roofline"
+UNIT = "beam·head steps/s"
+
+
+# ------------------------------------------------------------------ helpers
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", 0)), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "linear_attention_beam_shared_b200", "csrc", "*"))):
+        with open(p, "rb") as f:
+            h.update(os.path.basename(p).encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_kind):
+    """DRAM bytes per launch of the decode kernel from the committed ncu
+    summary, or None when the kernel sources changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    entry = d.get(kernel_kind)
+    if not entry or entry.get("source_hash") != kernel_source_hash():
+        return None
+    return entry
+
+
+def s0_by_prefill_gpu(wl, device):
+    """S0 for the workload: the GDN recurrence from zero over its synthetic
+    prompt, run with plain torch fp64 ops on the device (input synthesis for
+    the benchmark only; not part of the timed decode)."""
+    k, v, a, b = synth.draw_prompt(wl)
+    k = torch.from_numpy(k).to(device)
+    v = torch.from_numpy(v).to(device)
+    a = torch.from_numpy(a).to(device)
+    b = torch.from_numpy(b).to(device)
+    R, L, H, dk = k.shape
+    S = torch.zeros((R, H, wl.d_v, dk), dtype=torch.float64, device=device)
+    for l in range(L):
+        kl, vl = k[:, l], v[:, l]
+        al, bl = a[:, l, :, None], b[:, l, :, None]
+        u = torch.einsum("rhij,rhj->rhi", S, kl)
+        delta = bl * (vl - al * u)
+        S = al[..., None] * S + delta[..., :, None] * kl[..., None, :]
+    S32 = S.float().cpu()
+    return S32.to(torch.bfloat16) if wl.s0_dtype == "bf16" else S32
+
+
+def byte_model(wl, steps):
+    """Algorithmic bytes of one whole decode (all T steps): every byte the
+    method must move at least once, with each distinct ancestor record counted
+    once; plus the per-beam-gather upper bound."""
+    s = 2 if wl.s0_dtype == "bf16" else 4
+    e = 2 if wl.qkv_dtype == "bf16" else 4
+    d_k, d_v, H, R = wl.d_k, wl.d_v, wl.H, wl.R
+    rec = 4 + 4 * d_v + e * d_k
+    total = upper = 0
+    per_step = []
+    for t, st in enumerate(steps, start=1):
+        W = st["W"]
+        plist = [x["parents"].numpy() for x in steps[:t]]
+        U = [synth.distinct_ancestors([p[r] for p in plist], t) for r in range(R)]
+        base = R * H * (d_k * d_v * s + W * ((2 * d_k + d_v) * e + 8) + W * (4 * d_v + 4 * d_v + 4 + d_k * e))
+        idx = R * (W * 4 + W * (t - 1) * 4)
+        b_t = base + idx + H * sum(U) * rec
+        u_t = base + idx + H * R * W * (t - 1) * rec
+        per_step.append(b_t)
+        total += b_t
+        upper += u_t
+    return total, upper, per_step
+
+
+class ClockSampler:
+    """nvidia-smi samples during the timed region."""
+
+    def __init__(self, gpu_index):
+        self.proc = None
+        self.gpu = gpu_index
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv") if os.path.isdir(
+            os.path.join(ROOT, "gpurun_out")) else f"/tmp/onela_clocks_{os.getpid()}.csv"
+
+    def __enter__(self):
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.gpu)], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def time_cpu_oracle(wl, S0, steps, budget_s=10.0, nthreads=0):
+    """The C fp64 full-state oracle as it stands, on the host cores.  Runs the
+    whole decode repeatedly until about budget_s of CPU work is done."""
+    from oracle import cref
+    cref.beam_decode_fullstate(S0[:, :1], [{k: (v[:, :, :1] if k in ("q", "k", "v", "g", "beta") else v)
+                                            for k, v in s.items()} for s in steps[:1]], nthreads=nthreads)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        cref.beam_decode_fullstate(S0, steps, nthreads=nthreads)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or reps >= 50:
+            break
+    units = wl.units * reps
+    threads = nthreads if nthreads > 0 else cref.max_threads()
+    return units / el, reps, el, threads
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args):
+    ws, rank, local = dist_env()
+    if ws > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    device = torch.device("cuda", torch.cuda.current_device())
+    import linear_attention_beam_shared_b200 as L
+
+    base = synth.workload(args.workload)
+    # Every rank decodes its own request: own S0, own inputs.
+    wl = base.replace(seed_id=base.seed_id + 1000 * rank)
+    if args.s0 == "prefill":
+        S0 = s0_by_prefill_gpu(wl, device)
+    else:   # same shapes and dtype, entries drawn directly (for quick profiling runs)
+        S0 = synth.cast_state(0.1 * np.random.default_rng(wl.seed_id).standard_normal(
+            (wl.R, wl.H, wl.d_v, wl.d_k)), wl.s0_dtype)
+    steps = synth.draw_decode(wl)
+    kernel = {"auto": L.ONELA_KERNEL_AUTO, "simt": L.ONELA_KERNEL_SIMT, "tc": L.ONELA_KERNEL_TC}[args.kernel]
+    dec = L.BeamDecoder(wl.R, wl.H, wl.d_k, wl.d_v, wl.W, wl.T, wl.s0_dtype, wl.qkv_dtype,
+                        kernel=kernel, device=device.index)
+    kind = {L.ONELA_KERNEL_SIMT: "simt", L.ONELA_KERNEL_TC: "tc"}[dec.kernel]
+    dec.set_prompt_state(S0.to(device))
+    dsteps = [{k: (v.to(device) if isinstance(v, torch.Tensor) else v) for k, v in s.items()} for s in steps]
+    outs = [torch.empty((wl.R, s["W"], wl.H, wl.d_v), dtype=torch.float32, device=device) for s in steps]
+
+    stream = torch.cuda.Stream(device=device)
+    # Eager warm-up of the API (also loads the module), then capture.
+    with torch.cuda.stream(stream):
+        for s, o in zip(dsteps, outs):
+            dec.step(s["q"], s["k"], s["v"], s["g"], s["beta"], s["parents"], o=o, stream=stream)
+    stream.synchronize()
+    assert dec.status() == 0
+    dec.reset(stream)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for s, o in zip(dsteps, outs):
+            dec.step(s["q"], s["k"], s["v"], s["g"], s["beta"], s["parents"], o=o, stream=stream)
+    dec.reset(stream)
+
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=device)
+    for _ in range(args.warmup):
+        with torch.cuda.stream(stream):
+            flush.fill_(1)
+            graph.replay()
+    stream.synchronize()
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if ws > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(device.index) as clk:
+        with torch.cuda.stream(stream):
+            for i in range(args.steps):
+                flush.fill_(i & 0xFF)
+                starts[i].record(stream)
+                graph.replay()
+                ends[i].record(stream)
+        torch.cuda.synchronize()
+    if ws > 1:
+        torch.distributed.barrier()
+    times_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = float(sum(times_ms))
+    if ws > 1:
+        t = torch.tensor([total_ms], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    assert dec.status() == 0
+    ms_per_step = total_ms / args.steps
+    units_per_step = wl.units * ws
+    value = units_per_step / (ms_per_step / 1e3)
+
+    # Roofline of the decode kernel (the only kernel in the step).
+    alg_bytes, upper_bytes, _ = byte_model(wl, steps)
+    launches = wl.T
+    hbm, bf16_tf, bf16_sus, src = measured_peaks()
+    achieved = alg_bytes / (ms_per_step / 1e3) / 1e9
+    traffic = ncu_traffic(kind)
+    roofline = {
+        "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+        "frac": round(achieved / hbm, 4),
+        "traffic": traffic["bytes_per_launch"] if traffic else None,
+        "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else "fallback",
+        "kernel": f"onela step kernel ({kind})",
+        "alg_bytes_per_launch": round(alg_bytes / launches),
+        "upper_bound_bytes_per_launch": round(upper_bytes / launches),
+        "avg_launch_us": round(ms_per_step * 1e3 / launches, 3),
+    }
+    flops = 4 * wl.d_k * wl.d_v * wl.W * wl.H * wl.R * wl.T
+    roofline["tensor_frac_of_sustained_bf16"] = round(flops / (ms_per_step / 1e3) / 1e12 / bf16_sus, 5) if bf16_sus else None
+
+    # End to end through the public API with host buffers: per step the H2D
+    # copy of that step's inputs from pinned memory, the decode call, and the
+    # D2H read of its output o.
+    host_in = [{k: (v.pin_memory() if isinstance(v, torch.Tensor) else v) for k, v in s.items()} for s in steps]
+    host_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+    h2d = sum(v.numel() * v.element_size() for s in steps for v in s.values() if isinstance(v, torch.Tensor))
+    d2h = sum(o.numel() * o.element_size() for o in outs)
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(1, min(args.steps, 20))
+    e2e_ms = 0.0
+    for it in range(e2e_steps + 1):
+        with torch.cuda.stream(stream):
+            flush.fill_(3)
+            dec.reset(stream)
+            e_start.record(stream)
+            for hs, ds, o, ho in zip(host_in, dsteps, outs, host_out):
+                for key in ("q", "k", "v", "g", "beta", "parents"):
+                    ds[key].copy_(hs[key], non_blocking=True)
+                dec.step(ds["q"], ds["k"], ds["v"], ds["g"], ds["beta"], ds["parents"], o=o, stream=stream)
+                ho.copy_(o, non_blocking=True)
+            e_end.record(stream)
+        stream.synchronize()
+        if it > 0:
+            e2e_ms += e_start.elapsed_time(e_end)
+    if ws > 1:
+        t = torch.tensor([e2e_ms], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e = {"value": round(units_per_step / (e2e_ms / e2e_steps / 1e3), 1), "unit": UNIT,
+           "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+    assert dec.status() == 0
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu:
+        rate, reps, el, threads = time_cpu_oracle(wl, S0, steps, budget_s=args.cpu_budget)
+        cpu = {"value": round(rate, 1), "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"whole {args.workload} decode (R=1,H={wl.H},W={wl.W},T={wl.T}) x{reps} "
+                         f"in {el:.1f} s, plain-C fp64 full-state oracle"}
+
+    del graph
+    dec.close()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 6),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": f"{args.workload}: R={wl.R} per GPU, H={wl.H}, d_k=d_v={wl.d_k}, "
+                                   f"W={wl.W}, T={wl.T}, L_prompt={wl.L_prompt}, S0 {wl.s0_dtype}, "
+                                   f"q/k/v {wl.qkv_dtype}, parents Zipf(1.1)",
+                       "global_batch": wl.R * ws, "seq_len": wl.T, "parallelism": f"replicas{ws}",
+                       "l2": "flushed (512 MiB write) before every timed step", "kernel": kind,
+                       "step": f"one whole {wl.T}-step decode in a CUDA graph"},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "clocks": clk.summary(), "gpu_launches": launches * args.steps,
+        }
+        print(json.dumps(line))
+    if ws > 1:
+        torch.distributed.destroy_process_group()
+
+
+# ---------------------------------------------------------- reference arm
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return
+    from oracle import cref
+    wl = synth.workload(args.workload)
+    # S0 values do not change the oracle's running time; draw them directly
+    # instead of running a long prefill on the host.
+    S0 = synth.cast_state(0.1 * np.random.default_rng(0).standard_normal((wl.R, wl.H, wl.d_v, wl.d_k)),
+                          wl.s0_dtype)
+    steps = synth.draw_decode(wl)
+    for _ in range(args.warmup):
+        cref.beam_decode_fullstate(S0, steps)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        cref.beam_decode_fullstate(S0, steps)
+    el = time.perf_counter() - t0
+    value = wl.units * args.steps / el
+    threads = cref.max_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": f"{args.workload}: R={wl.R}, H={wl.H}, d_k=d_v={wl.d_k}, W={wl.W}, "
+                               f"T={wl.T}", "global_batch": wl.R, "seq_len": wl.T,
+                   "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(value, 1), "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"whole {args.workload} decode per step, plain-C fp64 full-state oracle"},
+        "e2e": {"value": round(value, 1), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="long5k")
+    ap.add_argument("--kernel", choices=["auto", "simt", "tc"], default="auto")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline leg")
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--s0", choices=["prefill", "direct"], default="prefill",
+                    help="S0 from the GDN recurrence over the synthetic prompt (default) or drawn "
+                         "directly; the decode's work does not depend on the S0 values")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -43,6 +43,12 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define ONELA_API __attribute__((visibility("default")))
+#else
+#define ONELA_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -97,10 +103,11 @@ typedef struct {
 /* Create a handle: validates cfg and allocates, on cfg->device, the S0 copy,
  * the record store (alpha fp32 [T_max][R][H][W_max], delta fp32
  * [T_max][R][H][W_max][d_v], k [T_max][R][H][W_max][d_k] in qkv_dtype), the
- * ancestry index (int32 [T_max][R][W_max][T_max]) and a device error word.
+ * ancestry index (int32 [T_max][R][W_max][T_max]) and an error word in
+ * mapped, pinned host memory that the kernels write and the host reads.
  * Host-side allocation only; no kernel runs.  *out receives the handle.
  * Errors: ONELA_ERR_ARG (null pointer or invalid field), ONELA_ERR_CUDA. */
-int onela_create(const onela_config *cfg, onela_handle **out);
+ONELA_API int onela_create(const onela_config *cfg, onela_handle **out);
 
 /* Install the shared prompt-derived state (abstract: "a single shared
  * prompt-derived state") and rewind the decode to step 0.
@@ -108,7 +115,7 @@ int onela_create(const onela_config *cfg, onela_handle **out);
  *       (and, for the tensor-core kernel, converted once into the bf16
  *       operand layout); S0 may be freed once the stream has passed the call.
  * Errors: ONELA_ERR_ARG, ONELA_ERR_CUDA. */
-int onela_set_prompt_state(onela_handle *h, const void *S0, onela_stream stream);
+ONELA_API int onela_set_prompt_state(onela_handle *h, const void *S0, onela_stream stream);
 
 /* One decode step t = (number of previous steps since the last rewind) + 1.
  *   W_prev      beams of the previous step; must be 1 at t = 1 (the prompt
@@ -129,48 +136,50 @@ int onela_set_prompt_state(onela_handle *h, const void *S0, onela_stream stream)
  * meaningless.
  * Errors: ONELA_ERR_ARG, ONELA_ERR_STATE, ONELA_ERR_CAPACITY,
  * ONELA_ERR_PARENT, ONELA_ERR_UNSUPPORTED, ONELA_ERR_CUDA. */
-int onela_decode_step(onela_handle *h, int32_t W_prev, int32_t W,
+ONELA_API int onela_decode_step(onela_handle *h, int32_t W_prev, int32_t W,
                       const void *q, const void *k, const void *v,
                       const float *g, const float *beta,
                       const int32_t *parent_idx, float *o,
                       onela_stream stream);
 
 /* Rewind to step 0 keeping S0 (records are logically dropped, nothing is
- * freed) and clear the device error word on `stream`.
+ * freed) and clear the error word.  Waits for `stream` first, so that no
+ * step still in flight can set the word after it is cleared; not meant for
+ * the inside of a captured region.
  * Errors: ONELA_ERR_ARG, ONELA_ERR_CUDA. */
-int onela_reset(onela_handle *h, onela_stream stream);
+ONELA_API int onela_reset(onela_handle *h, onela_stream stream);
 
 /* Wait for the handle's device (cudaDeviceSynchronize on it) and report the
- * device error word in *device_err (0: none; bit 0: a bad parent index).
+ * error word in *device_err (0: none; bit 0: a bad parent index).
  * Returns ONELA_ERR_PARENT when bit 0 is set, ONELA_OK otherwise.
  * Errors: ONELA_ERR_ARG, ONELA_ERR_CUDA. */
-int onela_status(onela_handle *h, int32_t *device_err);
+ONELA_API int onela_status(onela_handle *h, int32_t *device_err);
 
 /* Free everything the handle owns (synchronises its device first).
  * Errors: ONELA_ERR_ARG. */
-int onela_destroy(onela_handle *h);
+ONELA_API int onela_destroy(onela_handle *h);
 
 /* Copy the records of depth t (1 <= t <= steps done) into caller DEVICE
  * buffers on `stream`: alpha fp32 [R][H][W_t], delta fp32 [R][H][W_t][d_v],
  * k [R][H][W_t][d_k] in qkv_dtype.  Any of the three may be NULL.
  * Errors: ONELA_ERR_ARG, ONELA_ERR_CUDA. */
-int onela_read_records(onela_handle *h, int32_t t, float *alpha, float *delta,
+ONELA_API int onela_read_records(onela_handle *h, int32_t t, float *alpha, float *delta,
                        void *k, onela_stream stream);
 
 /* Copy the ancestry rows of depth t (1 <= t <= steps done) into a caller
  * DEVICE buffer on `stream`: int32 [R][W_t][t-1], entry [r][b][j] = index of
  * the beam at depth j+1 on the path from the root to beam b of step t.
  * Errors: ONELA_ERR_ARG, ONELA_ERR_CUDA. */
-int onela_read_ancestry(onela_handle *h, int32_t t, int32_t *anc,
+ONELA_API int onela_read_ancestry(onela_handle *h, int32_t t, int32_t *anc,
                         onela_stream stream);
 
 /* Query: number of decode steps done since the last rewind, and the kernel
  * the handle runs (ONELA_KERNEL_SIMT or ONELA_KERNEL_TC). */
-int onela_steps_done(const onela_handle *h);
-int onela_kernel_kind(const onela_handle *h);
+ONELA_API int onela_steps_done(const onela_handle *h);
+ONELA_API int onela_kernel_kind(const onela_handle *h);
 
 /* Static description of a return code (never NULL). */
-const char *onela_error_string(int code);
+ONELA_API const char *onela_error_string(int code);
 
 #ifdef __cplusplus
 }

@@ -1,0 +1,81 @@
+"""Shared-state Gated DeltaNet beam decode for B200 (sm_100a).
+
+One GDN decode step for W beams that share one prompt-derived state S0 per
+(request, head): beams are chains of append-only transition records
+(alpha, delta, k) reached through an ancestry index, and S_{t-1}[k; q] is
+formed as S0 [k; q] (S0 read once, shared by all beams) plus a gated replay
+over the beam's ancestor records (OneLA abstract; evolve.pub review, key
+claims on section 3.2, equations 2-4).
+
+The work runs in the CUDA library ``libonela_b200.so`` (C ABI in
+``include/onela.h``); this package is its Python binding.  ``onela_*``
+functions mirror the C entry points one to one; ``BeamDecoder`` is a small
+convenience wrapper around a handle.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _lib
+from ._lib import (  # noqa: F401
+    ONELA_BF16, ONELA_ERR_ARG, ONELA_ERR_CAPACITY, ONELA_ERR_CUDA, ONELA_ERR_PARENT,
+    ONELA_ERR_STATE, ONELA_ERR_UNSUPPORTED, ONELA_F32, ONELA_KERNEL_AUTO, ONELA_KERNEL_SIMT,
+    ONELA_KERNEL_TC, ONELA_OK, Handle, OnelaError, error_string, onela_create, onela_decode_step,
+    onela_destroy, onela_kernel_kind, onela_read_ancestry, onela_read_records, onela_reset,
+    onela_set_prompt_state, onela_status, onela_status_code, onela_steps_done,
+)
+
+LIB_PATH = _lib.LIB_PATH
+
+
+class BeamDecoder:
+    """Owns one handle; tracks the beam count of the previous step."""
+
+    def __init__(self, R, H, d_k, d_v, W_max, T_max, s0_dtype="f32", qkv_dtype="bf16",
+                 kernel=ONELA_KERNEL_AUTO, s0_split=0, device=0):
+        self.h = onela_create(R, H, d_k, d_v, W_max, T_max, s0_dtype, qkv_dtype, kernel,
+                              s0_split, device)
+        self.device = torch.device("cuda", device)
+        self.W_prev = 1
+        self.Ws = []
+
+    @property
+    def kernel(self) -> int:
+        return onela_kernel_kind(self.h)
+
+    def set_prompt_state(self, S0, stream=None):
+        onela_set_prompt_state(self.h, S0, stream)
+        self.W_prev, self.Ws = 1, []
+
+    def step(self, q, k, v, g, beta, parent_idx, o=None, stream=None):
+        c = self.h.cfg
+        W = int(parent_idx.shape[-1])
+        if o is None:
+            o = torch.empty((c.R, W, c.H, c.d_v), dtype=torch.float32, device=self.device)
+        onela_decode_step(self.h, self.W_prev, W, q, k, v, g, beta, parent_idx, o, stream)
+        self.W_prev = W
+        self.Ws.append(W)
+        return o
+
+    def reset(self, stream=None):
+        onela_reset(self.h, stream)
+        self.W_prev, self.Ws = 1, []
+
+    def status(self) -> int:
+        return onela_status(self.h)
+
+    def records(self, t: int):
+        return onela_read_records(self.h, t, self.Ws[t - 1])
+
+    def ancestry(self, t: int):
+        return onela_read_ancestry(self.h, t, self.Ws[t - 1])
+
+    def close(self):
+        onela_destroy(self.h)
+
+    def __del__(self):  # pragma: no cover - best effort
+        try:
+            if self.h.ptr:
+                onela_destroy(self.h)
+        except Exception:
+            pass

@@ -1,0 +1,295 @@
+// Host runtime of the decode library: handle, validation, record store,
+// ancestry index, error word, and the C ABI declared in include/onela.h.
+#include <cuda_runtime.h>
+
+#include <cstdlib>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "../../include/onela.h"
+#include "internal.h"
+
+struct onela_handle {
+  onela_config cfg;
+  int kernel;        // ONELA_KERNEL_SIMT or ONELA_KERNEL_TC
+  int planes;        // bf16 terms of the S0 operand image (tensor-core kernel)
+  int steps_done;    // decode steps since the last rewind
+  int has_prompt;
+  std::vector<int> Ws;  // beams of each step done
+  void *S0;
+  void *S0img;
+  float *rec_alpha;
+  float *rec_delta;
+  void *rec_k;
+  int32_t *anc;
+  int32_t *err_host;  // host-mapped error word
+  int32_t *err_dev;   // its device view
+};
+
+namespace {
+
+size_t esize(int dtype) { return dtype == ONELA_BF16 ? 2 : 4; }
+
+bool valid_dtype(int d) { return d == ONELA_F32 || d == ONELA_BF16; }
+
+// Switch to the handle's device for the duration of a call.
+struct DeviceGuard {
+  int prev = -1;
+  bool ok = false;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) return;
+    ok = (prev == dev) || (cudaSetDevice(dev) == cudaSuccess);
+  }
+  ~DeviceGuard() {
+    if (ok && prev >= 0) cudaSetDevice(prev);
+  }
+};
+
+void free_all(onela_handle *h) {
+  cudaFree(h->S0);
+  cudaFree(h->S0img);
+  cudaFree(h->rec_alpha);
+  cudaFree(h->rec_delta);
+  cudaFree(h->rec_k);
+  cudaFree(h->anc);
+  if (h->err_host) cudaFreeHost(h->err_host);
+}
+
+onela::StepParams base_params(const onela_handle *h) {
+  onela::StepParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.R = h->cfg.R;
+  p.H = h->cfg.H;
+  p.dk = h->cfg.d_k;
+  p.dv = h->cfg.d_v;
+  p.W_max = h->cfg.W_max;
+  p.T_max = h->cfg.T_max;
+  p.S0 = h->S0;
+  p.S0img = h->S0img;
+  p.s0_planes = h->planes;
+  p.rec_alpha = h->rec_alpha;
+  p.rec_delta = h->rec_delta;
+  p.rec_k = h->rec_k;
+  p.anc = h->anc;
+  p.err = h->err_dev;
+  return p;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *onela_error_string(int code) {
+  switch (code) {
+    case ONELA_OK: return "ok";
+    case ONELA_ERR_ARG: return "invalid argument";
+    case ONELA_ERR_STATE: return "no prompt state installed";
+    case ONELA_ERR_CAPACITY: return "step or beam count beyond the handle's capacity";
+    case ONELA_ERR_PARENT: return "parent index outside [0, W_prev) seen on the device";
+    case ONELA_ERR_CUDA: return "CUDA call failed";
+    case ONELA_ERR_UNSUPPORTED: return "kernel does not support this shape";
+    default: return "unknown error";
+  }
+}
+
+int onela_create(const onela_config *cfg, onela_handle **out) {
+  if (!cfg || !out) return ONELA_ERR_ARG;
+  *out = nullptr;
+  const onela_config c = *cfg;
+  if (c.R < 1 || c.H < 1 || c.d_k < 1 || c.d_k > 256 || c.d_v < 1 || c.d_v > 256 || c.W_max < 1 ||
+      c.T_max < 1 || c.T_max > 64 || !valid_dtype(c.s0_dtype) || !valid_dtype(c.qkv_dtype) ||
+      c.kernel < ONELA_KERNEL_AUTO || c.kernel > ONELA_KERNEL_TC || c.device < 0 ||
+      !(c.s0_split == 0 || c.s0_split == 2 || c.s0_split == 3))
+    return ONELA_ERR_ARG;
+  // Sizes must stay addressable with 64-bit offsets and the kernels' int grid.
+  const double rows = (double)c.T_max * c.R * c.H * c.W_max;
+  if (rows * (4.0 + 4.0 * c.d_v + esize(c.qkv_dtype) * (double)c.d_k) > 1.5e11) return ONELA_ERR_ARG;
+  if ((double)c.R * c.W_max * c.H * (c.d_k > c.d_v ? c.d_k : c.d_v) > 2.0e9) return ONELA_ERR_ARG;
+
+  const int qkv_bf16 = c.qkv_dtype == ONELA_BF16;
+  int kernel = c.kernel;
+  if (kernel == ONELA_KERNEL_AUTO) kernel = onela::tc_supports(c.d_k, c.d_v, qkv_bf16, c.T_max) ? ONELA_KERNEL_TC : ONELA_KERNEL_SIMT;
+  if (kernel == ONELA_KERNEL_TC && !onela::tc_supports(c.d_k, c.d_v, qkv_bf16, c.T_max)) return ONELA_ERR_UNSUPPORTED;
+
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || c.device >= ndev) return ONELA_ERR_CUDA;
+  DeviceGuard g(c.device);
+  if (!g.ok) return ONELA_ERR_CUDA;
+
+  onela_handle *h = new (std::nothrow) onela_handle();
+  if (!h) return ONELA_ERR_CUDA;
+  h->cfg = c;
+  h->kernel = kernel;
+  h->planes = c.s0_dtype == ONELA_BF16 ? 1 : (c.s0_split == 0 ? 2 : c.s0_split);
+  h->steps_done = 0;
+  h->has_prompt = 0;
+  const size_t nS0 = (size_t)c.R * c.H * c.d_v * c.d_k;
+  const size_t nrow = (size_t)c.T_max * c.R * c.H * c.W_max;
+  bool ok = cudaMalloc(&h->S0, nS0 * esize(c.s0_dtype)) == cudaSuccess;
+  if (ok && kernel == ONELA_KERNEL_TC)
+    ok = cudaMalloc(&h->S0img, onela::s0_image_bytes(c.R, c.H, c.d_k, c.d_v, h->planes)) == cudaSuccess;
+  ok = ok && cudaMalloc((void **)&h->rec_alpha, nrow * sizeof(float)) == cudaSuccess;
+  ok = ok && cudaMalloc((void **)&h->rec_delta, nrow * c.d_v * sizeof(float)) == cudaSuccess;
+  ok = ok && cudaMalloc(&h->rec_k, nrow * c.d_k * esize(c.qkv_dtype)) == cudaSuccess;
+  ok = ok && cudaMalloc((void **)&h->anc, (size_t)c.T_max * c.R * c.W_max * c.T_max * sizeof(int32_t)) == cudaSuccess;
+  ok = ok && cudaHostAlloc((void **)&h->err_host, sizeof(int32_t), cudaHostAllocMapped) == cudaSuccess;
+  ok = ok && cudaHostGetDevicePointer((void **)&h->err_dev, h->err_host, 0) == cudaSuccess;
+  if (ok) {
+    *h->err_host = 0;
+    // Zeroed so that nothing uninitialised is ever read, even after a bad parent.
+    ok = cudaMemset(h->rec_alpha, 0, nrow * sizeof(float)) == cudaSuccess &&
+         cudaMemset(h->anc, 0, (size_t)c.T_max * c.R * c.W_max * c.T_max * sizeof(int32_t)) == cudaSuccess &&
+         cudaDeviceSynchronize() == cudaSuccess;
+  }
+  if (!ok) {
+    cudaGetLastError();
+    free_all(h);
+    delete h;
+    return ONELA_ERR_CUDA;
+  }
+  *out = h;
+  return ONELA_OK;
+}
+
+int onela_set_prompt_state(onela_handle *h, const void *S0, onela_stream stream) {
+  if (!h || !S0) return ONELA_ERR_ARG;
+  DeviceGuard g(h->cfg.device);
+  if (!g.ok) return ONELA_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const onela_config &c = h->cfg;
+  const size_t bytes = (size_t)c.R * c.H * c.d_v * c.d_k * esize(c.s0_dtype);
+  if (cudaMemcpyAsync(h->S0, S0, bytes, cudaMemcpyDeviceToDevice, s) != cudaSuccess) return ONELA_ERR_CUDA;
+  if (h->kernel == ONELA_KERNEL_TC) {
+    if (onela::launch_s0_image(h->S0, h->S0img, c.R, c.H, c.d_k, c.d_v, c.s0_dtype == ONELA_BF16, h->planes, s) !=
+        cudaSuccess)
+      return ONELA_ERR_CUDA;
+  }
+  h->has_prompt = 1;
+  h->steps_done = 0;
+  h->Ws.clear();
+  return ONELA_OK;
+}
+
+int onela_decode_step(onela_handle *h, int32_t W_prev, int32_t W, const void *q, const void *k, const void *v,
+                      const float *gate, const float *beta, const int32_t *parent_idx, float *o,
+                      onela_stream stream) {
+  if (!h || !q || !k || !v || !gate || !beta || !parent_idx || !o) return ONELA_ERR_ARG;
+  if (*reinterpret_cast<volatile int32_t *>(h->err_host) & onela::kErrParent) return ONELA_ERR_PARENT;
+  if (!h->has_prompt) return ONELA_ERR_STATE;
+  const onela_config &c = h->cfg;
+  if (W < 1) return ONELA_ERR_ARG;
+  if (W > c.W_max || h->steps_done >= c.T_max) return ONELA_ERR_CAPACITY;
+  const int expect_prev = h->steps_done == 0 ? 1 : h->Ws.back();
+  if (W_prev != expect_prev) return ONELA_ERR_ARG;
+  DeviceGuard g(c.device);
+  if (!g.ok) return ONELA_ERR_CUDA;
+
+  onela::StepParams p = base_params(h);
+  p.W = W;
+  p.W_prev = W_prev;
+  p.t = h->steps_done + 1;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.g = gate;
+  p.beta = beta;
+  p.parents = parent_idx;
+  p.o = o;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (h->kernel == ONELA_KERNEL_TC)
+    e = onela::launch_step_tc(p, c.s0_dtype == ONELA_BF16, s);
+  else
+    e = onela::launch_step_simt(p, c.qkv_dtype == ONELA_BF16, c.s0_dtype == ONELA_BF16, s);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return ONELA_ERR_CUDA;
+  }
+  h->steps_done += 1;
+  h->Ws.push_back(W);
+  return ONELA_OK;
+}
+
+int onela_reset(onela_handle *h, onela_stream stream) {
+  if (!h) return ONELA_ERR_ARG;
+  DeviceGuard g(h->cfg.device);
+  if (!g.ok) return ONELA_ERR_CUDA;
+  // Work still in flight could set the error word after it is cleared.
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ONELA_ERR_CUDA;
+  *reinterpret_cast<volatile int32_t *>(h->err_host) = 0;
+  h->steps_done = 0;
+  h->Ws.clear();
+  return ONELA_OK;
+}
+
+int onela_status(onela_handle *h, int32_t *device_err) {
+  if (!h) return ONELA_ERR_ARG;
+  DeviceGuard g(h->cfg.device);
+  if (!g.ok) return ONELA_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return ONELA_ERR_CUDA;
+  const int32_t e = *reinterpret_cast<volatile int32_t *>(h->err_host);
+  if (device_err) *device_err = e;
+  return (e & onela::kErrParent) ? ONELA_ERR_PARENT : ONELA_OK;
+}
+
+int onela_destroy(onela_handle *h) {
+  if (!h) return ONELA_ERR_ARG;
+  {
+    DeviceGuard g(h->cfg.device);
+    cudaDeviceSynchronize();
+    free_all(h);
+  }
+  delete h;
+  return ONELA_OK;
+}
+
+int onela_read_records(onela_handle *h, int32_t t, float *alpha, float *delta, void *k, onela_stream stream) {
+  if (!h || t < 1 || t > h->steps_done) return ONELA_ERR_ARG;
+  DeviceGuard g(h->cfg.device);
+  if (!g.ok) return ONELA_ERR_CUDA;
+  const onela_config &c = h->cfg;
+  const int Wt = h->Ws[t - 1];
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t ks = esize(c.qkv_dtype);
+  // Rows are [R][H][W_max]: copy the first W_t rows of each (r, h) block.
+  const size_t nblk = (size_t)c.R * c.H;
+  const size_t base = (size_t)(t - 1) * nblk * c.W_max;
+  bool ok = true;
+  if (alpha)
+    ok = ok && cudaMemcpy2DAsync(alpha, Wt * sizeof(float), h->rec_alpha + base, (size_t)c.W_max * sizeof(float),
+                                 Wt * sizeof(float), nblk, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
+  if (delta)
+    ok = ok && cudaMemcpy2DAsync(delta, (size_t)Wt * c.d_v * sizeof(float), h->rec_delta + base * c.d_v,
+                                 (size_t)c.W_max * c.d_v * sizeof(float), (size_t)Wt * c.d_v * sizeof(float), nblk,
+                                 cudaMemcpyDeviceToDevice, s) == cudaSuccess;
+  if (k)
+    ok = ok && cudaMemcpy2DAsync(k, (size_t)Wt * c.d_k * ks, static_cast<char *>(h->rec_k) + base * c.d_k * ks,
+                                 (size_t)c.W_max * c.d_k * ks, (size_t)Wt * c.d_k * ks, nblk,
+                                 cudaMemcpyDeviceToDevice, s) == cudaSuccess;
+  return ok ? ONELA_OK : ONELA_ERR_CUDA;
+}
+
+int onela_read_ancestry(onela_handle *h, int32_t t, int32_t *anc, onela_stream stream) {
+  if (!h || !anc || t < 1 || t > h->steps_done) return ONELA_ERR_ARG;
+  if (t == 1) return ONELA_OK;  // the chain of a depth-1 beam is empty
+  DeviceGuard g(h->cfg.device);
+  if (!g.ok) return ONELA_ERR_CUDA;
+  const onela_config &c = h->cfg;
+  const int Wt = h->Ws[t - 1];
+  // Source rows [R][W_max][T_max] -> dest [R][W_t][t-1].
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  for (int r = 0; r < c.R; ++r) {
+    const int32_t *src = h->anc + ((size_t)(t - 1) * c.R + r) * c.W_max * c.T_max;
+    if (cudaMemcpy2DAsync(anc + (size_t)r * Wt * (t - 1), (t - 1) * sizeof(int32_t), src, c.T_max * sizeof(int32_t),
+                          (t - 1) * sizeof(int32_t), Wt, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+      return ONELA_ERR_CUDA;
+  }
+  return ONELA_OK;
+}
+
+int onela_steps_done(const onela_handle *h) { return h ? h->steps_done : -1; }
+
+int onela_kernel_kind(const onela_handle *h) { return h ? h->kernel : -1; }
+
+}  // extern "C"
