@@ -15,7 +15,7 @@ pytestmark = pytest.mark.gpu
 def kernels_for(dk, dv, qkv):
     import linear_attention_beam_shared_b200 as L
     ks = [L.ONELA_KERNEL_SIMT]
-    if qkv == "bf16" and dk == dv and dk in (64, 128, 256) and _tc_available():
+    if qkv == "bf16" and dk == dv and dk in (64, 128) and _tc_available():
         ks.append(L.ONELA_KERNEL_TC)
     return ks
 
