@@ -69,7 +69,9 @@ enum {
                                 [0, W_prev); reported by the next call or by
                                 onela_status                                 */
   ONELA_ERR_CUDA = 5,        /* a CUDA call failed (allocation, launch ...)  */
-  ONELA_ERR_UNSUPPORTED = 6  /* the requested kernel cannot run this shape   */
+  ONELA_ERR_UNSUPPORTED = 6, /* the requested kernel cannot run this shape   */
+  ONELA_ERR_SCRATCH = 7      /* onela_decode_step_noalloc: the decode does not
+                                fit in its fixed 32 MiB device array         */
 };
 
 /* Which decode kernel runs.  AUTO picks the tensor-core kernel when the
@@ -177,6 +179,48 @@ ONELA_API int onela_read_ancestry(onela_handle *h, int32_t t, int32_t *anc,
  * the handle runs (ONELA_KERNEL_SIMT or ONELA_KERNEL_TC). */
 ONELA_API int onela_steps_done(const onela_handle *h);
 ONELA_API int onela_kernel_kind(const onela_handle *h);
+
+/* Decode step without any device allocation.
+ *
+ * The paper has no counterpart to this entry point; it exists for callers
+ * that cannot allocate device memory: code running while a CUDA stream is
+ * being captured (cudaMalloc is refused there) and plug-ins whose host engine
+ * owns all device memory and passes them nothing but their input and output
+ * tensors.  It computes exactly what onela_decode_step computes (same SIMT
+ * kernel), but keeps the record store, the ancestry index and the error word
+ * in one fixed array of 32 MiB that is part of the library (a file-scope
+ * __device__ array), instead of in memory owned by a handle.
+ *
+ *   cfg        shapes and dtypes (R, H, d_k, d_v, W_max, T_max, s0_dtype,
+ *              qkv_dtype, device); kernel and s0_split are ignored.  W_max and
+ *              T_max fix the array's layout and must stay the same for all
+ *              steps of one decode.
+ *   t          this step's depth, 1..T_max; call t = 1, 2, ... in order.
+ *              A call with t = 1 starts a new decode and clears the error
+ *              word.
+ *   W_prev, W  beams of the previous step (1 at t = 1) and of this one.
+ *   S0         [R][H][d_v][d_k] in s0_dtype, read directly at every step.
+ *   q, k, v, g, beta, parent_idx, o   as for onela_decode_step.
+ *   status     DEVICE pointer to one int32, written on `stream` with the
+ *              error word after the step: 0, or bit 0 set when some parent
+ *              index of this decode was outside [0, W_prev) (the index was
+ *              clamped to 0 and the outputs are meaningless).
+ * Memory: the array lives on every device where the library's module holding
+ * it is loaded, from the first call on that device until the process exits.
+ * Set-up: the first call on a device, with that device current, looks up the
+ * array's device address once; make that first call before any stream
+ * capture begins.  No call allocates or frees device memory.
+ * Sharing: every call, from any thread or stream, uses the same array and
+ * sees what the previous call left there, so decodes whose calls overlap on
+ * the GPU race with one another and give wrong results; run one decode at a
+ * time per device.
+ * Errors: ONELA_ERR_ARG (null pointer, invalid shape, t or W out of range),
+ * ONELA_ERR_SCRATCH (T_max * R * H * W_max records plus the ancestry rows do
+ * not fit in 32 MiB), ONELA_ERR_CUDA. */
+ONELA_API int onela_decode_step_noalloc(const onela_config *cfg, int32_t t, int32_t W_prev, int32_t W,
+                                        const void *S0, const void *q, const void *k, const void *v,
+                                        const float *g, const float *beta, const int32_t *parent_idx,
+                                        float *o, int32_t *status, onela_stream stream);
 
 /* Static description of a return code (never NULL). */
 ONELA_API const char *onela_error_string(int code);

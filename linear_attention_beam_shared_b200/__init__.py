@@ -20,8 +20,8 @@ from . import _lib
 from ._lib import (  # noqa: F401
     ONELA_BF16, ONELA_ERR_ARG, ONELA_ERR_CAPACITY, ONELA_ERR_CUDA, ONELA_ERR_PARENT,
     ONELA_ERR_STATE, ONELA_ERR_UNSUPPORTED, ONELA_F32, ONELA_KERNEL_AUTO, ONELA_KERNEL_SIMT,
-    ONELA_KERNEL_TC, ONELA_OK, Handle, OnelaError, error_string, onela_create, onela_decode_step,
-    onela_destroy, onela_kernel_kind, onela_read_ancestry, onela_read_records, onela_reset,
+    ONELA_ERR_SCRATCH, ONELA_KERNEL_TC, ONELA_OK, Handle, OnelaError, error_string, onela_create,
+    onela_decode_step, onela_decode_step_noalloc, onela_destroy, onela_kernel_kind, onela_read_ancestry, onela_read_records, onela_reset,
     onela_set_prompt_state, onela_status, onela_status_code, onela_steps_done,
 )
 

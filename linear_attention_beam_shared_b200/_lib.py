@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_PKG, "libonela_b200.so")
 
 ONELA_F32, ONELA_BF16 = 0, 1
 ONELA_OK, ONELA_ERR_ARG, ONELA_ERR_STATE, ONELA_ERR_CAPACITY = 0, 1, 2, 3
-ONELA_ERR_PARENT, ONELA_ERR_CUDA, ONELA_ERR_UNSUPPORTED = 4, 5, 6
+ONELA_ERR_PARENT, ONELA_ERR_CUDA, ONELA_ERR_UNSUPPORTED, ONELA_ERR_SCRATCH = 4, 5, 6, 7
 ONELA_KERNEL_AUTO, ONELA_KERNEL_SIMT, ONELA_KERNEL_TC = 0, 1, 2
 
 _DT = {ONELA_F32: torch.float32, ONELA_BF16: torch.bfloat16}
@@ -57,6 +57,8 @@ def _load() -> ctypes.CDLL:
         "onela_steps_done": ([vp], ctypes.c_int),
         "onela_kernel_kind": ([vp], ctypes.c_int),
         "onela_error_string": ([ctypes.c_int], ctypes.c_char_p),
+        "onela_decode_step_noalloc": ([ctypes.POINTER(onela_config), i32, i32, i32, vp, vp, vp, vp, vp,
+                                       vp, vp, vp, vp, vp], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -202,3 +204,27 @@ def onela_steps_done(h: Handle) -> int:
 
 def onela_kernel_kind(h: Handle) -> int:
     return int(lib.onela_kernel_kind(h.ptr))
+
+
+def onela_decode_step_noalloc(R: int, H: int, d_k: int, d_v: int, W_max: int, T_max: int,
+                              s0_dtype, qkv_dtype, t: int, W_prev: int, W: int, S0, q, k, v, g,
+                              beta, parent_idx, o, status, device: int = 0, stream=None) -> None:
+    """Decode step t that allocates no device memory (state in the library's
+    fixed 32 MiB array).  status: int32 CUDA tensor of one element, written
+    with the error word."""
+    cfg = onela_config(R, H, d_k, d_v, W_max, T_max, _DT_CODE[s0_dtype], _DT_CODE[qkv_dtype],
+                       0, 0, device)
+    dt = _DT[cfg.qkv_dtype]
+    args = (
+        _ptr(S0, "S0", _DT[cfg.s0_dtype], (R, H, d_v, d_k), device),
+        _ptr(q, "q", dt, (R, W, H, d_k), device),
+        _ptr(k, "k", dt, (R, W, H, d_k), device),
+        _ptr(v, "v", dt, (R, W, H, d_v), device),
+        _ptr(g, "g", torch.float32, (R, W, H), device),
+        _ptr(beta, "beta", torch.float32, (R, W, H), device),
+        _ptr(parent_idx, "parent_idx", torch.int32, (R, W), device),
+        _ptr(o, "o", torch.float32, (R, W, H, d_v), device),
+        _ptr(status, "status", torch.int32, (1,), device),
+    )
+    _check(lib.onela_decode_step_noalloc(ctypes.byref(cfg), int(t), int(W_prev), int(W), *args,
+                                         _stream(stream)), "onela_decode_step_noalloc")

@@ -89,6 +89,7 @@ const char *onela_error_string(int code) {
     case ONELA_ERR_PARENT: return "parent index outside [0, W_prev) seen on the device";
     case ONELA_ERR_CUDA: return "CUDA call failed";
     case ONELA_ERR_UNSUPPORTED: return "kernel does not support this shape";
+    case ONELA_ERR_SCRATCH: return "decode does not fit in the 32 MiB array of onela_decode_step_noalloc";
     default: return "unknown error";
   }
 }
