@@ -219,8 +219,11 @@ def run_ours(args):
             (wl.R, wl.H, wl.d_v, wl.d_k)), wl.s0_dtype)
     steps = synth.draw_decode(wl)
     kernel = {"auto": L.ONELA_KERNEL_AUTO, "simt": L.ONELA_KERNEL_SIMT, "tc": L.ONELA_KERNEL_TC}[args.kernel]
+    # Inputs are resident before the graph runs and the steps follow one
+    # another directly, so steps 2..T may start while the previous one ends.
+    flags = 0 if args.no_pdl else L.ONELA_FLAG_PDL
     dec = L.BeamDecoder(wl.R, wl.H, wl.d_k, wl.d_v, wl.W, wl.T, wl.s0_dtype, wl.qkv_dtype,
-                        kernel=kernel, device=device.index)
+                        kernel=kernel, device=device.index, flags=flags)
     kind = {L.ONELA_KERNEL_SIMT: "simt", L.ONELA_KERNEL_TC: "tc"}[dec.kernel]
     dec.set_prompt_state(S0.to(device))
     dsteps = [{k: (v.to(device) if isinstance(v, torch.Tensor) else v) for k, v in s.items()} for s in steps]
@@ -294,7 +297,13 @@ def run_ours(args):
 
     # End to end through the public API with host buffers: per step the H2D
     # copy of that step's inputs from pinned memory, the decode call, and the
-    # D2H read of its output o.
+    # D2H read of its output o.  A handle without the programmatic-launch
+    # flag: here a copy, not the previous step, precedes each step.
+    del graph
+    dec.close()
+    dec = L.BeamDecoder(wl.R, wl.H, wl.d_k, wl.d_v, wl.W, wl.T, wl.s0_dtype, wl.qkv_dtype,
+                        kernel=kernel, device=device.index)
+    dec.set_prompt_state(S0.to(device))
     host_in = [{k: (v.pin_memory() if isinstance(v, torch.Tensor) else v) for k, v in s.items()} for s in steps]
     host_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
     h2d = sum(v.numel() * v.element_size() for s in steps for v in s.values() if isinstance(v, torch.Tensor))
@@ -332,7 +341,6 @@ def run_ours(args):
                "sample": f"whole {args.workload} decode (R=1,H={wl.H},W={wl.W},T={wl.T}) x{reps} "
                          f"in {el:.1f} s, plain-C fp64 full-state oracle"}
 
-    del graph
     dec.close()
     if rank == 0:
         line = {
@@ -345,7 +353,8 @@ def run_ours(args):
                                    f"q/k/v {wl.qkv_dtype}, parents Zipf(1.1)",
                        "global_batch": wl.R * ws, "seq_len": wl.T, "parallelism": f"replicas{ws}",
                        "l2": "flushed (512 MiB write) before every timed step", "kernel": kind,
-                       "step": f"one whole {wl.T}-step decode in a CUDA graph"},
+                       "step": f"one whole {wl.T}-step decode in a CUDA graph",
+                       "programmatic_launch": not args.no_pdl},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "clocks": clk.summary(), "gpu_launches": launches * args.steps,
         }
@@ -398,6 +407,8 @@ def main():
     ap.add_argument("--workload", default="long5k")
     ap.add_argument("--kernel", choices=["auto", "simt", "tc"], default="auto")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline leg")
+    ap.add_argument("--no-pdl", action="store_true",
+                    help="launch every step only after the previous one has finished")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--s0", choices=["prefill", "direct"], default="prefill",
                     help="S0 from the GDN recurrence over the synthetic prompt (default) or drawn "

@@ -74,9 +74,21 @@ enum {
                                 fit in its fixed 32 MiB device array         */
 };
 
+/* onela_config.flags bits.
+ *   ONELA_FLAG_PDL  launch decode steps t >= 2 of the tensor-core kernel as
+ *                   programmatic dependents of the kernel before them in the
+ *                   stream: step t starts loading its inputs and S0 while
+ *                   step t-1 finishes, and waits for step t-1 only before it
+ *                   touches the records.  Set it only when that earlier
+ *                   kernel does not produce any input of step t (q, k, v, g,
+ *                   beta, parent_idx) -- e.g. back-to-back decode steps whose
+ *                   inputs were all written before the first of them, as in
+ *                   a CUDA graph of a whole decode.  Step 1 never overlaps. */
+enum { ONELA_FLAG_PDL = 1 };
+
 /* Which decode kernel runs.  AUTO picks the tensor-core kernel when the
- * shape allows it (bf16 q/k/v, d_k and d_v in {64, 128, 256}) and the SIMT
- * kernel otherwise. */
+ * shape allows it (bf16 q/k/v, d_k = d_v in {64, 128}, T_max <= 16,
+ * W_max <= 1024) and the SIMT kernel otherwise. */
 enum { ONELA_KERNEL_AUTO = 0, ONELA_KERNEL_SIMT = 1, ONELA_KERNEL_TC = 2 };
 
 /* Handle configuration.
@@ -92,6 +104,7 @@ enum { ONELA_KERNEL_AUTO = 0, ONELA_KERNEL_SIMT = 1, ONELA_KERNEL_TC = 2 };
  *                   terms S0 is split into (2 or 3; 0 means 2).  Ignored
  *                   otherwise.
  *   device          CUDA device ordinal the handle lives on.
+ *   flags           ONELA_FLAG_* bits (0: none).
  */
 typedef struct {
   int32_t R, H, d_k, d_v, W_max, T_max;
@@ -100,11 +113,14 @@ typedef struct {
   int32_t kernel;
   int32_t s0_split;
   int32_t device;
+  int32_t flags;
 } onela_config;
 
 /* Create a handle: validates cfg and allocates, on cfg->device, the S0 copy,
  * the record store (alpha fp32 [T_max][R][H][W_max], delta fp32
- * [T_max][R][H][W_max][d_v], k [T_max][R][H][W_max][d_k] in qkv_dtype), the
+ * [T_max][R][H][W_max][d_v], k [T_max][R][H][W_max][d_k] in qkv_dtype; the
+ * tensor-core kernel also keeps, per record, the product of the gates on its
+ * path from the root, fp32 [T_max][R][H][W_max]), the
  * ancestry index (int32 [T_max][R][W_max][T_max]) and an error word in
  * mapped, pinned host memory that the kernels write and the host reads.
  * Host-side allocation only; no kernel runs.  *out receives the handle.
@@ -192,7 +208,7 @@ ONELA_API int onela_kernel_kind(const onela_handle *h);
  * __device__ array), instead of in memory owned by a handle.
  *
  *   cfg        shapes and dtypes (R, H, d_k, d_v, W_max, T_max, s0_dtype,
- *              qkv_dtype, device); kernel and s0_split are ignored.  W_max and
+ *              qkv_dtype, device); kernel, s0_split and flags are ignored.  W_max and
  *              T_max fix the array's layout and must stay the same for all
  *              steps of one decode.
  *   t          this step's depth, 1..T_max; call t = 1, 2, ... in order.

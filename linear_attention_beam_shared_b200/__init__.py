@@ -19,7 +19,7 @@ import torch
 from . import _lib
 from ._lib import (  # noqa: F401
     ONELA_BF16, ONELA_ERR_ARG, ONELA_ERR_CAPACITY, ONELA_ERR_CUDA, ONELA_ERR_PARENT,
-    ONELA_ERR_STATE, ONELA_ERR_UNSUPPORTED, ONELA_F32, ONELA_KERNEL_AUTO, ONELA_KERNEL_SIMT,
+    ONELA_ERR_STATE, ONELA_ERR_UNSUPPORTED, ONELA_F32, ONELA_FLAG_PDL, ONELA_KERNEL_AUTO, ONELA_KERNEL_SIMT,
     ONELA_ERR_SCRATCH, ONELA_KERNEL_TC, ONELA_OK, Handle, OnelaError, error_string, onela_create,
     onela_decode_step, onela_decode_step_noalloc, onela_destroy, onela_kernel_kind, onela_read_ancestry, onela_read_records, onela_reset,
     onela_set_prompt_state, onela_status, onela_status_code, onela_steps_done,
@@ -32,9 +32,9 @@ class BeamDecoder:
     """Owns one handle; tracks the beam count of the previous step."""
 
     def __init__(self, R, H, d_k, d_v, W_max, T_max, s0_dtype="f32", qkv_dtype="bf16",
-                 kernel=ONELA_KERNEL_AUTO, s0_split=0, device=0):
+                 kernel=ONELA_KERNEL_AUTO, s0_split=0, device=0, flags=0):
         self.h = onela_create(R, H, d_k, d_v, W_max, T_max, s0_dtype, qkv_dtype, kernel,
-                              s0_split, device)
+                              s0_split, device, flags)
         self.device = torch.device("cuda", device)
         self.W_prev = 1
         self.Ws = []

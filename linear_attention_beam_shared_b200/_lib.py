@@ -21,6 +21,7 @@ ONELA_F32, ONELA_BF16 = 0, 1
 ONELA_OK, ONELA_ERR_ARG, ONELA_ERR_STATE, ONELA_ERR_CAPACITY = 0, 1, 2, 3
 ONELA_ERR_PARENT, ONELA_ERR_CUDA, ONELA_ERR_UNSUPPORTED, ONELA_ERR_SCRATCH = 4, 5, 6, 7
 ONELA_KERNEL_AUTO, ONELA_KERNEL_SIMT, ONELA_KERNEL_TC = 0, 1, 2
+ONELA_FLAG_PDL = 1
 
 _DT = {ONELA_F32: torch.float32, ONELA_BF16: torch.bfloat16}
 _DT_CODE = {"f32": ONELA_F32, "bf16": ONELA_BF16, torch.float32: ONELA_F32, torch.bfloat16: ONELA_BF16}
@@ -29,7 +30,7 @@ _DT_CODE = {"f32": ONELA_F32, "bf16": ONELA_BF16, torch.float32: ONELA_F32, torc
 class onela_config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "R", "H", "d_k", "d_v", "W_max", "T_max", "s0_dtype", "qkv_dtype",
-        "kernel", "s0_split", "device")]
+        "kernel", "s0_split", "device", "flags")]
 
 
 class OnelaError(RuntimeError):
@@ -120,9 +121,9 @@ class Handle:
 
 def onela_create(R: int, H: int, d_k: int, d_v: int, W_max: int, T_max: int,
                  s0_dtype="f32", qkv_dtype="bf16", kernel: int = ONELA_KERNEL_AUTO,
-                 s0_split: int = 0, device: int = 0) -> Handle:
+                 s0_split: int = 0, device: int = 0, flags: int = 0) -> Handle:
     cfg = onela_config(R, H, d_k, d_v, W_max, T_max, _DT_CODE[s0_dtype], _DT_CODE[qkv_dtype],
-                       kernel, s0_split, device)
+                       kernel, s0_split, device, flags)
     out = ctypes.c_void_p()
     _check(lib.onela_create(ctypes.byref(cfg), ctypes.byref(out)), "onela_create")
     return Handle(out.value, cfg)

@@ -21,6 +21,9 @@ struct StepParams {
   const void *S0img;      // tensor-core operand image of S0 (see step_tc.cu)
   int s0_planes;          // bf16 terms in S0img (1 for bf16 S0)
   float *rec_alpha;       // [T_max][R][H][W_max]
+  float *rec_P;           // [T_max][R][H][W_max]: product of the gates on the
+                          // path from the root to the record, inclusive
+                          // (tensor-core kernel only; may be null otherwise)
   float *rec_delta;       // [T_max][R][H][W_max][dv]
   void *rec_k;            // [T_max][R][H][W_max][dk] in the qkv type
   int32_t *anc;           // [T_max][R][W_max][T_max]
@@ -41,10 +44,10 @@ constexpr int32_t kErrParent = 1;
 
 // Kernel launchers (step_simt.cu, step_tc.cu).  Return a cudaError_t.
 cudaError_t launch_step_simt(const StepParams &p, int qkv_bf16, int s0_bf16, cudaStream_t s);
-cudaError_t launch_step_tc(const StepParams &p, int s0_bf16, cudaStream_t s);
+cudaError_t launch_step_tc(const StepParams &p, int pdl, cudaStream_t s);
 cudaError_t launch_s0_image(const void *S0, void *img, int R, int H, int dk, int dv,
                             int s0_bf16, int planes, cudaStream_t s);
 size_t s0_image_bytes(int R, int H, int dk, int dv, int planes);
-bool tc_supports(int dk, int dv, int qkv_bf16, int T_max);
+bool tc_supports(int dk, int dv, int qkv_bf16, int T_max, int W_max);
 
 }  // namespace onela

@@ -20,6 +20,7 @@ struct onela_handle {
   void *S0;
   void *S0img;
   float *rec_alpha;
+  float *rec_P;
   float *rec_delta;
   void *rec_k;
   int32_t *anc;
@@ -50,6 +51,7 @@ void free_all(onela_handle *h) {
   cudaFree(h->S0);
   cudaFree(h->S0img);
   cudaFree(h->rec_alpha);
+  cudaFree(h->rec_P);
   cudaFree(h->rec_delta);
   cudaFree(h->rec_k);
   cudaFree(h->anc);
@@ -69,6 +71,7 @@ onela::StepParams base_params(const onela_handle *h) {
   p.S0img = h->S0img;
   p.s0_planes = h->planes;
   p.rec_alpha = h->rec_alpha;
+  p.rec_P = h->rec_P;
   p.rec_delta = h->rec_delta;
   p.rec_k = h->rec_k;
   p.anc = h->anc;
@@ -101,7 +104,7 @@ int onela_create(const onela_config *cfg, onela_handle **out) {
   if (c.R < 1 || c.H < 1 || c.d_k < 1 || c.d_k > 256 || c.d_v < 1 || c.d_v > 256 || c.W_max < 1 ||
       c.T_max < 1 || c.T_max > 64 || !valid_dtype(c.s0_dtype) || !valid_dtype(c.qkv_dtype) ||
       c.kernel < ONELA_KERNEL_AUTO || c.kernel > ONELA_KERNEL_TC || c.device < 0 ||
-      !(c.s0_split == 0 || c.s0_split == 2 || c.s0_split == 3))
+      !(c.s0_split == 0 || c.s0_split == 2 || c.s0_split == 3) || (c.flags & ~ONELA_FLAG_PDL) != 0)
     return ONELA_ERR_ARG;
   // Sizes must stay addressable with 64-bit offsets and the kernels' int grid.
   const double rows = (double)c.T_max * c.R * c.H * c.W_max;
@@ -110,8 +113,8 @@ int onela_create(const onela_config *cfg, onela_handle **out) {
 
   const int qkv_bf16 = c.qkv_dtype == ONELA_BF16;
   int kernel = c.kernel;
-  if (kernel == ONELA_KERNEL_AUTO) kernel = onela::tc_supports(c.d_k, c.d_v, qkv_bf16, c.T_max) ? ONELA_KERNEL_TC : ONELA_KERNEL_SIMT;
-  if (kernel == ONELA_KERNEL_TC && !onela::tc_supports(c.d_k, c.d_v, qkv_bf16, c.T_max)) return ONELA_ERR_UNSUPPORTED;
+  if (kernel == ONELA_KERNEL_AUTO) kernel = onela::tc_supports(c.d_k, c.d_v, qkv_bf16, c.T_max, c.W_max) ? ONELA_KERNEL_TC : ONELA_KERNEL_SIMT;
+  if (kernel == ONELA_KERNEL_TC && !onela::tc_supports(c.d_k, c.d_v, qkv_bf16, c.T_max, c.W_max)) return ONELA_ERR_UNSUPPORTED;
 
   int ndev = 0;
   if (cudaGetDeviceCount(&ndev) != cudaSuccess || c.device >= ndev) return ONELA_ERR_CUDA;
@@ -131,6 +134,7 @@ int onela_create(const onela_config *cfg, onela_handle **out) {
   if (ok && kernel == ONELA_KERNEL_TC)
     ok = cudaMalloc(&h->S0img, onela::s0_image_bytes(c.R, c.H, c.d_k, c.d_v, h->planes)) == cudaSuccess;
   ok = ok && cudaMalloc((void **)&h->rec_alpha, nrow * sizeof(float)) == cudaSuccess;
+  if (ok && kernel == ONELA_KERNEL_TC) ok = cudaMalloc((void **)&h->rec_P, nrow * sizeof(float)) == cudaSuccess;
   ok = ok && cudaMalloc((void **)&h->rec_delta, nrow * c.d_v * sizeof(float)) == cudaSuccess;
   ok = ok && cudaMalloc(&h->rec_k, nrow * c.d_k * esize(c.qkv_dtype)) == cudaSuccess;
   ok = ok && cudaMalloc((void **)&h->anc, (size_t)c.T_max * c.R * c.W_max * c.T_max * sizeof(int32_t)) == cudaSuccess;
@@ -200,7 +204,7 @@ int onela_decode_step(onela_handle *h, int32_t W_prev, int32_t W, const void *q,
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (h->kernel == ONELA_KERNEL_TC)
-    e = onela::launch_step_tc(p, c.s0_dtype == ONELA_BF16, s);
+    e = onela::launch_step_tc(p, (c.flags & ONELA_FLAG_PDL) && p.t >= 2, s);
   else
     e = onela::launch_step_simt(p, c.qkv_dtype == ONELA_BF16, c.s0_dtype == ONELA_BF16, s);
   if (e != cudaSuccess) {

@@ -1,39 +1,51 @@
 // Tensor-core decode-step kernel (tcgen05, sm_100a) for bf16 q/k/v and
 // d_k = d_v in {64, 128}.
 //
-// One CTA per (request r, head h, tile of 32 beams); 256 threads.  The step
-// of the shared-state GDN beam decode (OneLA, evolve.pub review, key claims
-// on section 3.2, equations 2-4) becomes two small dense contractions on the
-// tensor cores plus a SIMT epilogue:
+// One CTA per (request r, head h, tile of 32 beams); 256 threads; two CTAs
+// fit on an SM, so a step launched as a programmatic dependent runs its
+// input phase beside the previous step.  The step of the shared-state GDN
+// beam decode (OneLA, evolve.pub review, key claims on section 3.2,
+// equations 2-4) runs as dense products on the tensor cores, fp32
+// accumulators in TMEM:
 //
-//   D1 = S0 . X^T    S0 [d_v x d_k] (M = 128, rows beyond d_v are zero) times
-//                    the tile's 64 vectors X = [k_0..k_31; q_0..q_31]
-//                    (N = 64, K = d_k).  S0 is the shared prompt state: its
-//                    operand image is read once per CTA and used by every
-//                    beam of the tile (abstract: "reuses the shared state
-//                    across beams").
-//   D2 = KA . X^T    KA = the tile's own keys (rows 0..31) followed by the
-//                    distinct ancestor keys of the tile's beams (rows 32..),
-//                    so D2 holds every dot product k_j . x the projection
-//                    replay needs plus k_b . q_b.
+//   D1  = S0 . X^T      S0 k_b and S0 q_b for the tile's 64 vectors
+//                       X = [k_0..k_31; q_0..q_31].  The S0 operand image is
+//                       read once per CTA and used by every beam of the tile
+//                       (abstract: "reuses the shared state across beams");
+//                       fp32 S0 is split once, when the prompt state is
+//                       installed, into two or three bf16 terms.
+//   Dkq = X . K^T       gives k_b . q_b.
+//   D2  = X . KA^T      k_a . x for every vector x and every distinct
+//                       ancestor a of the tile (KA: their keys).
+//   D1 += Delta'^T . C  the projection replay (review, Summary: records
+//                       replayed "in vector form without ever materializing a
+//                       per-beam matrix").  With P(a) the product of the
+//                       gates on the path from the root to record a (kept in
+//                       the record store), the weight of record a in the
+//                       replay of a beam whose parent is p is P(p) / P(a), so
+//                         S_{t-1} x = P(p) [ S0 x + sum_a (delta_a / P(a)) (k_a . x) ]
+//                       over the beam's ancestors a.  Delta' holds
+//                       delta_a / P(a); C[x][a] is k_a . x where a is an
+//                       ancestor of x's beam and 0 elsewhere.  Delta' and C
+//                       are split into fp16 hi + lo terms; the passes hi.hi,
+//                       hi.lo and lo.hi keep fp32-level accuracy.
 //
-// fp32 S0 is split once (when the prompt state is installed) into two or
-// three bf16 terms S0 = hi + mid (+ lo); each term is one more pass of D1
-// (bf16 x bf16 products are exact in the fp32 accumulator).
+// The epilogue (TMEM lane i = output element i) forms u_x = P(p) D1_x,
+// delta_b = beta_b (v_b - alpha_b u_k), o_b = alpha_b u_q + delta_b (k_b . q_b),
+// and appends the record (alpha_b, delta_b, k_b) with P(b) = P(p) alpha_b.
 //
-// The epilogue (TMEM lane i = row i of S0, i.e. output element i) forms
-//   u_x = G (S0 x) + sum_j w_j (k_j . x) delta_j          x in {k_b, q_b}
-//   delta_b = beta_b (v_b - alpha_b u_k),  o_b = alpha_b u_q + delta_b (k_b . q_b)
-// reading each ancestor delta_j row with coalesced loads, and appends the
-// record (alpha_b, delta_b, k_b) (review, Summary: records replayed "in
-// vector form without ever materializing a per-beam matrix").
-//
-// The ancestry update (abstract: "lightweight ancestry index ... without
-// moving or copying existing records") runs in warp 0: a beam's row is its
-// parent's row plus the parent; parents are range-checked, and distinct
-// ancestors are found with a warp-wide match so each ancestor key is staged
-// once per CTA.
+// Before griddepcontrol.wait the kernel touches inputs only (S0 image, q, k,
+// v, g, beta, parents): it stages X, runs D1 and Dkq and finds the tile's
+// distinct parents.  After the wait it reads, in one round, the parents'
+// ancestor rows (the parent's row plus the parent form the beam's row;
+// abstract: "lightweight ancestry index ... without moving or copying
+// existing records") and the parents' records, then, in a second round, the
+// deeper ancestors' records.  Distinct ancestors are found with warp-wide
+// matches and staged once per CTA.  Every global write happens after the
+// wait, so a step never overwrites records that the step before it may still
+// be reading.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "internal.h"
 #include "sm100_ptx.h"
@@ -41,37 +53,53 @@
 namespace onela {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kBT = 32;            // beams per CTA
-constexpr int kN = 2 * kBT;        // MMA N: k vectors then q vectors
-constexpr int kM = 128;            // MMA M
-constexpr int kTmemCols = 128;     // D1: columns [0, 64), D2: [64, 128)
-constexpr int kTableStride = kN + 1;
-constexpr int kMaxT = 32;          // deepest decode the kernel serves
+constexpr int kThreads = 256;       // 8 warps
+constexpr int kBT = 32;             // beams per CTA
+constexpr int kN = 2 * kBT;         // vectors: k rows 0..31, q rows 32..63
+constexpr int kM = 128;             // MMA M
+constexpr int kBlk = 64;            // distinct ancestors per staging block
+constexpr int kTmemCols = 256;      // D1 [0,64), D2 [64,128), Dkq [128,160)
+constexpr int kMaxT = 16;           // deepest decode the kernel serves
+constexpr int kMaxW = 1 << 20;      // beam index must fit the packed slot entry
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far beyond any legal wait
 constexpr int32_t kErrTimeout = 2;
 
-struct Smem {
-  // byte offsets from the 1024-aligned base
-  uint32_t s0, x, ka, table, book, total;
+struct Layout {
+  uint32_t x;                        // X [NK][64 rows][128 B]
+  uint32_t a;                        // S0 image, then the block operands
+  uint32_t ka, dhi, dlo, chi, clo;   // block operands inside region a
+  uint32_t book;                     // barriers and bookkeeping
+  uint32_t total;
 };
 
-__host__ __device__ inline Smem smem_layout(int nk, int planes, int TM) {
-  Smem s;
-  s.s0 = 0;
-  s.x = s.s0 + (uint32_t)planes * nk * 16384u;
-  s.ka = s.x + (uint32_t)nk * 8192u;
-  s.table = s.ka + (uint32_t)nk * 16384u;
-  s.book = s.table + (uint32_t)kM * kTableStride * 4u;
-  // book: 2 mbarriers + tmem addr (32 B), then per-beam arrays
-  const uint32_t per_beam = (uint32_t)kBT * TM * 4u;
-  s.total = s.book + 64u + 5u * per_beam + 4u * kBT * 4u + (uint32_t)(kBT * TM + kBT) * 4u + 16u;
-  return s;
+__host__ __device__ inline Layout layout(int nk, int planes, int TM) {
+  Layout L;
+  L.x = 0;
+  L.a = (uint32_t)nk * 8192u;
+  L.ka = L.a;                                // [NK][64 rows][128 B]
+  L.dhi = L.ka + (uint32_t)nk * 8192u;       // [2 M-atoms][8 groups][8 rows][128 B]
+  L.dlo = L.dhi + 16384u;
+  L.chi = L.dlo + 16384u;                    // [64 rows][128 B]
+  L.clo = L.chi + 8192u;
+  const uint32_t post_end = L.clo + 8192u;
+  const uint32_t pre_end = L.a + (uint32_t)planes * nk * 16384u;
+  L.book = post_end > pre_end ? post_end : pre_end;
+  // 64 B barriers/counters; 5 per-beam scalars; chain, slot [32][TM];
+  // list [32 * TM]; per-depth counts [TM].
+  L.total = L.book + 64u + 5u * kBT * 4u + 3u * kBT * TM * 4u + TM * 4u + 16u;
+  return L;
+}
+
+__device__ __forceinline__ void split_f16(float x, __half &hi, __half &lo) {
+  hi = __float2half_rn(x);
+  lo = __float2half_rn(x - __half2float(hi));
 }
 
 template <int DK>
-__global__ void __launch_bounds__(kThreads, 1) step_tc_kernel(const StepParams p) {
-  constexpr int NK = DK / 64;  // 128-byte K atoms per row
+__global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const StepParams p) {
+  constexpr int NK = DK / 64;  // 128-byte K atoms per key row
+  constexpr int DV = DK;
+  constexpr int C4 = DV / 4;   // float4 chunks per delta row
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = ptx::smem_u32(smem_raw);
   uint8_t *base = smem_raw + ((1024u - (raw_u32 & 1023u)) & 1023u);
@@ -80,38 +108,38 @@ __global__ void __launch_bounds__(kThreads, 1) step_tc_kernel(const StepParams p
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int b0 = tile * kBT;
   const int nb = min(kBT, p.W - b0);
-  const int dv = p.dv, H = p.H, t = p.t, TM = p.T_max, P = p.s0_planes;
+  const int H = p.H, t = p.t, TM = p.T_max, P = p.s0_planes;
   const int nanc = t - 1;
+  const int jp = nanc - 1;  // depth index of the parents (depth t-1)
 
-  const Smem L = smem_layout(NK, P, TM);
-  uint8_t *s_s0 = base + L.s0;
+  const Layout L = layout(NK, P, TM);
   uint8_t *s_x = base + L.x;
-  uint8_t *s_ka = base + L.ka;
-  float *s_table = reinterpret_cast<float *>(base + L.table);
-  uint64_t *bar_load = reinterpret_cast<uint64_t *>(base + L.book);
-  uint64_t *bar_mma = bar_load + 1;
-  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bar_load + 2);
-  int *s_U = reinterpret_cast<int *>(s_tmem + 1);
-  int *s_chain = reinterpret_cast<int *>(base + L.book + 64);  // [BT][TM]
-  int *s_slot = s_chain + kBT * TM;                            // [BT][TM]
-  float *s_w = reinterpret_cast<float *>(s_slot + kBT * TM);   // [BT][TM]
-  float *s_ck = s_w + kBT * TM;                                // [BT][TM]
-  float *s_cq = s_ck + kBT * TM;                               // [BT][TM]
-  float *s_G = s_cq + kBT * TM;                                // [BT]
-  float *s_alpha = s_G + kBT;
+  uint64_t *bar_s0 = reinterpret_cast<uint64_t *>(base + L.book);
+  uint64_t *bar1 = bar_s0 + 1, *bar2 = bar_s0 + 2, *bar3 = bar_s0 + 3;
+  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bar_s0 + 4);
+  int *s_U1 = reinterpret_cast<int *>(s_tmem + 1);
+  int *s_par = reinterpret_cast<int *>(base + L.book + 64);
+  float *s_alpha = reinterpret_cast<float *>(s_par + kBT);
   float *s_beta = s_alpha + kBT;
-  float *s_kq = s_beta + kBT;
-  int *s_list = reinterpret_cast<int *>(s_kq + kBT);  // packed (beam << 6 | depth-1), by slot
+  float *s_Gp = s_beta + kBT;  // P(parent): the beam's gate product so far
+  float *s_kq = s_Gp + kBT;
+  int *s_chain = reinterpret_cast<int *>(s_kq + kBT);  // [32][TM] ancestor beam by depth
+  int *s_slot = s_chain + kBT * TM;                     // [32][TM] ancestor slot by depth
+  int *s_list = s_slot + kBT * TM;                      // slot -> (beam << 5 | depth-1)
+  int *s_cnt = s_list + kBT * TM;                       // distinct ancestors per depth
 
   const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(p.q);
   const __nv_bfloat16 *k = static_cast<const __nv_bfloat16 *>(p.k);
   const __nv_bfloat16 *v = static_cast<const __nv_bfloat16 *>(p.v);
   __nv_bfloat16 *rec_k = static_cast<__nv_bfloat16 *>(p.rec_k);
+  const int64_t row0 = (int64_t)(r * p.W + b0) * H + h;  // (r, b0, h) row of [R][W][H][d]
 
-  // ---- setup: barriers, TMEM
+  // ------------------------------------------------------------ setup
   if (tid == 0) {
-    ptx::mbar_init(bar_load, 1);
-    ptx::mbar_init(bar_mma, 1);
+    ptx::mbar_init(bar_s0, 1);
+    ptx::mbar_init(bar1, 1);
+    ptx::mbar_init(bar2, 1);
+    ptx::mbar_init(bar3, 1);
     ptx::mbar_fence_init();
   }
   if (warp == 0) {
@@ -122,200 +150,355 @@ __global__ void __launch_bounds__(kThreads, 1) step_tc_kernel(const StepParams p
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *s_tmem;
+  ptx::pdl_launch_dependents();
 
-  // ---- S0 operand image (planes x K atoms x 128 rows x 128 B) by bulk copy
+  // ------------------------------------------- inputs (before the wait)
   const uint32_t s0_bytes = (uint32_t)P * NK * 16384u;
-  if (tid == 0) {
-    ptx::mbar_arrive_expect_tx(bar_load, s0_bytes);
+  if (tid == kThreads - 32) {
+    ptx::mbar_arrive_expect_tx(bar_s0, s0_bytes);
     const uint8_t *src = static_cast<const uint8_t *>(p.S0img) + (size_t)(r * H + h) * s0_bytes;
-    for (uint32_t off = 0; off < s0_bytes; off += 16384u) ptx::bulk_g2s(s_s0 + off, src + off, 16384u, bar_load);
+    for (uint32_t off = 0; off < s0_bytes; off += 16384u)
+      ptx::bulk_g2s(base + L.a + off, src + off, 16384u, bar_s0);
   }
-
-  // ---- X tile (k rows 0..31, q rows 32..63), record k, own keys into KA
   for (int e = tid; e < kN * NK * 8; e += kThreads) {
     const int n = e / (NK * 8), cc = e - n * (NK * 8);
-    const int ka = cc >> 3, c = cc & 7;
     const int bb = n & (kBT - 1);
-    const bool is_q = n >= kBT;
-    uint4 val = make_uint4(0u, 0u, 0u, 0u);
-    if (bb < nb) {
-      const int64_t row = (int64_t)(r * p.W + b0 + bb) * H + h;
-      const uint4 *src = reinterpret_cast<const uint4 *>((is_q ? q : k) + row * DK) + cc;
-      val = __ldg(src);
-      if (!is_q) reinterpret_cast<uint4 *>(rec_k + rec_row(p, t, r, h, b0 + bb) * DK)[cc] = val;
-    }
-    *reinterpret_cast<uint4 *>(s_x + ka * (kN * 128) + ptx::swz128(n, c)) = val;
-    if (!is_q) *reinterpret_cast<uint4 *>(s_ka + ka * (kM * 128) + ptx::swz128(bb, c)) = val;
+    const bool valid = bb < nb;
+    const __nv_bfloat16 *src = (n >= kBT ? q : k) + (row0 + (int64_t)(valid ? bb : 0) * H) * DK + cc * 8;
+    ptx::cp_async16(s_x + (cc >> 3) * (kN * 128) + ptx::swz128(n, cc & 7), src, valid ? 16u : 0u);
   }
-
-  // ---- ancestry, gates, distinct ancestors (warp 0, one lane per beam)
-  if (warp == 0) {
+  ptx::cp_async_commit();
+  if (warp == 1) {
     const int b = lane;
-    const bool valid = b < nb;
-    float G = 1.f, alpha = 0.f, beta = 0.f;
-    int *chain = s_chain + b * TM;
-    if (valid) {
-      const int gb = b0 + b;
-      int par = p.parents[r * p.W + gb];
+    int par = -1;
+    float alpha = 0.f, beta = 0.f;
+    if (b < nb) {
+      par = nanc >= 1 ? p.parents[r * p.W + b0 + b] : 0;
       if (par < 0 || par >= p.W_prev) {
         *reinterpret_cast<volatile int32_t *>(p.err) = kErrParent;
         par = 0;
       }
-      if (nanc >= 1) {
-        chain[nanc - 1] = par;
-        if (nanc >= 2) {
-          const int32_t *prow = p.anc + anc_row(p, t - 1, r, par);
-          for (int j = 0; j < nanc - 1; ++j) chain[j] = prow[j];
-        }
-        if (h == 0) {
-          int32_t *row = p.anc + anc_row(p, t, r, gb);
-          for (int j = 0; j < nanc; ++j) row[j] = chain[j];
-        }
-      }
-      float run = 1.f;
-      for (int j = nanc - 1; j >= 0; --j) {
-        s_w[b * TM + j] = run;
-        run *= p.rec_alpha[rec_row(p, j + 1, r, h, chain[j])];
-      }
-      G = run;
-      const int64_t si = (int64_t)(r * p.W + gb) * H + h;
+      const int64_t si = row0 + (int64_t)b * H;
       alpha = expf(p.g[si]);
       beta = p.beta[si];
-      p.rec_alpha[rec_row(p, t, r, h, gb)] = alpha;
     }
-    s_G[b] = G;
+    s_par[b] = par;
     s_alpha[b] = alpha;
     s_beta[b] = beta;
-    // Distinct (depth, beam) ancestors; slots 0..31 are the tile's own keys.
-    int U = kBT;
-    for (int j = 0; j < nanc; ++j) {
-      const int a = valid ? chain[j] : -1;
-      const unsigned same = __match_any_sync(0xffffffffu, a);
+    // Distinct parents (the depth-(t-1) ancestors) take slots 0..U1-1.
+    if (nanc >= 1) {
+      const unsigned same = __match_any_sync(0xffffffffu, par);
       const int leader = __ffs(same) - 1;
-      const bool lead = valid && leader == lane;
+      const bool lead = b < nb && leader == lane;
       const unsigned leaders = __ballot_sync(0xffffffffu, lead);
-      const int my = U + __popc(leaders & ((1u << lane) - 1u));
-      if (lead) s_list[my] = (a << 6) | j;
+      const int my = __popc(leaders & ((1u << lane) - 1u));
+      if (lead) s_list[my] = (par << 5) | jp;
       const int slot = __shfl_sync(0xffffffffu, my, leader);
-      if (valid) s_slot[b * TM + j] = slot;
-      U += __popc(leaders);
+      if (b < nb) {
+        s_slot[b * TM + jp] = slot;
+        s_chain[b * TM + jp] = par;
+      }
+      if (lane == 0) *s_U1 = __popc(leaders);
+    } else if (lane == 0) {
+      *s_U1 = 0;
     }
-    if (lane == 0) *s_U = U;
+  }
+  // Epilogue mapping: warp w serves TMEM lanes 32*(w%4).. (output elements)
+  // and beams 16*(w/4)..+15; v is loaded now, used at the end.
+  const int ei = (warp & 3) * 32 + lane;
+  const int half = warp >> 2;
+  __nv_bfloat16 vreg[16];
+#pragma unroll
+  for (int m = 0; m < 16; ++m) {
+    const int b = half * 16 + m;
+    vreg[m] = (b < nb && ei < DV) ? v[(row0 + (int64_t)b * H) * DV + ei] : __float2bfloat16(0.f);
+  }
+  ptx::cp_async_wait_all();
+  ptx::fence_proxy_async_smem();
+  __syncthreads();
+
+  bool ok = true;
+  const uint32_t x_u32 = ptx::smem_u32(s_x), a_u32 = ptx::smem_u32(base + L.a);
+  const uint32_t ka_u32 = ptx::smem_u32(base + L.ka);
+  const uint32_t dhi_u32 = ptx::smem_u32(base + L.dhi), dlo_u32 = ptx::smem_u32(base + L.dlo);
+  const uint32_t chi_u32 = ptx::smem_u32(base + L.chi), clo_u32 = ptx::smem_u32(base + L.clo);
+  if (tid == 0) {
+    ok = ptx::mbar_wait(bar_s0, 0, kWaitLimitNs);
+    ptx::tc_fence_after();
+    constexpr uint32_t idesc1 = ptx::idesc_bf16_f32(kM, kN);
+    int acc = 0;
+    for (int pl = 0; pl < P; ++pl)
+#pragma unroll
+      for (int ka = 0; ka < NK; ++ka)
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t ad = ptx::desc_k128(a_u32 + (pl * NK + ka) * 16384 + kk * 32);
+          const uint64_t bd = ptx::desc_k128(x_u32 + ka * (kN * 128) + kk * 32);
+          ptx::mma_bf16(tmem, ad, bd, idesc1, acc);
+          acc = 1;
+        }
+    // Dkq = X . K^T (M = 128 rows from X: rows past 63 are not used).
+    constexpr uint32_t idesc_kq = ptx::idesc_bf16_f32(kM, kBT);
+#pragma unroll
+    for (int ka = 0; ka < NK; ++ka)
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t ad = ptx::desc_k128(x_u32 + ka * (kN * 128) + kk * 32);
+        const uint64_t bd = ptx::desc_k128(x_u32 + ka * (kN * 128) + kk * 32);
+        ptx::mma_bf16(tmem + 128, ad, bd, idesc_kq, (ka | kk) != 0);
+      }
+    ptx::mma_commit(bar1);
+  }
+  if (warp == 1) {
+    // k_b . q_b = Dkq[32 + b][b]: TMEM lanes 32..63 belong to warp 1.
+    if (!ptx::mbar_wait(bar1, 0, kWaitLimitNs)) ok = false;
+    ptx::tc_fence_after();
+    float d[32];
+    ptx::tmem_ld32(tmem + (32u << 16) + 128, d);
+    ptx::tmem_ld_wait();
+    float kq = 0.f;
+#pragma unroll
+    for (int z = 0; z < 32; ++z)
+      if (z == lane) kq = d[z];
+    s_kq[lane] = kq;
+  }
+
+  // ------------------------------- records of earlier steps (after the wait)
+  ptx::pdl_wait();
+  // Round 1: the parents' ancestor rows and P values (warp 0), this step's
+  // keys into the record store, the parents' records into the operands.
+  if (warp == 0 && lane < nb) {
+    const int b = lane, gb = b0 + lane;
+    const int par = s_par[b];
+    float Gp = 1.f;
+    if (nanc >= 1) {
+      Gp = p.rec_P[rec_row(p, nanc, r, h, par)];
+      int tmp[kMaxT - 1];
+      if (nanc >= 2) {
+        const int32_t *prow = p.anc + anc_row(p, nanc, r, par);
+#pragma unroll
+        for (int j = 0; j < kMaxT - 1; ++j)
+          if (j < nanc - 1) tmp[j] = prow[j];
+#pragma unroll
+        for (int j = 0; j < kMaxT - 1; ++j)
+          if (j < nanc - 1) s_chain[b * TM + j] = tmp[j];
+      }
+      if (h == 0) {
+        int32_t *row = p.anc + anc_row(p, t, r, gb);
+#pragma unroll
+        for (int j = 0; j < kMaxT - 1; ++j)
+          if (j < nanc - 1) row[j] = tmp[j];
+        row[nanc - 1] = par;
+      }
+    }
+    s_Gp[b] = Gp;
+    p.rec_alpha[rec_row(p, t, r, h, gb)] = s_alpha[b];
+    p.rec_P[rec_row(p, t, r, h, gb)] = Gp * s_alpha[b];
+  }
+  for (int e = tid; e < kBT * NK * 8; e += kThreads) {
+    const int n = e / (NK * 8), cc = e - n * (NK * 8);
+    if (n < nb)
+      reinterpret_cast<uint4 *>(rec_k + rec_row(p, t, r, h, b0 + n) * DK)[cc] =
+          *reinterpret_cast<const uint4 *>(s_x + (cc >> 3) * (kN * 128) + ptx::swz128(n, cc & 7));
+  }
+  // Region A holds the S0 image until D1 is complete.
+  if (!ptx::mbar_wait(bar1, 0, kWaitLimitNs)) ok = false;
+
+  // Stage slots [lo, hi) of block blk: keys (cp.async) into KA; deltas / P(a)
+  // as fp16 hi + lo into the MN-major Delta' operand.
+  auto stage = [&](int blk, int lo, int hi) {
+    for (int e = tid; e < (hi - lo) * NK * 8; e += kThreads) {
+      const int s = lo + e / (NK * 8), cc = e % (NK * 8);
+      const int packed = s_list[s];
+      const int lr = s - blk * kBlk;
+      ptx::cp_async16(base + L.ka + (cc >> 3) * (kBlk * 128) + ptx::swz128(lr, cc & 7),
+                      rec_k + rec_row(p, (packed & 31) + 1, r, h, packed >> 5) * DK + cc * 8, 16u);
+    }
+    ptx::cp_async_commit();
+    for (int e0 = tid; e0 < (hi - lo) * C4; e0 += 4 * kThreads) {
+      float4 val[4];
+      float pa[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = e0 + u * kThreads;
+        val[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        pa[u] = 1.f;
+        if (e < (hi - lo) * C4) {
+          const int packed = s_list[lo + e / C4];
+          const int64_t rr = rec_row(p, (packed & 31) + 1, r, h, packed >> 5);
+          val[u] = __ldcg(reinterpret_cast<const float4 *>(p.rec_delta + rr * DV) + e % C4);
+          pa[u] = __ldcg(p.rec_P + rr);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = e0 + u * kThreads;
+        if (e < (hi - lo) * C4) {
+          const int lr = lo + e / C4 - blk * kBlk;
+          const int i0 = (e % C4) * 4;
+          const uint32_t off = (uint32_t)(i0 >> 6) * 8192u + (uint32_t)(lr >> 3) * 1024u +
+                               (uint32_t)(lr & 7) * 128u + (uint32_t)((((i0 & 63) >> 3) ^ (lr & 7)) << 4) +
+                               (uint32_t)(i0 & 7) * 2u;
+          const float inv = 1.f / pa[u];
+          const float f[4] = {val[u].x * inv, val[u].y * inv, val[u].z * inv, val[u].w * inv};
+          __align__(8) __half hi4[4], lo4[4];
+#pragma unroll
+          for (int z = 0; z < 4; ++z) split_f16(f[z], hi4[z], lo4[z]);
+          *reinterpret_cast<uint2 *>(base + L.dhi + off) = *reinterpret_cast<const uint2 *>(hi4);
+          *reinterpret_cast<uint2 *>(base + L.dlo + off) = *reinterpret_cast<const uint2 *>(lo4);
+        }
+      }
+    }
+  };
+  const int U1 = *s_U1;
+  if (U1 > 0) stage(0, 0, U1);
+  __syncthreads();  // ancestor rows in s_chain
+
+  // Deeper ancestors: one warp per depth finds the distinct ones, then the
+  // slots U1.. are handed out depth by depth.
+  for (int j = warp; j < nanc - 1; j += kThreads / 32) {
+    const int a = lane < nb ? s_chain[lane * TM + j] : -1;
+    const unsigned same = __match_any_sync(0xffffffffu, a);
+    const int leader = __ffs(same) - 1;
+    const bool lead = lane < nb && leader == lane;
+    const unsigned leaders = __ballot_sync(0xffffffffu, lead);
+    const int my = __popc(leaders & ((1u << lane) - 1u));
+    const int rank = __shfl_sync(0xffffffffu, my, leader);
+    if (lane < nb) s_slot[lane * TM + j] = rank;
+    if (lane == 0) s_cnt[j] = __popc(leaders);
   }
   __syncthreads();
-  const int U = *s_U;
-
-  // ---- blocks of up to 128 KA rows: stage ancestor keys, run the MMAs
-  const uint32_t idesc = ptx::idesc_bf16_f32(kM, kN);
-  const uint32_t x_u32 = ptx::smem_u32(s_x), ka_u32 = ptx::smem_u32(s_ka), s0_u32 = ptx::smem_u32(s_s0);
-  bool ok = true;
-  const int nblocks = (U + kM - 1) / kM;
-  for (int blk = 0; blk < nblocks; ++blk) {
-    const int row0 = blk == 0 ? kBT : 0;
-    const int nrows = min(kM, U - blk * kM);
-    if (blk > 0) __syncthreads();  // previous block's table fully consumed
-    for (int e = tid; e < (nrows - row0) * NK * 8; e += kThreads) {
-      const int lr = row0 + e / (NK * 8), cc = e % (NK * 8);
-      const int packed = s_list[blk * kM + lr];
-      const int beam = packed >> 6, depth = (packed & 63) + 1;
-      const uint4 val =
-          __ldg(reinterpret_cast<const uint4 *>(rec_k + rec_row(p, depth, r, h, beam) * DK) + cc);
-      *reinterpret_cast<uint4 *>(s_ka + (cc >> 3) * (kM * 128) + ptx::swz128(lr, cc & 7)) = val;
+  int U = U1;
+  for (int j = 0; j < nanc - 1; ++j) U += s_cnt[j];
+  if (warp == 0 && lane < nb) {
+    int run = U1;
+    for (int j = 0; j < nanc - 1; ++j) {
+      const int slot = run + s_slot[lane * TM + j];
+      s_slot[lane * TM + j] = slot;
+      s_list[slot] = (s_chain[lane * TM + j] << 5) | j;
+      run += s_cnt[j];
     }
+  }
+  __syncthreads();
+  const int nblk = (U + kBlk - 1) / kBlk;
+
+  for (int blk = 0; blk < nblk; ++blk) {
+    const int lo = blk * kBlk, hi = min(U, lo + kBlk);
+    const int nrows = hi - lo;
+    const int kpad = (nrows + 15) & ~15;  // slots the MMAs read (multiple of 16)
+    if (blk > 0) {
+      if (!ptx::mbar_wait(bar3, (blk - 1) & 1, kWaitLimitNs)) ok = false;
+      stage(blk, lo, hi);
+    } else if (hi > U1) {
+      stage(0, U1, hi);
+    }
+    // Slots past the block's last ancestor but inside the MMA K range hold
+    // zero deltas.
+    for (int e = tid; e < (kpad - nrows) * 2 * 8; e += kThreads) {
+      const int lr = nrows + e / 16, rem = e % 16, ma = rem >> 3, c = rem & 7;
+      const uint32_t off = (uint32_t)ma * 8192u + (uint32_t)(lr >> 3) * 1024u + ptx::swz128(lr & 7, c);
+      *reinterpret_cast<uint4 *>(base + L.dhi + off) = make_uint4(0u, 0u, 0u, 0u);
+      *reinterpret_cast<uint4 *>(base + L.dlo + off) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    ptx::cp_async_wait_all();
     ptx::fence_proxy_async_smem();
     __syncthreads();
     if (tid == 0) {
       ptx::tc_fence_after();
-      if (blk == 0) {
-        ok = ptx::mbar_wait(bar_load, 0, kWaitLimitNs);
-        ptx::tc_fence_after();
-        int acc = 0;
-        for (int pl = 0; pl < P; ++pl)
-          for (int ka = 0; ka < NK; ++ka)
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t a = ptx::desc_k128(s0_u32 + (pl * NK + ka) * 16384 + kk * 32);
-              const uint64_t bd = ptx::desc_k128(x_u32 + ka * (kN * 128) + kk * 32);
-              ptx::mma_bf16(tmem, a, bd, idesc, acc);
-              acc = 1;
-            }
-      }
+      const uint32_t idesc2 = ptx::idesc_bf16_f32(kM, kpad);
+#pragma unroll
       for (int ka = 0; ka < NK; ++ka)
+#pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t a = ptx::desc_k128(ka_u32 + ka * (kM * 128) + kk * 32);
-          const uint64_t bd = ptx::desc_k128(x_u32 + ka * (kN * 128) + kk * 32);
-          ptx::mma_bf16(tmem + kN, a, bd, idesc, (ka | kk) != 0);
+          const uint64_t ad = ptx::desc_k128(x_u32 + ka * (kN * 128) + kk * 32);
+          const uint64_t bd = ptx::desc_k128(ka_u32 + ka * (kBlk * 128) + kk * 32);
+          ptx::mma_bf16(tmem + 64, ad, bd, idesc2, (ka | kk) != 0);
         }
-      ptx::mma_commit(bar_mma);
+      ptx::mma_commit(bar2);
     }
-    // Everyone waits for this block's MMAs.
-    if (!ptx::mbar_wait(bar_mma, blk & 1, kWaitLimitNs)) ok = false;
+    // C build: TMEM lanes 0..63 (vector n) belong to warps 0, 1, 4, 5; each
+    // takes a 16-slot column group.  C[n][a] = D2[n][a] where a is an
+    // ancestor of n's beam, else 0, stored as fp16 hi + lo, K-major.
+    const bool c_warp = (warp & 2) == 0;  // warps 0,1,4,5: column groups 0,2 / 1,3
+    if (!ptx::mbar_wait(bar2, blk & 1, kWaitLimitNs)) ok = false;
     ptx::tc_fence_after();
-    // D2 rows -> table (warps 0..3: TMEM lanes 0..127 = KA rows).
-    if (warp < 4) {
-      const int lr = warp * 32 + lane;
-#pragma unroll
-      for (int c0 = 0; c0 < kN; c0 += 16) {
-        float vals[16];
-        ptx::tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + kN + c0, vals);
-        ptx::tmem_ld_wait();
-        if (lr < nrows) {
-#pragma unroll
-          for (int c = 0; c < 16; ++c) s_table[lr * kTableStride + c0 + c] = vals[c];
+    for (int g = (warp >> 2); c_warp && g * 16 < kpad; g += 2) {
+      const int n = (warp & 1) * 32 + lane;
+      const int b = n & (kBT - 1);
+      float d[16];
+      ptx::tmem_ld16(tmem + ((uint32_t)((warp & 1) * 32) << 16) + 64 + g * 16, d);
+      ptx::tmem_ld_wait();
+      uint32_t mask = 0u;
+      if (b < nb)
+        for (int j = 0; j < nanc; ++j) {
+          const int s = s_slot[b * TM + j] - lo - g * 16;
+          if (s >= 0 && s < 16) mask |= 1u << s;
         }
+      __align__(16) __half h16[16], l16[16];
+#pragma unroll
+      for (int z = 0; z < 16; ++z) split_f16(((mask >> z) & 1u) ? d[z] : 0.f, h16[z], l16[z]);
+#pragma unroll
+      for (int c2 = 0; c2 < 2; ++c2) {
+        const uint32_t off = ptx::swz128(n, g * 2 + c2);
+        *reinterpret_cast<uint4 *>(base + L.chi + off) = reinterpret_cast<const uint4 *>(h16)[c2];
+        *reinterpret_cast<uint4 *>(base + L.clo + off) = reinterpret_cast<const uint4 *>(l16)[c2];
       }
     }
+    ptx::fence_proxy_async_smem();
     ptx::tc_fence_before();
     __syncthreads();
-    // Coefficients of the slots that fall in this block.
-    if (warp == 0 && lane < nb) {
-      const int b = lane;
-      if (blk == 0) s_kq[b] = s_table[b * kTableStride + kBT + b];
-      for (int j = 0; j < nanc; ++j) {
-        const int s = s_slot[b * TM + j] - blk * kM;
-        if (s >= 0 && s < kM) {
-          const float w = s_w[b * TM + j];
-          s_ck[b * TM + j] = w * s_table[s * kTableStride + b];
-          s_cq[b * TM + j] = w * s_table[s * kTableStride + kBT + b];
-        }
-      }
-    }
-  }
-  if (!ok && tid == 0) *reinterpret_cast<volatile int32_t *>(p.err) = kErrTimeout;
-  __syncthreads();
-
-  // ---- epilogue: warp w serves TMEM lanes 32*(w%4).. and beams 16*(w/4)..
-  {
-    const int i = (warp & 3) * 32 + lane;  // output element (row of S0)
-    const int half = warp >> 2;
-    float uk[16], uq[16];
-    ptx::tc_fence_after();
-    ptx::tmem_ld16(tmem + ((uint32_t)((warp & 3) * 32) << 16) + half * 16, uk);
-    ptx::tmem_ld16(tmem + ((uint32_t)((warp & 3) * 32) << 16) + kBT + half * 16, uq);
-    ptx::tmem_ld_wait();
-    if (i < dv && ok) {
+    if (tid == 0) {
+      ptx::tc_fence_after();
+      constexpr uint32_t idesc3 = ptx::idesc_f16_amn_f32(kM, kN);
+      const uint32_t dA[3] = {dhi_u32, dhi_u32, dlo_u32};
+      const uint32_t cB[3] = {chi_u32, clo_u32, chi_u32};
 #pragma unroll
-      for (int m = 0; m < 16; ++m) {
-        const int b = half * 16 + m;
-        if (b >= nb) continue;
-        const int gb = b0 + b;
-        float xk = s_G[b] * uk[m];
-        float xq = s_G[b] * uq[m];
-        for (int j = 0; j < nanc; ++j) {
-          const int a = s_chain[b * TM + j];
-          const float d = __ldg(p.rec_delta + rec_row(p, j + 1, r, h, a) * dv + i);
-          xk = fmaf(s_ck[b * TM + j], d, xk);
-          xq = fmaf(s_cq[b * TM + j], d, xq);
+      for (int term = 0; term < 3; ++term)
+        for (int ks = 0; ks < kpad / 16; ++ks) {
+          const uint64_t ad = ptx::desc_mn128(dA[term] + ks * 2048, 8192u, 1024u);
+          const uint64_t bd = ptx::desc_k128(cB[term] + ks * 32);
+          ptx::mma_bf16(tmem, ad, bd, idesc3, 1u);
         }
-        const int64_t vi = ((int64_t)(r * p.W + gb) * H + h) * dv + i;
-        const float alpha = s_alpha[b];
-        const float delta = s_beta[b] * (__bfloat162float(v[vi]) - alpha * xk);
-        p.o[vi] = fmaf(alpha, xq, delta * s_kq[b]);
-        p.rec_delta[rec_row(p, t, r, h, gb) * dv + i] = delta;
+      ptx::mma_commit(bar3);
+    }
+  }
+
+  // --------------------------------------------------------- epilogue
+  if (nblk > 0 && !ptx::mbar_wait(bar3, (nblk - 1) & 1, kWaitLimitNs)) ok = false;
+  if (!ok) *reinterpret_cast<volatile int32_t *>(p.err) = kErrTimeout;
+  ptx::tc_fence_after();
+  {
+    const uint32_t lb = (uint32_t)((warp & 3) * 32) << 16;
+    float uk[16], uq[16];
+    ptx::tmem_ld16(tmem + lb + half * 16, uk);
+    ptx::tmem_ld16(tmem + lb + kBT + half * 16, uq);
+    ptx::tmem_ld_wait();
+    if (ei < DV && ok) {
+      const float4 *G4 = reinterpret_cast<const float4 *>(s_Gp + half * 16);
+      const float4 *A4 = reinterpret_cast<const float4 *>(s_alpha + half * 16);
+      const float4 *B4 = reinterpret_cast<const float4 *>(s_beta + half * 16);
+      const float4 *K4 = reinterpret_cast<const float4 *>(s_kq + half * 16);
+#pragma unroll
+      for (int m4 = 0; m4 < 4; ++m4) {
+        const float4 G = G4[m4], A = A4[m4], B = B4[m4], KQ = K4[m4];
+        const float Gv[4] = {G.x, G.y, G.z, G.w}, Av[4] = {A.x, A.y, A.z, A.w};
+        const float Bv[4] = {B.x, B.y, B.z, B.w}, Kv[4] = {KQ.x, KQ.y, KQ.z, KQ.w};
+#pragma unroll
+        for (int z = 0; z < 4; ++z) {
+          const int m = m4 * 4 + z;
+          const int b = half * 16 + m;
+          if (b < nb) {
+            const float ag = Av[z] * Gv[z];  // alpha P(p)
+            const float delta = Bv[z] * fmaf(-ag, uk[m], __bfloat162float(vreg[m]));
+            p.o[(row0 + (int64_t)b * H) * DV + ei] = fmaf(ag, uq[m], delta * Kv[z]);
+            p.rec_delta[rec_row(p, t, r, h, b0 + b) * DV + ei] = delta;
+          }
+        }
       }
     }
   }
 
-  // ---- teardown
+  // --------------------------------------------------------- teardown
   ptx::tc_fence_before();
   __syncthreads();
   if (warp == 0) ptx::tmem_dealloc(tmem, kTmemCols);
@@ -358,29 +541,9 @@ __global__ void s0_image_kernel(const void *S0, uint4 *img, int R, int H, int dk
   }
 }
 
-}  // namespace
-
-bool tc_supports(int dk, int dv, int qkv_bf16, int T_max) {
-  return qkv_bf16 && dk == dv && (dk == 64 || dk == 128) && T_max <= kMaxT;
-}
-
-size_t s0_image_bytes(int R, int H, int dk, int dv, int planes) {
-  (void)dv;
-  return (size_t)R * H * planes * (dk / 64) * 16384u;
-}
-
-cudaError_t launch_s0_image(const void *S0, void *img, int R, int H, int dk, int dv, int s0_bf16, int planes,
-                            cudaStream_t s) {
-  const int64_t total = (int64_t)R * H * planes * (dk / 64) * kM * 8;
-  const int threads = 256;
-  const int blocks = (int)((total + threads - 1) / threads < 148 * 16 ? (total + threads - 1) / threads : 148 * 16);
-  s0_image_kernel<<<blocks, threads, 0, s>>>(S0, static_cast<uint4 *>(img), R, H, dk, dv, s0_bf16, planes);
-  return cudaGetLastError();
-}
-
 template <int DK>
-static cudaError_t launch_dk(const StepParams &p, cudaStream_t s) {
-  const Smem L = smem_layout(DK / 64, p.s0_planes, p.T_max);
+cudaError_t launch_dk(const StepParams &p, bool pdl, cudaStream_t s) {
+  const Layout L = layout(DK / 64, p.s0_planes, p.T_max);
   const size_t smem = L.total + 1024;
   static size_t configured[64] = {0};
   int dev = 0;
@@ -392,16 +555,45 @@ static cudaError_t launch_dk(const StepParams &p, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     configured[dev] = smem;
   }
-  dim3 grid((p.W + kBT - 1) / kBT, p.H, p.R);
-  step_tc_kernel<DK><<<grid, kThreads, smem, s>>>(p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((p.W + kBT - 1) / kBT, p.H, p.R);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, step_tc_kernel<DK>, p);
+}
+
+}  // namespace
+
+bool tc_supports(int dk, int dv, int qkv_bf16, int T_max, int W_max) {
+  return qkv_bf16 && dk == dv && (dk == 64 || dk == 128) && T_max <= kMaxT && W_max <= kMaxW;
+}
+
+size_t s0_image_bytes(int R, int H, int dk, int dv, int planes) {
+  (void)dv;
+  return (size_t)R * H * planes * (dk / 64) * 16384u;
+}
+
+cudaError_t launch_s0_image(const void *S0, void *img, int R, int H, int dk, int dv, int s0_bf16, int planes,
+                            cudaStream_t s) {
+  const int64_t total = (int64_t)R * H * planes * (dk / 64) * kM * 8;
+  const int threads = 256;
+  const int64_t want = (total + threads - 1) / threads;
+  const int blocks = (int)(want < 148 * 16 ? want : 148 * 16);
+  s0_image_kernel<<<blocks, threads, 0, s>>>(S0, static_cast<uint4 *>(img), R, H, dk, dv, s0_bf16, planes);
   return cudaGetLastError();
 }
 
-cudaError_t launch_step_tc(const StepParams &p, int s0_bf16, cudaStream_t s) {
-  (void)s0_bf16;
-  if (p.T_max > kMaxT || p.s0_planes < 1 || p.s0_planes > 3) return cudaErrorNotSupported;
-  if (p.dk == 64 && p.dv == 64) return launch_dk<64>(p, s);
-  if (p.dk == 128 && p.dv == 128) return launch_dk<128>(p, s);
+cudaError_t launch_step_tc(const StepParams &p, int pdl, cudaStream_t s) {
+  if (p.T_max > kMaxT || p.W_max > kMaxW || p.s0_planes < 1 || p.s0_planes > 3 || !p.rec_P)
+    return cudaErrorNotSupported;
+  if (p.dk == 64 && p.dv == 64) return launch_dk<64>(p, pdl != 0, s);
+  if (p.dk == 128 && p.dv == 128) return launch_dk<128>(p, pdl != 0, s);
   return cudaErrorNotSupported;
 }
 

@@ -44,17 +44,17 @@ def to_dev(steps, device="cuda"):
 
 def run_gpu(S0: torch.Tensor, steps: List[Dict], qkv_dtype: str, kernel: int,
             T_max: Optional[int] = None, W_max: Optional[int] = None, read_back=True,
-            s0_split: int = 0):
+            s0_split: int = 0, flags: int = 0):
     import linear_attention_beam_shared_b200 as L
     R, H, dv, dk = S0.shape
     s0_dtype = "bf16" if S0.dtype == torch.bfloat16 else "f32"
     T = len(steps)
     W_max = W_max or max(s["W"] for s in steps)
     dec = L.BeamDecoder(R, H, dk, dv, W_max, T_max or T, s0_dtype, qkv_dtype, kernel=kernel,
-                        s0_split=s0_split)
+                        s0_split=s0_split, flags=flags)
     try:
+        dsteps = to_dev(steps)          # every input resident before the first step
         dec.set_prompt_state(S0.cuda())
-        dsteps = to_dev(steps)
         outs = []
         for s in dsteps:
             o = dec.step(s["q"], s["k"], s["v"], s["g"], s["beta"], s["parents"])

@@ -42,16 +42,27 @@ def _skip_unavailable(kernel, dk, dv, qkv):
         pytest.skip("kernel does not serve this shape")
 
 
-def run_workload(name, kernel, s0_dtype=None):
+def run_workload(name, kernel, s0_dtype=None, flags=0, s0_split=0):
     wl = synth.workload(name)
     if s0_dtype:
         wl = wl.replace(s0_dtype=s0_dtype)
     _skip_unavailable(kernel, wl.d_k, wl.d_v, wl.qkv_dtype)
     S0 = P.prompt_state(wl)
     steps = synth.draw_decode(wl)
-    gpu, _ = P.run_gpu(S0, steps, wl.qkv_dtype, kernel)
+    gpu, _ = P.run_gpu(S0, steps, wl.qkv_dtype, kernel, flags=flags, s0_split=s0_split)
     ref = P.oracle(S0, steps)
     return P.compare(gpu, ref, steps, wl.s0_dtype)
+
+
+@pytest.mark.parametrize("name", ["op1k", "long5k", "long5k_bf16"])
+def test_tc_with_programmatic_launch(name):
+    """Steps 2..T start before the previous step ends (inputs resident)."""
+    import linear_attention_beam_shared_b200 as L
+    run_workload(name, 2, flags=L.ONELA_FLAG_PDL)
+
+
+def test_tc_three_term_split():
+    run_workload("long5k", 2, s0_split=3)
 
 
 @pytest.mark.parametrize("kernel", [1, 2])
@@ -140,7 +151,12 @@ def test_identity_gate_keeps_s0(kernel):
 
 
 @pytest.mark.parametrize("kernel", [1, 2])
-def test_linearity_is_bitwise(kernel):
+def test_linearity(kernel):
+    """o and delta are linear in (S0, v).  The SIMT kernel is bitwise linear
+    (scaling by 2 is exact in every fp32 operation).  The tensor-core kernel
+    splits deltas and replay coefficients into fp16 hi + lo terms, and the lo
+    term of a tiny value is an fp16 subnormal whose rounding changes with the
+    scale, so there linearity holds to within fp32 rounding instead."""
     _skip_unavailable(kernel, 128, 128, "bf16")
     wl, S0, steps = P.custom_steps(10, 1, 2, 128, 128, (8, 33, 33, 20))
     S0c = synth.cast_state(S0, "f32")
@@ -148,8 +164,12 @@ def test_linearity_is_bitwise(kernel):
     steps2 = [dict(s, v=(2 * s["v"].float()).to(s["v"].dtype)) for s in steps]
     b, _ = P.run_gpu(2 * S0c, steps2, "bf16", kernel)
     for x, y in zip(a, b):
-        assert torch.equal(2 * x["o"], y["o"])
-        assert torch.equal(2 * x["delta"], y["delta"])
+        if kernel == 1:
+            assert torch.equal(2 * x["o"], y["o"])
+            assert torch.equal(2 * x["delta"], y["delta"])
+        else:
+            assert float((2 * x["o"] - y["o"]).abs().max()) <= 2e-6
+            assert float((2 * x["delta"] - y["delta"]).abs().max()) <= 2e-6
 
 
 @pytest.mark.parametrize("kernel", [1, 2])
@@ -163,15 +183,15 @@ def test_deterministic(kernel):
         assert torch.equal(x["o"], y["o"]) and torch.equal(x["delta"], y["delta"])
 
 
-@pytest.mark.parametrize("kernel", [1, 2])
-def test_graph_replay_matches_eager(kernel):
+@pytest.mark.parametrize("kernel,flags", [(1, 0), (2, 0), (2, 1)])
+def test_graph_replay_matches_eager(kernel, flags):
     import linear_attention_beam_shared_b200 as L
     _skip_unavailable(kernel, 128, 128, "bf16")
     wl, S0, steps = P.custom_steps(12, 1, 4, 128, 128, (32, 96, 96, 96))
     S0c = synth.cast_state(S0, "f32").cuda()
     dsteps = P.to_dev(steps)
     eager, _ = P.run_gpu(S0c.cpu(), steps, "bf16", kernel, read_back=False)
-    dec = L.BeamDecoder(1, 4, 128, 128, 96, 4, "f32", "bf16", kernel=kernel)
+    dec = L.BeamDecoder(1, 4, 128, 128, 96, 4, "f32", "bf16", kernel=kernel, flags=flags)
     try:
         dec.set_prompt_state(S0c)
         outs = [torch.empty((1, s["W"], 4, 128), device="cuda") for s in steps]
