@@ -31,7 +31,8 @@
  *     decode path synchronises the host, so the calls can be captured in a
  *     CUDA graph.
  *   - Inputs are borrowed for the stream-ordered duration of the call; the
- *     library never keeps a pointer to caller memory.  The library owns its
+ *     library keeps no pointer to caller memory beyond it (one exception,
+ *     opt-in: ONELA_FLAG_PDL, below).  The library owns its
  *     copy of S0, the record store and the ancestry index and frees them in
  *     onela_destroy.
  *   - Return value: ONELA_OK or one of the ONELA_ERR_* codes below.  A call
@@ -77,11 +78,14 @@ enum {
 /* onela_config.flags bits.
  *   ONELA_FLAG_PDL  launch decode steps t >= 2 of the tensor-core kernel as
  *                   programmatic dependents of the kernel before them in the
- *                   stream: step t starts loading its inputs and S0 while
- *                   step t-1 finishes, and waits for step t-1 only before it
- *                   touches the records.  Set it only when that earlier
- *                   kernel does not produce any input of step t (q, k, v, g,
- *                   beta, parent_idx) -- e.g. back-to-back decode steps whose
+ *                   stream: step t loads its inputs, S0 and the part of each
+ *                   beam's ancestry that steps up to t-2 produced while step
+ *                   t-1 finishes, and waits for step t-1 only before it
+ *                   touches step t-1's records.  Set it only when (a) that
+ *                   earlier kernel does not produce any input of step t (q,
+ *                   k, v, g, beta, parent_idx), and (b) the parent_idx array
+ *                   of step t-1 stays unchanged and allocated until step t
+ *                   has completed -- e.g. back-to-back decode steps whose
  *                   inputs were all written before the first of them, as in
  *                   a CUDA graph of a whole decode.  Step 1 never overlaps. */
 enum { ONELA_FLAG_PDL = 1 };
@@ -144,7 +148,9 @@ ONELA_API int onela_set_prompt_state(onela_handle *h, const void *S0, onela_stre
  *   g           [R][W][H] fp32, the log of the decay gate: alpha = exp(g).
  *   beta        [R][W][H] fp32, the delta-rule write strength.
  *   parent_idx  [R][W] int32, beam b's parent among the previous step's
- *               beams, in [0, W_prev).  One array serves all heads.
+ *               beams, in [0, W_prev).  One array serves all heads.  With
+ *               ONELA_FLAG_PDL the library reads it again during the next
+ *               step (see the flag).
  *   o           [R][W][H][d_v] fp32, written: o_t = S_t q_t.
  * Also appends the records (alpha_t, delta_t, k_t) of every (beam, head) at
  * depth t and the ancestry rows of depth t; earlier records are never moved.

@@ -16,6 +16,12 @@ struct StepParams {
   const void *q, *k, *v;  // [R][W][H][d] in the qkv type
   const float *g, *beta;  // [R][W][H]
   const int32_t *parents; // [R][W]
+  // Parents of the previous step (step t-1), [R][prev_stride] with W_prev
+  // valid entries per request, and the beam count of step t-2 (W_prev2).
+  // Used by the tensor-core kernel for t >= 3; may be null otherwise.
+  const int32_t *prev_parents;
+  int prev_stride, W_prev2;
+  int32_t *par_store;     // [T_max][R][W_max]: each step's parents (tensor-core kernel)
   float *o;               // [R][W][H][dv]
   const void *S0;         // [R][H][dv][dk] in the S0 type
   const void *S0img;      // tensor-core operand image of S0 (see step_tc.cu)

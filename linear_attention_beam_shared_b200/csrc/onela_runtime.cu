@@ -19,6 +19,8 @@ struct onela_handle {
   std::vector<int> Ws;  // beams of each step done
   void *S0;
   void *S0img;
+  int32_t *par_store;         // each step's parents, written by the kernel
+  const int32_t *last_parents;  // the previous call's parent_idx (caller memory)
   float *rec_alpha;
   float *rec_P;
   float *rec_delta;
@@ -52,6 +54,7 @@ void free_all(onela_handle *h) {
   cudaFree(h->S0img);
   cudaFree(h->rec_alpha);
   cudaFree(h->rec_P);
+  cudaFree(h->par_store);
   cudaFree(h->rec_delta);
   cudaFree(h->rec_k);
   cudaFree(h->anc);
@@ -72,6 +75,7 @@ onela::StepParams base_params(const onela_handle *h) {
   p.s0_planes = h->planes;
   p.rec_alpha = h->rec_alpha;
   p.rec_P = h->rec_P;
+  p.par_store = h->par_store;
   p.rec_delta = h->rec_delta;
   p.rec_k = h->rec_k;
   p.anc = h->anc;
@@ -135,6 +139,8 @@ int onela_create(const onela_config *cfg, onela_handle **out) {
     ok = cudaMalloc(&h->S0img, onela::s0_image_bytes(c.R, c.H, c.d_k, c.d_v, h->planes)) == cudaSuccess;
   ok = ok && cudaMalloc((void **)&h->rec_alpha, nrow * sizeof(float)) == cudaSuccess;
   if (ok && kernel == ONELA_KERNEL_TC) ok = cudaMalloc((void **)&h->rec_P, nrow * sizeof(float)) == cudaSuccess;
+  if (ok && kernel == ONELA_KERNEL_TC)
+    ok = cudaMalloc((void **)&h->par_store, (size_t)c.T_max * c.R * c.W_max * sizeof(int32_t)) == cudaSuccess;
   ok = ok && cudaMalloc((void **)&h->rec_delta, nrow * c.d_v * sizeof(float)) == cudaSuccess;
   ok = ok && cudaMalloc(&h->rec_k, nrow * c.d_k * esize(c.qkv_dtype)) == cudaSuccess;
   ok = ok && cudaMalloc((void **)&h->anc, (size_t)c.T_max * c.R * c.W_max * c.T_max * sizeof(int32_t)) == cudaSuccess;
@@ -203,8 +209,21 @@ int onela_decode_step(onela_handle *h, int32_t W_prev, int32_t W, const void *q,
   p.o = o;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
+  const bool pdl = (c.flags & ONELA_FLAG_PDL) && p.t >= 2;
+  if (p.t >= 3) {
+    p.W_prev2 = h->Ws[p.t - 3];
+    if (pdl) {
+      // The previous call's parents, still valid by the ONELA_FLAG_PDL contract.
+      p.prev_parents = h->last_parents;
+      p.prev_stride = W_prev;
+    } else {
+      // The copy the previous step's kernel wrote (it has completed).
+      p.prev_parents = h->par_store + (size_t)(p.t - 2) * c.R * c.W_max;
+      p.prev_stride = c.W_max;
+    }
+  }
   if (h->kernel == ONELA_KERNEL_TC)
-    e = onela::launch_step_tc(p, (c.flags & ONELA_FLAG_PDL) && p.t >= 2, s);
+    e = onela::launch_step_tc(p, pdl, s);
   else
     e = onela::launch_step_simt(p, c.qkv_dtype == ONELA_BF16, c.s0_dtype == ONELA_BF16, s);
   if (e != cudaSuccess) {
@@ -213,6 +232,7 @@ int onela_decode_step(onela_handle *h, int32_t W_prev, int32_t W, const void *q,
   }
   h->steps_done += 1;
   h->Ws.push_back(W);
+  h->last_parents = parent_idx;
   return ONELA_OK;
 }
 

@@ -34,16 +34,19 @@
 // delta_b = beta_b (v_b - alpha_b u_k), o_b = alpha_b u_q + delta_b (k_b . q_b),
 // and appends the record (alpha_b, delta_b, k_b) with P(b) = P(p) alpha_b.
 //
-// Before griddepcontrol.wait the kernel touches inputs only (S0 image, q, k,
-// v, g, beta, parents): it stages X, runs D1 and Dkq and finds the tile's
-// distinct parents.  After the wait it reads, in one round, the parents'
-// ancestor rows (the parent's row plus the parent form the beam's row;
-// abstract: "lightweight ancestry index ... without moving or copying
-// existing records") and the parents' records, then, in a second round, the
-// deeper ancestors' records.  Distinct ancestors are found with warp-wide
-// matches and staged once per CTA.  Every global write happens after the
-// wait, so a step never overwrites records that the step before it may still
-// be reading.
+// The ancestry (abstract: "lightweight ancestry index ... without moving or
+// copying existing records"): beam b with parent p, grandparent g = the
+// parent of p at step t-1, has the ancestor row [row of g at depth t-2, g, p].
+// The kernel signals its dependents only after its own griddepcontrol.wait,
+// so when step t starts, step t-2 has completed: before its wait, step t
+// reads only inputs (S0 image, q, k, v, g, beta, parents of steps t and t-1)
+// and what steps up to t-2 wrote (ancestor rows of depth t-2).  There it
+// stages X, runs D1 and Dkq, forms every beam's ancestor row and finds the
+// tile's distinct ancestors with warp-wide matches (parents first, then one
+// warp per depth).  After the wait one round of loads stages all the distinct
+// ancestors' records (keys, deltas, P) once per CTA.  Every global write
+// happens after the wait, so a step never overwrites records that the step
+// before it may still be reading.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -60,22 +63,26 @@ constexpr int kM = 128;             // MMA M
 constexpr int kBlk = 64;            // distinct ancestors per staging block
 constexpr int kTmemCols = 256;      // D1 [0,64), D2 [64,128), Dkq [128,160)
 constexpr int kMaxT = 16;           // deepest decode the kernel serves
-constexpr int kMaxW = 1 << 20;      // beam index must fit the packed slot entry
+constexpr int kMaxW = 1024;         // widest beam set the kernel serves
+constexpr int kSliceMax = 4096;     // ancestor-row slice copied to shared memory when
+                                    // W_max * T_max fits (ints); otherwise rows are gathered
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far beyond any legal wait
 constexpr int32_t kErrTimeout = 2;
 
 struct Layout {
-  uint32_t x;                        // X [NK][64 rows][128 B]
+  uint32_t x;                        // X [NK][128 rows][128 B]: k, q, k, q
   uint32_t a;                        // S0 image, then the block operands
   uint32_t ka, dhi, dlo, chi, clo;   // block operands inside region a
   uint32_t book;                     // barriers and bookkeeping
   uint32_t total;
 };
 
-__host__ __device__ inline Layout layout(int nk, int planes, int TM) {
+__host__ __device__ inline bool use_slice(int W_max, int TM) { return W_max * TM <= kSliceMax; }
+
+__host__ __device__ inline Layout layout(int nk, int planes, int TM, int W_max) {
   Layout L;
   L.x = 0;
-  L.a = (uint32_t)nk * 8192u;
+  L.a = (uint32_t)nk * 16384u;
   L.ka = L.a;                                // [NK][64 rows][128 B]
   L.dhi = L.ka + (uint32_t)nk * 8192u;       // [2 M-atoms][8 groups][8 rows][128 B]
   L.dlo = L.dhi + 16384u;
@@ -85,8 +92,10 @@ __host__ __device__ inline Layout layout(int nk, int planes, int TM) {
   const uint32_t pre_end = L.a + (uint32_t)planes * nk * 16384u;
   L.book = post_end > pre_end ? post_end : pre_end;
   // 64 B barriers/counters; 5 per-beam scalars; chain, slot [32][TM];
-  // list [32 * TM]; per-depth counts [TM].
-  L.total = L.book + 64u + 5u * kBT * 4u + 3u * kBT * TM * 4u + TM * 4u + 16u;
+  // list [32 * TM]; per-depth counts [TM]; the previous step's parents
+  // [W_max]; the ancestor-row slice of depth t-2 [W_max][TM] if it fits.
+  L.total = L.book + 64u + 5u * kBT * 4u + 3u * kBT * TM * 4u + (uint32_t)(TM + 4) * 4u + (uint32_t)W_max * 4u +
+            (use_slice(W_max, TM) ? (uint32_t)W_max * TM * 4u : 0u) + 16u;
   return L;
 }
 
@@ -100,6 +109,8 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const StepParams p
   constexpr int NK = DK / 64;  // 128-byte K atoms per key row
   constexpr int DV = DK;
   constexpr int C4 = DV / 4;   // float4 chunks per delta row
+  constexpr int XA = 2 * kN * 128;  // bytes of one K atom of X (128 rows)
+  constexpr int NF = kBlk * C4 / kThreads;  // delta float4 chunks per thread per block
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = ptx::smem_u32(smem_raw);
   uint8_t *base = smem_raw + ((1024u - (raw_u32 & 1023u)) & 1023u);
@@ -111,8 +122,9 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const StepParams p
   const int H = p.H, t = p.t, TM = p.T_max, P = p.s0_planes;
   const int nanc = t - 1;
   const int jp = nanc - 1;  // depth index of the parents (depth t-1)
+  const bool slice = use_slice(p.W_max, TM);
 
-  const Layout L = layout(NK, P, TM);
+  const Layout L = layout(NK, P, TM, p.W_max);
   uint8_t *s_x = base + L.x;
   uint64_t *bar_s0 = reinterpret_cast<uint64_t *>(base + L.book);
   uint64_t *bar1 = bar_s0 + 1, *bar2 = bar_s0 + 2, *bar3 = bar_s0 + 3;
@@ -126,7 +138,9 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const StepParams p
   int *s_chain = reinterpret_cast<int *>(s_kq + kBT);  // [32][TM] ancestor beam by depth
   int *s_slot = s_chain + kBT * TM;                     // [32][TM] ancestor slot by depth
   int *s_list = s_slot + kBT * TM;                      // slot -> (beam << 5 | depth-1)
-  int *s_cnt = s_list + kBT * TM;                       // distinct ancestors per depth
+  int *s_cnt = s_list + kBT * TM;                       // distinct ancestors per depth [TM + 4]
+  int *s_pp = s_cnt + TM + 4;                           // parents of step t-1 [W_max]
+  int *s_slice = s_pp + p.W_max;                        // ancestor rows of depth t-2 [W_max][TM]
 
   const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(p.q);
   const __nv_bfloat16 *k = static_cast<const __nv_bfloat16 *>(p.k);
@@ -150,9 +164,9 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const StepParams p
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *s_tmem;
-  ptx::pdl_launch_dependents();
 
-  // ------------------------------------------- inputs (before the wait)
+  // ------------------------------------------- before the wait
+  // Every load of this phase is issued up front: one round trip.
   const uint32_t s0_bytes = (uint32_t)P * NK * 16384u;
   if (tid == kThreads - 32) {
     ptx::mbar_arrive_expect_tx(bar_s0, s0_bytes);
@@ -160,48 +174,36 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const StepParams p
     for (uint32_t off = 0; off < s0_bytes; off += 16384u)
       ptx::bulk_g2s(base + L.a + off, src + off, 16384u, bar_s0);
   }
-  for (int e = tid; e < kN * NK * 8; e += kThreads) {
+  // X: rows 0..31 k_b, 32..63 q_b, then the same 64 rows again (so that all
+  // four TMEM lane quarters of D2 hold vectors).  Zeros past the last beam.
+  for (int e = tid; e < 2 * kN * NK * 8; e += kThreads) {
     const int n = e / (NK * 8), cc = e - n * (NK * 8);
-    const int bb = n & (kBT - 1);
+    const int vec = n & (kN - 1);
+    const int bb = vec & (kBT - 1);
     const bool valid = bb < nb;
-    const __nv_bfloat16 *src = (n >= kBT ? q : k) + (row0 + (int64_t)(valid ? bb : 0) * H) * DK + cc * 8;
-    ptx::cp_async16(s_x + (cc >> 3) * (kN * 128) + ptx::swz128(n, cc & 7), src, valid ? 16u : 0u);
+    const __nv_bfloat16 *src = (vec >= kBT ? q : k) + (row0 + (int64_t)(valid ? bb : 0) * H) * DK + cc * 8;
+    ptx::cp_async16(s_x + (cc >> 3) * XA + ptx::swz128(n, cc & 7), src, valid ? 16u : 0u);
+  }
+  // The previous step's parents (an input of step t-1) and the ancestor rows
+  // of depth t-2 (written by step t-2, which has completed).
+  if (nanc >= 2)
+    for (int e = tid; e < p.W_prev; e += kThreads) ptx::cp_async4(s_pp + e, p.prev_parents + r * p.prev_stride + e);
+  if (nanc >= 3 && slice) {
+    const int w2 = nanc - 2;  // entries per row
+    const int32_t *src = p.anc + anc_row(p, nanc - 1, r, 0);
+    for (int e = tid; e < p.W_prev2 * w2; e += kThreads) {
+      const int row = e / w2, j = e - row * w2;
+      ptx::cp_async4(s_slice + e, src + (int64_t)row * TM + j);
+    }
   }
   ptx::cp_async_commit();
-  if (warp == 1) {
-    const int b = lane;
-    int par = -1;
-    float alpha = 0.f, beta = 0.f;
-    if (b < nb) {
-      par = nanc >= 1 ? p.parents[r * p.W + b0 + b] : 0;
-      if (par < 0 || par >= p.W_prev) {
-        *reinterpret_cast<volatile int32_t *>(p.err) = kErrParent;
-        par = 0;
-      }
-      const int64_t si = row0 + (int64_t)b * H;
-      alpha = expf(p.g[si]);
-      beta = p.beta[si];
-    }
-    s_par[b] = par;
-    s_alpha[b] = alpha;
-    s_beta[b] = beta;
-    // Distinct parents (the depth-(t-1) ancestors) take slots 0..U1-1.
-    if (nanc >= 1) {
-      const unsigned same = __match_any_sync(0xffffffffu, par);
-      const int leader = __ffs(same) - 1;
-      const bool lead = b < nb && leader == lane;
-      const unsigned leaders = __ballot_sync(0xffffffffu, lead);
-      const int my = __popc(leaders & ((1u << lane) - 1u));
-      if (lead) s_list[my] = (par << 5) | jp;
-      const int slot = __shfl_sync(0xffffffffu, my, leader);
-      if (b < nb) {
-        s_slot[b * TM + jp] = slot;
-        s_chain[b * TM + jp] = par;
-      }
-      if (lane == 0) *s_U1 = __popc(leaders);
-    } else if (lane == 0) {
-      *s_U1 = 0;
-    }
+  int par = -1;
+  float g_alpha = 0.f, g_beta = 0.f;
+  if (warp == 1 && lane < nb) {
+    par = nanc >= 1 ? p.parents[r * p.W + b0 + lane] : 0;
+    const int64_t si = row0 + (int64_t)lane * H;
+    g_alpha = p.g[si];
+    g_beta = p.beta[si];
   }
   // Epilogue mapping: warp w serves TMEM lanes 32*(w%4).. (output elements)
   // and beams 16*(w/4)..+15; v is loaded now, used at the end.
@@ -233,129 +235,73 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const StepParams p
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint64_t ad = ptx::desc_k128(a_u32 + (pl * NK + ka) * 16384 + kk * 32);
-          const uint64_t bd = ptx::desc_k128(x_u32 + ka * (kN * 128) + kk * 32);
+          const uint64_t bd = ptx::desc_k128(x_u32 + ka * XA + kk * 32);
           ptx::mma_bf16(tmem, ad, bd, idesc1, acc);
           acc = 1;
         }
-    // Dkq = X . K^T (M = 128 rows from X: rows past 63 are not used).
+    // Dkq = X . K^T: row 32 + b, column b is k_b . q_b.
     constexpr uint32_t idesc_kq = ptx::idesc_bf16_f32(kM, kBT);
 #pragma unroll
     for (int ka = 0; ka < NK; ++ka)
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t ad = ptx::desc_k128(x_u32 + ka * (kN * 128) + kk * 32);
-        const uint64_t bd = ptx::desc_k128(x_u32 + ka * (kN * 128) + kk * 32);
-        ptx::mma_bf16(tmem + 128, ad, bd, idesc_kq, (ka | kk) != 0);
+        const uint64_t ad = ptx::desc_k128(x_u32 + ka * XA + kk * 32);
+        ptx::mma_bf16(tmem + 128, ad, ad, idesc_kq, (ka | kk) != 0);
       }
     ptx::mma_commit(bar1);
   }
   if (warp == 1) {
-    // k_b . q_b = Dkq[32 + b][b]: TMEM lanes 32..63 belong to warp 1.
-    if (!ptx::mbar_wait(bar1, 0, kWaitLimitNs)) ok = false;
-    ptx::tc_fence_after();
-    float d[32];
-    ptx::tmem_ld32(tmem + (32u << 16) + 128, d);
-    ptx::tmem_ld_wait();
-    float kq = 0.f;
-#pragma unroll
-    for (int z = 0; z < 32; ++z)
-      if (z == lane) kq = d[z];
-    s_kq[lane] = kq;
-  }
-
-  // ------------------------------- records of earlier steps (after the wait)
-  ptx::pdl_wait();
-  // Round 1: the parents' ancestor rows and P values (warp 0), this step's
-  // keys into the record store, the parents' records into the operands.
-  if (warp == 0 && lane < nb) {
-    const int b = lane, gb = b0 + lane;
-    const int par = s_par[b];
-    float Gp = 1.f;
+    // Each beam's ancestor row: [row of g at depth t-2, g, p].
+    const int b = lane;
+    if (b < nb) {
+      if (par < 0 || par >= p.W_prev) {
+        *reinterpret_cast<volatile int32_t *>(p.err) = kErrParent;
+        par = 0;
+      }
+    }
+    s_par[b] = b < nb ? par : 0;
+    s_alpha[b] = b < nb ? expf(g_alpha) : 0.f;
+    s_beta[b] = g_beta;
     if (nanc >= 1) {
-      Gp = p.rec_P[rec_row(p, nanc, r, h, par)];
-      int tmp[kMaxT - 1];
-      if (nanc >= 2) {
-        const int32_t *prow = p.anc + anc_row(p, nanc, r, par);
+      // Distinct parents take slots 0..U1-1.
+      const unsigned same = __match_any_sync(0xffffffffu, par);
+      const int leader = __ffs(same) - 1;
+      const bool lead = b < nb && leader == lane;
+      const unsigned leaders = __ballot_sync(0xffffffffu, lead);
+      const int my = __popc(leaders & ((1u << lane) - 1u));
+      if (lead) s_list[my] = (par << 5) | jp;
+      const int slot = __shfl_sync(0xffffffffu, my, leader);
+      if (lane == 0) *s_U1 = __popc(leaders);
+      if (b < nb) {
+        s_slot[b * TM + jp] = slot;
+        s_chain[b * TM + jp] = par;
+        if (nanc >= 2) {
+          int gp = s_pp[par];
+          if (gp < 0 || gp >= p.W_prev2) gp = 0;  // already reported by step t-1
+          s_chain[b * TM + nanc - 2] = gp;
+          if (nanc >= 3) {
+            if (slice) {
+              for (int j = 0; j < nanc - 2; ++j) s_chain[b * TM + j] = s_slice[gp * (nanc - 2) + j];
+            } else {
+              const int32_t *grow = p.anc + anc_row(p, nanc - 1, r, gp);
+              int tmp[kMaxT - 2];
 #pragma unroll
-        for (int j = 0; j < kMaxT - 1; ++j)
-          if (j < nanc - 1) tmp[j] = prow[j];
+              for (int j = 0; j < kMaxT - 2; ++j)
+                if (j < nanc - 2) tmp[j] = grow[j];
 #pragma unroll
-        for (int j = 0; j < kMaxT - 1; ++j)
-          if (j < nanc - 1) s_chain[b * TM + j] = tmp[j];
-      }
-      if (h == 0) {
-        int32_t *row = p.anc + anc_row(p, t, r, gb);
-#pragma unroll
-        for (int j = 0; j < kMaxT - 1; ++j)
-          if (j < nanc - 1) row[j] = tmp[j];
-        row[nanc - 1] = par;
-      }
-    }
-    s_Gp[b] = Gp;
-    p.rec_alpha[rec_row(p, t, r, h, gb)] = s_alpha[b];
-    p.rec_P[rec_row(p, t, r, h, gb)] = Gp * s_alpha[b];
-  }
-  for (int e = tid; e < kBT * NK * 8; e += kThreads) {
-    const int n = e / (NK * 8), cc = e - n * (NK * 8);
-    if (n < nb)
-      reinterpret_cast<uint4 *>(rec_k + rec_row(p, t, r, h, b0 + n) * DK)[cc] =
-          *reinterpret_cast<const uint4 *>(s_x + (cc >> 3) * (kN * 128) + ptx::swz128(n, cc & 7));
-  }
-  // Region A holds the S0 image until D1 is complete.
-  if (!ptx::mbar_wait(bar1, 0, kWaitLimitNs)) ok = false;
-
-  // Stage slots [lo, hi) of block blk: keys (cp.async) into KA; deltas / P(a)
-  // as fp16 hi + lo into the MN-major Delta' operand.
-  auto stage = [&](int blk, int lo, int hi) {
-    for (int e = tid; e < (hi - lo) * NK * 8; e += kThreads) {
-      const int s = lo + e / (NK * 8), cc = e % (NK * 8);
-      const int packed = s_list[s];
-      const int lr = s - blk * kBlk;
-      ptx::cp_async16(base + L.ka + (cc >> 3) * (kBlk * 128) + ptx::swz128(lr, cc & 7),
-                      rec_k + rec_row(p, (packed & 31) + 1, r, h, packed >> 5) * DK + cc * 8, 16u);
-    }
-    ptx::cp_async_commit();
-    for (int e0 = tid; e0 < (hi - lo) * C4; e0 += 4 * kThreads) {
-      float4 val[4];
-      float pa[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int e = e0 + u * kThreads;
-        val[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-        pa[u] = 1.f;
-        if (e < (hi - lo) * C4) {
-          const int packed = s_list[lo + e / C4];
-          const int64_t rr = rec_row(p, (packed & 31) + 1, r, h, packed >> 5);
-          val[u] = __ldcg(reinterpret_cast<const float4 *>(p.rec_delta + rr * DV) + e % C4);
-          pa[u] = __ldcg(p.rec_P + rr);
+              for (int j = 0; j < kMaxT - 2; ++j)
+                if (j < nanc - 2) s_chain[b * TM + j] = tmp[j];
+            }
+          }
         }
       }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int e = e0 + u * kThreads;
-        if (e < (hi - lo) * C4) {
-          const int lr = lo + e / C4 - blk * kBlk;
-          const int i0 = (e % C4) * 4;
-          const uint32_t off = (uint32_t)(i0 >> 6) * 8192u + (uint32_t)(lr >> 3) * 1024u +
-                               (uint32_t)(lr & 7) * 128u + (uint32_t)((((i0 & 63) >> 3) ^ (lr & 7)) << 4) +
-                               (uint32_t)(i0 & 7) * 2u;
-          const float inv = 1.f / pa[u];
-          const float f[4] = {val[u].x * inv, val[u].y * inv, val[u].z * inv, val[u].w * inv};
-          __align__(8) __half hi4[4], lo4[4];
-#pragma unroll
-          for (int z = 0; z < 4; ++z) split_f16(f[z], hi4[z], lo4[z]);
-          *reinterpret_cast<uint2 *>(base + L.dhi + off) = *reinterpret_cast<const uint2 *>(hi4);
-          *reinterpret_cast<uint2 *>(base + L.dlo + off) = *reinterpret_cast<const uint2 *>(lo4);
-        }
-      }
+    } else if (lane == 0) {
+      *s_U1 = 0;
     }
-  };
-  const int U1 = *s_U1;
-  if (U1 > 0) stage(0, 0, U1);
-  __syncthreads();  // ancestor rows in s_chain
-
-  // Deeper ancestors: one warp per depth finds the distinct ones, then the
-  // slots U1.. are handed out depth by depth.
+  }
+  __syncthreads();
+  // Deeper ancestors (depths 1..t-2): one warp per depth finds the distinct
+  // ones; their slots follow the parents', depth by depth.
   for (int j = warp; j < nanc - 1; j += kThreads / 32) {
     const int a = lane < nb ? s_chain[lane * TM + j] : -1;
     const unsigned same = __match_any_sync(0xffffffffu, a);
@@ -368,18 +314,105 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const StepParams p
     if (lane == 0) s_cnt[j] = __popc(leaders);
   }
   __syncthreads();
+  const int U1 = *s_U1;
   int U = U1;
   for (int j = 0; j < nanc - 1; ++j) U += s_cnt[j];
-  if (warp == 0 && lane < nb) {
-    int run = U1;
-    for (int j = 0; j < nanc - 1; ++j) {
-      const int slot = run + s_slot[lane * TM + j];
+  for (int j = warp; j < nanc - 1; j += kThreads / 32) {
+    int base_j = U1;
+    for (int j2 = 0; j2 < j; ++j2) base_j += s_cnt[j2];
+    if (lane < nb) {
+      const int slot = base_j + s_slot[lane * TM + j];
       s_slot[lane * TM + j] = slot;
       s_list[slot] = (s_chain[lane * TM + j] << 5) | j;
-      run += s_cnt[j];
     }
   }
-  __syncthreads();
+  __syncthreads();  // slots and the slot list complete
+
+  // ------------------------------- after the wait: step t-1's records
+  ptx::pdl_wait();
+  ptx::pdl_launch_dependents();
+  // Region A holds the S0 image until D1 is complete.
+  if (!ptx::mbar_wait(bar1, 0, kWaitLimitNs)) ok = false;
+
+  // Stage slots [lo, hi) of block blk: keys (cp.async) into KA; deltas / P(a)
+  // as fp16 hi + lo into the MN-major Delta' operand.  All loads in flight
+  // at once.
+  auto stage = [&](int blk, int lo, int hi) {
+    for (int e = tid; e < (hi - lo) * NK * 8; e += kThreads) {
+      const int s = lo + e / (NK * 8), cc = e % (NK * 8);
+      const int packed = s_list[s];
+      const int lr = s - blk * kBlk;
+      ptx::cp_async16(base + L.ka + (cc >> 3) * (kBlk * 128) + ptx::swz128(lr, cc & 7),
+                      rec_k + rec_row(p, (packed & 31) + 1, r, h, packed >> 5) * DK + cc * 8, 16u);
+    }
+    ptx::cp_async_commit();
+    float4 val[NF];
+    float pa[NF];
+#pragma unroll
+    for (int u = 0; u < NF; ++u) {
+      const int e = tid + u * kThreads;
+      val[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      pa[u] = 1.f;
+      if (e < (hi - lo) * C4) {
+        const int packed = s_list[lo + e / C4];
+        const int64_t rr = rec_row(p, (packed & 31) + 1, r, h, packed >> 5);
+        val[u] = __ldcg(reinterpret_cast<const float4 *>(p.rec_delta + rr * DV) + e % C4);
+        pa[u] = __ldcg(p.rec_P + rr);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < NF; ++u) {
+      const int e = tid + u * kThreads;
+      if (e < (hi - lo) * C4) {
+        const int lr = lo + e / C4 - blk * kBlk;
+        const int i0 = (e % C4) * 4;
+        const uint32_t off = (uint32_t)(i0 >> 6) * 8192u + (uint32_t)(lr >> 3) * 1024u +
+                             (uint32_t)(lr & 7) * 128u + (uint32_t)((((i0 & 63) >> 3) ^ (lr & 7)) << 4) +
+                             (uint32_t)(i0 & 7) * 2u;
+        const float inv = 1.f / pa[u];
+        const float f[4] = {val[u].x * inv, val[u].y * inv, val[u].z * inv, val[u].w * inv};
+        __align__(8) __half hi4[4], lo4[4];
+#pragma unroll
+        for (int z = 0; z < 4; ++z) split_f16(f[z], hi4[z], lo4[z]);
+        *reinterpret_cast<uint2 *>(base + L.dhi + off) = *reinterpret_cast<const uint2 *>(hi4);
+        *reinterpret_cast<uint2 *>(base + L.dlo + off) = *reinterpret_cast<const uint2 *>(lo4);
+      }
+    }
+  };
+  // This step's outputs that need no arithmetic (records of depth t: alpha,
+  // P, k; the ancestor row and parents of depth t) and P(parent): issued
+  // first so that they overlap the staging loads.
+  if (warp == 2 && lane < nb) {
+    const int b = lane, gb = b0 + lane;
+    const float Gp = nanc >= 1 ? __ldcg(p.rec_P + rec_row(p, nanc, r, h, s_par[b])) : 1.f;
+    s_Gp[b] = Gp;
+    p.rec_alpha[rec_row(p, t, r, h, gb)] = s_alpha[b];
+    p.rec_P[rec_row(p, t, r, h, gb)] = Gp * s_alpha[b];
+    if (h == 0) {
+      int32_t *row = p.anc + anc_row(p, t, r, gb);
+      for (int j = 0; j < nanc; ++j) row[j] = s_chain[b * TM + j];
+      p.par_store[((int64_t)(t - 1) * p.R + r) * p.W_max + gb] = s_par[b];
+    }
+  }
+  if (U > 0) stage(0, 0, min(U, kBlk));
+  for (int e = tid; e < kBT * NK * 8; e += kThreads) {
+    const int n = e / (NK * 8), cc = e - n * (NK * 8);
+    if (n < nb)
+      reinterpret_cast<uint4 *>(rec_k + rec_row(p, t, r, h, b0 + n) * DK)[cc] =
+          *reinterpret_cast<const uint4 *>(s_x + (cc >> 3) * XA + ptx::swz128(n, cc & 7));
+  }
+  if (warp == 1) {
+    // k_b . q_b from Dkq (TMEM lanes 32..63 belong to warp 1).
+    ptx::tc_fence_after();
+    float d[32];
+    ptx::tmem_ld32(tmem + (32u << 16) + 128, d);
+    ptx::tmem_ld_wait();
+    float kq = 0.f;
+#pragma unroll
+    for (int z = 0; z < 32; ++z)
+      if (z == lane) kq = d[z];
+    s_kq[lane] = kq;
+  }
   const int nblk = (U + kBlk - 1) / kBlk;
 
   for (int blk = 0; blk < nblk; ++blk) {
@@ -389,8 +422,6 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const StepParams p
     if (blk > 0) {
       if (!ptx::mbar_wait(bar3, (blk - 1) & 1, kWaitLimitNs)) ok = false;
       stage(blk, lo, hi);
-    } else if (hi > U1) {
-      stage(0, U1, hi);
     }
     // Slots past the block's last ancestor but inside the MMA K range hold
     // zero deltas.
@@ -410,38 +441,42 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const StepParams p
       for (int ka = 0; ka < NK; ++ka)
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t ad = ptx::desc_k128(x_u32 + ka * (kN * 128) + kk * 32);
+          const uint64_t ad = ptx::desc_k128(x_u32 + ka * XA + kk * 32);
           const uint64_t bd = ptx::desc_k128(ka_u32 + ka * (kBlk * 128) + kk * 32);
           ptx::mma_bf16(tmem + 64, ad, bd, idesc2, (ka | kk) != 0);
         }
       ptx::mma_commit(bar2);
     }
-    // C build: TMEM lanes 0..63 (vector n) belong to warps 0, 1, 4, 5; each
-    // takes a 16-slot column group.  C[n][a] = D2[n][a] where a is an
-    // ancestor of n's beam, else 0, stored as fp16 hi + lo, K-major.
-    const bool c_warp = (warp & 2) == 0;  // warps 0,1,4,5: column groups 0,2 / 1,3
+    // C build: D2 row n (TMEM lane n) is vector n % 64; warp w takes the
+    // lane quarter w % 4 and the 16-slot column group (w % 4) / 2 + 2 (w / 4).
+    // C[vec][a] = D2[vec][a] where a is an ancestor of vec's beam, else 0,
+    // stored as fp16 hi + lo, K-major (row vec, K = slot).
     if (!ptx::mbar_wait(bar2, blk & 1, kWaitLimitNs)) ok = false;
     ptx::tc_fence_after();
-    for (int g = (warp >> 2); c_warp && g * 16 < kpad; g += 2) {
-      const int n = (warp & 1) * 32 + lane;
-      const int b = n & (kBT - 1);
-      float d[16];
-      ptx::tmem_ld16(tmem + ((uint32_t)((warp & 1) * 32) << 16) + 64 + g * 16, d);
-      ptx::tmem_ld_wait();
-      uint32_t mask = 0u;
-      if (b < nb)
-        for (int j = 0; j < nanc; ++j) {
-          const int s = s_slot[b * TM + j] - lo - g * 16;
-          if (s >= 0 && s < 16) mask |= 1u << s;
+    {
+      const int qq = warp & 3;
+      const int g = (qq >> 1) + 2 * (warp >> 2);
+      if (g * 16 < kpad) {
+        const int vec = (qq * 32 + lane) & (kN - 1);
+        const int b = vec & (kBT - 1);
+        float d[16];
+        ptx::tmem_ld16(tmem + ((uint32_t)(qq * 32) << 16) + 64 + g * 16, d);
+        ptx::tmem_ld_wait();
+        uint32_t mask = 0u;
+        if (b < nb)
+          for (int j = 0; j < nanc; ++j) {
+            const int sl = s_slot[b * TM + j] - lo - g * 16;
+            if (sl >= 0 && sl < 16) mask |= 1u << sl;
+          }
+        __align__(16) __half h16[16], l16[16];
+#pragma unroll
+        for (int z = 0; z < 16; ++z) split_f16(((mask >> z) & 1u) ? d[z] : 0.f, h16[z], l16[z]);
+#pragma unroll
+        for (int c2 = 0; c2 < 2; ++c2) {
+          const uint32_t off = ptx::swz128(vec, g * 2 + c2);
+          *reinterpret_cast<uint4 *>(base + L.chi + off) = reinterpret_cast<const uint4 *>(h16)[c2];
+          *reinterpret_cast<uint4 *>(base + L.clo + off) = reinterpret_cast<const uint4 *>(l16)[c2];
         }
-      __align__(16) __half h16[16], l16[16];
-#pragma unroll
-      for (int z = 0; z < 16; ++z) split_f16(((mask >> z) & 1u) ? d[z] : 0.f, h16[z], l16[z]);
-#pragma unroll
-      for (int c2 = 0; c2 < 2; ++c2) {
-        const uint32_t off = ptx::swz128(n, g * 2 + c2);
-        *reinterpret_cast<uint4 *>(base + L.chi + off) = reinterpret_cast<const uint4 *>(h16)[c2];
-        *reinterpret_cast<uint4 *>(base + L.clo + off) = reinterpret_cast<const uint4 *>(l16)[c2];
       }
     }
     ptx::fence_proxy_async_smem();
@@ -466,6 +501,7 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const StepParams p
   // --------------------------------------------------------- epilogue
   if (nblk > 0 && !ptx::mbar_wait(bar3, (nblk - 1) & 1, kWaitLimitNs)) ok = false;
   if (!ok) *reinterpret_cast<volatile int32_t *>(p.err) = kErrTimeout;
+  __syncthreads();  // s_Gp and s_kq visible
   ptx::tc_fence_after();
   {
     const uint32_t lb = (uint32_t)((warp & 3) * 32) << 16;
@@ -478,6 +514,9 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const StepParams p
       const float4 *A4 = reinterpret_cast<const float4 *>(s_alpha + half * 16);
       const float4 *B4 = reinterpret_cast<const float4 *>(s_beta + half * 16);
       const float4 *K4 = reinterpret_cast<const float4 *>(s_kq + half * 16);
+      const int64_t ostride = (int64_t)H * DV;
+      float *op = p.o + (row0 + (int64_t)(half * 16) * H) * DV + ei;
+      float *dp = p.rec_delta + (rec_row(p, t, r, h, b0) + half * 16) * DV + ei;
 #pragma unroll
       for (int m4 = 0; m4 < 4; ++m4) {
         const float4 G = G4[m4], A = A4[m4], B = B4[m4], KQ = K4[m4];
@@ -486,12 +525,11 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const StepParams p
 #pragma unroll
         for (int z = 0; z < 4; ++z) {
           const int m = m4 * 4 + z;
-          const int b = half * 16 + m;
-          if (b < nb) {
+          if (half * 16 + m < nb) {
             const float ag = Av[z] * Gv[z];  // alpha P(p)
             const float delta = Bv[z] * fmaf(-ag, uk[m], __bfloat162float(vreg[m]));
-            p.o[(row0 + (int64_t)b * H) * DV + ei] = fmaf(ag, uq[m], delta * Kv[z]);
-            p.rec_delta[rec_row(p, t, r, h, b0 + b) * DV + ei] = delta;
+            op[m * ostride] = fmaf(ag, uq[m], delta * Kv[z]);
+            dp[m * DV] = delta;
           }
         }
       }
@@ -543,7 +581,7 @@ __global__ void s0_image_kernel(const void *S0, uint4 *img, int R, int H, int dk
 
 template <int DK>
 cudaError_t launch_dk(const StepParams &p, bool pdl, cudaStream_t s) {
-  const Layout L = layout(DK / 64, p.s0_planes, p.T_max);
+  const Layout L = layout(DK / 64, p.s0_planes, p.T_max, p.W_max);
   const size_t smem = L.total + 1024;
   static size_t configured[64] = {0};
   int dev = 0;

@@ -125,6 +125,17 @@ def test_adversarial_parents(kernel, kind):
 
 
 @pytest.mark.parametrize("kernel", [1, 2])
+def test_wide_beams_gathered_ancestry(kernel):
+    """W_max * T_max too large for the tensor-core kernel's shared-memory
+    copy of the ancestor rows: it gathers them row by row instead."""
+    _skip_unavailable(kernel, 64, 64, "bf16")
+    wl, S0, steps = P.custom_steps(16, 1, 2, 64, 64, (600, 600, 600, 600, 600))
+    S0c = synth.cast_state(S0, "f32")
+    gpu, _ = P.run_gpu(S0c, steps, "bf16", kernel, T_max=8)
+    P.compare(gpu, P.oracle(S0c, steps), steps, "f32")
+
+
+@pytest.mark.parametrize("kernel", [1, 2])
 def test_deep_decode(kernel):
     _skip_unavailable(kernel, 64, 64, "bf16")
     wl, S0, steps = P.custom_steps(8, 1, 2, 64, 64, (24,) * 12)
