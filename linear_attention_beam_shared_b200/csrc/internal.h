@@ -1,6 +1,7 @@
 // Internal declarations shared by the runtime and the decode kernels.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -34,6 +35,10 @@ struct StepParams {
   void *rec_k;            // [T_max][R][H][W_max][dk] in the qkv type
   int32_t *anc;           // [T_max][R][W_max][T_max]
   int32_t *err;           // host-mapped error word (device view)
+  // TMA descriptors of k and q (tensor-core kernel; encoded per call):
+  // 4-D {d_k, H, W, R} bf16, box {64, 1, 32, 1}, 128-byte swizzle.
+  alignas(64) CUtensorMap tm_k;
+  alignas(64) CUtensorMap tm_q;
 };
 
 // Row index of the record of beam b, head h, request r at depth s (1-based).

@@ -49,6 +49,7 @@
 // before it may still be reading.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cudaTypedefs.h>
 
 #include "internal.h"
 #include "sm100_ptx.h"
@@ -105,7 +106,7 @@ __device__ __forceinline__ void split_f16(float x, __half &hi, __half &lo) {
 }
 
 template <int DK>
-__global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const StepParams p) {
+__global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_constant__ StepParams p) {
   constexpr int NK = DK / 64;  // 128-byte K atoms per key row
   constexpr int DV = DK;
   constexpr int C4 = DV / 4;   // float4 chunks per delta row
@@ -142,8 +143,6 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const StepParams p
   int *s_pp = s_cnt + TM + 4;                           // parents of step t-1 [W_max]
   int *s_slice = s_pp + p.W_max;                        // ancestor rows of depth t-2 [W_max][TM]
 
-  const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(p.q);
-  const __nv_bfloat16 *k = static_cast<const __nv_bfloat16 *>(p.k);
   const __nv_bfloat16 *v = static_cast<const __nv_bfloat16 *>(p.v);
   __nv_bfloat16 *rec_k = static_cast<__nv_bfloat16 *>(p.rec_k);
   const int64_t row0 = (int64_t)(r * p.W + b0) * H + h;  // (r, b0, h) row of [R][W][H][d]
@@ -169,20 +168,21 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const StepParams p
   // Every load of this phase is issued up front: one round trip.
   const uint32_t s0_bytes = (uint32_t)P * NK * 16384u;
   if (tid == kThreads - 32) {
-    ptx::mbar_arrive_expect_tx(bar_s0, s0_bytes);
+    // S0 image (bulk copy) and X by TMA: rows 0..31 k_b, 32..63 q_b, then
+    // the same 64 rows again (so that all four TMEM lane quarters of D2 hold
+    // vectors).  Beams past W read as zeros.
+    ptx::mbar_arrive_expect_tx(bar_s0, s0_bytes + 2u * kN * 128u * NK);
     const uint8_t *src = static_cast<const uint8_t *>(p.S0img) + (size_t)(r * H + h) * s0_bytes;
     for (uint32_t off = 0; off < s0_bytes; off += 16384u)
       ptx::bulk_g2s(base + L.a + off, src + off, 16384u, bar_s0);
-  }
-  // X: rows 0..31 k_b, 32..63 q_b, then the same 64 rows again (so that all
-  // four TMEM lane quarters of D2 hold vectors).  Zeros past the last beam.
-  for (int e = tid; e < 2 * kN * NK * 8; e += kThreads) {
-    const int n = e / (NK * 8), cc = e - n * (NK * 8);
-    const int vec = n & (kN - 1);
-    const int bb = vec & (kBT - 1);
-    const bool valid = bb < nb;
-    const __nv_bfloat16 *src = (vec >= kBT ? q : k) + (row0 + (int64_t)(valid ? bb : 0) * H) * DK + cc * 8;
-    ptx::cp_async16(s_x + (cc >> 3) * XA + ptx::swz128(n, cc & 7), src, valid ? 16u : 0u);
+#pragma unroll
+    for (int copy = 0; copy < 2; ++copy)
+#pragma unroll
+      for (int ka = 0; ka < NK; ++ka) {
+        uint8_t *dst = s_x + ka * XA + copy * (kN * 128);
+        ptx::tma_load_4d(dst, &p.tm_k, ka * 64, h, b0, r, bar_s0);
+        ptx::tma_load_4d(dst + kBT * 128, &p.tm_q, ka * 64, h, b0, r, bar_s0);
+      }
   }
   // The previous step's parents (an input of step t-1) and the ancestor rows
   // of depth t-2 (written by step t-2, which has completed).
@@ -300,9 +300,10 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const StepParams p
     }
   }
   __syncthreads();
-  // Deeper ancestors (depths 1..t-2): one warp per depth finds the distinct
-  // ones; their slots follow the parents', depth by depth.
-  for (int j = warp; j < nanc - 1; j += kThreads / 32) {
+  // Deeper ancestors (depths 1..t-2): one warp per depth (warps 1..7; warp 0
+  // issues the MMAs) finds the distinct ones; their slots follow the
+  // parents', depth by depth.
+  for (int j = warp - 1; warp > 0 && j < nanc - 1; j += kThreads / 32 - 1) {
     const int a = lane < nb ? s_chain[lane * TM + j] : -1;
     const unsigned same = __match_any_sync(0xffffffffu, a);
     const int leader = __ffs(same) - 1;
@@ -317,7 +318,7 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const StepParams p
   const int U1 = *s_U1;
   int U = U1;
   for (int j = 0; j < nanc - 1; ++j) U += s_cnt[j];
-  for (int j = warp; j < nanc - 1; j += kThreads / 32) {
+  for (int j = warp - 1; warp > 0 && j < nanc - 1; j += kThreads / 32 - 1) {
     int base_j = U1;
     for (int j2 = 0; j2 < j; ++j2) base_j += s_cnt[j2];
     if (lane < nb) {
@@ -379,12 +380,14 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const StepParams p
       }
     }
   };
-  // This step's outputs that need no arithmetic (records of depth t: alpha,
-  // P, k; the ancestor row and parents of depth t) and P(parent): issued
-  // first so that they overlap the staging loads.
+  // P(parent): loaded now, consumed after the staging loads are issued.
+  float Gp = 1.f;
+  if (warp == 2 && lane < nb && nanc >= 1) Gp = __ldcg(p.rec_P + rec_row(p, nanc, r, h, s_par[lane]));
+  if (U > 0) stage(0, 0, min(U, kBlk));
+  // This step's outputs that need no arithmetic: records of depth t (alpha,
+  // P, k), the ancestor row and the parents of depth t.
   if (warp == 2 && lane < nb) {
     const int b = lane, gb = b0 + lane;
-    const float Gp = nanc >= 1 ? __ldcg(p.rec_P + rec_row(p, nanc, r, h, s_par[b])) : 1.f;
     s_Gp[b] = Gp;
     p.rec_alpha[rec_row(p, t, r, h, gb)] = s_alpha[b];
     p.rec_P[rec_row(p, t, r, h, gb)] = Gp * s_alpha[b];
@@ -394,7 +397,7 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const StepParams p
       p.par_store[((int64_t)(t - 1) * p.R + r) * p.W_max + gb] = s_par[b];
     }
   }
-  if (U > 0) stage(0, 0, min(U, kBlk));
+  if (!ptx::mbar_wait(bar_s0, 0, kWaitLimitNs)) ok = false;  // X visible to this thread
   for (int e = tid; e < kBT * NK * 8; e += kThreads) {
     const int n = e / (NK * 8), cc = e - n * (NK * 8);
     if (n < nb)
@@ -579,8 +582,38 @@ __global__ void s0_image_kernel(const void *S0, uint4 *img, int R, int H, int dk
   }
 }
 
+// cuTensorMapEncodeTiled, fetched once from the driver.
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// 4-D map over a [R][W][H][d] bf16 tensor: {d, H, W, R}, box {64, 1, 32, 1},
+// 128-byte swizzle (the K-major operand layout), zeros outside the tensor.
+bool encode_rows(CUtensorMap *m, const void *base, int d, int H, int W, int R) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)W, (cuuint64_t)R};
+  const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, (cuuint64_t)W * H * d * 2};
+  const cuuint32_t box[4] = {64, 1, (cuuint32_t)kBT, 1};
+  const cuuint32_t es[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int DK>
-cudaError_t launch_dk(const StepParams &p, bool pdl, cudaStream_t s) {
+cudaError_t launch_dk(const StepParams &p_in, bool pdl, cudaStream_t s) {
+  StepParams p = p_in;
+  if (!encode_rows(&p.tm_k, p.k, DK, p.H, p.W, p.R) || !encode_rows(&p.tm_q, p.q, DK, p.H, p.W, p.R))
+    return cudaErrorInvalidValue;
   const Layout L = layout(DK / 64, p.s0_planes, p.T_max, p.W_max);
   const size_t smem = L.total + 1024;
   static size_t configured[64] = {0};
