@@ -7,6 +7,10 @@
 
 namespace onela {
 
+constexpr int kHistSteps = 17;     // steps 1..16: the deepest tensor-core decode
+constexpr int kHistMaxInts = 4096;  // parents of earlier steps the tensor-core kernel
+                                    // keeps in shared memory (more: read from global memory)
+
 // Everything one decode step needs.  Record store and ancestry index are the
 // handle's; all other pointers are the caller's tensors for this step.
 struct StepParams {
@@ -17,28 +21,36 @@ struct StepParams {
   const void *q, *k, *v;  // [R][W][H][d] in the qkv type
   const float *g, *beta;  // [R][W][H]
   const int32_t *parents; // [R][W]
-  // Parents of the previous step (step t-1), [R][prev_stride] with W_prev
-  // valid entries per request, and the beam count of step t-2 (W_prev2).
-  // Used by the tensor-core kernel for t >= 3; may be null otherwise.
-  const int32_t *prev_parents;
-  int prev_stride, W_prev2;
   int32_t *par_store;     // [T_max][R][W_max]: each step's parents (tensor-core kernel)
+  // History of the decode for the tensor-core kernel, indexed by step j
+  // (1 <= j < t): keys, gates and parents of every earlier step.
+  // hist_inputs = 1: the callers' own arrays of step j, valid under
+  // ONELA_FLAG_PDL -- hk[j] [R][W_j][H][d_k], hg[j] [R][W_j][H] (the gate
+  // before exp), hpar[j] [R][W_j].  hist_inputs = 0: the record store
+  // (rec_k, rec_alpha) and the par_store row of step j.  Parents of request r
+  // start at hpar[j] + r * hpar_rs[j]; hW[j] = W_j.
+  int hist_inputs;
+  const void *hk[kHistSteps];
+  const float *hg[kHistSteps];
+  const int32_t *hpar[kHistSteps];
+  int hpar_rs[kHistSteps];
+  int hW[kHistSteps];
+  int hoff[kHistSteps];  // where step j's parents start in the kernel's shared copy (ints)
+  int hist_cap;  // ints of shared memory for the parents of steps 2..t-1 (0: read them from global memory)
   float *o;               // [R][W][H][dv]
   const void *S0;         // [R][H][dv][dk] in the S0 type
   const void *S0img;      // tensor-core operand image of S0 (see step_tc.cu)
   int s0_planes;          // bf16 terms in S0img (1 for bf16 S0)
   float *rec_alpha;       // [T_max][R][H][W_max]
-  float *rec_P;           // [T_max][R][H][W_max]: product of the gates on the
-                          // path from the root to the record, inclusive
-                          // (tensor-core kernel only; may be null otherwise)
   float *rec_delta;       // [T_max][R][H][W_max][dv]
   void *rec_k;            // [T_max][R][H][W_max][dk] in the qkv type
   int32_t *anc;           // [T_max][R][W_max][T_max]
   int32_t *err;           // host-mapped error word (device view)
-  // TMA descriptors of k and q (tensor-core kernel; encoded per call):
-  // 4-D {d_k, H, W, R} bf16, box {64, 1, 32, 1}, 128-byte swizzle.
+  // TMA descriptors of k, q and v (tensor-core kernel; encoded per call):
+  // 4-D {d, H, W, R} bf16, box {64, 1, 32, 1}, 128-byte swizzle.
   alignas(64) CUtensorMap tm_k;
   alignas(64) CUtensorMap tm_q;
+  alignas(64) CUtensorMap tm_v;
 };
 
 // Row index of the record of beam b, head h, request r at depth s (1-based).

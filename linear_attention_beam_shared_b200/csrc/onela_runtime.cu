@@ -20,9 +20,12 @@ struct onela_handle {
   void *S0;
   void *S0img;
   int32_t *par_store;         // each step's parents, written by the kernel
-  const int32_t *last_parents;  // the previous call's parent_idx (caller memory)
+  // Every earlier call's k, gate and parent_idx (caller memory; read again
+  // only under ONELA_FLAG_PDL).
+  std::vector<const void *> hist_k;
+  std::vector<const float *> hist_g;
+  std::vector<const int32_t *> hist_par;
   float *rec_alpha;
-  float *rec_P;
   float *rec_delta;
   void *rec_k;
   int32_t *anc;
@@ -53,7 +56,6 @@ void free_all(onela_handle *h) {
   cudaFree(h->S0);
   cudaFree(h->S0img);
   cudaFree(h->rec_alpha);
-  cudaFree(h->rec_P);
   cudaFree(h->par_store);
   cudaFree(h->rec_delta);
   cudaFree(h->rec_k);
@@ -74,7 +76,6 @@ onela::StepParams base_params(const onela_handle *h) {
   p.S0img = h->S0img;
   p.s0_planes = h->planes;
   p.rec_alpha = h->rec_alpha;
-  p.rec_P = h->rec_P;
   p.par_store = h->par_store;
   p.rec_delta = h->rec_delta;
   p.rec_k = h->rec_k;
@@ -138,7 +139,6 @@ int onela_create(const onela_config *cfg, onela_handle **out) {
   if (ok && kernel == ONELA_KERNEL_TC)
     ok = cudaMalloc(&h->S0img, onela::s0_image_bytes(c.R, c.H, c.d_k, c.d_v, h->planes)) == cudaSuccess;
   ok = ok && cudaMalloc((void **)&h->rec_alpha, nrow * sizeof(float)) == cudaSuccess;
-  if (ok && kernel == ONELA_KERNEL_TC) ok = cudaMalloc((void **)&h->rec_P, nrow * sizeof(float)) == cudaSuccess;
   if (ok && kernel == ONELA_KERNEL_TC)
     ok = cudaMalloc((void **)&h->par_store, (size_t)c.T_max * c.R * c.W_max * sizeof(int32_t)) == cudaSuccess;
   ok = ok && cudaMalloc((void **)&h->rec_delta, nrow * c.d_v * sizeof(float)) == cudaSuccess;
@@ -179,6 +179,9 @@ int onela_set_prompt_state(onela_handle *h, const void *S0, onela_stream stream)
   h->has_prompt = 1;
   h->steps_done = 0;
   h->Ws.clear();
+  h->hist_k.clear();
+  h->hist_g.clear();
+  h->hist_par.clear();
   return ONELA_OK;
 }
 
@@ -210,17 +213,33 @@ int onela_decode_step(onela_handle *h, int32_t W_prev, int32_t W, const void *q,
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   const bool pdl = (c.flags & ONELA_FLAG_PDL) && p.t >= 2;
-  if (p.t >= 3) {
-    p.W_prev2 = h->Ws[p.t - 3];
-    if (pdl) {
-      // The previous call's parents, still valid by the ONELA_FLAG_PDL contract.
-      p.prev_parents = h->last_parents;
-      p.prev_stride = W_prev;
-    } else {
-      // The copy the previous step's kernel wrote (it has completed).
-      p.prev_parents = h->par_store + (size_t)(p.t - 2) * c.R * c.W_max;
-      p.prev_stride = c.W_max;
+  if (h->kernel == ONELA_KERNEL_TC) {
+    // The tensor-core kernel reads tiles of q, k, v and o with 16-byte accesses.
+    const uintptr_t any = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
+                          reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(o);
+    if (any & 15u) return ONELA_ERR_ARG;
+    // Keys, gates and parents of the earlier steps: the callers' arrays under
+    // ONELA_FLAG_PDL (still valid by its contract), else the record store
+    // and the parents the earlier kernels stored (they have completed).
+    p.hist_inputs = pdl ? 1 : 0;
+    int hist = 0;
+    for (int j = 1; j < p.t; ++j) {
+      p.hW[j] = h->Ws[j - 1];
+      if (pdl) {
+        p.hk[j] = h->hist_k[j - 1];
+        p.hg[j] = h->hist_g[j - 1];
+        p.hpar[j] = h->hist_par[j - 1];
+        p.hpar_rs[j] = h->Ws[j - 1];
+      } else {
+        p.hpar[j] = h->par_store + (size_t)(j - 1) * c.R * c.W_max;
+        p.hpar_rs[j] = c.W_max;
+      }
+      if (j >= 2) {
+        p.hoff[j] = hist;
+        hist += (h->Ws[j - 1] + 3) & ~3;
+      }
     }
+    p.hist_cap = hist <= onela::kHistMaxInts ? hist : 0;
   }
   if (h->kernel == ONELA_KERNEL_TC)
     e = onela::launch_step_tc(p, pdl, s);
@@ -232,7 +251,9 @@ int onela_decode_step(onela_handle *h, int32_t W_prev, int32_t W, const void *q,
   }
   h->steps_done += 1;
   h->Ws.push_back(W);
-  h->last_parents = parent_idx;
+  h->hist_k.push_back(k);
+  h->hist_g.push_back(gate);
+  h->hist_par.push_back(parent_idx);
   return ONELA_OK;
 }
 
@@ -245,6 +266,9 @@ int onela_reset(onela_handle *h, onela_stream stream) {
   *reinterpret_cast<volatile int32_t *>(h->err_host) = 0;
   h->steps_done = 0;
   h->Ws.clear();
+  h->hist_k.clear();
+  h->hist_g.clear();
+  h->hist_par.clear();
   return ONELA_OK;
 }
 

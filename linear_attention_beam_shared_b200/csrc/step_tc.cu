@@ -2,51 +2,42 @@
 // d_k = d_v in {64, 128}.
 //
 // One CTA per (request r, head h, tile of 32 beams); 256 threads; two CTAs
-// fit on an SM, so a step launched as a programmatic dependent runs its
-// input phase beside the previous step.  The step of the shared-state GDN
-// beam decode (OneLA, evolve.pub review, key claims on section 3.2,
-// equations 2-4) runs as dense products on the tensor cores, fp32
-// accumulators in TMEM:
+// fit on an SM.  The step of the shared-state GDN beam decode (OneLA,
+// evolve.pub review, key claims on section 3.2, equations 2-4).  For beam b
+// with ancestors a_1 .. a_{t-1} (a_{t-1} = p, its parent) and P(a) the
+// product of the gates on the path from the root to record a:
 //
-//   D1  = S0 . X^T      S0 k_b and S0 q_b for the tile's 64 vectors
-//                       X = [k_0..k_31; q_0..q_31].  The S0 operand image is
-//                       read once per CTA and used by every beam of the tile
-//                       (abstract: "reuses the shared state across beams");
-//                       fp32 S0 is split once, when the prompt state is
-//                       installed, into two or three bf16 terms.
-//   Dkq = X . K^T       gives k_b . q_b.
-//   D2  = X . KA^T      k_a . x for every vector x and every distinct
-//                       ancestor a of the tile (KA: their keys).
-//   D1 += Delta'^T . C  the projection replay (review, Summary: records
-//                       replayed "in vector form without ever materializing a
-//                       per-beam matrix").  With P(a) the product of the
-//                       gates on the path from the root to record a (kept in
-//                       the record store), the weight of record a in the
-//                       replay of a beam whose parent is p is P(p) / P(a), so
-//                         S_{t-1} x = P(p) [ S0 x + sum_a (delta_a / P(a)) (k_a . x) ]
-//                       over the beam's ancestors a.  Delta' holds
-//                       delta_a / P(a); C[x][a] is k_a . x where a is an
-//                       ancestor of x's beam and 0 elsewhere.  Delta' and C
-//                       are split into fp16 hi + lo terms; the passes hi.hi,
-//                       hi.lo and lo.hi keep fp32-level accuracy.
+//   S_{t-1} x = P(p) S0 x + sum_j delta_{a_j} w_j (k_{a_j} . x),
+//   w_j = alpha_{a_{j+1}} ... alpha_{a_{t-1}}   (w = 1 for the parent),
 //
-// The epilogue (TMEM lane i = output element i) forms u_x = P(p) D1_x,
-// delta_b = beta_b (v_b - alpha_b u_k), o_b = alpha_b u_q + delta_b (k_b . q_b),
-// and appends the record (alpha_b, delta_b, k_b) with P(b) = P(p) alpha_b.
+// for x = k_b and x = q_b (review, Summary: records replayed "in vector form
+// without ever materializing a per-beam matrix").  Then
+// delta_b = beta_b (v_b - alpha_b S_{t-1} k_b) and
+// o_b = alpha_b S_{t-1} q_b + delta_b (k_b . q_b), and the record
+// (alpha_b, delta_b, k_b) is appended.
 //
-// The ancestry (abstract: "lightweight ancestry index ... without moving or
-// copying existing records"): beam b with parent p, grandparent g = the
-// parent of p at step t-1, has the ancestor row [row of g at depth t-2, g, p].
-// The kernel signals its dependents only after its own griddepcontrol.wait,
-// so when step t starts, step t-2 has completed: before its wait, step t
-// reads only inputs (S0 image, q, k, v, g, beta, parents of steps t and t-1)
-// and what steps up to t-2 wrote (ancestor rows of depth t-2).  There it
-// stages X, runs D1 and Dkq, forms every beam's ancestor row and finds the
-// tile's distinct ancestors with warp-wide matches (parents first, then one
-// warp per depth).  After the wait one round of loads stages all the distinct
-// ancestors' records (keys, deltas, P) once per CTA.  Every global write
-// happens after the wait, so a step never overwrites records that the step
-// before it may still be reading.
+//   D1 = S0 . X^T   tensor cores, fp32 accumulators in TMEM, for the tile's
+//                   64 vectors X = [k_0..k_31; q_0..q_31].  The S0 operand
+//                   image is read once per CTA and serves every beam of the
+//                   tile (abstract: "reuses the shared state across beams");
+//                   fp32 S0 is split once, when the prompt state is
+//                   installed, into two or three bf16 terms.
+//   D2 = KA . X^T   tensor cores: k_a . x for every distinct ancestor a of
+//                   the tile (KA: their keys).
+//   replay         fp32 FMAs, one thread per (beam, eighth of the elements).
+//
+// Only the deltas are outputs of earlier steps; ancestors (from the parents
+// of every step), their keys and their gates are inputs.  So each kernel
+// lets its dependent launch start at once, and before its
+// griddepcontrol.wait it reads inputs only: the callers' arrays of the
+// earlier steps under ONELA_FLAG_PDL, the record store otherwise (then the
+// earlier steps have completed).  It computes D1, the ancestry (abstract:
+// "lightweight ancestry index ... without moving or copying existing
+// records"), D2 and every weight, and writes the depth-t entries that need
+// no delta (alpha, k, the ancestry row).  After the wait it stages the
+// distinct ancestors' deltas with one round of bulk copies, replays, and
+// writes o and delta.  No kernel reads a depth-t entry before step t has
+// completed, so the early writes race with nothing.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cudaTypedefs.h>
@@ -61,57 +52,72 @@ constexpr int kThreads = 256;       // 8 warps
 constexpr int kBT = 32;             // beams per CTA
 constexpr int kN = 2 * kBT;         // vectors: k rows 0..31, q rows 32..63
 constexpr int kM = 128;             // MMA M
-constexpr int kBlk = 64;            // distinct ancestors per staging block
-constexpr int kTmemCols = 256;      // D1 [0,64), D2 [64,128), Dkq [128,160)
+constexpr int kBlk = 128;           // ancestors per D2 block (the MMA's M)
+constexpr int kDRows = 128;         // ancestor deltas per staging round after the wait
+constexpr int kTmemCols = 128;      // D1 [0,64), D2 [64,128)
 constexpr int kMaxT = 16;           // deepest decode the kernel serves
 constexpr int kMaxW = 1024;         // widest beam set the kernel serves
-constexpr int kSliceMax = 4096;     // ancestor-row slice copied to shared memory when
-                                    // W_max * T_max fits (ints); otherwise rows are gathered
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far beyond any legal wait
 constexpr int32_t kErrTimeout = 2;
 
 struct Layout {
-  uint32_t x;                        // X [NK][128 rows][128 B]: k, q, k, q
-  uint32_t a;                        // S0 image, then the block operands
-  uint32_t ka, dhi, dlo, chi, clo;   // block operands inside region a
-  uint32_t book;                     // barriers and bookkeeping
+  uint32_t x;     // X [NK][64 rows][128 B]: k rows, then q rows
+  uint32_t v;     // v [NK][32 rows][128 B]
+  uint32_t a;     // region A: the S0 image; then KA and D1^T; then the deltas
+  uint32_t ka;    // keys of a D2 block [NK][128 rows][128 B]
+  uint32_t d1;    // D1^T [64 vectors][d_v] fp32
+  uint32_t dst;   // ancestor deltas [kDRows][d_v] fp32
+  uint32_t book;  // barriers and bookkeeping
   uint32_t total;
 };
 
-__host__ __device__ inline bool use_slice(int W_max, int TM) { return W_max * TM <= kSliceMax; }
+// Shared-memory ints of the per-depth counts, rounded to whole 16-byte pieces.
+__host__ __device__ inline int cnt_ints(int TM) { return (TM + 7) & ~3; }
 
-__host__ __device__ inline Layout layout(int nk, int planes, int TM, int W_max) {
+__host__ __device__ inline Layout layout(int nk, int planes, int TM, int hist_cap) {
   Layout L;
   L.x = 0;
-  L.a = (uint32_t)nk * 16384u;
-  L.ka = L.a;                                // [NK][64 rows][128 B]
-  L.dhi = L.ka + (uint32_t)nk * 8192u;       // [2 M-atoms][8 groups][8 rows][128 B]
-  L.dlo = L.dhi + 16384u;
-  L.chi = L.dlo + 16384u;                    // [64 rows][128 B]
-  L.clo = L.chi + 8192u;
-  const uint32_t post_end = L.clo + 8192u;
-  const uint32_t pre_end = L.a + (uint32_t)planes * nk * 16384u;
-  L.book = post_end > pre_end ? post_end : pre_end;
-  // 64 B barriers/counters; 5 per-beam scalars; chain, slot [32][TM];
-  // list [32 * TM]; per-depth counts [TM]; the previous step's parents
-  // [W_max]; the ancestor-row slice of depth t-2 [W_max][TM] if it fits.
-  L.total = L.book + 64u + 5u * kBT * 4u + 3u * kBT * TM * 4u + (uint32_t)(TM + 4) * 4u + (uint32_t)W_max * 4u +
-            (use_slice(W_max, TM) ? (uint32_t)W_max * TM * 4u : 0u) + 16u;
+  L.v = (uint32_t)nk * 8192u;
+  L.a = (uint32_t)nk * 12288u;
+  L.ka = L.a;
+  L.d1 = L.a + (uint32_t)nk * 16384u;
+  L.dst = L.a;
+  const uint32_t s0 = (uint32_t)planes * nk * 16384u, ops = (uint32_t)nk * 32768u;
+  L.book = L.a + (s0 > ops ? s0 : ops);
+  // 64 B barriers/counters; 5 per-beam scalars; per (beam, depth) the replay
+  // coefficients (float4), the chain, slot, slot-list ints and weights; per-depth
+  // counts; the parents of steps 2..t-1.
+  L.total = L.book + 64u + 5u * kBT * 4u + (uint32_t)kBT * TM * 16u + 4u * kBT * TM * 4u +
+            (uint32_t)cnt_ints(TM) * 4u + (uint32_t)((hist_cap + 3) & ~3) * 4u + 16u;
   return L;
 }
 
-__device__ __forceinline__ void split_f16(float x, __half &hi, __half &lo) {
-  hi = __float2half_rn(x);
-  lo = __float2half_rn(x - __half2float(hi));
+// Copies n ints from global src to shared dst with cp.async, by the 32 lanes
+// of one warp: 16-byte pieces when both ends allow it, single ints otherwise.
+__device__ __forceinline__ void copy_ints_warp(int *dst, const int32_t *src, int n, int lane) {
+  int done = 0;
+  if (((ptx::smem_u32(dst) | (uint32_t)reinterpret_cast<uintptr_t>(src)) & 15u) == 0) {
+    done = n & ~3;
+    for (int e = lane * 4; e < done; e += 128) ptx::cp_async16(dst + e, src + e, 16u);
+  }
+  for (int e = done + lane; e < n; e += 32) ptx::cp_async4(dst + e, src + e);
+}
+
+// Four consecutive bf16 elements at p (8-byte aligned) as floats.
+__device__ __forceinline__ float4 bf16x4(const uint8_t *p) {
+  const uint2 u = *reinterpret_cast<const uint2 *>(p);
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+  return make_float4(a.x, a.y, b.x, b.y);
 }
 
 template <int DK>
 __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_constant__ StepParams p) {
-  constexpr int NK = DK / 64;  // 128-byte K atoms per key row
+  constexpr int NK = DK / 64;        // 128-byte K atoms per key row
   constexpr int DV = DK;
-  constexpr int C4 = DV / 4;   // float4 chunks per delta row
-  constexpr int XA = 2 * kN * 128;  // bytes of one K atom of X (128 rows)
-  constexpr int NF = kBlk * C4 / kThreads;  // delta float4 chunks per thread per block
+  constexpr uint32_t XA = kN * 128;  // bytes of one K atom of X (64 rows)
+  constexpr uint32_t VA = kBT * 128; // bytes of one K atom of v (32 rows)
+  constexpr int NU = DV / 32;        // 4-element groups per thread, beam-major phase
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = ptx::smem_u32(smem_raw);
   uint8_t *base = smem_raw + ((1024u - (raw_u32 & 1023u)) & 1023u);
@@ -121,82 +127,70 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
   const int b0 = tile * kBT;
   const int nb = min(kBT, p.W - b0);
   const int H = p.H, t = p.t, TM = p.T_max, P = p.s0_planes;
-  const int nanc = t - 1;
+  const int nanc = t - 1;   // ancestors per beam (depths 1..t-1)
   const int jp = nanc - 1;  // depth index of the parents (depth t-1)
-  const bool slice = use_slice(p.W_max, TM);
+  const bool hin = p.hist_inputs != 0;
 
-  const Layout L = layout(NK, P, TM, p.W_max);
+  const Layout L = layout(NK, P, TM, p.hist_cap);
   uint8_t *s_x = base + L.x;
+  const uint8_t *s_v = base + L.v;
+  float *s_d1 = reinterpret_cast<float *>(base + L.d1);
+  const float *s_dst = reinterpret_cast<const float *>(base + L.dst);
   uint64_t *bar_s0 = reinterpret_cast<uint64_t *>(base + L.book);
-  uint64_t *bar1 = bar_s0 + 1, *bar2 = bar_s0 + 2, *bar3 = bar_s0 + 3;
+  uint64_t *bar1 = bar_s0 + 1, *bar2 = bar_s0 + 2, *bar_d = bar_s0 + 3;
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bar_s0 + 4);
   int *s_U1 = reinterpret_cast<int *>(s_tmem + 1);
   int *s_par = reinterpret_cast<int *>(base + L.book + 64);
   float *s_alpha = reinterpret_cast<float *>(s_par + kBT);
   float *s_beta = s_alpha + kBT;
-  float *s_Gp = s_beta + kBT;  // P(parent): the beam's gate product so far
-  float *s_kq = s_Gp + kBT;
-  int *s_chain = reinterpret_cast<int *>(s_kq + kBT);  // [32][TM] ancestor beam by depth
-  int *s_slot = s_chain + kBT * TM;                     // [32][TM] ancestor slot by depth
-  int *s_list = s_slot + kBT * TM;                      // slot -> (beam << 5 | depth-1)
-  int *s_cnt = s_list + kBT * TM;                       // distinct ancestors per depth [TM + 4]
-  int *s_pp = s_cnt + TM + 4;                           // parents of step t-1 [W_max]
-  int *s_slice = s_pp + p.W_max;                        // ancestor rows of depth t-2 [W_max][TM]
+  float *s_Gp = s_beta + kBT;  // P(parent)
+  float *s_spare = s_Gp + kBT;
+  // [32][TM]: (w k_a . k_b, w k_a . q_b, slot of a) for the ancestor a of
+  // beam b at each depth.
+  float4 *s_c = reinterpret_cast<float4 *>(s_spare + kBT);
+  int *s_chain = reinterpret_cast<int *>(s_c + kBT * TM);  // [32][TM] ancestor beam by depth
+  int *s_slot = s_chain + kBT * TM;                         // [32][TM] ancestor slot by depth
+  int *s_list = s_slot + kBT * TM;                          // slot -> (beam << 5 | depth-1)
+  float *s_w = reinterpret_cast<float *>(s_list + kBT * TM);  // [32][TM] replay weight by depth
+  int *s_cnt = reinterpret_cast<int *>(s_w + kBT * TM);       // distinct ancestors per depth
+  int *s_hist = s_cnt + cnt_ints(TM);                          // parents of steps 2..t-1
 
-  const __nv_bfloat16 *v = static_cast<const __nv_bfloat16 *>(p.v);
   __nv_bfloat16 *rec_k = static_cast<__nv_bfloat16 *>(p.rec_k);
   const int64_t row0 = (int64_t)(r * p.W + b0) * H + h;  // (r, b0, h) row of [R][W][H][d]
 
-  // ------------------------------------------------------------ setup
+  // --------------------------------------- setup; every load issued at once
+  const uint32_t s0_bytes = (uint32_t)P * NK * 16384u;
   if (tid == 0) {
     ptx::mbar_init(bar_s0, 1);
     ptx::mbar_init(bar1, 1);
     ptx::mbar_init(bar2, 1);
-    ptx::mbar_init(bar3, 1);
+    ptx::mbar_init(bar_d, kDRows);
     ptx::mbar_fence_init();
-  }
-  if (warp == 0) {
-    ptx::tmem_alloc(s_tmem, kTmemCols);
-    ptx::tmem_relinquish();
-  }
-  ptx::tc_fence_before();
-  __syncthreads();
-  ptx::tc_fence_after();
-  const uint32_t tmem = *s_tmem;
-
-  // ------------------------------------------- before the wait
-  // Every load of this phase is issued up front: one round trip.
-  const uint32_t s0_bytes = (uint32_t)P * NK * 16384u;
-  if (tid == kThreads - 32) {
-    // S0 image (bulk copy) and X by TMA: rows 0..31 k_b, 32..63 q_b, then
-    // the same 64 rows again (so that all four TMEM lane quarters of D2 hold
-    // vectors).  Beams past W read as zeros.
-    ptx::mbar_arrive_expect_tx(bar_s0, s0_bytes + 2u * kN * 128u * NK);
+    // S0 image (bulk copy); k, q, v tiles by TMA, beams past W read as zeros.
+    ptx::mbar_arrive_expect_tx(bar_s0, s0_bytes + NK * (XA + VA));
     const uint8_t *src = static_cast<const uint8_t *>(p.S0img) + (size_t)(r * H + h) * s0_bytes;
     for (uint32_t off = 0; off < s0_bytes; off += 16384u)
       ptx::bulk_g2s(base + L.a + off, src + off, 16384u, bar_s0);
 #pragma unroll
-    for (int copy = 0; copy < 2; ++copy)
-#pragma unroll
-      for (int ka = 0; ka < NK; ++ka) {
-        uint8_t *dst = s_x + ka * XA + copy * (kN * 128);
-        ptx::tma_load_4d(dst, &p.tm_k, ka * 64, h, b0, r, bar_s0);
-        ptx::tma_load_4d(dst + kBT * 128, &p.tm_q, ka * 64, h, b0, r, bar_s0);
-      }
-  }
-  // The previous step's parents (an input of step t-1) and the ancestor rows
-  // of depth t-2 (written by step t-2, which has completed).
-  if (nanc >= 2)
-    for (int e = tid; e < p.W_prev; e += kThreads) ptx::cp_async4(s_pp + e, p.prev_parents + r * p.prev_stride + e);
-  if (nanc >= 3 && slice) {
-    const int w2 = nanc - 2;  // entries per row
-    const int32_t *src = p.anc + anc_row(p, nanc - 1, r, 0);
-    for (int e = tid; e < p.W_prev2 * w2; e += kThreads) {
-      const int row = e / w2, j = e - row * w2;
-      ptx::cp_async4(s_slice + e, src + (int64_t)row * TM + j);
+    for (int ka = 0; ka < NK; ++ka) {
+      ptx::tma_load_4d(s_x + ka * XA, &p.tm_k, ka * 64, h, b0, r, bar_s0);
+      ptx::tma_load_4d(s_x + ka * XA + kBT * 128, &p.tm_q, ka * 64, h, b0, r, bar_s0);
+      ptx::tma_load_4d(base + L.v + ka * VA, &p.tm_v, ka * 64, h, b0, r, bar_s0);
     }
   }
+  if (warp == 3) {
+    ptx::tmem_alloc(s_tmem, kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  // The parents of steps 2..t-1 for this request, back to back, each array
+  // starting on a 16-byte boundary; warp w copies steps w + 2, w + 10.
+  if (p.hist_cap > 0)
+#pragma unroll 1
+    for (int j = warp + 2; j < t; j += kThreads / 32)
+      copy_ints_warp(s_hist + p.hoff[j], p.hpar[j] + (int64_t)r * p.hpar_rs[j], p.hW[j], lane);
   ptx::cp_async_commit();
+  // Before its wait this kernel reads inputs only, so the next step may start.
+  ptx::pdl_launch_dependents();
   int par = -1;
   float g_alpha = 0.f, g_beta = 0.f;
   if (warp == 1 && lane < nb) {
@@ -205,25 +199,15 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
     g_alpha = p.g[si];
     g_beta = p.beta[si];
   }
-  // Epilogue mapping: warp w serves TMEM lanes 32*(w%4).. (output elements)
-  // and beams 16*(w/4)..+15; v is loaded now, used at the end.
-  const int ei = (warp & 3) * 32 + lane;
-  const int half = warp >> 2;
-  __nv_bfloat16 vreg[16];
-#pragma unroll
-  for (int m = 0; m < 16; ++m) {
-    const int b = half * 16 + m;
-    vreg[m] = (b < nb && ei < DV) ? v[(row0 + (int64_t)b * H) * DV + ei] : __float2bfloat16(0.f);
-  }
   ptx::cp_async_wait_all();
-  ptx::fence_proxy_async_smem();
+  ptx::tc_fence_before();
   __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *s_tmem;
 
   bool ok = true;
   const uint32_t x_u32 = ptx::smem_u32(s_x), a_u32 = ptx::smem_u32(base + L.a);
   const uint32_t ka_u32 = ptx::smem_u32(base + L.ka);
-  const uint32_t dhi_u32 = ptx::smem_u32(base + L.dhi), dlo_u32 = ptx::smem_u32(base + L.dlo);
-  const uint32_t chi_u32 = ptx::smem_u32(base + L.chi), clo_u32 = ptx::smem_u32(base + L.clo);
   if (tid == 0) {
     ok = ptx::mbar_wait(bar_s0, 0, kWaitLimitNs);
     ptx::tc_fence_after();
@@ -239,29 +223,32 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
           ptx::mma_bf16(tmem, ad, bd, idesc1, acc);
           acc = 1;
         }
-    // Dkq = X . K^T: row 32 + b, column b is k_b . q_b.
-    constexpr uint32_t idesc_kq = ptx::idesc_bf16_f32(kM, kBT);
-#pragma unroll
-    for (int ka = 0; ka < NK; ++ka)
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t ad = ptx::desc_k128(x_u32 + ka * XA + kk * 32);
-        ptx::mma_bf16(tmem + 128, ad, ad, idesc_kq, (ka | kk) != 0);
-      }
     ptx::mma_commit(bar1);
   }
   if (warp == 1) {
-    // Each beam's ancestor row: [row of g at depth t-2, g, p].
+    // Beam b's ancestors: a[j] at depth j + 1, a[t-2] = its parent; a[j] is
+    // the parent, at step j + 2, of a[j + 1].
     const int b = lane;
-    if (b < nb) {
-      if (par < 0 || par >= p.W_prev) {
-        *reinterpret_cast<volatile int32_t *>(p.err) = kErrParent;
-        par = 0;
+    if (b < nb && nanc >= 1 && (par < 0 || par >= p.W_prev)) {
+      *reinterpret_cast<volatile int32_t *>(p.err) = kErrParent;
+      par = 0;
+    }
+    if (b >= nb) par = 0;
+    const float alpha_b = b < nb ? expf(g_alpha) : 0.f;
+    s_par[b] = par;
+    s_alpha[b] = alpha_b;
+    s_beta[b] = g_beta;
+    if (b < nb && nanc >= 1) {
+      int a = par;
+      s_chain[b * TM + jp] = a;
+#pragma unroll 1
+      for (int j = jp - 1; j >= 0; --j) {
+        int pa = p.hist_cap > 0 ? s_hist[p.hoff[j + 2] + a] : p.hpar[j + 2][(int64_t)r * p.hpar_rs[j + 2] + a];
+        if (pa < 0 || pa >= p.hW[j + 1]) pa = 0;  // reported by step j + 2
+        a = pa;
+        s_chain[b * TM + j] = a;
       }
     }
-    s_par[b] = b < nb ? par : 0;
-    s_alpha[b] = b < nb ? expf(g_alpha) : 0.f;
-    s_beta[b] = g_beta;
     if (nanc >= 1) {
       // Distinct parents take slots 0..U1-1.
       const unsigned same = __match_any_sync(0xffffffffu, par);
@@ -272,38 +259,53 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
       if (lead) s_list[my] = (par << 5) | jp;
       const int slot = __shfl_sync(0xffffffffu, my, leader);
       if (lane == 0) *s_U1 = __popc(leaders);
-      if (b < nb) {
-        s_slot[b * TM + jp] = slot;
-        s_chain[b * TM + jp] = par;
-        if (nanc >= 2) {
-          int gp = s_pp[par];
-          if (gp < 0 || gp >= p.W_prev2) gp = 0;  // already reported by step t-1
-          s_chain[b * TM + nanc - 2] = gp;
-          if (nanc >= 3) {
-            if (slice) {
-              for (int j = 0; j < nanc - 2; ++j) s_chain[b * TM + j] = s_slice[gp * (nanc - 2) + j];
-            } else {
-              const int32_t *grow = p.anc + anc_row(p, nanc - 1, r, gp);
-              int tmp[kMaxT - 2];
-#pragma unroll
-              for (int j = 0; j < kMaxT - 2; ++j)
-                if (j < nanc - 2) tmp[j] = grow[j];
-#pragma unroll
-              for (int j = 0; j < kMaxT - 2; ++j)
-                if (j < nanc - 2) s_chain[b * TM + j] = tmp[j];
-            }
-          }
-        }
-      }
+      if (b < nb) s_slot[b * TM + jp] = slot;
     } else if (lane == 0) {
       *s_U1 = 0;
     }
+    // Entries of depth t that need no delta.
+    if (b < nb) {
+      const int gb = b0 + b;
+      p.rec_alpha[rec_row(p, t, r, h, gb)] = alpha_b;
+      if (h == 0) {
+        int32_t *row = p.anc + anc_row(p, t, r, gb);
+#pragma unroll 1
+        for (int j = 0; j < nanc; ++j) row[j] = s_chain[b * TM + j];
+        p.par_store[((int64_t)(t - 1) * p.R + r) * p.W_max + gb] = par;
+      }
+    }
   }
   __syncthreads();
+  if (warp == 0) {
+    // The gates along beam b's chain give the replay weights (products of the
+    // later gates) and P(p).  The gates land in s_w first (one round trip);
+    // each entry is then overwritten by the weight of its depth.
+    const int b = lane;
+    if (b < nb) {
+#pragma unroll 1
+      for (int j = 0; j <= jp; ++j) {
+        const int a = s_chain[b * TM + j];
+        ptx::cp_async4(s_w + b * TM + j, hin ? p.hg[j + 1] + ((int64_t)r * p.hW[j + 1] + a) * H + h
+                                             : p.rec_alpha + rec_row(p, j + 1, r, h, a));
+      }
+    }
+    ptx::cp_async_commit();
+    ptx::cp_async_wait_all();
+    float w = 1.f;
+    if (b < nb) {
+#pragma unroll 1
+      for (int j = jp; j >= 0; --j) {
+        const float gj = s_w[b * TM + j];
+        s_w[b * TM + j] = w;
+        w *= hin ? expf(gj) : gj;
+      }
+    }
+    s_Gp[b] = w;  // P(p): all the gates on the path
+  }
   // Deeper ancestors (depths 1..t-2): one warp per depth (warps 1..7; warp 0
-  // issues the MMAs) finds the distinct ones; their slots follow the
+  // gathers the gates) finds the distinct ones; their slots follow the
   // parents', depth by depth.
-  for (int j = warp - 1; warp > 0 && j < nanc - 1; j += kThreads / 32 - 1) {
+  for (int j = warp - 1; warp > 0 && j < jp; j += kThreads / 32 - 1) {
     const int a = lane < nb ? s_chain[lane * TM + j] : -1;
     const unsigned same = __match_any_sync(0xffffffffu, a);
     const int leader = __ffs(same) - 1;
@@ -317,232 +319,222 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
   __syncthreads();
   const int U1 = *s_U1;
   int U = U1;
-  for (int j = 0; j < nanc - 1; ++j) U += s_cnt[j];
-  for (int j = warp - 1; warp > 0 && j < nanc - 1; j += kThreads / 32 - 1) {
+  for (int j = 0; j < jp; ++j) U += s_cnt[j];
+  for (int j = warp - 1; warp > 0 && j < jp; j += kThreads / 32 - 1) {
     int base_j = U1;
     for (int j2 = 0; j2 < j; ++j2) base_j += s_cnt[j2];
     if (lane < nb) {
       const int slot = base_j + s_slot[lane * TM + j];
       s_slot[lane * TM + j] = slot;
       s_list[slot] = (s_chain[lane * TM + j] << 5) | j;
+      // The slot is known now; the coefficients follow with the slot's block.
+      s_c[lane * TM + j] = make_float4(0.f, 0.f, __int_as_float(slot), 0.f);
     }
   }
-  __syncthreads();  // slots and the slot list complete
 
-  // ------------------------------- after the wait: step t-1's records
-  ptx::pdl_wait();
-  ptx::pdl_launch_dependents();
-  // Region A holds the S0 image until D1 is complete.
-  if (!ptx::mbar_wait(bar1, 0, kWaitLimitNs)) ok = false;
-
-  // Stage slots [lo, hi) of block blk: keys (cp.async) into KA; deltas / P(a)
-  // as fp16 hi + lo into the MN-major Delta' operand.  All loads in flight
-  // at once.
-  auto stage = [&](int blk, int lo, int hi) {
-    for (int e = tid; e < (hi - lo) * NK * 8; e += kThreads) {
-      const int s = lo + e / (NK * 8), cc = e % (NK * 8);
-      const int packed = s_list[s];
-      const int lr = s - blk * kBlk;
-      ptx::cp_async16(base + L.ka + (cc >> 3) * (kBlk * 128) + ptx::swz128(lr, cc & 7),
-                      rec_k + rec_row(p, (packed & 31) + 1, r, h, packed >> 5) * DK + cc * 8, 16u);
+  __syncthreads();  // slot list complete
+  // D1 is complete, so region A is free: the keys of the first D2 block go
+  // in flight now and land while the beam-major work below runs.  KA holds
+  // the keys of slots [lo, lo + nrows), K-major with the 128-byte swizzle.
+  auto stage_keys = [&](int lo, int nrows) {
+    constexpr int KPT = kBlk * NK * 8 / kThreads;  // 16-byte key pieces per thread
+    int kp[KPT];
+#pragma unroll
+    for (int u = 0; u < KPT; ++u) {
+      const int e = tid + u * kThreads;
+      kp[u] = e < nrows * NK * 8 ? s_list[lo + e / (NK * 8)] : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < KPT; ++u) {
+      const int e = tid + u * kThreads;
+      if (kp[u] >= 0) {
+        const int a = kp[u] >> 5, j = kp[u] & 31, cc = e % (NK * 8);
+        const __nv_bfloat16 *src =
+            hin ? static_cast<const __nv_bfloat16 *>(p.hk[j + 1]) + (((int64_t)r * p.hW[j + 1] + a) * H + h) * DK
+                : rec_k + rec_row(p, j + 1, r, h, a) * DK;
+        ptx::cp_async16(base + L.ka + (cc >> 3) * 16384 + ptx::swz128(e / (NK * 8), cc & 7), src + cc * 8, 16u);
+      }
     }
     ptx::cp_async_commit();
-    float4 val[NF];
-    float pa[NF];
-#pragma unroll
-    for (int u = 0; u < NF; ++u) {
-      const int e = tid + u * kThreads;
-      val[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-      pa[u] = 1.f;
-      if (e < (hi - lo) * C4) {
-        const int packed = s_list[lo + e / C4];
-        const int64_t rr = rec_row(p, (packed & 31) + 1, r, h, packed >> 5);
-        val[u] = __ldcg(reinterpret_cast<const float4 *>(p.rec_delta + rr * DV) + e % C4);
-        pa[u] = __ldcg(p.rec_P + rr);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < NF; ++u) {
-      const int e = tid + u * kThreads;
-      if (e < (hi - lo) * C4) {
-        const int lr = lo + e / C4 - blk * kBlk;
-        const int i0 = (e % C4) * 4;
-        const uint32_t off = (uint32_t)(i0 >> 6) * 8192u + (uint32_t)(lr >> 3) * 1024u +
-                             (uint32_t)(lr & 7) * 128u + (uint32_t)((((i0 & 63) >> 3) ^ (lr & 7)) << 4) +
-                             (uint32_t)(i0 & 7) * 2u;
-        const float inv = 1.f / pa[u];
-        const float f[4] = {val[u].x * inv, val[u].y * inv, val[u].z * inv, val[u].w * inv};
-        __align__(8) __half hi4[4], lo4[4];
-#pragma unroll
-        for (int z = 0; z < 4; ++z) split_f16(f[z], hi4[z], lo4[z]);
-        *reinterpret_cast<uint2 *>(base + L.dhi + off) = *reinterpret_cast<const uint2 *>(hi4);
-        *reinterpret_cast<uint2 *>(base + L.dlo + off) = *reinterpret_cast<const uint2 *>(lo4);
-      }
-    }
   };
-  // P(parent): loaded now, consumed after the staging loads are issued.
-  float Gp = 1.f;
-  if (warp == 2 && lane < nb && nanc >= 1) Gp = __ldcg(p.rec_P + rec_row(p, nanc, r, h, s_par[lane]));
-  if (U > 0) stage(0, 0, min(U, kBlk));
-  // This step's outputs that need no arithmetic: records of depth t (alpha,
-  // P, k), the ancestor row and the parents of depth t.
-  if (warp == 2 && lane < nb) {
-    const int b = lane, gb = b0 + lane;
-    s_Gp[b] = Gp;
-    p.rec_alpha[rec_row(p, t, r, h, gb)] = s_alpha[b];
-    p.rec_P[rec_row(p, t, r, h, gb)] = Gp * s_alpha[b];
-    if (h == 0) {
-      int32_t *row = p.anc + anc_row(p, t, r, gb);
-      for (int j = 0; j < nanc; ++j) row[j] = s_chain[b * TM + j];
-      p.par_store[((int64_t)(t - 1) * p.R + r) * p.W_max + gb] = s_par[b];
-    }
+  if (!ptx::mbar_wait(bar1, 0, kWaitLimitNs)) ok = false;
+  ptx::tc_fence_after();
+  if (U > 0) stage_keys(0, min(U, kBlk));
+
+  // Beam-major phase: thread (bb, l) owns elements 32 u + 4 l + z (z < 4) of
+  // beam bb.  k_b . q_b, v, and the key records of depth t, from X and v.
+  const int bb = tid >> 3, l = tid & 7;
+  if (!ptx::mbar_wait(bar_s0, 0, kWaitLimitNs)) ok = false;
+  float kq = 0.f;
+  float4 vf[NU];
+#pragma unroll
+  for (int u = 0; u < NU; ++u) {
+    const uint32_t off = (uint32_t)(u >> 1) * XA + (uint32_t)(l & 1) * 8u;
+    const int c = 4 * (u & 1) + (l >> 1);
+    const float4 kf = bf16x4(s_x + off + ptx::swz128(bb, c));
+    const float4 qf = bf16x4(s_x + off + ptx::swz128(kBT + bb, c));
+    kq = fmaf(kf.x, qf.x, kq);
+    kq = fmaf(kf.y, qf.y, kq);
+    kq = fmaf(kf.z, qf.z, kq);
+    kq = fmaf(kf.w, qf.w, kq);
+    vf[u] = bf16x4(s_v + (u >> 1) * VA + ptx::swz128(bb, c) + (l & 1) * 8);
   }
-  if (!ptx::mbar_wait(bar_s0, 0, kWaitLimitNs)) ok = false;  // X visible to this thread
+  kq += __shfl_xor_sync(0xffffffffu, kq, 4);
+  kq += __shfl_xor_sync(0xffffffffu, kq, 2);
+  kq += __shfl_xor_sync(0xffffffffu, kq, 1);
   for (int e = tid; e < kBT * NK * 8; e += kThreads) {
     const int n = e / (NK * 8), cc = e - n * (NK * 8);
     if (n < nb)
       reinterpret_cast<uint4 *>(rec_k + rec_row(p, t, r, h, b0 + n) * DK)[cc] =
           *reinterpret_cast<const uint4 *>(s_x + (cc >> 3) * XA + ptx::swz128(n, cc & 7));
   }
-  if (warp == 1) {
-    // k_b . q_b from Dkq (TMEM lanes 32..63 belong to warp 1).
-    ptx::tc_fence_after();
-    float d[32];
-    ptx::tmem_ld32(tmem + (32u << 16) + 128, d);
-    ptx::tmem_ld_wait();
-    float kq = 0.f;
-#pragma unroll
-    for (int z = 0; z < 32; ++z)
-      if (z == lane) kq = d[z];
-    s_kq[lane] = kq;
-  }
-  const int nblk = (U + kBlk - 1) / kBlk;
 
-  for (int blk = 0; blk < nblk; ++blk) {
-    const int lo = blk * kBlk, hi = min(U, lo + kBlk);
+  // D1^T to shared memory: warp w reads TMEM lanes 32 (w % 4).. (elements)
+  // and the k (w < 4) or q columns.
+  const int ei = (warp & 3) * 32 + lane, half = warp >> 2;
+  const uint32_t lb = (uint32_t)((warp & 3) * 32) << 16;
+  if ((warp & 3) * 32 < DV) {
+    float d[32];
+    ptx::tmem_ld32(tmem + lb + half * 32, d);
+    ptx::tmem_ld_wait();
+#pragma unroll
+    for (int n = 0; n < 32; ++n) s_d1[(half * 32 + n) * DV + ei] = d[n];
+  }
+  // (made visible by the barrier before the first D2 block)
+
+  // Keys of the tile's distinct ancestors, D2 = KA . X^T, and the weighted
+  // coefficients, block by block.
+  for (int lo = 0, blk = 0; lo < U; lo += kBlk, ++blk) {
+    const int hi = min(U, lo + kBlk);
     const int nrows = hi - lo;
-    const int kpad = (nrows + 15) & ~15;  // slots the MMAs read (multiple of 16)
     if (blk > 0) {
-      if (!ptx::mbar_wait(bar3, (blk - 1) & 1, kWaitLimitNs)) ok = false;
-      stage(blk, lo, hi);
-    }
-    // Slots past the block's last ancestor but inside the MMA K range hold
-    // zero deltas.
-    for (int e = tid; e < (kpad - nrows) * 2 * 8; e += kThreads) {
-      const int lr = nrows + e / 16, rem = e % 16, ma = rem >> 3, c = rem & 7;
-      const uint32_t off = (uint32_t)ma * 8192u + (uint32_t)(lr >> 3) * 1024u + ptx::swz128(lr & 7, c);
-      *reinterpret_cast<uint4 *>(base + L.dhi + off) = make_uint4(0u, 0u, 0u, 0u);
-      *reinterpret_cast<uint4 *>(base + L.dlo + off) = make_uint4(0u, 0u, 0u, 0u);
+      __syncthreads();  // the previous block's keys are consumed
+      stage_keys(lo, nrows);
     }
     ptx::cp_async_wait_all();
     ptx::fence_proxy_async_smem();
     __syncthreads();
     if (tid == 0) {
       ptx::tc_fence_after();
-      const uint32_t idesc2 = ptx::idesc_bf16_f32(kM, kpad);
+      constexpr uint32_t idesc2 = ptx::idesc_bf16_f32(kM, kN);
 #pragma unroll
       for (int ka = 0; ka < NK; ++ka)
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t ad = ptx::desc_k128(x_u32 + ka * XA + kk * 32);
-          const uint64_t bd = ptx::desc_k128(ka_u32 + ka * (kBlk * 128) + kk * 32);
+          const uint64_t ad = ptx::desc_k128(ka_u32 + ka * 16384 + kk * 32);
+          const uint64_t bd = ptx::desc_k128(x_u32 + ka * XA + kk * 32);
           ptx::mma_bf16(tmem + 64, ad, bd, idesc2, (ka | kk) != 0);
         }
       ptx::mma_commit(bar2);
     }
-    // C build: D2 row n (TMEM lane n) is vector n % 64; warp w takes the
-    // lane quarter w % 4 and the 16-slot column group (w % 4) / 2 + 2 (w / 4).
-    // C[vec][a] = D2[vec][a] where a is an ancestor of vec's beam, else 0,
-    // stored as fp16 hi + lo, K-major (row vec, K = slot).
-    if (!ptx::mbar_wait(bar2, blk & 1, kWaitLimitNs)) ok = false;
-    ptx::tc_fence_after();
+    // D2 row (TMEM lane) = slot lo + row, column = vector.  Warp w reads rows
+    // 32 (w % 4).. for the beams of half w / 4.  The slot's thread writes the
+    // coefficients of every beam that replays it.
     {
-      const int qq = warp & 3;
-      const int g = (qq >> 1) + 2 * (warp >> 2);
-      if (g * 16 < kpad) {
-        const int vec = (qq * 32 + lane) & (kN - 1);
-        const int b = vec & (kBT - 1);
-        float d[16];
-        ptx::tmem_ld16(tmem + ((uint32_t)(qq * 32) << 16) + 64 + g * 16, d);
-        ptx::tmem_ld_wait();
-        uint32_t mask = 0u;
-        if (b < nb)
-          for (int j = 0; j < nanc; ++j) {
-            const int sl = s_slot[b * TM + j] - lo - g * 16;
-            if (sl >= 0 && sl < 16) mask |= 1u << sl;
+      const int s = lo + (warp & 3) * 32 + lane;
+      const bool act = s < hi;
+      const int js = act ? (s_list[s] & 31) : 0;
+      int sl[16];
+#pragma unroll
+      for (int m = 0; m < 16; ++m) sl[m] = s_slot[(half * 16 + m) * TM + js];
+      if (!ptx::mbar_wait(bar2, blk & 1, kWaitLimitNs)) ok = false;
+      ptx::tc_fence_after();
+      float dk[16], dq[16];
+      ptx::tmem_ld16(tmem + lb + 64 + half * 16, dk);
+      ptx::tmem_ld16(tmem + lb + 64 + kBT + half * 16, dq);
+      ptx::tmem_ld_wait();
+      if (act) {
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+          const int b = half * 16 + m;
+          if (b < nb && sl[m] == s) {
+            const float w = s_w[b * TM + js];
+            s_c[b * TM + js] = make_float4(dk[m] * w, dq[m] * w, __int_as_float(s), 0.f);
           }
-        __align__(16) __half h16[16], l16[16];
-#pragma unroll
-        for (int z = 0; z < 16; ++z) split_f16(((mask >> z) & 1u) ? d[z] : 0.f, h16[z], l16[z]);
-#pragma unroll
-        for (int c2 = 0; c2 < 2; ++c2) {
-          const uint32_t off = ptx::swz128(vec, g * 2 + c2);
-          *reinterpret_cast<uint4 *>(base + L.chi + off) = reinterpret_cast<const uint4 *>(h16)[c2];
-          *reinterpret_cast<uint4 *>(base + L.clo + off) = reinterpret_cast<const uint4 *>(l16)[c2];
         }
       }
     }
-    ptx::fence_proxy_async_smem();
     ptx::tc_fence_before();
     __syncthreads();
-    if (tid == 0) {
-      ptx::tc_fence_after();
-      constexpr uint32_t idesc3 = ptx::idesc_f16_amn_f32(kM, kN);
-      const uint32_t dA[3] = {dhi_u32, dhi_u32, dlo_u32};
-      const uint32_t cB[3] = {chi_u32, clo_u32, chi_u32};
+  }
+
+  if (U == 0) __syncthreads();  // D1^T visible (otherwise the block loop's barriers did it)
+  // u = P(p) D1 + (replayed terms, after the wait).
+  float acc_k[4 * NU], acc_q[4 * NU];
+  const float Gp = s_Gp[bb], alpha = s_alpha[bb], beta = s_beta[bb];
 #pragma unroll
-      for (int term = 0; term < 3; ++term)
-        for (int ks = 0; ks < kpad / 16; ++ks) {
-          const uint64_t ad = ptx::desc_mn128(dA[term] + ks * 2048, 8192u, 1024u);
-          const uint64_t bd = ptx::desc_k128(cB[term] + ks * 32);
-          ptx::mma_bf16(tmem, ad, bd, idesc3, 1u);
+  for (int u = 0; u < NU; ++u) {
+    const float4 dk = reinterpret_cast<const float4 *>(s_d1 + bb * DV)[8 * u + l];
+    const float4 dq = reinterpret_cast<const float4 *>(s_d1 + (kBT + bb) * DV)[8 * u + l];
+    acc_k[4 * u + 0] = Gp * dk.x, acc_k[4 * u + 1] = Gp * dk.y, acc_k[4 * u + 2] = Gp * dk.z, acc_k[4 * u + 3] = Gp * dk.w;
+    acc_q[4 * u + 0] = Gp * dq.x, acc_q[4 * u + 1] = Gp * dq.y, acc_q[4 * u + 2] = Gp * dq.z, acc_q[4 * u + 3] = Gp * dq.w;
+  }
+  ptx::tc_fence_before();
+  __syncthreads();  // D1^T consumed, TMEM reads done
+  if (warp == 3) ptx::tmem_dealloc(tmem, kTmemCols);
+
+  // ------------------------------- after the wait: the ancestors' deltas
+  ptx::pdl_wait();
+  for (int lo = 0, rnd = 0; lo < U; lo += kDRows, ++rnd) {
+    const int hi = min(U, lo + kDRows);
+    const int nrows = hi - lo;
+    if (rnd > 0) __syncthreads();  // the previous round's deltas are consumed
+    if (tid < kDRows) {
+      const int s = lo + tid;
+      if (s < hi) {
+        const int packed = s_list[s];
+        ptx::fence_proxy_async_smem();
+        ptx::mbar_arrive_expect_tx(bar_d, DV * 4);
+        ptx::bulk_g2s(base + L.dst + tid * DV * 4,
+                      p.rec_delta + rec_row(p, (packed & 31) + 1, r, h, packed >> 5) * DV, DV * 4, bar_d);
+      } else {
+        ptx::mbar_arrive(bar_d);
+      }
+    }
+    if (!ptx::mbar_wait(bar_d, rnd & 1, kWaitLimitNs)) ok = false;
+    if (bb < nb) {
+      for (int j = 0; j < nanc; ++j) {
+        const float4 c = s_c[bb * TM + j];
+        const unsigned sl = (unsigned)(__float_as_int(c.z) - lo);
+        if (sl < (unsigned)nrows) {
+          const float4 *row = reinterpret_cast<const float4 *>(s_dst + sl * DV) + l;
+#pragma unroll
+          for (int u = 0; u < NU; ++u) {
+            const float4 d = row[8 * u];
+            acc_k[4 * u + 0] = fmaf(d.x, c.x, acc_k[4 * u + 0]);
+            acc_k[4 * u + 1] = fmaf(d.y, c.x, acc_k[4 * u + 1]);
+            acc_k[4 * u + 2] = fmaf(d.z, c.x, acc_k[4 * u + 2]);
+            acc_k[4 * u + 3] = fmaf(d.w, c.x, acc_k[4 * u + 3]);
+            acc_q[4 * u + 0] = fmaf(d.x, c.y, acc_q[4 * u + 0]);
+            acc_q[4 * u + 1] = fmaf(d.y, c.y, acc_q[4 * u + 1]);
+            acc_q[4 * u + 2] = fmaf(d.z, c.y, acc_q[4 * u + 2]);
+            acc_q[4 * u + 3] = fmaf(d.w, c.y, acc_q[4 * u + 3]);
+          }
         }
-      ptx::mma_commit(bar3);
+      }
     }
   }
 
   // --------------------------------------------------------- epilogue
-  if (nblk > 0 && !ptx::mbar_wait(bar3, (nblk - 1) & 1, kWaitLimitNs)) ok = false;
   if (!ok) *reinterpret_cast<volatile int32_t *>(p.err) = kErrTimeout;
-  __syncthreads();  // s_Gp and s_kq visible
-  ptx::tc_fence_after();
-  {
-    const uint32_t lb = (uint32_t)((warp & 3) * 32) << 16;
-    float uk[16], uq[16];
-    ptx::tmem_ld16(tmem + lb + half * 16, uk);
-    ptx::tmem_ld16(tmem + lb + kBT + half * 16, uq);
-    ptx::tmem_ld_wait();
-    if (ei < DV && ok) {
-      const float4 *G4 = reinterpret_cast<const float4 *>(s_Gp + half * 16);
-      const float4 *A4 = reinterpret_cast<const float4 *>(s_alpha + half * 16);
-      const float4 *B4 = reinterpret_cast<const float4 *>(s_beta + half * 16);
-      const float4 *K4 = reinterpret_cast<const float4 *>(s_kq + half * 16);
-      const int64_t ostride = (int64_t)H * DV;
-      float *op = p.o + (row0 + (int64_t)(half * 16) * H) * DV + ei;
-      float *dp = p.rec_delta + (rec_row(p, t, r, h, b0) + half * 16) * DV + ei;
+  if (bb < nb && ok) {
+    float4 *op = reinterpret_cast<float4 *>(p.o + (row0 + (int64_t)bb * H) * DV) + l;
+    float4 *dp = reinterpret_cast<float4 *>(p.rec_delta + rec_row(p, t, r, h, b0 + bb) * DV) + l;
 #pragma unroll
-      for (int m4 = 0; m4 < 4; ++m4) {
-        const float4 G = G4[m4], A = A4[m4], B = B4[m4], KQ = K4[m4];
-        const float Gv[4] = {G.x, G.y, G.z, G.w}, Av[4] = {A.x, A.y, A.z, A.w};
-        const float Bv[4] = {B.x, B.y, B.z, B.w}, Kv[4] = {KQ.x, KQ.y, KQ.z, KQ.w};
-#pragma unroll
-        for (int z = 0; z < 4; ++z) {
-          const int m = m4 * 4 + z;
-          if (half * 16 + m < nb) {
-            const float ag = Av[z] * Gv[z];  // alpha P(p)
-            const float delta = Bv[z] * fmaf(-ag, uk[m], __bfloat162float(vreg[m]));
-            op[m * ostride] = fmaf(ag, uq[m], delta * Kv[z]);
-            dp[m * DV] = delta;
-          }
-        }
-      }
+    for (int u = 0; u < NU; ++u) {
+      float4 d, o;
+      d.x = beta * fmaf(-alpha, acc_k[4 * u + 0], vf[u].x);
+      d.y = beta * fmaf(-alpha, acc_k[4 * u + 1], vf[u].y);
+      d.z = beta * fmaf(-alpha, acc_k[4 * u + 2], vf[u].z);
+      d.w = beta * fmaf(-alpha, acc_k[4 * u + 3], vf[u].w);
+      o.x = fmaf(alpha, acc_q[4 * u + 0], d.x * kq);
+      o.y = fmaf(alpha, acc_q[4 * u + 1], d.y * kq);
+      o.z = fmaf(alpha, acc_q[4 * u + 2], d.z * kq);
+      o.w = fmaf(alpha, acc_q[4 * u + 3], d.w * kq);
+      op[8 * u] = o;
+      dp[8 * u] = d;
     }
   }
-
-  // --------------------------------------------------------- teardown
-  ptx::tc_fence_before();
-  __syncthreads();
-  if (warp == 0) ptx::tmem_dealloc(tmem, kTmemCols);
 }
 
 __global__ void s0_image_kernel(const void *S0, uint4 *img, int R, int H, int dk, int dv, int s0_bf16,
@@ -612,9 +604,10 @@ bool encode_rows(CUtensorMap *m, const void *base, int d, int H, int W, int R) {
 template <int DK>
 cudaError_t launch_dk(const StepParams &p_in, bool pdl, cudaStream_t s) {
   StepParams p = p_in;
-  if (!encode_rows(&p.tm_k, p.k, DK, p.H, p.W, p.R) || !encode_rows(&p.tm_q, p.q, DK, p.H, p.W, p.R))
+  if (!encode_rows(&p.tm_k, p.k, DK, p.H, p.W, p.R) || !encode_rows(&p.tm_q, p.q, DK, p.H, p.W, p.R) ||
+      !encode_rows(&p.tm_v, p.v, DK, p.H, p.W, p.R))
     return cudaErrorInvalidValue;
-  const Layout L = layout(DK / 64, p.s0_planes, p.T_max, p.W_max);
+  const Layout L = layout(DK / 64, p.s0_planes, p.T_max, p.hist_cap);
   const size_t smem = L.total + 1024;
   static size_t configured[64] = {0};
   int dev = 0;
@@ -661,7 +654,7 @@ cudaError_t launch_s0_image(const void *S0, void *img, int R, int H, int dk, int
 }
 
 cudaError_t launch_step_tc(const StepParams &p, int pdl, cudaStream_t s) {
-  if (p.T_max > kMaxT || p.W_max > kMaxW || p.s0_planes < 1 || p.s0_planes > 3 || !p.rec_P)
+  if (p.T_max > kMaxT || p.W_max > kMaxW || p.s0_planes < 1 || p.s0_planes > 3 || p.hist_cap > kHistMaxInts)
     return cudaErrorNotSupported;
   if (p.dk == 64 && p.dv == 64) return launch_dk<64>(p, pdl != 0, s);
   if (p.dk == 128 && p.dv == 128) return launch_dk<128>(p, pdl != 0, s);
