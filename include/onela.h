@@ -78,16 +78,21 @@ enum {
 /* onela_config.flags bits.
  *   ONELA_FLAG_PDL  launch decode steps t >= 2 of the tensor-core kernel as
  *                   programmatic dependents of the kernel before them in the
- *                   stream: step t loads its inputs, S0 and the part of each
- *                   beam's ancestry that steps up to t-2 produced while step
- *                   t-1 finishes, and waits for step t-1 only before it
- *                   touches step t-1's records.  Set it only when (a) that
- *                   earlier kernel does not produce any input of step t (q,
- *                   k, v, g, beta, parent_idx), and (b) the parent_idx array
- *                   of step t-1 stays unchanged and allocated until step t
- *                   has completed -- e.g. back-to-back decode steps whose
- *                   inputs were all written before the first of them, as in
- *                   a CUDA graph of a whole decode.  Step 1 never overlaps. */
+ *                   stream: step t starts while step t-1 still runs, does
+ *                   all its work that needs no delta of an earlier step
+ *                   (S0 products, ancestry, key products, gate weights), and
+ *                   waits for step t-1 only before it stages the ancestors'
+ *                   deltas.  For that it reads the k, gate and parent_idx
+ *                   arrays of every earlier step of the decode again.  Set
+ *                   it only when (a) the kernel before step t in the stream
+ *                   produces no input of step t (q, k, v, g, beta,
+ *                   parent_idx), and (b) the k, gate and parent_idx arrays of
+ *                   every earlier step of the decode stay unchanged and
+ *                   allocated until step t has completed -- e.g. back-to-back
+ *                   decode steps whose inputs were all written before the
+ *                   first of them, as in a CUDA graph of a whole decode, or
+ *                   the verification of a tree of drafted tokens.  Step 1
+ *                   never overlaps. */
 enum { ONELA_FLAG_PDL = 1 };
 
 /* Which decode kernel runs.  AUTO picks the tensor-core kernel when the
@@ -149,9 +154,11 @@ ONELA_API int onela_set_prompt_state(onela_handle *h, const void *S0, onela_stre
  *   beta        [R][W][H] fp32, the delta-rule write strength.
  *   parent_idx  [R][W] int32, beam b's parent among the previous step's
  *               beams, in [0, W_prev).  One array serves all heads.  With
- *               ONELA_FLAG_PDL the library reads it again during the next
- *               step (see the flag).
+ *               ONELA_FLAG_PDL the library reads it, k and gate again during
+ *               the later steps of the decode (see the flag).
  *   o           [R][W][H][d_v] fp32, written: o_t = S_t q_t.
+ * With the tensor-core kernel, q, k, v and o must start on 16-byte
+ * boundaries (ONELA_ERR_ARG otherwise).
  * Also appends the records (alpha_t, delta_t, k_t) of every (beam, head) at
  * depth t and the ancestry rows of depth t; earlier records are never moved.
  * A parent index outside [0, W_prev) is clamped to 0 on the device, recorded

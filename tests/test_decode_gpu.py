@@ -268,6 +268,11 @@ def test_host_side_errors():
             dec.step(d[2]["q"], d[2]["k"], d[2]["v"], d[2]["g"], d[2]["beta"], d[2]["parents"])
         assert ei.value.code == L.ONELA_ERR_CAPACITY
         dec.reset()
+        if dec.kernel == L.ONELA_KERNEL_TC:    # 16-byte aligned tiles
+            o_off = torch.empty(1 * 4 * 2 * 64 + 1, device="cuda")[1:].view(1, 4, 2, 64)
+            with pytest.raises(L.OnelaError) as ei:
+                L.onela_decode_step(dec.h, 1, 4, s["q"], s["k"], s["v"], s["g"], s["beta"], s["parents"], o_off)
+            assert ei.value.code == L.ONELA_ERR_ARG
         big = P.custom_steps(15, 1, 2, 64, 64, (5,))[2]
         b = P.to_dev(big)[0]
         with pytest.raises(L.OnelaError) as ei:        # W_max = 4
