@@ -188,7 +188,7 @@ def time_cpu_oracle(wl, S0, steps, budget_s=10.0, nthreads=0):
         cref.beam_decode_fullstate(S0, steps, nthreads=nthreads)
         reps += 1
         el = time.perf_counter() - t0
-        if el >= budget_s or reps >= 50:
+        if el >= budget_s or reps >= 1000:
             break
     units = wl.units * reps
     threads = nthreads if nthreads > 0 else cref.max_threads()
