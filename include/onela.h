@@ -12,16 +12,14 @@
  *     delta_t = beta_t (v_t - alpha_t S_{t-1} k_t),   alpha_t = exp(g_t)
  *     o_t     = S_t q_t = alpha_t S_{t-1} q_t + delta_t (k_t . q_t)
  *
- * No per-beam state is ever formed.  Every beam is a chain of transition
- * records (alpha, delta, k) reached through an ancestry index (review,
- * Summary: "compact append-only GDN Transition Records"; abstract: "a
- * lightweight ancestry index ... without moving or copying existing
- * records").  S_{t-1} x for x in {k_t, q_t} is computed as
+ * No per-beam state is ever formed.  Every beam is a chain of small
+ * transition records (alpha, delta, k), written once and never moved, that
+ * an index of parent pointers ties together (review, Summary; abstract).
+ * S_{t-1} x for x in {k_t, q_t} is computed as
  *     G (S0 x) + sum_j w_j (k_j . x) delta_j
  * over the beam's ancestor records j (w_j: product of the gates of the
  * records after j, G: product of all of them), with S0 read once per head and
- * shared by every beam (abstract: "A fused GPU kernel further reuses the
- * shared state across beams").
+ * used for every beam (the abstract's fused kernel shares S0 across beams).
  *
  * Conventions for every entry point
  *   - All tensor pointers are DEVICE pointers on the handle's device unless a
@@ -136,8 +134,8 @@ typedef struct {
  * Errors: ONELA_ERR_ARG (null pointer or invalid field), ONELA_ERR_CUDA. */
 ONELA_API int onela_create(const onela_config *cfg, onela_handle **out);
 
-/* Install the shared prompt-derived state (abstract: "a single shared
- * prompt-derived state") and rewind the decode to step 0.
+/* Install the state that every beam of a request starts from (the one state
+ * built from the prompt, abstract) and rewind the decode to step 0.
  *   S0  device pointer, [R][H][d_v][d_k] in cfg.s0_dtype.  Copied on `stream`
  *       (and, for the tensor-core kernel, converted once into the bf16
  *       operand layout); S0 may be freed once the stream has passed the call.

@@ -4,14 +4,13 @@
 // shared-state GDN beam decode (OneLA, evolve.pub review, key claims on
 // section 3.2, equations 2-4) runs in this one launch:
 //   1. ancestry update: the beam's ancestor row is its parent's row plus the
-//      parent itself (abstract: "lightweight ancestry index ... without
-//      moving or copying existing records"); parents are range-checked;
+//      parent itself, so only indices move and records stay where they
+//      were written (abstract); parents are range-checked;
 //   2. the shared-state products S0 k_b and S0 q_b (S0 staged through shared
 //      memory in column chunks and reused by every beam of the tile);
-//   3. projection replay over the ancestor records (review, Summary: the
-//      records are replayed "in vector form without ever materializing a
-//      per-beam matrix"): gate weights, dot products k_j . x, and the two
-//      d_v-wide accumulators;
+//   3. projection replay over the ancestor records, with vectors only and
+//      no per-beam matrix (review, Summary): gate weights, dot products
+//      k_j . x, and the two d_v-wide accumulators;
 //   4. the step epilogue: delta = beta (v - alpha u_k), o = alpha u_q +
 //      delta (k . q), and the append of the record (alpha, delta, k).
 // This kernel serves shapes the tensor-core kernel does not (fp32 q/k/v, odd

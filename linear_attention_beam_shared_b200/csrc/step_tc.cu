@@ -10,8 +10,8 @@
 //   S_{t-1} x = P(p) S0 x + sum_j delta_{a_j} w_j (k_{a_j} . x),
 //   w_j = alpha_{a_{j+1}} ... alpha_{a_{t-1}}   (w = 1 for the parent),
 //
-// for x = k_b and x = q_b (review, Summary: records replayed "in vector form
-// without ever materializing a per-beam matrix").  Then
+// for x = k_b and x = q_b: the records are replayed with vectors only, no
+// per-beam matrix is formed (review, Summary).  Then
 // delta_b = beta_b (v_b - alpha_b S_{t-1} k_b) and
 // o_b = alpha_b S_{t-1} q_b + delta_b (k_b . q_b), and the record
 // (alpha_b, delta_b, k_b) is appended.
@@ -19,7 +19,7 @@
 //   D1 = S0 . X^T   tensor cores, fp32 accumulators in TMEM, for the tile's
 //                   64 vectors X = [k_0..k_31; q_0..q_31].  The S0 operand
 //                   image is read once per CTA and serves every beam of the
-//                   tile (abstract: "reuses the shared state across beams");
+//                   tile (the abstract's shared-state reuse across beams);
 //                   fp32 S0 is split once, when the prompt state is
 //                   installed, into two or three bf16 terms.
 //   D2 = KA . X^T   tensor cores: k_a . x for every distinct ancestor a of
@@ -31,9 +31,9 @@
 // lets its dependent launch start at once, and before its
 // griddepcontrol.wait it reads inputs only: the callers' arrays of the
 // earlier steps under ONELA_FLAG_PDL, the record store otherwise (then the
-// earlier steps have completed).  It computes D1, the ancestry (abstract:
-// "lightweight ancestry index ... without moving or copying existing
-// records"), D2 and every weight, and writes the depth-t entries that need
+// earlier steps have completed).  It computes D1, the ancestry (parent
+// indices only; records never move, abstract), D2 and every weight, and
+// writes the depth-t entries that need
 // no delta (alpha, k, the ancestry row).  After the wait it stages the
 // distinct ancestors' deltas with one round of bulk copies, replays, and
 // writes o and delta.  No kernel reads a depth-t entry before step t has

@@ -14,9 +14,10 @@ and is advanced once per decode step,
     o_t = S_t q_t,
 
 where S_{t-1} is the state of the beam's parent (the beam it was expanded
-from).  The pages call the method exact ("reproduces GDN exactly", review
-section 3.2 and FAQ), so this oracle is that plain definition written out: the
-"FullState" semantics (review, Scope & Claims), a full d_v x d_k state per
+from).  The pages state that the method is exact, with no approximation
+(review, key claims on section 3.2), so this oracle is that plain definition
+written out: the FullState baseline's semantics (review, Summary and report
+preview "Scope & Claims"), a full d_v x d_k state per
 beam, copied from the parent at every step, and the output taken literally as
 S_t q_t.  Nothing is blocked, fused or reordered beyond numpy's own matrix
 products.

@@ -3,7 +3,8 @@ oracle itself (closed forms, exact rational arithmetic, the textbook matrix
 form of the gated delta rule, invariants, brute force, a hand-worked example).
 
 The method and its exactness claim: OneLA abstract and the evolve.pub review
-(key claims on section 3.2, equations 2-4; FAQ "mathematically exact").
+(key claims on section 3.2, equations 2-4, which state that the replay
+reproduces GDN exactly).
 """
 import json
 import os
