@@ -48,6 +48,29 @@ def dist_env():
     return ws, rank, local
 
 
+def rank_workload(base, rank):
+    """Every rank decodes its own request: the same shapes, its own S0 and
+    inputs (its own random stream)."""
+    return base.replace(seed_id=base.seed_id + 1000 * rank)
+
+
+def max_over_ranks(x, device):
+    """The largest value of x over all ranks (x itself with one rank).  The
+    tensor lives on ``device``: the GPU for NCCL, the CPU for gloo."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(units_per_rank, ws, max_ms_per_step):
+    """Whole-job throughput: the units all ranks processed / the slowest
+    rank's device time."""
+    return units_per_rank * ws / (max_ms_per_step / 1e3)
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -209,9 +232,7 @@ def run_ours(args):
     device = torch.device("cuda", torch.cuda.current_device())
     import linear_attention_beam_shared_b200 as L
 
-    base = synth.workload(args.workload)
-    # Every rank decodes its own request: own S0, own inputs.
-    wl = base.replace(seed_id=base.seed_id + 1000 * rank)
+    wl = rank_workload(synth.workload(args.workload), rank)
     if args.s0 == "prefill":
         S0 = s0_by_prefill_gpu(wl, device)
     else:   # same shapes and dtype, entries drawn directly (for quick profiling runs)
@@ -266,15 +287,10 @@ def run_ours(args):
     if ws > 1:
         torch.distributed.barrier()
     times_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = float(sum(times_ms))
-    if ws > 1:
-        t = torch.tensor([total_ms], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(times_ms), device)
     assert dec.status() == 0
     ms_per_step = total_ms / args.steps
-    units_per_step = wl.units * ws
-    value = units_per_step / (ms_per_step / 1e3)
+    value = whole_job_value(wl.units, ws, ms_per_step)
 
     # Roofline of the decode kernel (the only kernel in the step).
     alg_bytes, upper_bytes, _ = byte_model(wl, steps)
@@ -326,11 +342,8 @@ def run_ours(args):
         stream.synchronize()
         if it > 0:
             e2e_ms += e_start.elapsed_time(e_end)
-    if ws > 1:
-        t = torch.tensor([e2e_ms], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e = {"value": round(units_per_step / (e2e_ms / e2e_steps / 1e3), 1), "unit": UNIT,
+    e2e_ms = max_over_ranks(e2e_ms, device)
+    e2e = {"value": round(whole_job_value(wl.units, ws, e2e_ms / e2e_steps), 1), "unit": UNIT,
            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
     assert dec.status() == 0
 
