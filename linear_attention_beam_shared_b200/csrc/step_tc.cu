@@ -52,7 +52,6 @@ constexpr int kThreads = 256;       // 8 warps
 constexpr int kBT = 32;             // beams per CTA
 constexpr int kN = 2 * kBT;         // vectors: k rows 0..31, q rows 32..63
 constexpr int kM = 128;             // MMA M
-constexpr int kBlk = 128;           // ancestors per D2 block (the MMA's M)
 constexpr int kDRows = 128;         // ancestor deltas per staging round after the wait
 constexpr int kTmemCols = 128;      // D1 [0,64), D2 [64,128)
 constexpr int kMaxT = 16;           // deepest decode the kernel serves
@@ -71,10 +70,7 @@ struct Layout {
   uint32_t total;
 };
 
-// Shared-memory ints of the per-depth counts, rounded to whole 16-byte pieces.
-__host__ __device__ inline int cnt_ints(int TM) { return (TM + 7) & ~3; }
-
-__host__ __device__ inline Layout layout(int nk, int planes, int TM, int hist_cap) {
+__host__ __device__ inline Layout layout(int nk, int planes, int TM, int W_max, int hist_cap) {
   Layout L;
   L.x = 0;
   L.v = (uint32_t)nk * 8192u;
@@ -84,11 +80,12 @@ __host__ __device__ inline Layout layout(int nk, int planes, int TM, int hist_ca
   L.dst = L.a;
   const uint32_t s0 = (uint32_t)planes * nk * 16384u, ops = (uint32_t)nk * 32768u;
   L.book = L.a + (s0 > ops ? s0 : ops);
-  // 64 B barriers/counters; 5 per-beam scalars; per (beam, depth) the replay
-  // coefficients (float4), the chain, slot, slot-list ints and weights; per-depth
-  // counts; the parents of steps 2..t-1.
-  L.total = L.book + 64u + 5u * kBT * 4u + (uint32_t)kBT * TM * 16u + 4u * kBT * TM * 4u +
-            (uint32_t)cnt_ints(TM) * 4u + (uint32_t)((hist_cap + 3) & ~3) * 4u + 16u;
+  // 128 B of barriers and counters; 4 per-beam scalars; per (beam, depth)
+  // the replay coefficients (float4), the chain, slot, slot-list ints and
+  // weights; per slot the key row's address; a beam-index scratch [W_max];
+  // the parents of steps 2..t-1.
+  L.total = L.book + 128u + 4u * kBT * 4u + (uint32_t)kBT * TM * 16u + 4u * kBT * TM * 4u +
+            (uint32_t)kBT * TM * 8u + (uint32_t)((W_max + 3) & ~3) * 4u + (uint32_t)((hist_cap + 3) & ~3) * 4u + 16u;
   return L;
 }
 
@@ -118,6 +115,9 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
   constexpr uint32_t XA = kN * 128;  // bytes of one K atom of X (64 rows)
   constexpr uint32_t VA = kBT * 128; // bytes of one K atom of v (32 rows)
   constexpr int NU = DV / 32;        // 4-element groups per thread, beam-major phase
+  // Ancestors per D2 block: the MMA's M (128), or 64 at d = 64, where D2^T of
+  // a block must fit in the 16 KB key area.
+  constexpr int kBlk = DK == 128 ? 128 : 64;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = ptx::smem_u32(smem_raw);
   uint8_t *base = smem_raw + ((1024u - (raw_u32 & 1023u)) & 1023u);
@@ -131,29 +131,39 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
   const int jp = nanc - 1;  // depth index of the parents (depth t-1)
   const bool hin = p.hist_inputs != 0;
 
-  const Layout L = layout(NK, P, TM, p.hist_cap);
+  const Layout L = layout(NK, P, TM, p.W_max, p.hist_cap);
   uint8_t *s_x = base + L.x;
   const uint8_t *s_v = base + L.v;
   float *s_d1 = reinterpret_cast<float *>(base + L.d1);
   const float *s_dst = reinterpret_cast<const float *>(base + L.dst);
-  uint64_t *bar_s0 = reinterpret_cast<uint64_t *>(base + L.book);
-  uint64_t *bar1 = bar_s0 + 1, *bar2 = bar_s0 + 2, *bar_d = bar_s0 + 3;
-  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bar_s0 + 4);
-  int *s_U1 = reinterpret_cast<int *>(s_tmem + 1);
-  int *s_par = reinterpret_cast<int *>(base + L.book + 64);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(base + L.book);
+  uint64_t *bar_s0 = bars + 0;     // S0 image, X and v landed
+  uint64_t *bar1 = bars + 1;       // D1 complete
+  uint64_t *bar2 = bars + 2;       // D2 of the current block complete
+  uint64_t *bar_d = bars + 3;      // ancestor deltas landed
+  uint64_t *bar_chain = bars + 4;  // warp 1: every beam's chain in s_chain
+  uint64_t *bar_slots = bars + 5;  // warp 1: slots, slot list and U
+  uint64_t *bar_w = bars + 6;      // warp 2: replay weights and P(p)
+  uint64_t *bar_keys = bars + 7;   // warps 4-7: keys of the current block in KA
+  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(base + L.book + 64);
+  int *s_U = reinterpret_cast<int *>(s_tmem + 1);
+  int *s_par = reinterpret_cast<int *>(base + L.book + 128);
   float *s_alpha = reinterpret_cast<float *>(s_par + kBT);
   float *s_beta = s_alpha + kBT;
   float *s_Gp = s_beta + kBT;  // P(parent)
-  float *s_spare = s_Gp + kBT;
   // [32][TM]: (w k_a . k_b, w k_a . q_b, slot of a) for the ancestor a of
   // beam b at each depth.
-  float4 *s_c = reinterpret_cast<float4 *>(s_spare + kBT);
+  float4 *s_c = reinterpret_cast<float4 *>(s_Gp + kBT);
   int *s_chain = reinterpret_cast<int *>(s_c + kBT * TM);  // [32][TM] ancestor beam by depth
   int *s_slot = s_chain + kBT * TM;                         // [32][TM] ancestor slot by depth
   int *s_list = s_slot + kBT * TM;                          // slot -> (beam << 5 | depth-1)
   float *s_w = reinterpret_cast<float *>(s_list + kBT * TM);  // [32][TM] replay weight by depth
-  int *s_cnt = reinterpret_cast<int *>(s_w + kBT * TM);       // distinct ancestors per depth
-  int *s_hist = s_cnt + cnt_ints(TM);                          // parents of steps 2..t-1
+  const __nv_bfloat16 **s_ksrc =                               // slot -> key row of the ancestor
+      reinterpret_cast<const __nv_bfloat16 **>(s_w + kBT * TM);
+  int *s_seen = reinterpret_cast<int *>(s_ksrc + kBT * TM);    // beam index -> a lane (scratch)
+  int *s_hist = s_seen + ((p.W_max + 3) & ~3);                 // parents of steps 2..t-1
+  float *s_d2t = reinterpret_cast<float *>(base + L.ka);       // D2^T [64 vectors][kBlk slots]
+  static_assert(kN * kBlk * 4 <= NK * 16384, "D2^T must fit in the key area");
 
   __nv_bfloat16 *rec_k = static_cast<__nv_bfloat16 *>(p.rec_k);
   const int64_t row0 = (int64_t)(r * p.W + b0) * H + h;  // (r, b0, h) row of [R][W][H][d]
@@ -165,6 +175,10 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
     ptx::mbar_init(bar1, 1);
     ptx::mbar_init(bar2, 1);
     ptx::mbar_init(bar_d, kDRows);
+    ptx::mbar_init(bar_chain, 32);
+    ptx::mbar_init(bar_slots, 32);
+    ptx::mbar_init(bar_w, 32);
+    ptx::mbar_init(bar_keys, kThreads / 2);
     ptx::mbar_fence_init();
     // S0 image (bulk copy); k, q, v tiles by TMA, beams past W read as zeros.
     ptx::mbar_arrive_expect_tx(bar_s0, s0_bytes + NK * (XA + VA));
@@ -182,24 +196,19 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
     ptx::tmem_alloc(s_tmem, kTmemCols);
     ptx::tmem_relinquish();
   }
-  // The parents of steps 2..t-1 for this request, back to back, each array
-  // starting on a 16-byte boundary; warp w copies steps w + 2, w + 10.
-  if (p.hist_cap > 0)
-#pragma unroll 1
-    for (int j = warp + 2; j < t; j += kThreads / 32)
-      copy_ints_warp(s_hist + p.hoff[j], p.hpar[j] + (int64_t)r * p.hpar_rs[j], p.hW[j], lane);
-  ptx::cp_async_commit();
+  int par = 0;
+  float g_alpha = 0.f, g_beta = 0.f;
+  if (warp == 1) {
+    // This tile's parents, gates and betas.
+    if (lane < nb) {
+      par = nanc >= 1 ? p.parents[r * p.W + b0 + lane] : 0;
+      const int64_t si = row0 + (int64_t)lane * H;
+      g_alpha = p.g[si];
+      g_beta = p.beta[si];
+    }
+  }
   // Before its wait this kernel reads inputs only, so the next step may start.
   ptx::pdl_launch_dependents();
-  int par = -1;
-  float g_alpha = 0.f, g_beta = 0.f;
-  if (warp == 1 && lane < nb) {
-    par = nanc >= 1 ? p.parents[r * p.W + b0 + lane] : 0;
-    const int64_t si = row0 + (int64_t)lane * H;
-    g_alpha = p.g[si];
-    g_beta = p.beta[si];
-  }
-  ptx::cp_async_wait_all();
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
@@ -208,32 +217,63 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
   bool ok = true;
   const uint32_t x_u32 = ptx::smem_u32(s_x), a_u32 = ptx::smem_u32(base + L.a);
   const uint32_t ka_u32 = ptx::smem_u32(base + L.ka);
-  if (tid == 0) {
-    ok = ptx::mbar_wait(bar_s0, 0, kWaitLimitNs);
-    ptx::tc_fence_after();
-    constexpr uint32_t idesc1 = ptx::idesc_bf16_f32(kM, kN);
-    int acc = 0;
-    for (int pl = 0; pl < P; ++pl)
+  const int wq = warp & 3;                        // TMEM lane quarter of this warp
+  const uint32_t lb = (uint32_t)(wq * 32) << 16;  // its lane base
+
+  // ------------------------------------------------ warp roles before the wait
+  if (warp == 0) {
+    // The MMA issuer: D1 = S0 . X^T, then D2 = KA . X^T per block of keys.
+    if (lane == 0) {
+      ok = ptx::mbar_wait(bar_s0, 0, kWaitLimitNs);
+      ptx::tc_fence_after();
+      constexpr uint32_t idesc1 = ptx::idesc_bf16_f32(kM, kN);
+      int acc = 0;
+      for (int pl = 0; pl < P; ++pl)
 #pragma unroll
-      for (int ka = 0; ka < NK; ++ka)
+        for (int ka = 0; ka < NK; ++ka)
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t ad = ptx::desc_k128(a_u32 + (pl * NK + ka) * 16384 + kk * 32);
-          const uint64_t bd = ptx::desc_k128(x_u32 + ka * XA + kk * 32);
-          ptx::mma_bf16(tmem, ad, bd, idesc1, acc);
-          acc = 1;
-        }
-    ptx::mma_commit(bar1);
-  }
-  if (warp == 1) {
-    // Beam b's ancestors: a[j] at depth j + 1, a[t-2] = its parent; a[j] is
-    // the parent, at step j + 2, of a[j + 1].
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = ptx::desc_k128(a_u32 + (pl * NK + ka) * 16384 + kk * 32);
+            const uint64_t bd = ptx::desc_k128(x_u32 + ka * XA + kk * 32);
+            ptx::mma_bf16(tmem, ad, bd, idesc1, acc);
+            acc = 1;
+          }
+      ptx::mma_commit(bar1);
+      if (!ptx::mbar_wait(bar_slots, 0, kWaitLimitNs)) ok = false;
+      const int U = *s_U;
+      for (int lo = 0, blk = 0; lo < U; lo += kBlk, ++blk) {
+        if (!ptx::mbar_wait(bar_keys, blk & 1, kWaitLimitNs)) ok = false;
+        ptx::tc_fence_after();
+        constexpr uint32_t idesc2 = ptx::idesc_bf16_f32(kM, kN);
+#pragma unroll
+        for (int ka = 0; ka < NK; ++ka)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = ptx::desc_k128(ka_u32 + ka * 16384 + kk * 32);
+            const uint64_t bd = ptx::desc_k128(x_u32 + ka * XA + kk * 32);
+            ptx::mma_bf16(tmem + 64, ad, bd, idesc2, (ka | kk) != 0);
+          }
+        ptx::mma_commit(bar2);
+      }
+    }
+  } else if (warp == 1) {
+    // The ancestry: beam b's ancestors a[j] at depth j + 1 (a[t-2] = its
+    // parent; a[j] is the parent, at step j + 2, of a[j + 1]), the entries of
+    // depth t that need no delta, and the distinct ancestors of the tile.
     const int b = lane;
+    // The parents of steps 2..t-1 for this request, back to back, each array
+    // starting on a 16-byte boundary.
+    if (p.hist_cap > 0)
+#pragma unroll 1
+      for (int j = 2; j < t; ++j)
+        copy_ints_warp(s_hist + p.hoff[j], p.hpar[j] + (int64_t)r * p.hpar_rs[j], p.hW[j], lane);
+    ptx::cp_async_commit();
+    ptx::cp_async_wait_all();
+    __syncwarp();
     if (b < nb && nanc >= 1 && (par < 0 || par >= p.W_prev)) {
       *reinterpret_cast<volatile int32_t *>(p.err) = kErrParent;
       par = 0;
     }
-    if (b >= nb) par = 0;
     const float alpha_b = b < nb ? expf(g_alpha) : 0.f;
     s_par[b] = par;
     s_alpha[b] = alpha_b;
@@ -249,21 +289,7 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
         s_chain[b * TM + j] = a;
       }
     }
-    if (nanc >= 1) {
-      // Distinct parents take slots 0..U1-1.
-      const unsigned same = __match_any_sync(0xffffffffu, par);
-      const int leader = __ffs(same) - 1;
-      const bool lead = b < nb && leader == lane;
-      const unsigned leaders = __ballot_sync(0xffffffffu, lead);
-      const int my = __popc(leaders & ((1u << lane) - 1u));
-      if (lead) s_list[my] = (par << 5) | jp;
-      const int slot = __shfl_sync(0xffffffffu, my, leader);
-      if (lane == 0) *s_U1 = __popc(leaders);
-      if (b < nb) s_slot[b * TM + jp] = slot;
-    } else if (lane == 0) {
-      *s_U1 = 0;
-    }
-    // Entries of depth t that need no delta.
+    ptx::mbar_arrive(bar_chain);
     if (b < nb) {
       const int gb = b0 + b;
       p.rec_alpha[rec_row(p, t, r, h, gb)] = alpha_b;
@@ -274,13 +300,39 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
         p.par_store[((int64_t)(t - 1) * p.R + r) * p.W_max + gb] = par;
       }
     }
-  }
-  __syncthreads();
-  if (warp == 0) {
-    // The gates along beam b's chain give the replay weights (products of the
-    // later gates) and P(p).  The gates land in s_w first (one round trip);
+    // Distinct ancestors depth by depth: every lane writes its lane number
+    // at its ancestor's index, and the lane whose number survives leads that
+    // ancestor.  Slots in order of depth, then of the leading lane.
+    int U = 0;
+#pragma unroll 1
+    for (int j = 0; j < nanc; ++j) {
+      const int a = b < nb ? s_chain[b * TM + j] : 0;
+      if (b < nb) s_seen[a] = lane;
+      __syncwarp();
+      const int leader = b < nb ? s_seen[a] : 0;
+      __syncwarp();
+      const bool lead = b < nb && leader == lane;
+      const unsigned leaders = __ballot_sync(0xffffffffu, lead);
+      const int slot = U + __popc(leaders & ((1u << leader) - 1u));
+      if (lead) {
+        s_list[slot] = (a << 5) | j;
+        s_ksrc[slot] = hin ? static_cast<const __nv_bfloat16 *>(p.hk[j + 1]) + (((int64_t)r * p.hW[j + 1] + a) * H + h) * DK
+                           : rec_k + rec_row(p, j + 1, r, h, a) * DK;
+      }
+      if (b < nb) {
+        s_slot[b * TM + j] = slot;
+        s_c[b * TM + j] = make_float4(0.f, 0.f, __int_as_float(slot), 0.f);
+      }
+      U += __popc(leaders);
+    }
+    if (lane == 0) *s_U = U;
+    ptx::mbar_arrive(bar_slots);
+  } else if (warp == 2) {
+    // The gates along each beam's chain give the replay weights (products of
+    // the later gates) and P(p).  They land in s_w first (one round trip);
     // each entry is then overwritten by the weight of its depth.
     const int b = lane;
+    if (!ptx::mbar_wait(bar_chain, 0, kWaitLimitNs)) ok = false;
     if (b < nb) {
 #pragma unroll 1
       for (int j = 0; j <= jp; ++j) {
@@ -301,72 +353,119 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
       }
     }
     s_Gp[b] = w;  // P(p): all the gates on the path
-  }
-  // Deeper ancestors (depths 1..t-2): one warp per depth (warps 1..7; warp 0
-  // gathers the gates) finds the distinct ones; their slots follow the
-  // parents', depth by depth.
-  for (int j = warp - 1; warp > 0 && j < jp; j += kThreads / 32 - 1) {
-    const int a = lane < nb ? s_chain[lane * TM + j] : -1;
-    const unsigned same = __match_any_sync(0xffffffffu, a);
-    const int leader = __ffs(same) - 1;
-    const bool lead = lane < nb && leader == lane;
-    const unsigned leaders = __ballot_sync(0xffffffffu, lead);
-    const int my = __popc(leaders & ((1u << lane) - 1u));
-    const int rank = __shfl_sync(0xffffffffu, my, leader);
-    if (lane < nb) s_slot[lane * TM + j] = rank;
-    if (lane == 0) s_cnt[j] = __popc(leaders);
-  }
-  __syncthreads();
-  const int U1 = *s_U1;
-  int U = U1;
-  for (int j = 0; j < jp; ++j) U += s_cnt[j];
-  for (int j = warp - 1; warp > 0 && j < jp; j += kThreads / 32 - 1) {
-    int base_j = U1;
-    for (int j2 = 0; j2 < j; ++j2) base_j += s_cnt[j2];
-    if (lane < nb) {
-      const int slot = base_j + s_slot[lane * TM + j];
-      s_slot[lane * TM + j] = slot;
-      s_list[slot] = (s_chain[lane * TM + j] << 5) | j;
-      // The slot is known now; the coefficients follow with the slot's block.
-      s_c[lane * TM + j] = make_float4(0.f, 0.f, __int_as_float(slot), 0.f);
+    ptx::mbar_arrive(bar_w);
+  } else if (warp == 3) {
+    // The key records of depth t, from X.
+    if (!ptx::mbar_wait(bar_s0, 0, kWaitLimitNs)) ok = false;
+    for (int e = lane; e < kBT * NK * 8; e += 32) {
+      const int n = e / (NK * 8), cc = e - n * (NK * 8);
+      if (n < nb)
+        reinterpret_cast<uint4 *>(rec_k + rec_row(p, t, r, h, b0 + n) * DK)[cc] =
+            *reinterpret_cast<const uint4 *>(s_x + (cc >> 3) * XA + ptx::swz128(n, cc & 7));
     }
-  }
-
-  __syncthreads();  // slot list complete
-  // D1 is complete, so region A is free: the keys of the first D2 block go
-  // in flight now and land while the beam-major work below runs.  KA holds
-  // the keys of slots [lo, lo + nrows), K-major with the 128-byte swizzle.
-  auto stage_keys = [&](int lo, int nrows) {
-    constexpr int KPT = kBlk * NK * 8 / kThreads;  // 16-byte key pieces per thread
-    int kp[KPT];
+  } else {
+    // Warps 4-7: D1^T to shared memory, the keys of the tile's distinct
+    // ancestors into KA (K-major, 128-byte swizzle), and the weighted
+    // coefficients from D2 (row = slot, column = vector).
+    const int ei = wq * 32 + lane;  // TMEM lane: output element of D1, slot of D2
+    const int t4 = tid - kThreads / 2;
+    if (!ptx::mbar_wait(bar1, 0, kWaitLimitNs)) ok = false;
+    ptx::tc_fence_after();
+    if (!ptx::mbar_wait(bar_slots, 0, kWaitLimitNs)) ok = false;
+    const int U = *s_U;
+    bool have_w = false;
+    for (int lo = 0, blk = 0; lo < U; lo += kBlk, ++blk) {
+      const int hi = min(U, lo + kBlk);
+      const int nrows = hi - lo;
+      {
+        constexpr int KPT = kBlk * NK * 8 / (kThreads / 2);  // 16-byte key pieces per thread
+        const __nv_bfloat16 *src[KPT];
 #pragma unroll
-    for (int u = 0; u < KPT; ++u) {
-      const int e = tid + u * kThreads;
-      kp[u] = e < nrows * NK * 8 ? s_list[lo + e / (NK * 8)] : -1;
-    }
+        for (int u = 0; u < KPT; ++u) {
+          const int e = t4 + u * (kThreads / 2);
+          src[u] = e < nrows * NK * 8 ? s_ksrc[lo + e / (NK * 8)] : nullptr;
+        }
 #pragma unroll
-    for (int u = 0; u < KPT; ++u) {
-      const int e = tid + u * kThreads;
-      if (kp[u] >= 0) {
-        const int a = kp[u] >> 5, j = kp[u] & 31, cc = e % (NK * 8);
-        const __nv_bfloat16 *src =
-            hin ? static_cast<const __nv_bfloat16 *>(p.hk[j + 1]) + (((int64_t)r * p.hW[j + 1] + a) * H + h) * DK
-                : rec_k + rec_row(p, j + 1, r, h, a) * DK;
-        ptx::cp_async16(base + L.ka + (cc >> 3) * 16384 + ptx::swz128(e / (NK * 8), cc & 7), src + cc * 8, 16u);
+        for (int u = 0; u < KPT; ++u) {
+          const int e = t4 + u * (kThreads / 2);
+          const int cc = e % (NK * 8);
+          if (src[u])
+            ptx::cp_async16(base + L.ka + (cc >> 3) * 16384 + ptx::swz128(e / (NK * 8), cc & 7), src[u] + cc * 8,
+                            16u);
+        }
+        ptx::cp_async_commit();
       }
+      if (blk == 0) {
+        // D1^T while the keys are in flight.
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          float d[32];
+          ptx::tmem_ld32(tmem + lb + half * 32, d);
+          ptx::tmem_ld_wait();
+          if (wq * 32 < DV)
+#pragma unroll
+            for (int n = 0; n < 32; ++n) s_d1[(half * 32 + n) * DV + ei] = d[n];
+        }
+      }
+      ptx::cp_async_wait_all();
+      ptx::fence_proxy_async_smem();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(bar_keys);
+      if (!ptx::mbar_wait(bar2, blk & 1, kWaitLimitNs)) ok = false;
+      ptx::tc_fence_after();
+      // D2 (KA is consumed) to shared memory transposed: s_d2t[vector][row].
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        float d[32];
+        ptx::tmem_ld32(tmem + lb + 64 + half * 32, d);
+        ptx::tmem_ld_wait();
+        if (ei < kBlk)
+#pragma unroll
+          for (int n = 0; n < 32; ++n) s_d2t[(half * 32 + n) * kBlk + ei] = d[n];
+      }
+      ptx::tc_fence_before();
+      if (!have_w) {
+        if (!ptx::mbar_wait(bar_w, 0, kWaitLimitNs)) ok = false;
+        have_w = true;
+      }
+      ptx::named_sync(1, kThreads / 2);
+      // Every (beam, depth) pair whose ancestor is in this block takes its
+      // products from the ancestor's row, weighted.
+      for (int e = t4; e < nb * nanc; e += kThreads / 2) {
+        const int b = e / nanc, j = e - b * nanc;
+        const int sl = s_slot[b * TM + j] - lo;
+        if (sl >= 0 && sl < nrows) {
+          const float w = s_w[b * TM + j];
+          s_c[b * TM + j] = make_float4(s_d2t[b * kBlk + sl] * w, s_d2t[(kBT + b) * kBlk + sl] * w,
+                                        __int_as_float(sl + lo), 0.f);
+        }
+      }
+      ptx::named_sync(1, kThreads / 2);  // s_d2t and KA free for the next block
     }
-    ptx::cp_async_commit();
-  };
-  if (!ptx::mbar_wait(bar1, 0, kWaitLimitNs)) ok = false;
-  ptx::tc_fence_after();
-  if (U > 0) stage_keys(0, min(U, kBlk));
+    if (U == 0) {
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        float d[32];
+        ptx::tmem_ld32(tmem + lb + half * 32, d);
+        ptx::tmem_ld_wait();
+        if (wq * 32 < DV)
+#pragma unroll
+          for (int n = 0; n < 32; ++n) s_d1[(half * 32 + n) * DV + ei] = d[n];
+      }
+      if (!ptx::mbar_wait(bar_w, 0, kWaitLimitNs)) ok = false;
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();  // every role done: D1^T, coefficients, weights, k . q
+  if (warp == 3) ptx::tmem_dealloc(tmem, kTmemCols);
 
   // Beam-major phase: thread (bb, l) owns elements 32 u + 4 l + z (z < 4) of
-  // beam bb.  k_b . q_b, v, and the key records of depth t, from X and v.
+  // beam bb.  u = P(p) D1 + (replayed terms, after the wait); v from its tile.
   const int bb = tid >> 3, l = tid & 7;
-  if (!ptx::mbar_wait(bar_s0, 0, kWaitLimitNs)) ok = false;
-  float kq = 0.f;
+  float acc_k[4 * NU], acc_q[4 * NU];
   float4 vf[NU];
+  const float Gp = s_Gp[bb], alpha = s_alpha[bb], beta = s_beta[bb];
+  float kq = 0.f;
 #pragma unroll
   for (int u = 0; u < NU; ++u) {
     const uint32_t off = (uint32_t)(u >> 1) * XA + (uint32_t)(l & 1) * 8u;
@@ -377,101 +476,20 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
     kq = fmaf(kf.y, qf.y, kq);
     kq = fmaf(kf.z, qf.z, kq);
     kq = fmaf(kf.w, qf.w, kq);
-    vf[u] = bf16x4(s_v + (u >> 1) * VA + ptx::swz128(bb, c) + (l & 1) * 8);
   }
   kq += __shfl_xor_sync(0xffffffffu, kq, 4);
   kq += __shfl_xor_sync(0xffffffffu, kq, 2);
   kq += __shfl_xor_sync(0xffffffffu, kq, 1);
-  for (int e = tid; e < kBT * NK * 8; e += kThreads) {
-    const int n = e / (NK * 8), cc = e - n * (NK * 8);
-    if (n < nb)
-      reinterpret_cast<uint4 *>(rec_k + rec_row(p, t, r, h, b0 + n) * DK)[cc] =
-          *reinterpret_cast<const uint4 *>(s_x + (cc >> 3) * XA + ptx::swz128(n, cc & 7));
-  }
-
-  // D1^T to shared memory: warp w reads TMEM lanes 32 (w % 4).. (elements)
-  // and the k (w < 4) or q columns.
-  const int ei = (warp & 3) * 32 + lane, half = warp >> 2;
-  const uint32_t lb = (uint32_t)((warp & 3) * 32) << 16;
-  if ((warp & 3) * 32 < DV) {
-    float d[32];
-    ptx::tmem_ld32(tmem + lb + half * 32, d);
-    ptx::tmem_ld_wait();
-#pragma unroll
-    for (int n = 0; n < 32; ++n) s_d1[(half * 32 + n) * DV + ei] = d[n];
-  }
-  // (made visible by the barrier before the first D2 block)
-
-  // Keys of the tile's distinct ancestors, D2 = KA . X^T, and the weighted
-  // coefficients, block by block.
-  for (int lo = 0, blk = 0; lo < U; lo += kBlk, ++blk) {
-    const int hi = min(U, lo + kBlk);
-    const int nrows = hi - lo;
-    if (blk > 0) {
-      __syncthreads();  // the previous block's keys are consumed
-      stage_keys(lo, nrows);
-    }
-    ptx::cp_async_wait_all();
-    ptx::fence_proxy_async_smem();
-    __syncthreads();
-    if (tid == 0) {
-      ptx::tc_fence_after();
-      constexpr uint32_t idesc2 = ptx::idesc_bf16_f32(kM, kN);
-#pragma unroll
-      for (int ka = 0; ka < NK; ++ka)
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t ad = ptx::desc_k128(ka_u32 + ka * 16384 + kk * 32);
-          const uint64_t bd = ptx::desc_k128(x_u32 + ka * XA + kk * 32);
-          ptx::mma_bf16(tmem + 64, ad, bd, idesc2, (ka | kk) != 0);
-        }
-      ptx::mma_commit(bar2);
-    }
-    // D2 row (TMEM lane) = slot lo + row, column = vector.  Warp w reads rows
-    // 32 (w % 4).. for the beams of half w / 4.  The slot's thread writes the
-    // coefficients of every beam that replays it.
-    {
-      const int s = lo + (warp & 3) * 32 + lane;
-      const bool act = s < hi;
-      const int js = act ? (s_list[s] & 31) : 0;
-      int sl[16];
-#pragma unroll
-      for (int m = 0; m < 16; ++m) sl[m] = s_slot[(half * 16 + m) * TM + js];
-      if (!ptx::mbar_wait(bar2, blk & 1, kWaitLimitNs)) ok = false;
-      ptx::tc_fence_after();
-      float dk[16], dq[16];
-      ptx::tmem_ld16(tmem + lb + 64 + half * 16, dk);
-      ptx::tmem_ld16(tmem + lb + 64 + kBT + half * 16, dq);
-      ptx::tmem_ld_wait();
-      if (act) {
-#pragma unroll
-        for (int m = 0; m < 16; ++m) {
-          const int b = half * 16 + m;
-          if (b < nb && sl[m] == s) {
-            const float w = s_w[b * TM + js];
-            s_c[b * TM + js] = make_float4(dk[m] * w, dq[m] * w, __int_as_float(s), 0.f);
-          }
-        }
-      }
-    }
-    ptx::tc_fence_before();
-    __syncthreads();
-  }
-
-  if (U == 0) __syncthreads();  // D1^T visible (otherwise the block loop's barriers did it)
-  // u = P(p) D1 + (replayed terms, after the wait).
-  float acc_k[4 * NU], acc_q[4 * NU];
-  const float Gp = s_Gp[bb], alpha = s_alpha[bb], beta = s_beta[bb];
 #pragma unroll
   for (int u = 0; u < NU; ++u) {
     const float4 dk = reinterpret_cast<const float4 *>(s_d1 + bb * DV)[8 * u + l];
     const float4 dq = reinterpret_cast<const float4 *>(s_d1 + (kBT + bb) * DV)[8 * u + l];
     acc_k[4 * u + 0] = Gp * dk.x, acc_k[4 * u + 1] = Gp * dk.y, acc_k[4 * u + 2] = Gp * dk.z, acc_k[4 * u + 3] = Gp * dk.w;
     acc_q[4 * u + 0] = Gp * dq.x, acc_q[4 * u + 1] = Gp * dq.y, acc_q[4 * u + 2] = Gp * dq.z, acc_q[4 * u + 3] = Gp * dq.w;
+    vf[u] = bf16x4(s_v + (u >> 1) * VA + ptx::swz128(bb, 4 * (u & 1) + (l >> 1)) + (l & 1) * 8);
   }
-  ptx::tc_fence_before();
-  __syncthreads();  // D1^T consumed, TMEM reads done
-  if (warp == 3) ptx::tmem_dealloc(tmem, kTmemCols);
+  int U = *s_U;
+  __syncthreads();  // D1^T consumed before the deltas overwrite region A
 
   // ------------------------------- after the wait: the ancestors' deltas
   ptx::pdl_wait();
@@ -607,7 +625,7 @@ cudaError_t launch_dk(const StepParams &p_in, bool pdl, cudaStream_t s) {
   if (!encode_rows(&p.tm_k, p.k, DK, p.H, p.W, p.R) || !encode_rows(&p.tm_q, p.q, DK, p.H, p.W, p.R) ||
       !encode_rows(&p.tm_v, p.v, DK, p.H, p.W, p.R))
     return cudaErrorInvalidValue;
-  const Layout L = layout(DK / 64, p.s0_planes, p.T_max, p.hist_cap);
+  const Layout L = layout(DK / 64, p.s0_planes, p.T_max, p.W_max, p.hist_cap);
   const size_t smem = L.total + 1024;
   static size_t configured[64] = {0};
   int dev = 0;
