@@ -52,8 +52,9 @@ constexpr int kThreads = 256;       // 8 warps
 constexpr int kBT = 32;             // beams per CTA
 constexpr int kN = 2 * kBT;         // vectors: k rows 0..31, q rows 32..63
 constexpr int kM = 128;             // MMA M
-constexpr int kDRows = 128;         // ancestor deltas per staging round after the wait
-constexpr int kTmemCols = 128;      // D1 [0,64), D2 [64,128)
+constexpr int kDRows = 128;         // ancestor deltas per staging round after the wait (32 groups of 4)
+constexpr int kTmemCols = 64;       // D1
+constexpr int kKeyRows = 128;       // ancestor key rows per staging round
 constexpr int kMaxT = 16;           // deepest decode the kernel serves
 constexpr int kMaxW = 1024;         // widest beam set the kernel serves
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far beyond any legal wait
@@ -82,10 +83,10 @@ __host__ __device__ inline Layout layout(int nk, int planes, int TM, int W_max, 
   L.book = L.a + (s0 > ops ? s0 : ops);
   // 128 B of barriers and counters; 4 per-beam scalars; per (beam, depth)
   // the replay coefficients (float4), the chain, slot, slot-list ints and
-  // weights; per slot the key row's address; a beam-index scratch [W_max];
-  // the parents of steps 2..t-1.
-  L.total = L.book + 128u + 4u * kBT * 4u + (uint32_t)kBT * TM * 16u + 4u * kBT * TM * 4u +
-            (uint32_t)kBT * TM * 8u + (uint32_t)((W_max + 3) & ~3) * 4u + (uint32_t)((hist_cap + 3) & ~3) * 4u + 16u;
+  // weights (the slot list 4 TM longer); a beam-index scratch [W_max]; the
+  // parents of steps 2..t-1.
+  L.total = L.book + 128u + 4u * kBT * 4u + (uint32_t)kBT * TM * 16u + (4u * kBT + 4u) * TM * 4u +
+            (uint32_t)((W_max + 3) & ~3) * 4u + (uint32_t)((hist_cap + 3) & ~3) * 4u + 16u;
   return L;
 }
 
@@ -115,9 +116,6 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
   constexpr uint32_t XA = kN * 128;  // bytes of one K atom of X (64 rows)
   constexpr uint32_t VA = kBT * 128; // bytes of one K atom of v (32 rows)
   constexpr int NU = DV / 32;        // 4-element groups per thread, beam-major phase
-  // Ancestors per D2 block: the MMA's M (128), or 64 at d = 64, where D2^T of
-  // a block must fit in the 16 KB key area.
-  constexpr int kBlk = DK == 128 ? 128 : 64;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = ptx::smem_u32(smem_raw);
   uint8_t *base = smem_raw + ((1024u - (raw_u32 & 1023u)) & 1023u);
@@ -139,12 +137,11 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
   uint64_t *bars = reinterpret_cast<uint64_t *>(base + L.book);
   uint64_t *bar_s0 = bars + 0;     // S0 image, X and v landed
   uint64_t *bar1 = bars + 1;       // D1 complete
-  uint64_t *bar2 = bars + 2;       // D2 of the current block complete
   uint64_t *bar_d = bars + 3;      // ancestor deltas landed
   uint64_t *bar_chain = bars + 4;  // warp 1: every beam's chain in s_chain
   uint64_t *bar_slots = bars + 5;  // warp 1: slots, slot list and U
   uint64_t *bar_w = bars + 6;      // warp 2: replay weights and P(p)
-  uint64_t *bar_keys = bars + 7;   // warps 4-7: keys of the current block in KA
+  uint64_t *bar_keys = bars + 7;   // key rows of the current round landed
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(base + L.book + 64);
   int *s_U = reinterpret_cast<int *>(s_tmem + 1);
   int *s_par = reinterpret_cast<int *>(base + L.book + 128);
@@ -156,14 +153,14 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
   float4 *s_c = reinterpret_cast<float4 *>(s_Gp + kBT);
   int *s_chain = reinterpret_cast<int *>(s_c + kBT * TM);  // [32][TM] ancestor beam by depth
   int *s_slot = s_chain + kBT * TM;                         // [32][TM] ancestor slot by depth
-  int *s_list = s_slot + kBT * TM;                          // slot -> (beam << 5 | depth-1)
-  float *s_w = reinterpret_cast<float *>(s_list + kBT * TM);  // [32][TM] replay weight by depth
-  const __nv_bfloat16 **s_ksrc =                               // slot -> key row of the ancestor
-      reinterpret_cast<const __nv_bfloat16 **>(s_w + kBT * TM);
-  int *s_seen = reinterpret_cast<int *>(s_ksrc + kBT * TM);    // beam index -> a lane (scratch)
+  // slot -> (beam << 5 | depth-1); every depth's slots start on a multiple
+  // of 4 (padding slots repeat the depth's first ancestor), [(32 + 4) TM].
+  int *s_list = s_slot + kBT * TM;
+  float *s_w = reinterpret_cast<float *>(s_list + (kBT + 4) * TM);  // [32][TM] replay weight by depth
+  int *s_seen = reinterpret_cast<int *>(s_w + kBT * TM);           // beam index -> a lane (scratch)
   int *s_hist = s_seen + ((p.W_max + 3) & ~3);                 // parents of steps 2..t-1
-  float *s_d2t = reinterpret_cast<float *>(base + L.ka);       // D2^T [64 vectors][kBlk slots]
-  static_assert(kN * kBlk * 4 <= NK * 16384, "D2^T must fit in the key area");
+  uint8_t *s_keys = base + L.ka;                               // key rows [kKeyRows][d_k] bf16
+  static_assert(kKeyRows * DK * 2 <= NK * 16384, "the key rows must fit in their area");
 
   __nv_bfloat16 *rec_k = static_cast<__nv_bfloat16 *>(p.rec_k);
   const int64_t row0 = (int64_t)(r * p.W + b0) * H + h;  // (r, b0, h) row of [R][W][H][d]
@@ -173,12 +170,11 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
   if (tid == 0) {
     ptx::mbar_init(bar_s0, 1);
     ptx::mbar_init(bar1, 1);
-    ptx::mbar_init(bar2, 1);
-    ptx::mbar_init(bar_d, kDRows);
+    ptx::mbar_init(bar_d, 32);
     ptx::mbar_init(bar_chain, 32);
     ptx::mbar_init(bar_slots, 32);
     ptx::mbar_init(bar_w, 32);
-    ptx::mbar_init(bar_keys, kThreads / 2);
+    ptx::mbar_init(bar_keys, 32);
     ptx::mbar_fence_init();
     // S0 image (bulk copy); k, q, v tiles by TMA, beams past W read as zeros.
     ptx::mbar_arrive_expect_tx(bar_s0, s0_bytes + NK * (XA + VA));
@@ -216,13 +212,34 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
 
   bool ok = true;
   const uint32_t x_u32 = ptx::smem_u32(s_x), a_u32 = ptx::smem_u32(base + L.a);
-  const uint32_t ka_u32 = ptx::smem_u32(base + L.ka);
+  // Key rows of slots [lo, lo + n) (n a multiple of 4) into s_keys, by the
+  // 32 lanes of one warp: lane i gathers the 4 rows of slots lo + 4i .. + 3
+  // (one depth: the slots of a depth start on a multiple of 4) from that
+  // depth's row table.  Every lane arrives on bar_keys once.
+  auto stage_keys = [&](int lo, int n, int i) {
+    if (4 * i < n) {
+      const int s0 = lo + 4 * i;
+      const int j = s_list[s0] & 31;
+      const int Wj = p.hW[j + 1];
+      int row[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int a = s_list[s0 + q] >> 5;
+        row[q] = hin ? (r * Wj + a) * H + h : (int)rec_row(p, j + 1, r, h, a);
+      }
+      ptx::fence_proxy_async_smem();
+      ptx::mbar_arrive_expect_tx(bar_keys, 4 * DK * 2);
+      ptx::tma_gather4(s_keys + 4 * i * DK * 2, &p.tm_krows[j + 1], 0, row[0], row[1], row[2], row[3], bar_keys);
+    } else {
+      ptx::mbar_arrive(bar_keys);
+    }
+  };
   const int wq = warp & 3;                        // TMEM lane quarter of this warp
   const uint32_t lb = (uint32_t)(wq * 32) << 16;  // its lane base
 
   // ------------------------------------------------ warp roles before the wait
   if (warp == 0) {
-    // The MMA issuer: D1 = S0 . X^T, then D2 = KA . X^T per block of keys.
+    // The MMA issuer: D1 = S0 . X^T.
     if (lane == 0) {
       ok = ptx::mbar_wait(bar_s0, 0, kWaitLimitNs);
       ptx::tc_fence_after();
@@ -239,22 +256,6 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
             acc = 1;
           }
       ptx::mma_commit(bar1);
-      if (!ptx::mbar_wait(bar_slots, 0, kWaitLimitNs)) ok = false;
-      const int U = *s_U;
-      for (int lo = 0, blk = 0; lo < U; lo += kBlk, ++blk) {
-        if (!ptx::mbar_wait(bar_keys, blk & 1, kWaitLimitNs)) ok = false;
-        ptx::tc_fence_after();
-        constexpr uint32_t idesc2 = ptx::idesc_bf16_f32(kM, kN);
-#pragma unroll
-        for (int ka = 0; ka < NK; ++ka)
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = ptx::desc_k128(ka_u32 + ka * 16384 + kk * 32);
-            const uint64_t bd = ptx::desc_k128(x_u32 + ka * XA + kk * 32);
-            ptx::mma_bf16(tmem + 64, ad, bd, idesc2, (ka | kk) != 0);
-          }
-        ptx::mma_commit(bar2);
-      }
     }
   } else if (warp == 1) {
     // The ancestry: beam b's ancestors a[j] at depth j + 1 (a[t-2] = its
@@ -302,7 +303,8 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
     }
     // Distinct ancestors depth by depth: every lane writes its lane number
     // at its ancestor's index, and the lane whose number survives leads that
-    // ancestor.  Slots in order of depth, then of the leading lane.
+    // ancestor.  Slots in order of depth, then of the leading lane; each
+    // depth's first slot is a multiple of 4.
     int U = 0;
 #pragma unroll 1
     for (int j = 0; j < nanc; ++j) {
@@ -314,16 +316,16 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
       const bool lead = b < nb && leader == lane;
       const unsigned leaders = __ballot_sync(0xffffffffu, lead);
       const int slot = U + __popc(leaders & ((1u << leader) - 1u));
-      if (lead) {
-        s_list[slot] = (a << 5) | j;
-        s_ksrc[slot] = hin ? static_cast<const __nv_bfloat16 *>(p.hk[j + 1]) + (((int64_t)r * p.hW[j + 1] + a) * H + h) * DK
-                           : rec_k + rec_row(p, j + 1, r, h, a) * DK;
-      }
+      if (lead) s_list[slot] = (a << 5) | j;
       if (b < nb) {
         s_slot[b * TM + j] = slot;
         s_c[b * TM + j] = make_float4(0.f, 0.f, __int_as_float(slot), 0.f);
       }
-      U += __popc(leaders);
+      __syncwarp();
+      // Pad the depth to a whole group of 4 with its first ancestor.
+      const int cnt = __popc(leaders), cnt4 = (cnt + 3) & ~3;
+      if (lane >= cnt && lane < cnt4) s_list[U + lane] = s_list[U];
+      U += cnt4;
     }
     if (lane == 0) *s_U = U;
     ptx::mbar_arrive(bar_slots);
@@ -364,122 +366,93 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
             *reinterpret_cast<const uint4 *>(s_x + (cc >> 3) * XA + ptx::swz128(n, cc & 7));
     }
   } else {
-    // Warps 4-7: D1^T to shared memory, the keys of the tile's distinct
-    // ancestors into KA (K-major, 128-byte swizzle), and the weighted
-    // coefficients from D2 (row = slot, column = vector).
-    const int ei = wq * 32 + lane;  // TMEM lane: output element of D1, slot of D2
-    const int t4 = tid - kThreads / 2;
-    if (!ptx::mbar_wait(bar1, 0, kWaitLimitNs)) ok = false;
+    // Warps 4-7: the key rows of the tile's first kKeyRows distinct
+    // ancestors into shared memory (one bulk copy per row), and D1^T.
+    const int ei = wq * 32 + lane;  // TMEM lane: output element of D1
+    if (!ptx::mbar_wait(bar1, 0, kWaitLimitNs)) ok = false;  // region A is free
     ptx::tc_fence_after();
     if (!ptx::mbar_wait(bar_slots, 0, kWaitLimitNs)) ok = false;
-    const int U = *s_U;
-    bool have_w = false;
-    for (int lo = 0, blk = 0; lo < U; lo += kBlk, ++blk) {
-      const int hi = min(U, lo + kBlk);
-      const int nrows = hi - lo;
-      {
-        constexpr int KPT = kBlk * NK * 8 / (kThreads / 2);  // 16-byte key pieces per thread
-        const __nv_bfloat16 *src[KPT];
+    if (warp == 4) stage_keys(0, min(*s_U, kKeyRows), lane);
 #pragma unroll
-        for (int u = 0; u < KPT; ++u) {
-          const int e = t4 + u * (kThreads / 2);
-          src[u] = e < nrows * NK * 8 ? s_ksrc[lo + e / (NK * 8)] : nullptr;
-        }
+    for (int half = 0; half < 2; ++half) {
+      float d[32];
+      ptx::tmem_ld32(tmem + lb + half * 32, d);
+      ptx::tmem_ld_wait();
+      if (wq * 32 < DV)
 #pragma unroll
-        for (int u = 0; u < KPT; ++u) {
-          const int e = t4 + u * (kThreads / 2);
-          const int cc = e % (NK * 8);
-          if (src[u])
-            ptx::cp_async16(base + L.ka + (cc >> 3) * 16384 + ptx::swz128(e / (NK * 8), cc & 7), src[u] + cc * 8,
-                            16u);
-        }
-        ptx::cp_async_commit();
-      }
-      if (blk == 0) {
-        // D1^T while the keys are in flight.
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          float d[32];
-          ptx::tmem_ld32(tmem + lb + half * 32, d);
-          ptx::tmem_ld_wait();
-          if (wq * 32 < DV)
-#pragma unroll
-            for (int n = 0; n < 32; ++n) s_d1[(half * 32 + n) * DV + ei] = d[n];
-        }
-      }
-      ptx::cp_async_wait_all();
-      ptx::fence_proxy_async_smem();
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(bar_keys);
-      if (!ptx::mbar_wait(bar2, blk & 1, kWaitLimitNs)) ok = false;
-      ptx::tc_fence_after();
-      // D2 (KA is consumed) to shared memory transposed: s_d2t[vector][row].
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        float d[32];
-        ptx::tmem_ld32(tmem + lb + 64 + half * 32, d);
-        ptx::tmem_ld_wait();
-        if (ei < kBlk)
-#pragma unroll
-          for (int n = 0; n < 32; ++n) s_d2t[(half * 32 + n) * kBlk + ei] = d[n];
-      }
-      ptx::tc_fence_before();
-      if (!have_w) {
-        if (!ptx::mbar_wait(bar_w, 0, kWaitLimitNs)) ok = false;
-        have_w = true;
-      }
-      ptx::named_sync(1, kThreads / 2);
-      // Every (beam, depth) pair whose ancestor is in this block takes its
-      // products from the ancestor's row, weighted.
-      for (int e = t4; e < nb * nanc; e += kThreads / 2) {
-        const int b = e / nanc, j = e - b * nanc;
-        const int sl = s_slot[b * TM + j] - lo;
-        if (sl >= 0 && sl < nrows) {
-          const float w = s_w[b * TM + j];
-          s_c[b * TM + j] = make_float4(s_d2t[b * kBlk + sl] * w, s_d2t[(kBT + b) * kBlk + sl] * w,
-                                        __int_as_float(sl + lo), 0.f);
-        }
-      }
-      ptx::named_sync(1, kThreads / 2);  // s_d2t and KA free for the next block
-    }
-    if (U == 0) {
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        float d[32];
-        ptx::tmem_ld32(tmem + lb + half * 32, d);
-        ptx::tmem_ld_wait();
-        if (wq * 32 < DV)
-#pragma unroll
-          for (int n = 0; n < 32; ++n) s_d1[(half * 32 + n) * DV + ei] = d[n];
-      }
-      if (!ptx::mbar_wait(bar_w, 0, kWaitLimitNs)) ok = false;
+        for (int n = 0; n < 32; ++n) s_d1[(half * 32 + n) * DV + ei] = d[n];
     }
   }
   ptx::tc_fence_before();
-  __syncthreads();  // every role done: D1^T, coefficients, weights, k . q
+  __syncthreads();  // every role done: D1^T, slots, weights
   if (warp == 3) ptx::tmem_dealloc(tmem, kTmemCols);
 
   // Beam-major phase: thread (bb, l) owns elements 32 u + 4 l + z (z < 4) of
   // beam bb.  u = P(p) D1 + (replayed terms, after the wait); v from its tile.
   const int bb = tid >> 3, l = tid & 7;
-  float acc_k[4 * NU], acc_q[4 * NU];
-  float4 vf[NU];
-  const float Gp = s_Gp[bb], alpha = s_alpha[bb], beta = s_beta[bb];
+  const bool bval = bb < nb;
+  if (!ptx::mbar_wait(bar_s0, 0, kWaitLimitNs)) ok = false;  // X and v visible to this thread
+  // This thread's elements of k_b and q_b, and k_b . q_b.
+  float4 kb[NU], qb[NU];
   float kq = 0.f;
 #pragma unroll
   for (int u = 0; u < NU; ++u) {
     const uint32_t off = (uint32_t)(u >> 1) * XA + (uint32_t)(l & 1) * 8u;
     const int c = 4 * (u & 1) + (l >> 1);
-    const float4 kf = bf16x4(s_x + off + ptx::swz128(bb, c));
-    const float4 qf = bf16x4(s_x + off + ptx::swz128(kBT + bb, c));
-    kq = fmaf(kf.x, qf.x, kq);
-    kq = fmaf(kf.y, qf.y, kq);
-    kq = fmaf(kf.z, qf.z, kq);
-    kq = fmaf(kf.w, qf.w, kq);
+    kb[u] = bf16x4(s_x + off + ptx::swz128(bb, c));
+    qb[u] = bf16x4(s_x + off + ptx::swz128(kBT + bb, c));
+    kq = fmaf(kb[u].x, qb[u].x, kq);
+    kq = fmaf(kb[u].y, qb[u].y, kq);
+    kq = fmaf(kb[u].z, qb[u].z, kq);
+    kq = fmaf(kb[u].w, qb[u].w, kq);
   }
   kq += __shfl_xor_sync(0xffffffffu, kq, 4);
   kq += __shfl_xor_sync(0xffffffffu, kq, 2);
   kq += __shfl_xor_sync(0xffffffffu, kq, 1);
+  // k_a . k_b and k_a . q_b for the beam's ancestor a at every depth, from
+  // the staged key rows (rounds of kKeyRows slots), weighted.
+  const int U = *s_U;
+  for (int lo = 0, rnd = 0; lo < U; lo += kKeyRows, ++rnd) {
+    const int nrows = min(U - lo, kKeyRows);
+    if (rnd > 0) {
+      __syncthreads();  // the previous round's rows are consumed
+      if (warp == 0) stage_keys(lo, nrows, lane);
+    }
+    if (!ptx::mbar_wait(bar_keys, rnd & 1, kWaitLimitNs)) ok = false;
+#pragma unroll 1
+    for (int j = 0; j < nanc; ++j) {
+      const int slot = bval ? s_slot[bb * TM + j] : -1;
+      const unsigned sl = (unsigned)(slot - lo);
+      const bool in = sl < (unsigned)nrows;
+      const uint8_t *row = s_keys + (in ? sl : 0u) * (DK * 2) + l * 8;
+      float dk = 0.f, dq = 0.f;
+#pragma unroll
+      for (int u = 0; u < NU; ++u) {
+        const float4 kf = bf16x4(row + u * 64);
+        dk = fmaf(kf.x, kb[u].x, dk);
+        dk = fmaf(kf.y, kb[u].y, dk);
+        dk = fmaf(kf.z, kb[u].z, dk);
+        dk = fmaf(kf.w, kb[u].w, dk);
+        dq = fmaf(kf.x, qb[u].x, dq);
+        dq = fmaf(kf.y, qb[u].y, dq);
+        dq = fmaf(kf.z, qb[u].z, dq);
+        dq = fmaf(kf.w, qb[u].w, dq);
+      }
+#pragma unroll
+      for (int o = 4; o > 0; o >>= 1) {
+        dk += __shfl_xor_sync(0xffffffffu, dk, o);
+        dq += __shfl_xor_sync(0xffffffffu, dq, o);
+      }
+      if (in && l == 0) {
+        const float w = s_w[bb * TM + j];
+        s_c[bb * TM + j] = make_float4(dk * w, dq * w, __int_as_float(slot), 0.f);
+      }
+    }
+  }
+  // u = P(p) D1 + (replayed terms, after the wait); v from its tile.
+  float acc_k[4 * NU], acc_q[4 * NU];
+  float4 vf[NU];
+  const float Gp = s_Gp[bb], alpha = s_alpha[bb], beta = s_beta[bb];
 #pragma unroll
   for (int u = 0; u < NU; ++u) {
     const float4 dk = reinterpret_cast<const float4 *>(s_d1 + bb * DV)[8 * u + l];
@@ -488,8 +461,7 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
     acc_q[4 * u + 0] = Gp * dq.x, acc_q[4 * u + 1] = Gp * dq.y, acc_q[4 * u + 2] = Gp * dq.z, acc_q[4 * u + 3] = Gp * dq.w;
     vf[u] = bf16x4(s_v + (u >> 1) * VA + ptx::swz128(bb, 4 * (u & 1) + (l >> 1)) + (l & 1) * 8);
   }
-  int U = *s_U;
-  __syncthreads();  // D1^T consumed before the deltas overwrite region A
+  __syncthreads();  // D1^T and the key rows consumed before the deltas overwrite region A
 
   // ------------------------------- after the wait: the ancestors' deltas
   ptx::pdl_wait();
@@ -497,14 +469,18 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
     const int hi = min(U, lo + kDRows);
     const int nrows = hi - lo;
     if (rnd > 0) __syncthreads();  // the previous round's deltas are consumed
-    if (tid < kDRows) {
-      const int s = lo + tid;
-      if (s < hi) {
-        const int packed = s_list[s];
+    if (warp == 0) {
+      // Lane i gathers the delta rows of slots lo + 4i .. + 3.
+      if (4 * lane < nrows) {
+        int row[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int packed = s_list[lo + 4 * lane + q];
+          row[q] = (int)rec_row(p, (packed & 31) + 1, r, h, packed >> 5);
+        }
         ptx::fence_proxy_async_smem();
-        ptx::mbar_arrive_expect_tx(bar_d, DV * 4);
-        ptx::bulk_g2s(base + L.dst + tid * DV * 4,
-                      p.rec_delta + rec_row(p, (packed & 31) + 1, r, h, packed >> 5) * DV, DV * 4, bar_d);
+        ptx::mbar_arrive_expect_tx(bar_d, 4 * DV * 4);
+        ptx::tma_gather4(base + L.dst + 4 * lane * DV * 4, &p.tm_delta, 0, row[0], row[1], row[2], row[3], bar_d);
       } else {
         ptx::mbar_arrive(bar_d);
       }
@@ -651,6 +627,19 @@ cudaError_t launch_dk(const StepParams &p_in, bool pdl, cudaStream_t s) {
 }
 
 }  // namespace
+
+bool encode_row_table(CUtensorMap *m, const void *base, int bf16, int width, long long rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+  if (!fn || rows < 1 || rows > 0x7fffffffLL) return false;
+  const int es = bf16 ? 2 : 4;
+  const cuuint64_t dims[2] = {(cuuint64_t)width, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)width * es};
+  const cuuint32_t box[2] = {(cuuint32_t)width, 1};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(base),
+            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 bool tc_supports(int dk, int dv, int qkv_bf16, int T_max, int W_max) {
   return qkv_bf16 && dk == dv && (dk == 64 || dk == 128) && T_max <= kMaxT && W_max <= kMaxW;
