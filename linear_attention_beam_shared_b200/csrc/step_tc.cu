@@ -195,7 +195,13 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
   int par = 0;
   float g_alpha = 0.f, g_beta = 0.f;
   if (warp == 1) {
-    // This tile's parents, gates and betas.
+    // The parents of steps 2..t-1 for this request, back to back, each array
+    // starting on a 16-byte boundary; this tile's parents, gates and betas.
+    if (p.hist_cap > 0)
+#pragma unroll 1
+      for (int j = 2; j < t; ++j)
+        copy_ints_warp(s_hist + p.hoff[j], p.hpar[j] + (int64_t)r * p.hpar_rs[j], p.hW[j], lane);
+    ptx::cp_async_commit();
     if (lane < nb) {
       par = nanc >= 1 ? p.parents[r * p.W + b0 + lane] : 0;
       const int64_t si = row0 + (int64_t)lane * H;
@@ -262,13 +268,6 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
     // parent; a[j] is the parent, at step j + 2, of a[j + 1]), the entries of
     // depth t that need no delta, and the distinct ancestors of the tile.
     const int b = lane;
-    // The parents of steps 2..t-1 for this request, back to back, each array
-    // starting on a 16-byte boundary.
-    if (p.hist_cap > 0)
-#pragma unroll 1
-      for (int j = 2; j < t; ++j)
-        copy_ints_warp(s_hist + p.hoff[j], p.hpar[j] + (int64_t)r * p.hpar_rs[j], p.hW[j], lane);
-    ptx::cp_async_commit();
     ptx::cp_async_wait_all();
     __syncwarp();
     if (b < nb && nanc >= 1 && (par < 0 || par >= p.W_prev)) {
@@ -419,34 +418,46 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
       if (warp == 0) stage_keys(lo, nrows, lane);
     }
     if (!ptx::mbar_wait(bar_keys, rnd & 1, kWaitLimitNs)) ok = false;
+    // Two depths per pass: independent loads and shuffle chains interleave.
 #pragma unroll 1
-    for (int j = 0; j < nanc; ++j) {
-      const int slot = bval ? s_slot[bb * TM + j] : -1;
-      const unsigned sl = (unsigned)(slot - lo);
-      const bool in = sl < (unsigned)nrows;
-      const uint8_t *row = s_keys + (in ? sl : 0u) * (DK * 2) + l * 8;
-      float dk = 0.f, dq = 0.f;
+    for (int j0 = 0; j0 < nanc; j0 += 2) {
+      float dk[2], dq[2];
+      int slot[2];
+      bool in[2];
 #pragma unroll
-      for (int u = 0; u < NU; ++u) {
-        const float4 kf = bf16x4(row + u * 64);
-        dk = fmaf(kf.x, kb[u].x, dk);
-        dk = fmaf(kf.y, kb[u].y, dk);
-        dk = fmaf(kf.z, kb[u].z, dk);
-        dk = fmaf(kf.w, kb[u].w, dk);
-        dq = fmaf(kf.x, qb[u].x, dq);
-        dq = fmaf(kf.y, qb[u].y, dq);
-        dq = fmaf(kf.z, qb[u].z, dq);
-        dq = fmaf(kf.w, qb[u].w, dq);
+      for (int e = 0; e < 2; ++e) {
+        const int j = j0 + e;
+        slot[e] = bval && j < nanc ? s_slot[bb * TM + j] : -1;
+        const unsigned sl = (unsigned)(slot[e] - lo);
+        in[e] = sl < (unsigned)nrows;
+        const uint8_t *row = s_keys + (in[e] ? sl : 0u) * (DK * 2) + l * 8;
+        dk[e] = 0.f, dq[e] = 0.f;
+#pragma unroll
+        for (int u = 0; u < NU; ++u) {
+          const float4 kf = bf16x4(row + u * 64);
+          dk[e] = fmaf(kf.x, kb[u].x, dk[e]);
+          dk[e] = fmaf(kf.y, kb[u].y, dk[e]);
+          dk[e] = fmaf(kf.z, kb[u].z, dk[e]);
+          dk[e] = fmaf(kf.w, kb[u].w, dk[e]);
+          dq[e] = fmaf(kf.x, qb[u].x, dq[e]);
+          dq[e] = fmaf(kf.y, qb[u].y, dq[e]);
+          dq[e] = fmaf(kf.z, qb[u].z, dq[e]);
+          dq[e] = fmaf(kf.w, qb[u].w, dq[e]);
+        }
       }
 #pragma unroll
-      for (int o = 4; o > 0; o >>= 1) {
-        dk += __shfl_xor_sync(0xffffffffu, dk, o);
-        dq += __shfl_xor_sync(0xffffffffu, dq, o);
-      }
-      if (in && l == 0) {
-        const float w = s_w[bb * TM + j];
-        s_c[bb * TM + j] = make_float4(dk * w, dq * w, __int_as_float(slot), 0.f);
-      }
+      for (int o = 4; o > 0; o >>= 1)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          dk[e] += __shfl_xor_sync(0xffffffffu, dk[e], o);
+          dq[e] += __shfl_xor_sync(0xffffffffu, dq[e], o);
+        }
+#pragma unroll
+      for (int e = 0; e < 2; ++e)
+        if (in[e] && l == 0) {
+          const float w = s_w[bb * TM + j0 + e];
+          s_c[bb * TM + j0 + e] = make_float4(dk[e] * w, dq[e] * w, __int_as_float(slot[e]), 0.f);
+        }
     }
   }
   // u = P(p) D1 + (replayed terms, after the wait); v from its tile.
