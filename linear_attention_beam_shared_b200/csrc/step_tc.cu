@@ -55,6 +55,7 @@ constexpr int kM = 128;             // MMA M
 constexpr int kDRows = 128;         // ancestor deltas per staging round after the wait (32 groups of 4)
 constexpr int kTmemCols = 64;       // D1
 constexpr int kKeyRows = 128;       // ancestor key rows per staging round
+constexpr uint32_t kTabBytes = 2u * 8u * kHistSteps + 3u * 4u * kHistSteps;  // per-step table
 constexpr int kMaxT = 16;           // deepest decode the kernel serves
 constexpr int kMaxW = 1024;         // widest beam set the kernel serves
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far beyond any legal wait
@@ -84,9 +85,10 @@ __host__ __device__ inline Layout layout(int nk, int planes, int TM, int W_max, 
   // 128 B of barriers and counters; 4 per-beam scalars; per (beam, depth)
   // the replay coefficients (float4), the chain, slot, slot-list ints and
   // weights (the slot list 4 TM longer); a beam-index scratch [W_max]; the
-  // parents of steps 2..t-1.
+  // parents of steps 2..t-1; the per-step table (2 pointers and 3 ints per
+  // step).
   L.total = L.book + 128u + 4u * kBT * 4u + (uint32_t)kBT * TM * 16u + (4u * kBT + 4u) * TM * 4u +
-            (uint32_t)((W_max + 3) & ~3) * 4u + (uint32_t)((hist_cap + 3) & ~3) * 4u + 16u;
+            (uint32_t)((W_max + 3) & ~3) * 4u + (uint32_t)((hist_cap + 3) & ~3) * 4u + kTabBytes + 16u;
   return L;
 }
 
@@ -159,6 +161,14 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
   float *s_w = reinterpret_cast<float *>(s_list + (kBT + 4) * TM);  // [32][TM] replay weight by depth
   int *s_seen = reinterpret_cast<int *>(s_w + kBT * TM);           // beam index -> a lane (scratch)
   int *s_hist = s_seen + ((p.W_max + 3) & ~3);                 // parents of steps 2..t-1
+  // Per-step table (index = step j), filled by warp 1 before the first
+  // barrier with one load per lane: loops then read shared memory instead
+  // of indexing the parameters at run time.
+  const int32_t **s_tpar = reinterpret_cast<const int32_t **>(s_hist + ((p.hist_cap + 3) & ~3));
+  const float **s_tg = reinterpret_cast<const float **>(s_tpar + kHistSteps);
+  int *s_toff = reinterpret_cast<int *>(s_tg + kHistSteps);
+  int *s_tW = s_toff + kHistSteps;
+  int *s_trs = s_tW + kHistSteps;
   uint8_t *s_keys = base + L.ka;                               // key rows [kKeyRows][d_k] bf16
   static_assert(kKeyRows * DK * 2 <= NK * 16384, "the key rows must fit in their area");
 
@@ -192,25 +202,37 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
     ptx::tmem_alloc(s_tmem, kTmemCols);
     ptx::tmem_relinquish();
   }
+  // Before its wait this kernel reads inputs only, so the next step may start.
+  ptx::pdl_launch_dependents();
   int par = 0;
   float g_alpha = 0.f, g_beta = 0.f;
   if (warp == 1) {
-    // The parents of steps 2..t-1 for this request, back to back, each array
-    // starting on a 16-byte boundary; this tile's parents, gates and betas.
-    if (p.hist_cap > 0)
-#pragma unroll 1
-      for (int j = 2; j < t; ++j)
-        copy_ints_warp(s_hist + p.hoff[j], p.hpar[j] + (int64_t)r * p.hpar_rs[j], p.hW[j], lane);
-    ptx::cp_async_commit();
+    // This tile's parents, gates and betas; the per-step table (lane j loads
+    // step j: one load per lane, then loops read shared memory instead of
+    // indexing the parameters at run time).
     if (lane < nb) {
       par = nanc >= 1 ? p.parents[r * p.W + b0 + lane] : 0;
       const int64_t si = row0 + (int64_t)lane * H;
       g_alpha = p.g[si];
       g_beta = p.beta[si];
     }
+    if (lane < kHistSteps) {
+      s_tpar[lane] = p.hpar[lane];
+      s_tg[lane] = p.hg[lane];
+      s_toff[lane] = p.hoff[lane];
+      s_tW[lane] = p.hW[lane];
+      s_trs[lane] = p.hpar_rs[lane];
+    }
   }
-  // Before its wait this kernel reads inputs only, so the next step may start.
-  ptx::pdl_launch_dependents();
+  // The parents of steps 2..t-1 for this request, back to back, each array
+  // starting on a 16-byte boundary: warp w >= 1 copies steps w + 1, w + 8.
+  // Every thread waits for its own copies before the barrier below.
+  if (p.hist_cap > 0 && warp >= 1)
+#pragma unroll 1
+    for (int j = warp + 1; j < t; j += kThreads / 32 - 1)
+      copy_ints_warp(s_hist + p.hoff[j], p.hpar[j] + (int64_t)r * p.hpar_rs[j], p.hW[j], lane);
+  ptx::cp_async_commit();
+  ptx::cp_async_wait_all();
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
@@ -226,7 +248,7 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
     if (4 * i < n) {
       const int s0 = lo + 4 * i;
       const int j = s_list[s0] & 31;
-      const int Wj = p.hW[j + 1];
+      const int Wj = s_tW[j + 1];
       int row[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -268,8 +290,6 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
     // parent; a[j] is the parent, at step j + 2, of a[j + 1]), the entries of
     // depth t that need no delta, and the distinct ancestors of the tile.
     const int b = lane;
-    ptx::cp_async_wait_all();
-    __syncwarp();
     if (b < nb && nanc >= 1 && (par < 0 || par >= p.W_prev)) {
       *reinterpret_cast<volatile int32_t *>(p.err) = kErrParent;
       par = 0;
@@ -283,8 +303,8 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
       s_chain[b * TM + jp] = a;
 #pragma unroll 1
       for (int j = jp - 1; j >= 0; --j) {
-        int pa = p.hist_cap > 0 ? s_hist[p.hoff[j + 2] + a] : p.hpar[j + 2][(int64_t)r * p.hpar_rs[j + 2] + a];
-        if (pa < 0 || pa >= p.hW[j + 1]) pa = 0;  // reported by step j + 2
+        int pa = p.hist_cap > 0 ? s_hist[s_toff[j + 2] + a] : s_tpar[j + 2][(int64_t)r * s_trs[j + 2] + a];
+        if (pa < 0 || pa >= s_tW[j + 1]) pa = 0;  // reported by step j + 2
         a = pa;
         s_chain[b * TM + j] = a;
       }
@@ -338,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
 #pragma unroll 1
       for (int j = 0; j <= jp; ++j) {
         const int a = s_chain[b * TM + j];
-        ptx::cp_async4(s_w + b * TM + j, hin ? p.hg[j + 1] + ((int64_t)r * p.hW[j + 1] + a) * H + h
+        ptx::cp_async4(s_w + b * TM + j, hin ? s_tg[j + 1] + ((int64_t)r * s_tW[j + 1] + a) * H + h
                                              : p.rec_alpha + rec_row(p, j + 1, r, h, a));
       }
     }
