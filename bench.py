@@ -81,11 +81,17 @@ def measured_peaks():
 
 
 def kernel_source_hash():
+    """Hash of the kernel sources with comments and blank lines removed, so
+    that a change of wording alone keeps the recorded counters valid."""
+    import re
     h = hashlib.sha256()
     for p in sorted(glob.glob(os.path.join(ROOT, "linear_attention_beam_shared_b200", "csrc", "*"))):
-        with open(p, "rb") as f:
-            h.update(os.path.basename(p).encode())
-            h.update(f.read())
+        with open(p, "r", encoding="utf-8", errors="replace") as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = "\n".join(line.split("//")[0].rstrip() for line in text.splitlines() if line.split("//")[0].strip())
+        h.update(os.path.basename(p).encode())
+        h.update(text.encode())
     return h.hexdigest()[:16]
 
 

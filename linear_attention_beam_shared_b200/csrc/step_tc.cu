@@ -22,22 +22,28 @@
 //                   tile (the abstract's shared-state reuse across beams);
 //                   fp32 S0 is split once, when the prompt state is
 //                   installed, into two or three bf16 terms.
-//   D2 = KA . X^T   tensor cores: k_a . x for every distinct ancestor a of
-//                   the tile (KA: their keys).
-//   replay         fp32 FMAs, one thread per (beam, eighth of the elements).
+//   k_a . x         fp32 FMAs: the distinct ancestors' key rows are gathered
+//                   into shared memory (4 rows per TMA instruction) and
+//                   every beam's 8 threads form k_a . k_b, k_a . q_b and
+//                   k_b . q_b, reducing by shuffles.
+//   replay          fp32 FMAs, one thread per (beam, eighth of the elements).
 //
 // Only the deltas are outputs of earlier steps; ancestors (from the parents
 // of every step), their keys and their gates are inputs.  So each kernel
 // lets its dependent launch start at once, and before its
 // griddepcontrol.wait it reads inputs only: the callers' arrays of the
 // earlier steps under ONELA_FLAG_PDL, the record store otherwise (then the
-// earlier steps have completed).  It computes D1, the ancestry (parent
-// indices only; records never move, abstract), D2 and every weight, and
-// writes the depth-t entries that need
-// no delta (alpha, k, the ancestry row).  After the wait it stages the
-// distinct ancestors' deltas with one round of bulk copies, replays, and
-// writes o and delta.  No kernel reads a depth-t entry before step t has
-// completed, so the early writes race with nothing.
+// earlier steps have completed).  Warp roles (hand-offs on mbarriers with
+// bounded waits): warp 0 issues the loads and D1; warp 1 builds each beam's
+// ancestor chain (parent indices only; records never move, abstract), the
+// tile's distinct ancestors and the depth-t entries that need no delta
+// (alpha, the ancestry row); warp 2 gathers the gates along each chain into
+// the replay weights; warp 3 writes the key records; warps 4-7 stage the
+// ancestors' key rows and move D1 to shared memory.  Then all threads form
+// the key products.  After the wait the ancestors' delta rows arrive in one
+// round of 4-row gathers, every thread replays and writes o and delta.  No
+// kernel reads a depth-t entry before step t has completed, so the early
+// writes race with nothing.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cudaTypedefs.h>
