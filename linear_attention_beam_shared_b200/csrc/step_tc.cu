@@ -246,10 +246,10 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
 
   bool ok = true;
   const uint32_t x_u32 = ptx::smem_u32(s_x), a_u32 = ptx::smem_u32(base + L.a);
-  // Key rows of slots [lo, lo + n) (n a multiple of 4) into s_keys, by the
-  // 32 lanes of one warp: lane i gathers the 4 rows of slots lo + 4i .. + 3
+  // Key rows of slots [lo, lo + n) (n a multiple of 4) into s_keys, by 32
+  // callers i = 0..31: caller i gathers the 4 rows of slots lo + 4i .. + 3
   // (one depth: the slots of a depth start on a multiple of 4) from that
-  // depth's row table.  Every lane arrives on bar_keys once.
+  // depth's row table.  Every caller arrives on bar_keys once.
   auto stage_keys = [&](int lo, int n, int i) {
     if (4 * i < n) {
       const int s0 = lo + 4 * i;
@@ -397,7 +397,7 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
     if (!ptx::mbar_wait(bar1, 0, kWaitLimitNs)) ok = false;  // region A is free
     ptx::tc_fence_after();
     if (!ptx::mbar_wait(bar_slots, 0, kWaitLimitNs)) ok = false;
-    if (warp == 4) stage_keys(0, min(*s_U, kKeyRows), lane);
+    if (lane < 8) stage_keys(0, min(*s_U, kKeyRows), wq * 8 + lane);  // 8 groups per warp
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
       float d[32];
@@ -524,23 +524,31 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
     }
     if (!ptx::mbar_wait(bar_d, rnd & 1, kWaitLimitNs)) ok = false;
     if (bb < nb) {
-      for (int j = 0; j < nanc; ++j) {
-        const float4 c = s_c[bb * TM + j];
-        const unsigned sl = (unsigned)(__float_as_int(c.z) - lo);
-        if (sl < (unsigned)nrows) {
-          const float4 *row = reinterpret_cast<const float4 *>(s_dst + sl * DV) + l;
+      // Two depths per pass: their loads are independent.
+#pragma unroll 1
+      for (int j0 = 0; j0 < nanc; j0 += 2) {
+        float4 c[2];
+        bool in[2];
+        const float4 *row[2];
 #pragma unroll
-          for (int u = 0; u < NU; ++u) {
-            const float4 d = row[8 * u];
-            acc_k[4 * u + 0] = fmaf(d.x, c.x, acc_k[4 * u + 0]);
-            acc_k[4 * u + 1] = fmaf(d.y, c.x, acc_k[4 * u + 1]);
-            acc_k[4 * u + 2] = fmaf(d.z, c.x, acc_k[4 * u + 2]);
-            acc_k[4 * u + 3] = fmaf(d.w, c.x, acc_k[4 * u + 3]);
-            acc_q[4 * u + 0] = fmaf(d.x, c.y, acc_q[4 * u + 0]);
-            acc_q[4 * u + 1] = fmaf(d.y, c.y, acc_q[4 * u + 1]);
-            acc_q[4 * u + 2] = fmaf(d.z, c.y, acc_q[4 * u + 2]);
-            acc_q[4 * u + 3] = fmaf(d.w, c.y, acc_q[4 * u + 3]);
-          }
+        for (int e = 0; e < 2; ++e) {
+          c[e] = j0 + e < nanc ? s_c[bb * TM + j0 + e] : make_float4(0.f, 0.f, __int_as_float(-1), 0.f);
+          const unsigned sl = (unsigned)(__float_as_int(c[e].z) - lo);
+          in[e] = sl < (unsigned)nrows;
+          row[e] = reinterpret_cast<const float4 *>(s_dst + (in[e] ? sl : 0u) * DV) + l;
+          if (!in[e]) c[e].x = c[e].y = 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < NU; ++u) {
+          const float4 d0 = row[0][8 * u], d1 = row[1][8 * u];
+          acc_k[4 * u + 0] = fmaf(d1.x, c[1].x, fmaf(d0.x, c[0].x, acc_k[4 * u + 0]));
+          acc_k[4 * u + 1] = fmaf(d1.y, c[1].x, fmaf(d0.y, c[0].x, acc_k[4 * u + 1]));
+          acc_k[4 * u + 2] = fmaf(d1.z, c[1].x, fmaf(d0.z, c[0].x, acc_k[4 * u + 2]));
+          acc_k[4 * u + 3] = fmaf(d1.w, c[1].x, fmaf(d0.w, c[0].x, acc_k[4 * u + 3]));
+          acc_q[4 * u + 0] = fmaf(d1.x, c[1].y, fmaf(d0.x, c[0].y, acc_q[4 * u + 0]));
+          acc_q[4 * u + 1] = fmaf(d1.y, c[1].y, fmaf(d0.y, c[0].y, acc_q[4 * u + 1]));
+          acc_q[4 * u + 2] = fmaf(d1.z, c[1].y, fmaf(d0.z, c[0].y, acc_q[4 * u + 2]));
+          acc_q[4 * u + 3] = fmaf(d1.w, c[1].y, fmaf(d0.w, c[0].y, acc_q[4 * u + 3]));
         }
       }
     }
