@@ -51,12 +51,6 @@ struct StepParams {
   alignas(64) CUtensorMap tm_k;
   alignas(64) CUtensorMap tm_q;
   alignas(64) CUtensorMap tm_v;
-  // Row tables for 4-row gathers (tensor-core kernel): the delta records
-  // [T_max R H W_max][d_v] fp32, and per earlier step j the table its
-  // ancestors' key rows come from -- step j's own k input [R W_j H][d_k]
-  // (hist_inputs = 1) or the key records [T_max R H W_max][d_k].
-  alignas(64) CUtensorMap tm_delta;
-  alignas(64) CUtensorMap tm_krows[kHistSteps];
 };
 
 // Row index of the record of beam b, head h, request r at depth s (1-based).
@@ -74,9 +68,6 @@ constexpr int32_t kErrParent = 1;
 // Kernel launchers (step_simt.cu, step_tc.cu).  Return a cudaError_t.
 cudaError_t launch_step_simt(const StepParams &p, int qkv_bf16, int s0_bf16, cudaStream_t s);
 cudaError_t launch_step_tc(const StepParams &p, int pdl, cudaStream_t s);
-// A 2-D TMA map over `rows` rows of `width` elements (bf16 or fp32), with a
-// box of one row: the row table the tensor-core kernel gathers from.
-bool encode_row_table(CUtensorMap *m, const void *base, int bf16, int width, long long rows);
 cudaError_t launch_s0_image(const void *S0, void *img, int R, int H, int dk, int dv,
                             int s0_bf16, int planes, cudaStream_t s);
 size_t s0_image_bytes(int R, int H, int dk, int dv, int planes);

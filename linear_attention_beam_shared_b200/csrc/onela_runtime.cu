@@ -25,9 +25,6 @@ struct onela_handle {
   std::vector<const void *> hist_k;
   std::vector<const float *> hist_g;
   std::vector<const int32_t *> hist_par;
-  std::vector<CUtensorMap> hist_tmk;  // row table of every earlier call's k (tensor-core kernel)
-  CUtensorMap tm_delta;               // row tables of the delta and key records (tensor-core kernel)
-  CUtensorMap tm_reck;
   float *rec_alpha;
   float *rec_delta;
   void *rec_k;
@@ -156,10 +153,6 @@ int onela_create(const onela_config *cfg, onela_handle **out) {
          cudaMemset(h->anc, 0, (size_t)c.T_max * c.R * c.W_max * c.T_max * sizeof(int32_t)) == cudaSuccess &&
          cudaDeviceSynchronize() == cudaSuccess;
   }
-  if (ok && kernel == ONELA_KERNEL_TC) {
-    ok = onela::encode_row_table(&h->tm_delta, h->rec_delta, 0, c.d_v, (long long)nrow) &&
-         onela::encode_row_table(&h->tm_reck, h->rec_k, 1, c.d_k, (long long)nrow);
-  }
   if (!ok) {
     cudaGetLastError();
     free_all(h);
@@ -189,7 +182,6 @@ int onela_set_prompt_state(onela_handle *h, const void *S0, onela_stream stream)
   h->hist_k.clear();
   h->hist_g.clear();
   h->hist_par.clear();
-  h->hist_tmk.clear();
   return ONELA_OK;
 }
 
@@ -230,11 +222,9 @@ int onela_decode_step(onela_handle *h, int32_t W_prev, int32_t W, const void *q,
     // ONELA_FLAG_PDL (still valid by its contract), else the record store
     // and the parents the earlier kernels stored (they have completed).
     p.hist_inputs = pdl ? 1 : 0;
-    p.tm_delta = h->tm_delta;
     int hist = 0;
     for (int j = 1; j < p.t; ++j) {
       p.hW[j] = h->Ws[j - 1];
-      p.tm_krows[j] = pdl ? h->hist_tmk[j - 1] : h->tm_reck;
       if (pdl) {
         p.hk[j] = h->hist_k[j - 1];
         p.hg[j] = h->hist_g[j - 1];
@@ -250,11 +240,6 @@ int onela_decode_step(onela_handle *h, int32_t W_prev, int32_t W, const void *q,
       }
     }
     p.hist_cap = hist <= onela::kHistMaxInts ? hist : 0;
-    // This step's k as a row table, for the steps after it.
-    CUtensorMap tmk;
-    if (!onela::encode_row_table(&tmk, k, 1, c.d_k, (long long)c.R * W * c.H)) return ONELA_ERR_ARG;
-    h->hist_tmk.resize(p.t);
-    h->hist_tmk[p.t - 1] = tmk;
   }
   if (h->kernel == ONELA_KERNEL_TC)
     e = onela::launch_step_tc(p, pdl, s);
@@ -284,7 +269,6 @@ int onela_reset(onela_handle *h, onela_stream stream) {
   h->hist_k.clear();
   h->hist_g.clear();
   h->hist_par.clear();
-  h->hist_tmk.clear();
   return ONELA_OK;
 }
 

@@ -29,10 +29,6 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                : "memory");
 }
-// Hardware named barrier `id` (1..15) over `count` threads (a multiple of 32).
-__device__ __forceinline__ void named_sync(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
@@ -68,28 +64,7 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
       : "memory");
 }
 
-// Untiled bulk copy shared -> global (TMA store), tracked by bulk groups.
-__device__ __forceinline__ void bulk_s2g(void *dst, const void *src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(smem_u32(src)),
-               "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// Wait until the shared-memory sources of this thread's bulk stores have been read.
-__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-
 // Tiled TMA load of a 4-D box (no multicast); completes its bytes on bar.
-// Four rows r0..r3 of a 2-D tensor map (box: one row of the map's width,
-// starting at column col) into consecutive rows at dst (tile::gather4).
-__device__ __forceinline__ void tma_gather4(void *dst, const void *tmap, int col, int r0, int r1, int r2, int r3,
-                                            uint64_t *bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cta.global.tile::gather4.mbarrier::complete_tx::bytes [%0], "
-      "[%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
-      "l"(tmap), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(smem_u32(bar))
-      : "memory");
-}
-
 __device__ __forceinline__ void tma_load_4d(void *dst, const void *tmap, int c0, int c1, int c2, int c3,
                                             uint64_t *bar) {
   asm volatile(
@@ -97,12 +72,6 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const void *tmap, int c0,
       "[%6];" ::"r"(smem_u32(dst)),
       "l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
       : "memory");
-}
-
-// Make this thread's generic-proxy shared-memory writes visible to the async
-// proxy (tensor-core operand reads).
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // 16-byte asynchronous copy global -> shared (L2 only); src_bytes = 0 writes
@@ -162,19 +131,6 @@ __device__ __forceinline__ void mma_commit(uint64_t *bar) {
                : "memory");
 }
 
-// 32 lanes x 32 bit, 16 consecutive columns: thread i of the warp receives
-// columns [col, col + 16) of TMEM lane (lane base of the warp) + i.
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
-  uint32_t r[16];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-#pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-}
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // Shared-memory matrix descriptor, K-major, 128-byte swizzle: rows of 128 B
@@ -196,26 +152,9 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          | ((uint32_t)(M >> 4) << 24);  // M / 16
 }
 
-// Shared-memory matrix descriptor, MN-major (M or N contiguous), 128-byte
-// swizzle: 128-byte rows of 64 16-bit elements along M/N, one row per K
-// index; 8 K rows form a 1024-byte atom.  sbo = byte stride between groups of
-// 8 K rows, lbo = byte stride between 64-element groups along M/N.
-__device__ __forceinline__ uint64_t desc_mn128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-  return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
-         ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
 
-// Instruction descriptor: fp16 x fp16 -> fp32, A MN-major, B K-major.
-__host__ __device__ constexpr uint32_t idesc_f16_amn_f32(int M, int N) {
-  return (1u << 4)                      // D: fp32
-         | (0u << 7)                    // A: fp16
-         | (0u << 10)                   // B: fp16
-         | (1u << 15)                   // A is MN-major
-         | ((uint32_t)(N >> 3) << 17)   // N / 8
-         | ((uint32_t)(M >> 4) << 24);  // M / 16
-}
-
-// 32 lanes x 32 bit, 32 consecutive columns.
+// 32 lanes x 32 bit, 32 consecutive columns: thread i of the warp receives
+// columns [col, col + 32) of TMEM lane (lane base of the warp) + i.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   uint32_t r[32];
   asm volatile(

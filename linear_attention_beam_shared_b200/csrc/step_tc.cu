@@ -1,11 +1,12 @@
 // Tensor-core decode-step kernel (tcgen05, sm_100a) for bf16 q/k/v and
 // d_k = d_v in {64, 128}.
 //
-// One CTA per (request r, head h, tile of 32 beams); 256 threads; two CTAs
-// fit on an SM.  The step of the shared-state GDN beam decode (OneLA,
-// evolve.pub review, key claims on section 3.2, equations 2-4).  For beam b
-// with ancestors a_1 .. a_{t-1} (a_{t-1} = p, its parent) and P(a) the
-// product of the gates on the path from the root to record a:
+// One CTA per (request r, head h, tile of 32 beams); 320 threads (8 beam
+// warps, an ancestry warp and an MMA warp); two CTAs fit on an SM.  The step
+// of the shared-state GDN beam decode (OneLA, evolve.pub review, key claims
+// on section 3.2, equations 2-4).  For beam b with ancestors a_1 .. a_{t-1}
+// (a_{t-1} = p, its parent) and P(a) the product of the gates on the path
+// from the root to record a:
 //
 //   S_{t-1} x = P(p) S0 x + sum_j delta_{a_j} w_j (k_{a_j} . x),
 //   w_j = alpha_{a_{j+1}} ... alpha_{a_{t-1}}   (w = 1 for the parent),
@@ -22,28 +23,27 @@
 //                   tile (the abstract's shared-state reuse across beams);
 //                   fp32 S0 is split once, when the prompt state is
 //                   installed, into two or three bf16 terms.
-//   k_a . x         fp32 FMAs: the distinct ancestors' key rows are gathered
-//                   into shared memory (4 rows per TMA instruction) and
-//                   every beam's 8 threads form k_a . k_b, k_a . q_b and
-//                   k_b . q_b, reducing by shuffles.
-//   replay          fp32 FMAs, one thread per (beam, eighth of the elements).
+//   k_a . x         fp32 FMAs: every beam's 8 threads load their pieces of
+//                   each ancestor's key row from global memory and reduce
+//                   k_a . k_b, k_a . q_b by shuffles.
+//   replay          fp32 FMAs, one thread per (beam, eighth of the elements),
+//                   over the distinct ancestors' delta rows staged in shared
+//                   memory.
 //
 // Only the deltas are outputs of earlier steps; ancestors (from the parents
 // of every step), their keys and their gates are inputs.  So each kernel
 // lets its dependent launch start at once, and before its
 // griddepcontrol.wait it reads inputs only: the callers' arrays of the
 // earlier steps under ONELA_FLAG_PDL, the record store otherwise (then the
-// earlier steps have completed).  Warp roles (hand-offs on mbarriers with
-// bounded waits): warp 0 issues the loads and D1; warp 1 builds each beam's
-// ancestor chain (parent indices only; records never move, abstract), the
-// tile's distinct ancestors and the depth-t entries that need no delta
-// (alpha, the ancestry row); warp 2 gathers the gates along each chain into
-// the replay weights; warp 3 writes the key records; warps 4-7 stage the
-// ancestors' key rows and move D1 to shared memory.  Then all threads form
-// the key products.  After the wait the ancestors' delta rows arrive in one
-// round of 4-row gathers, every thread replays and writes o and delta.  No
-// kernel reads a depth-t entry before step t has completed, so the early
-// writes race with nothing.
+// earlier steps have completed).  Before the wait: the ancestry warp builds
+// each beam's ancestor chain (parent indices only; records never move,
+// abstract), then the tile's distinct ancestors and the replay weights; the
+// MMA warp issues D1 as soon as the image is in; the beam warps form the key
+// products as soon as the chains exist, then move D1 to shared memory and
+// write the entries of depth t that need no delta.  After the wait the
+// ancestors' delta rows arrive in one round of 16-byte copies, every beam
+// thread replays and writes o and delta.  No kernel reads a depth-t entry
+// before step t has completed, so the early writes race with nothing.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cudaTypedefs.h>
@@ -54,14 +54,15 @@
 namespace onela {
 namespace {
 
-constexpr int kThreads = 256;       // 8 warps
+constexpr int kThreads = 320;       // 8 beam warps, the ancestry warp and the MMA warp
+constexpr int kAncWarp = 8;         // the ancestry warp
+constexpr int kMmaWarp = 9;         // the MMA warp
 constexpr int kBT = 32;             // beams per CTA
 constexpr int kN = 2 * kBT;         // vectors: k rows 0..31, q rows 32..63
 constexpr int kM = 128;             // MMA M
-constexpr int kDRows = 128;         // ancestor deltas per staging round after the wait (32 groups of 4)
+constexpr int kDRows = 128;         // ancestor deltas per staging round after the wait
 constexpr int kTmemCols = 64;       // D1
-constexpr int kKeyRows = 128;       // ancestor key rows per staging round
-constexpr uint32_t kTabBytes = 2u * 8u * kHistSteps + 3u * 4u * kHistSteps;  // per-step table
+constexpr uint32_t kTabBytes = 3u * 8u * kHistSteps + 3u * 4u * kHistSteps;  // per-step table
 constexpr int kMaxT = 16;           // deepest decode the kernel serves
 constexpr int kMaxW = 1024;         // widest beam set the kernel serves
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far beyond any legal wait
@@ -70,8 +71,7 @@ constexpr int32_t kErrTimeout = 2;
 struct Layout {
   uint32_t x;     // X [NK][64 rows][128 B]: k rows, then q rows
   uint32_t v;     // v [NK][32 rows][128 B]
-  uint32_t a;     // region A: the S0 image; then KA and D1^T; then the deltas
-  uint32_t ka;    // keys of a D2 block [NK][128 rows][128 B]
+  uint32_t a;     // region A: the S0 image; then D1^T; then the deltas
   uint32_t d1;    // D1^T [64 vectors][d_v] fp32
   uint32_t dst;   // ancestor deltas [kDRows][d_v] fp32
   uint32_t book;  // barriers and bookkeeping
@@ -83,17 +83,15 @@ __host__ __device__ inline Layout layout(int nk, int planes, int TM, int W_max, 
   L.x = 0;
   L.v = (uint32_t)nk * 8192u;
   L.a = (uint32_t)nk * 12288u;
-  L.ka = L.a;
   L.d1 = L.a + (uint32_t)nk * 16384u;
   L.dst = L.a;
   const uint32_t s0 = (uint32_t)planes * nk * 16384u, ops = (uint32_t)nk * 32768u;
   L.book = L.a + (s0 > ops ? s0 : ops);
   // 128 B of barriers and counters; 4 per-beam scalars; per (beam, depth)
-  // the replay coefficients (float4), the chain, slot, slot-list ints and
-  // weights (the slot list 4 TM longer); a beam-index scratch [W_max]; the
-  // parents of steps 2..t-1; the per-step table (2 pointers and 3 ints per
-  // step).
-  L.total = L.book + 128u + 4u * kBT * 4u + (uint32_t)kBT * TM * 16u + (4u * kBT + 4u) * TM * 4u +
+  // the replay coefficients (float4), the chain, slot-list ints and gates
+  // (the slot list 4 TM longer); a beam-index scratch [W_max]; the parents
+  // of steps 2..t-1; the per-step table (3 pointers and 3 ints per step).
+  L.total = L.book + 128u + 4u * kBT * 4u + (uint32_t)kBT * TM * 16u + (3u * kBT + 4u) * TM * 4u +
             (uint32_t)((W_max + 3) & ~3) * 4u + (uint32_t)((hist_cap + 3) & ~3) * 4u + kTabBytes + 16u;
   return L;
 }
@@ -109,13 +107,13 @@ __device__ __forceinline__ void copy_ints_warp(int *dst, const int32_t *src, int
   for (int e = done + lane; e < n; e += 32) ptx::cp_async4(dst + e, src + e);
 }
 
-// Four consecutive bf16 elements at p (8-byte aligned) as floats.
-__device__ __forceinline__ float4 bf16x4(const uint8_t *p) {
-  const uint2 u = *reinterpret_cast<const uint2 *>(p);
+// Four consecutive bf16 elements (packed in u, or at p, 8-byte aligned) as floats.
+__device__ __forceinline__ float4 bf16x4(uint2 u) {
   const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
   const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
   return make_float4(a.x, a.y, b.x, b.y);
 }
+__device__ __forceinline__ float4 bf16x4(const uint8_t *p) { return bf16x4(*reinterpret_cast<const uint2 *>(p)); }
 
 template <int DK>
 __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_constant__ StepParams p) {
@@ -145,38 +143,31 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
   uint64_t *bars = reinterpret_cast<uint64_t *>(base + L.book);
   uint64_t *bar_s0 = bars + 0;     // S0 image, X and v landed
   uint64_t *bar1 = bars + 1;       // D1 complete
-  uint64_t *bar_d = bars + 3;      // ancestor deltas landed
-  uint64_t *bar_chain = bars + 4;  // warp 1: every beam's chain in s_chain
-  uint64_t *bar_slots = bars + 5;  // warp 1: slots, slot list and U
-  uint64_t *bar_w = bars + 6;      // warp 2: replay weights and P(p)
-  uint64_t *bar_keys = bars + 7;   // key rows of the current round landed
+  uint64_t *bar_chain = bars + 2;  // ancestry warp: every beam's chain in s_chain
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(base + L.book + 64);
   int *s_U = reinterpret_cast<int *>(s_tmem + 1);
   int *s_par = reinterpret_cast<int *>(base + L.book + 128);
   float *s_alpha = reinterpret_cast<float *>(s_par + kBT);
   float *s_beta = s_alpha + kBT;
   float *s_Gp = s_beta + kBT;  // P(parent)
-  // [32][TM]: (w k_a . k_b, w k_a . q_b, slot of a) for the ancestor a of
-  // beam b at each depth.
+  // [32][TM]: (k_a . k_b, k_a . q_b, slot of a, replay weight of a) for the
+  // ancestor a of beam b at each depth.  The beam warps write the first two
+  // words, the ancestry warp the last two.
   float4 *s_c = reinterpret_cast<float4 *>(s_Gp + kBT);
   int *s_chain = reinterpret_cast<int *>(s_c + kBT * TM);  // [32][TM] ancestor beam by depth
-  int *s_slot = s_chain + kBT * TM;                         // [32][TM] ancestor slot by depth
-  // slot -> (beam << 5 | depth-1); every depth's slots start on a multiple
-  // of 4 (padding slots repeat the depth's first ancestor), [(32 + 4) TM].
-  int *s_list = s_slot + kBT * TM;
-  float *s_w = reinterpret_cast<float *>(s_list + (kBT + 4) * TM);  // [32][TM] replay weight by depth
+  int *s_list = s_chain + kBT * TM;  // slot -> (beam << 5 | depth-1), [(32 + 4) TM]
+  float *s_w = reinterpret_cast<float *>(s_list + (kBT + 4) * TM);  // [32][TM] gates along the chains
   int *s_seen = reinterpret_cast<int *>(s_w + kBT * TM);           // beam index -> a lane (scratch)
-  int *s_hist = s_seen + ((p.W_max + 3) & ~3);                 // parents of steps 2..t-1
-  // Per-step table (index = step j), filled by warp 1 before the first
-  // barrier with one load per lane: loops then read shared memory instead
-  // of indexing the parameters at run time.
+  int *s_hist = s_seen + ((p.W_max + 3) & ~3);                      // parents of steps 2..t-1
+  // Per-step table (index = step j), filled by the ancestry warp before the
+  // first barrier with one load per lane: loops then read shared memory
+  // instead of indexing the parameters at run time.
   const int32_t **s_tpar = reinterpret_cast<const int32_t **>(s_hist + ((p.hist_cap + 3) & ~3));
   const float **s_tg = reinterpret_cast<const float **>(s_tpar + kHistSteps);
-  int *s_toff = reinterpret_cast<int *>(s_tg + kHistSteps);
+  const __nv_bfloat16 **s_tk = reinterpret_cast<const __nv_bfloat16 **>(s_tg + kHistSteps);
+  int *s_toff = reinterpret_cast<int *>(s_tk + kHistSteps);
   int *s_tW = s_toff + kHistSteps;
   int *s_trs = s_tW + kHistSteps;
-  uint8_t *s_keys = base + L.ka;                               // key rows [kKeyRows][d_k] bf16
-  static_assert(kKeyRows * DK * 2 <= NK * 16384, "the key rows must fit in their area");
 
   __nv_bfloat16 *rec_k = static_cast<__nv_bfloat16 *>(p.rec_k);
   const int64_t row0 = (int64_t)(r * p.W + b0) * H + h;  // (r, b0, h) row of [R][W][H][d]
@@ -186,11 +177,7 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
   if (tid == 0) {
     ptx::mbar_init(bar_s0, 1);
     ptx::mbar_init(bar1, 1);
-    ptx::mbar_init(bar_d, 32);
     ptx::mbar_init(bar_chain, 32);
-    ptx::mbar_init(bar_slots, 32);
-    ptx::mbar_init(bar_w, 32);
-    ptx::mbar_init(bar_keys, 32);
     ptx::mbar_fence_init();
     // S0 image (bulk copy); k, q, v tiles by TMA, beams past W read as zeros.
     ptx::mbar_arrive_expect_tx(bar_s0, s0_bytes + NK * (XA + VA));
@@ -204,7 +191,7 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
       ptx::tma_load_4d(base + L.v + ka * VA, &p.tm_v, ka * 64, h, b0, r, bar_s0);
     }
   }
-  if (warp == 3) {
+  if (warp == kMmaWarp) {
     ptx::tmem_alloc(s_tmem, kTmemCols);
     ptx::tmem_relinquish();
   }
@@ -212,10 +199,8 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
   ptx::pdl_launch_dependents();
   int par = 0;
   float g_alpha = 0.f, g_beta = 0.f;
-  if (warp == 1) {
-    // This tile's parents, gates and betas; the per-step table (lane j loads
-    // step j: one load per lane, then loops read shared memory instead of
-    // indexing the parameters at run time).
+  if (warp == kAncWarp) {
+    // This tile's parents, gates and betas, and the per-step table.
     if (lane < nb) {
       par = nanc >= 1 ? p.parents[r * p.W + b0 + lane] : 0;
       const int64_t si = row0 + (int64_t)lane * H;
@@ -225,17 +210,18 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
     if (lane < kHistSteps) {
       s_tpar[lane] = p.hpar[lane];
       s_tg[lane] = p.hg[lane];
+      s_tk[lane] = static_cast<const __nv_bfloat16 *>(p.hk[lane]);
       s_toff[lane] = p.hoff[lane];
       s_tW[lane] = p.hW[lane];
       s_trs[lane] = p.hpar_rs[lane];
     }
   }
   // The parents of steps 2..t-1 for this request, back to back, each array
-  // starting on a 16-byte boundary: warp w >= 1 copies steps w + 1, w + 8.
-  // Every thread waits for its own copies before the barrier below.
-  if (p.hist_cap > 0 && warp >= 1)
+  // starting on a 16-byte boundary: beam warp w >= 1 copies steps w + 1,
+  // w + 8, w + 15.  Every thread waits for its own copies before the barrier.
+  if (p.hist_cap > 0 && warp >= 1 && warp < kAncWarp)
 #pragma unroll 1
-    for (int j = warp + 1; j < t; j += kThreads / 32 - 1)
+    for (int j = warp + 1; j < t; j += kAncWarp - 1)
       copy_ints_warp(s_hist + p.hoff[j], p.hpar[j] + (int64_t)r * p.hpar_rs[j], p.hW[j], lane);
   ptx::cp_async_commit();
   ptx::cp_async_wait_all();
@@ -246,55 +232,23 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
 
   bool ok = true;
   const uint32_t x_u32 = ptx::smem_u32(s_x), a_u32 = ptx::smem_u32(base + L.a);
-  // Key rows of slots [lo, lo + n) (n a multiple of 4) into s_keys, by 32
-  // callers i = 0..31: caller i gathers the 4 rows of slots lo + 4i .. + 3
-  // (one depth: the slots of a depth start on a multiple of 4) from that
-  // depth's row table.  Every caller arrives on bar_keys once.
-  auto stage_keys = [&](int lo, int n, int i) {
-    if (4 * i < n) {
-      const int s0 = lo + 4 * i;
-      const int j = s_list[s0] & 31;
-      const int Wj = s_tW[j + 1];
-      int row[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int a = s_list[s0 + q] >> 5;
-        row[q] = hin ? (r * Wj + a) * H + h : (int)rec_row(p, j + 1, r, h, a);
-      }
-      ptx::fence_proxy_async_smem();
-      ptx::mbar_arrive_expect_tx(bar_keys, 4 * DK * 2);
-      ptx::tma_gather4(s_keys + 4 * i * DK * 2, &p.tm_krows[j + 1], 0, row[0], row[1], row[2], row[3], bar_keys);
-    } else {
-      ptx::mbar_arrive(bar_keys);
-    }
-  };
   const int wq = warp & 3;                        // TMEM lane quarter of this warp
   const uint32_t lb = (uint32_t)(wq * 32) << 16;  // its lane base
 
-  // ------------------------------------------------ warp roles before the wait
-  if (warp == 0) {
-    // The MMA issuer: D1 = S0 . X^T.
-    if (lane == 0) {
-      ok = ptx::mbar_wait(bar_s0, 0, kWaitLimitNs);
-      ptx::tc_fence_after();
-      constexpr uint32_t idesc1 = ptx::idesc_bf16_f32(kM, kN);
-      int acc = 0;
-      for (int pl = 0; pl < P; ++pl)
-#pragma unroll
-        for (int ka = 0; ka < NK; ++ka)
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = ptx::desc_k128(a_u32 + (pl * NK + ka) * 16384 + kk * 32);
-            const uint64_t bd = ptx::desc_k128(x_u32 + ka * XA + kk * 32);
-            ptx::mma_bf16(tmem, ad, bd, idesc1, acc);
-            acc = 1;
-          }
-      ptx::mma_commit(bar1);
-    }
-  } else if (warp == 1) {
-    // The ancestry: beam b's ancestors a[j] at depth j + 1 (a[t-2] = its
-    // parent; a[j] is the parent, at step j + 2, of a[j + 1]), the entries of
-    // depth t that need no delta, and the distinct ancestors of the tile.
+  // Beam-major phase (warps 0-7): thread (bb, l) owns elements
+  // 32 (u ^ sx) + 4 l + z (z < 4) of beam bb, where sx = bb & 1: odd beams
+  // take the 32-element groups in swapped pairs, so the four beams of a warp
+  // reading rows at the same step cover all 32 banks.
+  const int bb = tid >> 3, l = tid & 7, sx = bb & 1;
+  const bool bval = bb < nb;  // false in the ancestry warp (bb >= 32)
+  uint2 kb2[NU], qb2[NU];  // this thread's elements of k_b and q_b, bf16
+  float kq = 0.f;
+
+  if (warp == kAncWarp) {
+    // ------------------------------------------------ the ancestry warp
+    // Beam b's ancestors a[j] at depth j + 1 (a[t-2] = its parent; a[j] is
+    // the parent, at step j + 2, of a[j + 1]), the tile's distinct
+    // ancestors and the replay weights.
     const int b = lane;
     if (b < nb && nanc >= 1 && (par < 0 || par >= p.W_prev)) {
       *reinterpret_cast<volatile int32_t *>(p.err) = kErrParent;
@@ -316,20 +270,20 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
       }
     }
     ptx::mbar_arrive(bar_chain);
+    // The gates along the chain land in s_w (one round trip, overlapping
+    // the distinct-ancestor pass); they become the replay weights.
     if (b < nb) {
-      const int gb = b0 + b;
-      p.rec_alpha[rec_row(p, t, r, h, gb)] = alpha_b;
-      if (h == 0) {
-        int32_t *row = p.anc + anc_row(p, t, r, gb);
 #pragma unroll 1
-        for (int j = 0; j < nanc; ++j) row[j] = s_chain[b * TM + j];
-        p.par_store[((int64_t)(t - 1) * p.R + r) * p.W_max + gb] = par;
+      for (int j = 0; j <= jp; ++j) {
+        const int a = s_chain[b * TM + j];
+        ptx::cp_async4(s_w + b * TM + j, hin ? s_tg[j + 1] + ((int64_t)r * s_tW[j + 1] + a) * H + h
+                                             : p.rec_alpha + rec_row(p, j + 1, r, h, a));
       }
     }
+    ptx::cp_async_commit();
     // Distinct ancestors depth by depth: every lane writes its lane number
     // at its ancestor's index, and the lane whose number survives leads that
-    // ancestor.  Slots in order of depth, then of the leading lane; each
-    // depth's first slot is a multiple of 4.
+    // ancestor.  Slots in order of depth, then of the leading lane.
     int U = 0;
 #pragma unroll 1
     for (int j = 0; j < nanc; ++j) {
@@ -342,213 +296,234 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
       const unsigned leaders = __ballot_sync(0xffffffffu, lead);
       const int slot = U + __popc(leaders & ((1u << leader) - 1u));
       if (lead) s_list[slot] = (a << 5) | j;
-      if (b < nb) {
-        s_slot[b * TM + j] = slot;
-        s_c[b * TM + j] = make_float4(0.f, 0.f, __int_as_float(slot), 0.f);
-      }
-      __syncwarp();
-      // Pad the depth to a whole group of 4 with its first ancestor.
-      const int cnt = __popc(leaders), cnt4 = (cnt + 3) & ~3;
-      if (lane >= cnt && lane < cnt4) s_list[U + lane] = s_list[U];
-      U += cnt4;
+      if (b < nb) reinterpret_cast<float *>(s_c + b * TM + j)[2] = __int_as_float(slot);
+      U += __popc(leaders);
     }
     if (lane == 0) *s_U = U;
-    ptx::mbar_arrive(bar_slots);
-  } else if (warp == 2) {
-    // The gates along each beam's chain give the replay weights (products of
-    // the later gates) and P(p).  They land in s_w first (one round trip);
-    // each entry is then overwritten by the weight of its depth.
-    const int b = lane;
-    if (!ptx::mbar_wait(bar_chain, 0, kWaitLimitNs)) ok = false;
-    if (b < nb) {
-#pragma unroll 1
-      for (int j = 0; j <= jp; ++j) {
-        const int a = s_chain[b * TM + j];
-        ptx::cp_async4(s_w + b * TM + j, hin ? s_tg[j + 1] + ((int64_t)r * s_tW[j + 1] + a) * H + h
-                                             : p.rec_alpha + rec_row(p, j + 1, r, h, a));
-      }
-    }
-    ptx::cp_async_commit();
+    // Replay weights (products of the later gates) and P(p) (all of them).
     ptx::cp_async_wait_all();
     float w = 1.f;
     if (b < nb) {
 #pragma unroll 1
       for (int j = jp; j >= 0; --j) {
         const float gj = s_w[b * TM + j];
-        s_w[b * TM + j] = w;
+        reinterpret_cast<float *>(s_c + b * TM + j)[3] = w;
         w *= hin ? expf(gj) : gj;
       }
     }
-    s_Gp[b] = w;  // P(p): all the gates on the path
-    ptx::mbar_arrive(bar_w);
-  } else if (warp == 3) {
-    // The key records of depth t, from X.
-    if (!ptx::mbar_wait(bar_s0, 0, kWaitLimitNs)) ok = false;
-    for (int e = lane; e < kBT * NK * 8; e += 32) {
-      const int n = e / (NK * 8), cc = e - n * (NK * 8);
-      if (n < nb)
-        reinterpret_cast<uint4 *>(rec_k + rec_row(p, t, r, h, b0 + n) * DK)[cc] =
-            *reinterpret_cast<const uint4 *>(s_x + (cc >> 3) * XA + ptx::swz128(n, cc & 7));
+    s_Gp[b] = w;
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------ the MMA warp
+    // D1 = S0 . X^T on the tensor cores, issued by lane 0 once the image is
+    // here.
+    if (lane == 0) {
+      ok = ptx::mbar_wait(bar_s0, 0, kWaitLimitNs);
+      ptx::tc_fence_after();
+      constexpr uint32_t idesc1 = ptx::idesc_bf16_f32(kM, kN);
+      int acc = 0;
+      for (int pl = 0; pl < P; ++pl)
+#pragma unroll
+        for (int ka = 0; ka < NK; ++ka)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = ptx::desc_k128(a_u32 + (pl * NK + ka) * 16384 + kk * 32);
+            const uint64_t bd = ptx::desc_k128(x_u32 + ka * XA + kk * 32);
+            ptx::mma_bf16(tmem, ad, bd, idesc1, acc);
+            acc = 1;
+          }
+      ptx::mma_commit(bar1);
     }
   } else {
-    // Warps 4-7: the key rows of the tile's first kKeyRows distinct
-    // ancestors into shared memory (one bulk copy per row), and D1^T.
-    const int ei = wq * 32 + lane;  // TMEM lane: output element of D1
-    if (!ptx::mbar_wait(bar1, 0, kWaitLimitNs)) ok = false;  // region A is free
-    ptx::tc_fence_after();
-    if (!ptx::mbar_wait(bar_slots, 0, kWaitLimitNs)) ok = false;
-    if (lane < 8) stage_keys(0, min(*s_U, kKeyRows), wq * 8 + lane);  // 8 groups per warp
+    // ------------------------------------------------ the beam warps
+    if (!ptx::mbar_wait(bar_s0, 0, kWaitLimitNs)) ok = false;  // X and v visible to this thread
+    // This thread's elements of k_b and q_b, and k_b . q_b.
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      float d[32];
-      ptx::tmem_ld32(tmem + lb + half * 32, d);
-      ptx::tmem_ld_wait();
-      if (wq * 32 < DV)
-#pragma unroll
-        for (int n = 0; n < 32; ++n) s_d1[(half * 32 + n) * DV + ei] = d[n];
+    for (int u = 0; u < NU; ++u) {
+      const int uu = u ^ sx;
+      const uint32_t off = (uint32_t)(uu >> 1) * XA + (uint32_t)(l & 1) * 8u;
+      const int c = 4 * (uu & 1) + (l >> 1);
+      kb2[u] = *reinterpret_cast<const uint2 *>(s_x + off + ptx::swz128(bb, c));
+      qb2[u] = *reinterpret_cast<const uint2 *>(s_x + off + ptx::swz128(kBT + bb, c));
+      const float4 kf = bf16x4(kb2[u]), qf = bf16x4(qb2[u]);
+      kq = fmaf(kf.x, qf.x, kq);
+      kq = fmaf(kf.y, qf.y, kq);
+      kq = fmaf(kf.z, qf.z, kq);
+      kq = fmaf(kf.w, qf.w, kq);
     }
-  }
-  ptx::tc_fence_before();
-  __syncthreads();  // every role done: D1^T, slots, weights
-  if (warp == 3) ptx::tmem_dealloc(tmem, kTmemCols);
-
-  // Beam-major phase: thread (bb, l) owns elements 32 u + 4 l + z (z < 4) of
-  // beam bb.  u = P(p) D1 + (replayed terms, after the wait); v from its tile.
-  const int bb = tid >> 3, l = tid & 7;
-  const bool bval = bb < nb;
-  if (!ptx::mbar_wait(bar_s0, 0, kWaitLimitNs)) ok = false;  // X and v visible to this thread
-  // This thread's elements of k_b and q_b, and k_b . q_b.
-  float4 kb[NU], qb[NU];
-  float kq = 0.f;
-#pragma unroll
-  for (int u = 0; u < NU; ++u) {
-    const uint32_t off = (uint32_t)(u >> 1) * XA + (uint32_t)(l & 1) * 8u;
-    const int c = 4 * (u & 1) + (l >> 1);
-    kb[u] = bf16x4(s_x + off + ptx::swz128(bb, c));
-    qb[u] = bf16x4(s_x + off + ptx::swz128(kBT + bb, c));
-    kq = fmaf(kb[u].x, qb[u].x, kq);
-    kq = fmaf(kb[u].y, qb[u].y, kq);
-    kq = fmaf(kb[u].z, qb[u].z, kq);
-    kq = fmaf(kb[u].w, qb[u].w, kq);
-  }
-  kq += __shfl_xor_sync(0xffffffffu, kq, 4);
-  kq += __shfl_xor_sync(0xffffffffu, kq, 2);
-  kq += __shfl_xor_sync(0xffffffffu, kq, 1);
-  // k_a . k_b and k_a . q_b for the beam's ancestor a at every depth, from
-  // the staged key rows (rounds of kKeyRows slots), weighted.
-  const int U = *s_U;
-  for (int lo = 0, rnd = 0; lo < U; lo += kKeyRows, ++rnd) {
-    const int nrows = min(U - lo, kKeyRows);
-    if (rnd > 0) {
-      __syncthreads();  // the previous round's rows are consumed
-      if (warp == 0) stage_keys(lo, nrows, lane);
-    }
-    if (!ptx::mbar_wait(bar_keys, rnd & 1, kWaitLimitNs)) ok = false;
-    // Two depths per pass: independent loads and shuffle chains interleave.
-#pragma unroll 1
-    for (int j0 = 0; j0 < nanc; j0 += 2) {
-      float dk[2], dq[2];
-      int slot[2];
-      bool in[2];
+    kq += __shfl_xor_sync(0xffffffffu, kq, 4);
+    kq += __shfl_xor_sync(0xffffffffu, kq, 2);
+    kq += __shfl_xor_sync(0xffffffffu, kq, 1);
+    // k_a . k_b and k_a . q_b for the beam's ancestor a at every depth: the
+    // thread's pieces of each ancestor's key row come straight from global
+    // memory (step j's own k input, or the key records), two depths per
+    // pass, the next pass's loads in flight during this pass's arithmetic.
+    if (!ptx::mbar_wait(bar_chain, 0, kWaitLimitNs)) ok = false;
+    auto issue = [&](uint2 (&buf)[2][NU], int j0) {
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int j = j0 + e;
-        slot[e] = bval && j < nanc ? s_slot[bb * TM + j] : -1;
-        const unsigned sl = (unsigned)(slot[e] - lo);
-        in[e] = sl < (unsigned)nrows;
-        const uint8_t *row = s_keys + (in[e] ? sl : 0u) * (DK * 2) + l * 8;
-        dk[e] = 0.f, dq[e] = 0.f;
+        if (bval && j < nanc) {
+          const int a = s_chain[bb * TM + j];
+          const __nv_bfloat16 *row = hin ? s_tk[j + 1] + ((int64_t)(r * s_tW[j + 1] + a) * H + h) * DK
+                                         : rec_k + rec_row(p, j + 1, r, h, a) * DK;
+          const uint8_t *rb = reinterpret_cast<const uint8_t *>(row) + l * 8;
 #pragma unroll
-        for (int u = 0; u < NU; ++u) {
-          const float4 kf = bf16x4(row + u * 64);
-          dk[e] = fmaf(kf.x, kb[u].x, dk[e]);
-          dk[e] = fmaf(kf.y, kb[u].y, dk[e]);
-          dk[e] = fmaf(kf.z, kb[u].z, dk[e]);
-          dk[e] = fmaf(kf.w, kb[u].w, dk[e]);
-          dq[e] = fmaf(kf.x, qb[u].x, dq[e]);
-          dq[e] = fmaf(kf.y, qb[u].y, dq[e]);
-          dq[e] = fmaf(kf.z, qb[u].z, dq[e]);
-          dq[e] = fmaf(kf.w, qb[u].w, dq[e]);
+          for (int u = 0; u < NU; ++u) buf[e][u] = __ldg(reinterpret_cast<const uint2 *>(rb + (u ^ sx) * 64));
+        } else {
+#pragma unroll
+          for (int u = 0; u < NU; ++u) buf[e][u] = make_uint2(0u, 0u);
         }
       }
+    };
+    auto dots = [&](const uint2 (&buf)[2][NU], int j0) {
+      float dk[2], dq[2];
 #pragma unroll
-      for (int o = 4; o > 0; o >>= 1)
+      for (int e = 0; e < 2; ++e) dk[e] = 0.f, dq[e] = 0.f;
+#pragma unroll
+      for (int u = 0; u < NU; ++u) {
+        const float4 kbu = bf16x4(kb2[u]), qbu = bf16x4(qb2[u]);
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          dk[e] += __shfl_xor_sync(0xffffffffu, dk[e], o);
-          dq[e] += __shfl_xor_sync(0xffffffffu, dq[e], o);
+          const float4 kf = bf16x4(buf[e][u]);
+          dk[e] = fmaf(kf.x, kbu.x, dk[e]);
+          dk[e] = fmaf(kf.y, kbu.y, dk[e]);
+          dk[e] = fmaf(kf.z, kbu.z, dk[e]);
+          dk[e] = fmaf(kf.w, kbu.w, dk[e]);
+          dq[e] = fmaf(kf.x, qbu.x, dq[e]);
+          dq[e] = fmaf(kf.y, qbu.y, dq[e]);
+          dq[e] = fmaf(kf.z, qbu.z, dq[e]);
+          dq[e] = fmaf(kf.w, qbu.w, dq[e]);
         }
+      }
+      // Sum the four values over the beam's 8 threads in 4 shuffles: each
+      // level hands half of the values still held to the partner and keeps
+      // the other half, so thread l ends with value 2 (l >> 2) + ((l >> 1) & 1)
+      // (dk of depth j0, dq of j0, dk of j0 + 1, dq of j0 + 1).
+      const bool b2 = (l >> 2) & 1, b1 = (l >> 1) & 1;
+      const float s0v = __shfl_xor_sync(0xffffffffu, b2 ? dk[0] : dk[1], 4);
+      const float s1v = __shfl_xor_sync(0xffffffffu, b2 ? dq[0] : dq[1], 4);
+      const float w0 = (b2 ? dk[1] : dk[0]) + s0v, w1 = (b2 ? dq[1] : dq[0]) + s1v;
+      float x = (b1 ? w1 : w0) + __shfl_xor_sync(0xffffffffu, b1 ? w0 : w1, 2);
+      x += __shfl_xor_sync(0xffffffffu, x, 1);
+      const int j = j0 + (int)b2;
+      if ((l & 1) == 0 && bval && j < nanc) reinterpret_cast<float *>(s_c + bb * TM + j)[b1] = x;
+    };
+    uint2 kA[2][NU], kB[2][NU];
+    if (nanc > 0) issue(kA, 0);
+#pragma unroll 1
+    for (int j0 = 0; j0 < nanc; j0 += 4) {
+      if (j0 + 2 < nanc) issue(kB, j0 + 2);
+      dots(kA, j0);
+      if (j0 + 2 >= nanc) break;
+      if (j0 + 4 < nanc) issue(kA, j0 + 4);
+      dots(kB, j0 + 2);
+    }
+    if (warp >= 4) {
+      // D1^T into shared memory (region A: the image is consumed).
+      const int ei = wq * 32 + lane;  // TMEM lane: output element of D1
+      if (!ptx::mbar_wait(bar1, 0, kWaitLimitNs)) ok = false;
+      ptx::tc_fence_after();
 #pragma unroll
-      for (int e = 0; e < 2; ++e)
-        if (in[e] && l == 0) {
-          const float w = s_w[bb * TM + j0 + e];
-          s_c[bb * TM + j0 + e] = make_float4(dk[e] * w, dq[e] * w, __int_as_float(slot[e]), 0.f);
-        }
+      for (int half = 0; half < 2; ++half) {
+        float d[32];
+        ptx::tmem_ld32(tmem + lb + half * 32, d);
+        ptx::tmem_ld_wait();
+        if (wq * 32 < DV)
+#pragma unroll
+          for (int n = 0; n < 32; ++n) s_d1[(half * 32 + n) * DV + ei] = d[n];
+      }
+    } else {
+      // The key records of depth t, from X.
+      for (int e = tid; e < kBT * NK * 8; e += 128) {
+        const int n = e / (NK * 8), cc = e - n * (NK * 8);
+        if (n < nb)
+          reinterpret_cast<uint4 *>(rec_k + rec_row(p, t, r, h, b0 + n) * DK)[cc] =
+              *reinterpret_cast<const uint4 *>(s_x + (cc >> 3) * XA + ptx::swz128(n, cc & 7));
+      }
+    }
+    // alpha, the ancestry row and the parent of the beam.
+    if (bval && l == 0) {
+      const int gb = b0 + bb;
+      p.rec_alpha[rec_row(p, t, r, h, gb)] = s_alpha[bb];
+      if (h == 0) {
+        int32_t *row = p.anc + anc_row(p, t, r, gb);
+#pragma unroll 1
+        for (int j = 0; j < nanc; ++j) row[j] = s_chain[bb * TM + j];
+        p.par_store[((int64_t)(t - 1) * p.R + r) * p.W_max + gb] = s_par[bb];
+      }
     }
   }
+  ptx::tc_fence_before();
+  __syncthreads();  // every role done: D1^T, key products, slots, weights
+  if (warp == kMmaWarp) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, kTmemCols);
+  }
+
   // u = P(p) D1 + (replayed terms, after the wait); v from its tile.
+  const int U = *s_U;
   float acc_k[4 * NU], acc_q[4 * NU];
   float4 vf[NU];
-  const float Gp = s_Gp[bb], alpha = s_alpha[bb], beta = s_beta[bb];
+  const float Gp = warp < kAncWarp ? s_Gp[bb] : 0.f;  // beam warps only from here on
+  const float alpha = warp < kAncWarp ? s_alpha[bb] : 0.f, beta = warp < kAncWarp ? s_beta[bb] : 0.f;
+  if (warp < kAncWarp) {
 #pragma unroll
-  for (int u = 0; u < NU; ++u) {
-    const float4 dk = reinterpret_cast<const float4 *>(s_d1 + bb * DV)[8 * u + l];
-    const float4 dq = reinterpret_cast<const float4 *>(s_d1 + (kBT + bb) * DV)[8 * u + l];
-    acc_k[4 * u + 0] = Gp * dk.x, acc_k[4 * u + 1] = Gp * dk.y, acc_k[4 * u + 2] = Gp * dk.z, acc_k[4 * u + 3] = Gp * dk.w;
-    acc_q[4 * u + 0] = Gp * dq.x, acc_q[4 * u + 1] = Gp * dq.y, acc_q[4 * u + 2] = Gp * dq.z, acc_q[4 * u + 3] = Gp * dq.w;
-    vf[u] = bf16x4(s_v + (u >> 1) * VA + ptx::swz128(bb, 4 * (u & 1) + (l >> 1)) + (l & 1) * 8);
+    for (int u = 0; u < NU; ++u) {
+      const int uu = u ^ sx;
+      const float4 dk = reinterpret_cast<const float4 *>(s_d1 + bb * DV)[8 * uu + l];
+      const float4 dq = reinterpret_cast<const float4 *>(s_d1 + (kBT + bb) * DV)[8 * uu + l];
+      acc_k[4 * u + 0] = Gp * dk.x, acc_k[4 * u + 1] = Gp * dk.y, acc_k[4 * u + 2] = Gp * dk.z, acc_k[4 * u + 3] = Gp * dk.w;
+      acc_q[4 * u + 0] = Gp * dq.x, acc_q[4 * u + 1] = Gp * dq.y, acc_q[4 * u + 2] = Gp * dq.z, acc_q[4 * u + 3] = Gp * dq.w;
+      vf[u] = bf16x4(s_v + (uu >> 1) * VA + ptx::swz128(bb, 4 * (uu & 1) + (l >> 1)) + (l & 1) * 8);
+    }
   }
-  __syncthreads();  // D1^T and the key rows consumed before the deltas overwrite region A
+  __syncthreads();  // D1^T consumed before the deltas overwrite region A
 
   // ------------------------------- after the wait: the ancestors' deltas
   ptx::pdl_wait();
-  for (int lo = 0, rnd = 0; lo < U; lo += kDRows, ++rnd) {
+  constexpr int PD = DV / 4;  // 16-byte pieces of a delta row
+  for (int lo = 0; lo < U; lo += kDRows) {
     const int hi = min(U, lo + kDRows);
     const int nrows = hi - lo;
-    if (rnd > 0) __syncthreads();  // the previous round's deltas are consumed
-    if (warp == 0) {
-      // Lane i gathers the delta rows of slots lo + 4i .. + 3.
-      if (4 * lane < nrows) {
-        int row[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int packed = s_list[lo + 4 * lane + q];
-          row[q] = (int)rec_row(p, (packed & 31) + 1, r, h, packed >> 5);
-        }
-        ptx::fence_proxy_async_smem();
-        ptx::mbar_arrive_expect_tx(bar_d, 4 * DV * 4);
-        ptx::tma_gather4(base + L.dst + 4 * lane * DV * 4, &p.tm_delta, 0, row[0], row[1], row[2], row[3], bar_d);
-      } else {
-        ptx::mbar_arrive(bar_d);
-      }
+    if (lo > 0) __syncthreads();  // the previous round's deltas are consumed
+    // The rows of slots lo .. hi - 1 in 16-byte pieces (a warp copies whole
+    // rows), then every thread waits for its own pieces and the block syncs.
+#pragma unroll 1
+    for (int e = tid; e < nrows * PD; e += kThreads) {
+      const int rr = e / PD, c = e - rr * PD;
+      const int packed = s_list[lo + rr];
+      ptx::cp_async16(base + L.dst + (uint32_t)(rr * DV + c * 4) * 4u,
+                      p.rec_delta + rec_row(p, (packed & 31) + 1, r, h, packed >> 5) * DV + c * 4, 16u);
     }
-    if (!ptx::mbar_wait(bar_d, rnd & 1, kWaitLimitNs)) ok = false;
-    if (bb < nb) {
+    ptx::cp_async_commit();
+    ptx::cp_async_wait_all();
+    __syncthreads();
+    if (bval) {
       // Two depths per pass: their loads are independent.
 #pragma unroll 1
       for (int j0 = 0; j0 < nanc; j0 += 2) {
-        float4 c[2];
-        bool in[2];
+        float ck[2], cq[2];
         const float4 *row[2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          c[e] = j0 + e < nanc ? s_c[bb * TM + j0 + e] : make_float4(0.f, 0.f, __int_as_float(-1), 0.f);
-          const unsigned sl = (unsigned)(__float_as_int(c[e].z) - lo);
-          in[e] = sl < (unsigned)nrows;
-          row[e] = reinterpret_cast<const float4 *>(s_dst + (in[e] ? sl : 0u) * DV) + l;
-          if (!in[e]) c[e].x = c[e].y = 0.f;
+          const float4 c = j0 + e < nanc ? s_c[bb * TM + j0 + e] : make_float4(0.f, 0.f, __int_as_float(-1), 0.f);
+          const unsigned sl = (unsigned)(__float_as_int(c.z) - lo);
+          const bool in = sl < (unsigned)nrows;
+          row[e] = reinterpret_cast<const float4 *>(s_dst + (in ? sl : 0u) * DV) + l;
+          ck[e] = in ? c.x * c.w : 0.f;
+          cq[e] = in ? c.y * c.w : 0.f;
         }
 #pragma unroll
         for (int u = 0; u < NU; ++u) {
-          const float4 d0 = row[0][8 * u], d1 = row[1][8 * u];
-          acc_k[4 * u + 0] = fmaf(d1.x, c[1].x, fmaf(d0.x, c[0].x, acc_k[4 * u + 0]));
-          acc_k[4 * u + 1] = fmaf(d1.y, c[1].x, fmaf(d0.y, c[0].x, acc_k[4 * u + 1]));
-          acc_k[4 * u + 2] = fmaf(d1.z, c[1].x, fmaf(d0.z, c[0].x, acc_k[4 * u + 2]));
-          acc_k[4 * u + 3] = fmaf(d1.w, c[1].x, fmaf(d0.w, c[0].x, acc_k[4 * u + 3]));
-          acc_q[4 * u + 0] = fmaf(d1.x, c[1].y, fmaf(d0.x, c[0].y, acc_q[4 * u + 0]));
-          acc_q[4 * u + 1] = fmaf(d1.y, c[1].y, fmaf(d0.y, c[0].y, acc_q[4 * u + 1]));
-          acc_q[4 * u + 2] = fmaf(d1.z, c[1].y, fmaf(d0.z, c[0].y, acc_q[4 * u + 2]));
-          acc_q[4 * u + 3] = fmaf(d1.w, c[1].y, fmaf(d0.w, c[0].y, acc_q[4 * u + 3]));
+          const float4 d0 = row[0][8 * (u ^ sx)], d1 = row[1][8 * (u ^ sx)];
+          acc_k[4 * u + 0] = fmaf(d1.x, ck[1], fmaf(d0.x, ck[0], acc_k[4 * u + 0]));
+          acc_k[4 * u + 1] = fmaf(d1.y, ck[1], fmaf(d0.y, ck[0], acc_k[4 * u + 1]));
+          acc_k[4 * u + 2] = fmaf(d1.z, ck[1], fmaf(d0.z, ck[0], acc_k[4 * u + 2]));
+          acc_k[4 * u + 3] = fmaf(d1.w, ck[1], fmaf(d0.w, ck[0], acc_k[4 * u + 3]));
+          acc_q[4 * u + 0] = fmaf(d1.x, cq[1], fmaf(d0.x, cq[0], acc_q[4 * u + 0]));
+          acc_q[4 * u + 1] = fmaf(d1.y, cq[1], fmaf(d0.y, cq[0], acc_q[4 * u + 1]));
+          acc_q[4 * u + 2] = fmaf(d1.z, cq[1], fmaf(d0.z, cq[0], acc_q[4 * u + 2]));
+          acc_q[4 * u + 3] = fmaf(d1.w, cq[1], fmaf(d0.w, cq[0], acc_q[4 * u + 3]));
         }
       }
     }
@@ -556,7 +531,7 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
 
   // --------------------------------------------------------- epilogue
   if (!ok) *reinterpret_cast<volatile int32_t *>(p.err) = kErrTimeout;
-  if (bb < nb && ok) {
+  if (bval && ok) {
     float4 *op = reinterpret_cast<float4 *>(p.o + (row0 + (int64_t)bb * H) * DV) + l;
     float4 *dp = reinterpret_cast<float4 *>(p.rec_delta + rec_row(p, t, r, h, b0 + bb) * DV) + l;
 #pragma unroll
@@ -570,8 +545,8 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
       o.y = fmaf(alpha, acc_q[4 * u + 1], d.y * kq);
       o.z = fmaf(alpha, acc_q[4 * u + 2], d.z * kq);
       o.w = fmaf(alpha, acc_q[4 * u + 3], d.w * kq);
-      op[8 * u] = o;
-      dp[8 * u] = d;
+      op[8 * (u ^ sx)] = o;
+      dp[8 * (u ^ sx)] = d;
     }
   }
 }
@@ -672,19 +647,6 @@ cudaError_t launch_dk(const StepParams &p_in, bool pdl, cudaStream_t s) {
 }
 
 }  // namespace
-
-bool encode_row_table(CUtensorMap *m, const void *base, int bf16, int width, long long rows) {
-  PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
-  if (!fn || rows < 1 || rows > 0x7fffffffLL) return false;
-  const int es = bf16 ? 2 : 4;
-  const cuuint64_t dims[2] = {(cuuint64_t)width, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)width * es};
-  const cuuint32_t box[2] = {(cuuint32_t)width, 1};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(base),
-            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 bool tc_supports(int dk, int dv, int qkv_bf16, int T_max, int W_max) {
   return qkv_bf16 && dk == dv && (dk == 64 || dk == 128) && T_max <= kMaxT && W_max <= kMaxW;
