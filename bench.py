@@ -130,6 +130,63 @@ def s0_by_prefill_gpu(wl, device):
     return S32.to(torch.bfloat16) if wl.s0_dtype == "bf16" else S32
 
 
+# FP32 lanes per SM and SM count of the B200, for the ALU roofline of the
+# prefill (its recurrence runs on the CUDA cores in fp32).
+FP32_LANES_PER_SM, N_SMS = 128, 148
+
+
+def time_prefill(wl, device, stream, flush, reps=10, warmup=3):
+    """Device time of onela_prefill over the workload's prompt (every request
+    and head), L2 flushed before each call; and the oracle's prefill on a
+    bounded host sample.  Returns the JSON object for the bench line."""
+    import linear_attention_beam_shared_b200 as L
+    from oracle import gdn
+    k, v, a, b = synth.draw_prompt(wl)
+    kd = synth.cast_vec(k, wl.qkv_dtype).to(device)
+    vd = synth.cast_vec(v, wl.qkv_dtype).to(device)
+    g = torch.from_numpy(np.log(a)).float().to(device)
+    beta = torch.from_numpy(b).float().to(device)
+    dec = L.BeamDecoder(wl.R, wl.H, wl.d_k, wl.d_v, wl.W, wl.T, wl.s0_dtype, wl.qkv_dtype, device=device.index)
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            flush.fill_(5)
+            dec.prefill(kd, vd, g, beta, stream=stream)
+    stream.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    with torch.cuda.stream(stream):
+        for i, (e0, e1) in enumerate(ev):
+            flush.fill_(i & 0xFF)
+            e0.record(stream)
+            dec.prefill(kd, vd, g, beta, stream=stream)
+            e1.record(stream)
+    stream.synchronize()
+    assert dec.status() == 0
+    dec.close()
+    ms = max_over_ranks(sum(e0.elapsed_time(e1) for e0, e1 in ev) / reps, device)
+    units = wl.R * wl.L_prompt * wl.H
+    flops = 4.0 * wl.d_k * wl.d_v * units
+    peak = N_SMS * FP32_LANES_PER_SM * 2 * 1.965e9 / 1e9   # GFLOP/s at the 1965 MHz boost clock
+    achieved = flops / (ms / 1e3) / 1e9
+    e = 2 if wl.qkv_dtype == "bf16" else 4
+    bytes_ = units * (wl.d_k + wl.d_v) * e + units * 8 + wl.R * wl.H * wl.d_k * wl.d_v * (2 if wl.s0_dtype == "bf16" else 4)
+    # The oracle on the host: one head, the first 512 tokens.
+    Ls = min(512, wl.L_prompt)
+    t0 = time.perf_counter()
+    gdn.prefill(k[0, :Ls, :1], v[0, :Ls, :1], a[0, :Ls, :1], b[0, :Ls, :1])
+    el = time.perf_counter() - t0
+    return {
+        "workload": f"{wl.name} prompt: R={wl.R}, L={wl.L_prompt}, H={wl.H}, d_k=d_v={wl.d_k}, "
+                    f"k/v {wl.qkv_dtype}, S0 {wl.s0_dtype}",
+        "ms": round(ms, 4), "value": round(units / (ms / 1e3), 1), "unit": "prompt token·head steps/s",
+        "roofline": {"bound": "alu", "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "GFLOP/s",
+                     "frac": round(achieved / peak, 4),
+                     "peak_source": "148 SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz",
+                     "hbm_bytes": int(bytes_), "hbm_frac": round(bytes_ / (ms / 1e3) / 1e9 / measured_peaks()[0], 4)},
+        "cpu_baseline": {"value": round(Ls / el, 1), "unit": "prompt token·head steps/s", "cores": 1,
+                         "kind": "oracle", "sample": f"one head, first {Ls} tokens, numpy fp64 prefill, {el:.2f} s"},
+    }
+
+
 def byte_model(wl, steps):
     """Algorithmic bytes of one whole decode (all T steps): every byte the
     method must move at least once, with each distinct ancestor record counted
@@ -353,6 +410,8 @@ def run_ours(args):
            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
     assert dec.status() == 0
 
+    prefill = time_prefill(wl, device, stream, flush) if (wl.L_prompt > 0 and not args.no_prefill) else None
+
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu:
         rate, reps, el, threads = time_cpu_oracle(wl, S0, steps, budget_s=args.cpu_budget)
@@ -376,6 +435,7 @@ def run_ours(args):
                        "programmatic_launch": not args.no_pdl},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "clocks": clk.summary(), "gpu_launches": launches * args.steps,
+            "prefill": prefill,
         }
         print(json.dumps(line))
     if ws > 1:
@@ -429,6 +489,7 @@ def main():
     ap.add_argument("--no-pdl", action="store_true",
                     help="launch every step only after the previous one has finished")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill timing")
     ap.add_argument("--s0", choices=["prefill", "direct"], default="prefill",
                     help="S0 from the GDN recurrence over the synthetic prompt (default) or drawn "
                          "directly; the decode's work does not depend on the S0 values")

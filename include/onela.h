@@ -126,8 +126,8 @@ typedef struct {
 /* Create a handle: validates cfg and allocates, on cfg->device, the S0 copy,
  * the record store (alpha fp32 [T_max][R][H][W_max], delta fp32
  * [T_max][R][H][W_max][d_v], k [T_max][R][H][W_max][d_k] in qkv_dtype; the
- * tensor-core kernel also keeps, per record, the product of the gates on its
- * path from the root, fp32 [T_max][R][H][W_max]), the
+ * tensor-core kernel also keeps each step's parents, int32 [T_max][R][W_max],
+ * and the bf16 operand image of S0), the
  * ancestry index (int32 [T_max][R][W_max][T_max]) and an error word in
  * mapped, pinned host memory that the kernels write and the host reads.
  * Host-side allocation only; no kernel runs.  *out receives the handle.
@@ -141,6 +141,30 @@ ONELA_API int onela_create(const onela_config *cfg, onela_handle **out);
  *       operand layout); S0 may be freed once the stream has passed the call.
  * Errors: ONELA_ERR_ARG, ONELA_ERR_CUDA. */
 ONELA_API int onela_set_prompt_state(onela_handle *h, const void *S0, onela_stream stream);
+
+/* Build the state every beam of a request starts from out of the request's
+ * prompt, on the device, and install it as onela_set_prompt_state does (the
+ * one prompt-derived state of the abstract).  For every (request, head), the
+ * GDN recurrence of the review's section 3.2 (equation 2) from the zero state
+ * over the L prompt tokens,
+ *     S_l = alpha_l S_{l-1} + delta_l k_l^T,
+ *     delta_l = beta_l (v_l - alpha_l S_{l-1} k_l),   alpha_l = exp(g_l),
+ * in fp32, rounded to cfg.s0_dtype once at the end.
+ *   L        prompt tokens, L >= 1.
+ *   k        [R][L][H][d_k] in qkv_dtype.
+ *   v        [R][L][H][d_v] in qkv_dtype.
+ *   g        [R][L][H] fp32, the log of the decay gate.
+ *   beta     [R][L][H] fp32.
+ * Rewinds the decode to step 0.  The inputs may be freed once the stream has
+ * passed the call.
+ * Errors: ONELA_ERR_ARG, ONELA_ERR_CUDA. */
+ONELA_API int onela_prefill(onela_handle *h, int32_t L, const void *k, const void *v,
+                            const float *g, const float *beta, onela_stream stream);
+
+/* Copy the installed prompt state into a caller DEVICE buffer on `stream`:
+ * [R][H][d_v][d_k] in cfg.s0_dtype.
+ * Errors: ONELA_ERR_ARG, ONELA_ERR_STATE (no prompt state yet), ONELA_ERR_CUDA. */
+ONELA_API int onela_read_prompt_state(onela_handle *h, void *S0, onela_stream stream);
 
 /* One decode step t = (number of previous steps since the last rewind) + 1.
  *   W_prev      beams of the previous step; must be 1 at t = 1 (the prompt

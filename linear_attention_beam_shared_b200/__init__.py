@@ -21,8 +21,9 @@ from ._lib import (  # noqa: F401
     ONELA_BF16, ONELA_ERR_ARG, ONELA_ERR_CAPACITY, ONELA_ERR_CUDA, ONELA_ERR_PARENT,
     ONELA_ERR_STATE, ONELA_ERR_UNSUPPORTED, ONELA_F32, ONELA_FLAG_PDL, ONELA_KERNEL_AUTO, ONELA_KERNEL_SIMT,
     ONELA_ERR_SCRATCH, ONELA_KERNEL_TC, ONELA_OK, Handle, OnelaError, error_string, onela_create,
-    onela_decode_step, onela_decode_step_noalloc, onela_destroy, onela_kernel_kind, onela_read_ancestry, onela_read_records, onela_reset,
-    onela_set_prompt_state, onela_status, onela_status_code, onela_steps_done,
+    onela_decode_step, onela_decode_step_noalloc, onela_destroy, onela_kernel_kind, onela_prefill,
+    onela_read_ancestry, onela_read_prompt_state, onela_read_records, onela_reset, onela_set_prompt_state,
+    onela_status, onela_status_code, onela_steps_done,
 )
 
 LIB_PATH = _lib.LIB_PATH
@@ -46,6 +47,14 @@ class BeamDecoder:
     def set_prompt_state(self, S0, stream=None):
         onela_set_prompt_state(self.h, S0, stream)
         self.W_prev, self.Ws = 1, []
+
+    def prefill(self, k, v, g, beta, stream=None):
+        """Build S0 on the device from a prompt (see onela_prefill)."""
+        onela_prefill(self.h, k, v, g, beta, stream)
+        self.W_prev, self.Ws = 1, []
+
+    def prompt_state(self, stream=None):
+        return onela_read_prompt_state(self.h, stream)
 
     def step(self, q, k, v, g, beta, parent_idx, o=None, stream=None):
         c = self.h.cfg

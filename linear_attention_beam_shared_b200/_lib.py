@@ -49,6 +49,8 @@ def _load() -> ctypes.CDLL:
     sig = {
         "onela_create": ([ctypes.POINTER(onela_config), ctypes.POINTER(vp)], ctypes.c_int),
         "onela_set_prompt_state": ([vp, vp, vp], ctypes.c_int),
+        "onela_prefill": ([vp, i32, vp, vp, vp, vp, vp], ctypes.c_int),
+        "onela_read_prompt_state": ([vp, vp, vp], ctypes.c_int),
         "onela_decode_step": ([vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         "onela_reset": ([vp, vp], ctypes.c_int),
         "onela_status": ([vp, ctypes.POINTER(i32)], ctypes.c_int),
@@ -133,6 +135,29 @@ def onela_set_prompt_state(h: Handle, S0: torch.Tensor, stream=None) -> None:
     c = h.cfg
     p = _ptr(S0, "S0", _DT[c.s0_dtype], (c.R, c.H, c.d_v, c.d_k), c.device)
     _check(lib.onela_set_prompt_state(h.ptr, p, _stream(stream)), "onela_set_prompt_state")
+
+
+def onela_prefill(h: Handle, k, v, g, beta, stream=None) -> None:
+    """k, v: [R][L][H][d] in the handle's qkv dtype; g, beta: [R][L][H] fp32."""
+    c = h.cfg
+    dt = _DT[c.qkv_dtype]
+    if not isinstance(k, torch.Tensor) or k.dim() != 4:
+        raise ValueError("k must be a 4-D tensor [R][L][H][d_k]")
+    L = int(k.shape[1])
+    args = (
+        _ptr(k, "k", dt, (c.R, L, c.H, c.d_k), c.device),
+        _ptr(v, "v", dt, (c.R, L, c.H, c.d_v), c.device),
+        _ptr(g, "g", torch.float32, (c.R, L, c.H), c.device),
+        _ptr(beta, "beta", torch.float32, (c.R, L, c.H), c.device),
+    )
+    _check(lib.onela_prefill(h.ptr, L, *args, _stream(stream)), "onela_prefill")
+
+
+def onela_read_prompt_state(h: Handle, stream=None) -> torch.Tensor:
+    c = h.cfg
+    S0 = torch.empty((c.R, c.H, c.d_v, c.d_k), dtype=_DT[c.s0_dtype], device=torch.device("cuda", c.device))
+    _check(lib.onela_read_prompt_state(h.ptr, _ptr(S0, "S0"), _stream(stream)), "onela_read_prompt_state")
+    return S0
 
 
 def onela_decode_step(h: Handle, W_prev: int, W: int, q, k, v, g, beta, parent_idx, o,

@@ -71,6 +71,11 @@ cudaError_t launch_step_tc(const StepParams &p, int pdl, cudaStream_t s);
 cudaError_t launch_s0_image(const void *S0, void *img, int R, int H, int dk, int dv,
                             int s0_bf16, int planes, cudaStream_t s);
 size_t s0_image_bytes(int R, int H, int dk, int dv, int planes);
+// The GDN recurrence from the zero state over L prompt tokens for every
+// (request, head): k [R][L][H][dk], v [R][L][H][dv] (bf16 if qkv_bf16, else
+// fp32), g and beta [R][L][H] fp32 -> S0 [R][H][dv][dk] (bf16 if s0_bf16).
+cudaError_t launch_prefill(const void *k, const void *v, const float *g, const float *beta, void *S0, int R, int L,
+                           int H, int dk, int dv, int qkv_bf16, int s0_bf16, cudaStream_t s);
 bool tc_supports(int dk, int dv, int qkv_bf16, int T_max, int W_max);
 
 }  // namespace onela

@@ -52,6 +52,16 @@ struct DeviceGuard {
   }
 };
 
+// The prompt state is in place: the decode starts again at step 0.
+void rewind_to_prompt(onela_handle *h) {
+  h->has_prompt = 1;
+  h->steps_done = 0;
+  h->Ws.clear();
+  h->hist_k.clear();
+  h->hist_g.clear();
+  h->hist_par.clear();
+}
+
 void free_all(onela_handle *h) {
   cudaFree(h->S0);
   cudaFree(h->S0img);
@@ -176,12 +186,40 @@ int onela_set_prompt_state(onela_handle *h, const void *S0, onela_stream stream)
         cudaSuccess)
       return ONELA_ERR_CUDA;
   }
-  h->has_prompt = 1;
-  h->steps_done = 0;
-  h->Ws.clear();
-  h->hist_k.clear();
-  h->hist_g.clear();
-  h->hist_par.clear();
+  rewind_to_prompt(h);
+  return ONELA_OK;
+}
+
+int onela_prefill(onela_handle *h, int32_t L, const void *k, const void *v, const float *gate, const float *beta,
+                  onela_stream stream) {
+  if (!h || !k || !v || !gate || !beta || L < 1) return ONELA_ERR_ARG;
+  DeviceGuard g(h->cfg.device);
+  if (!g.ok) return ONELA_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const onela_config &c = h->cfg;
+  if (onela::launch_prefill(k, v, gate, beta, h->S0, c.R, L, c.H, c.d_k, c.d_v, c.qkv_dtype == ONELA_BF16,
+                            c.s0_dtype == ONELA_BF16, s) != cudaSuccess) {
+    cudaGetLastError();
+    return ONELA_ERR_CUDA;
+  }
+  if (h->kernel == ONELA_KERNEL_TC) {
+    if (onela::launch_s0_image(h->S0, h->S0img, c.R, c.H, c.d_k, c.d_v, c.s0_dtype == ONELA_BF16, h->planes, s) !=
+        cudaSuccess)
+      return ONELA_ERR_CUDA;
+  }
+  rewind_to_prompt(h);
+  return ONELA_OK;
+}
+
+int onela_read_prompt_state(onela_handle *h, void *S0, onela_stream stream) {
+  if (!h || !S0) return ONELA_ERR_ARG;
+  if (!h->has_prompt) return ONELA_ERR_STATE;
+  DeviceGuard g(h->cfg.device);
+  if (!g.ok) return ONELA_ERR_CUDA;
+  const onela_config &c = h->cfg;
+  const size_t bytes = (size_t)c.R * c.H * c.d_v * c.d_k * esize(c.s0_dtype);
+  if (cudaMemcpyAsync(S0, h->S0, bytes, cudaMemcpyDeviceToDevice, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return ONELA_ERR_CUDA;
   return ONELA_OK;
 }
 

@@ -23,8 +23,8 @@ def declared_symbols():
 
 def test_header_declares_the_decode_entry_points():
     names = declared_symbols()
-    for n in ("onela_create", "onela_set_prompt_state", "onela_decode_step", "onela_reset",
-              "onela_status", "onela_destroy"):
+    for n in ("onela_create", "onela_set_prompt_state", "onela_prefill", "onela_decode_step",
+              "onela_reset", "onela_status", "onela_destroy"):
         assert n in names
 
 
@@ -72,6 +72,8 @@ def test_null_arguments_are_rejected():
     assert lib.onela_destroy(None) == L.ONELA_ERR_ARG
     assert lib.onela_read_records(None, 1, None, None, None, None) == L.ONELA_ERR_ARG
     assert lib.onela_read_ancestry(None, 1, None, None) == L.ONELA_ERR_ARG
+    assert lib.onela_prefill(None, 4, None, None, None, None, None) == L.ONELA_ERR_ARG
+    assert lib.onela_read_prompt_state(None, None, None) == L.ONELA_ERR_ARG
     assert lib.onela_steps_done(None) == -1
 
 
