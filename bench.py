@@ -148,18 +148,25 @@ def time_prefill(wl, device, stream, flush, reps=10, warmup=3):
     beta = torch.from_numpy(b).float().to(device)
     dec = L.BeamDecoder(wl.R, wl.H, wl.d_k, wl.d_v, wl.W, wl.T, wl.s0_dtype, wl.qkv_dtype, device=device.index)
     with torch.cuda.stream(stream):
+        dec.prefill(kd, vd, g, beta, stream=stream)
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()   # the launches alone, without the host's call overhead
+    with torch.cuda.graph(graph, stream=stream):
+        dec.prefill(kd, vd, g, beta, stream=stream)
+    with torch.cuda.stream(stream):
         for _ in range(warmup):
             flush.fill_(5)
-            dec.prefill(kd, vd, g, beta, stream=stream)
+            graph.replay()
     stream.synchronize()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
     with torch.cuda.stream(stream):
         for i, (e0, e1) in enumerate(ev):
             flush.fill_(i & 0xFF)
             e0.record(stream)
-            dec.prefill(kd, vd, g, beta, stream=stream)
+            graph.replay()
             e1.record(stream)
     stream.synchronize()
+    del graph
     assert dec.status() == 0
     dec.close()
     ms = max_over_ranks(sum(e0.elapsed_time(e1) for e0, e1 in ev) / reps, device)
@@ -184,6 +191,62 @@ def time_prefill(wl, device, stream, flush, reps=10, warmup=3):
                      "hbm_bytes": int(bytes_), "hbm_frac": round(bytes_ / (ms / 1e3) / 1e9 / measured_peaks()[0], 4)},
         "cpu_baseline": {"value": round(Ls / el, 1), "unit": "prompt token·head steps/s", "cores": 1,
                          "kind": "oracle", "sample": f"one head, first {Ls} tokens, numpy fp64 prefill, {el:.2f} s"},
+    }
+
+
+def time_select(device, stream, flush, R=1, W_prev=256, C=256, W=256, reps=20, warmup=3):
+    """Device time of onela_select_beams for one decode step's beam set
+    (W_prev beams x C children -> W), L2 flushed before each call; the
+    oracle's selection on the host for the same inputs.  Returns the JSON
+    object for the bench line."""
+    import linear_attention_beam_shared_b200 as L
+    from oracle import beam
+    rng = np.random.default_rng(77)
+    bs = (-rng.exponential(3.0, (R, W_prev))).astype(np.float32)
+    lp = np.log(rng.dirichlet(np.ones(C), (R, W_prev))).astype(np.float32)
+    bsd, lpd = torch.from_numpy(bs).to(device), torch.from_numpy(lp).to(device)
+    out = (torch.empty((R, W), dtype=torch.int32, device=device), torch.empty((R, W), dtype=torch.int32, device=device),
+           torch.empty((R, W), dtype=torch.float32, device=device),
+           torch.empty(int(L._lib.lib.onela_select_scratch_bytes(R, W_prev, C, W)), dtype=torch.uint8, device=device))
+    with torch.cuda.stream(stream):
+        L.onela_select_beams(bsd, lpd, W, stream=stream, out=out)
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()   # the launches alone, without the host's call overhead
+    with torch.cuda.graph(graph, stream=stream):
+        L.onela_select_beams(bsd, lpd, W, stream=stream, out=out)
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            flush.fill_(7)
+            graph.replay()
+    stream.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    with torch.cuda.stream(stream):
+        for i, (e0, e1) in enumerate(ev):
+            flush.fill_(i & 0xFF)
+            e0.record(stream)
+            graph.replay()
+            e1.record(stream)
+    stream.synchronize()
+    del graph
+    ms = max_over_ranks(sum(e0.elapsed_time(e1) for e0, e1 in ev) / reps, device)
+    ref = beam.select_beams(bs, lp, W)
+    assert all(np.array_equal(o.cpu().numpy(), r) for o, r in zip(out[:2], ref[:2])), "selection differs from the oracle"
+    bytes_ = R * W_prev * C * 4 + R * W_prev * 4 + R * W * 12
+    t0 = time.perf_counter()
+    reps_cpu = 0
+    while time.perf_counter() - t0 < 1.0:
+        beam.select_beams(bs, lp, W)
+        reps_cpu += 1
+    el = time.perf_counter() - t0
+    hbm = measured_peaks()[0]
+    return {
+        "workload": f"R={R}, W_prev={W_prev} beams x C={C} children -> W={W}, fp32 scores",
+        "ms": round(ms, 5), "value": round(R * W_prev * C / (ms / 1e3), 1), "unit": "candidates/s",
+        "roofline": {"bound": "hbm", "achieved": round(bytes_ / (ms / 1e3) / 1e9, 2), "peak": hbm, "unit": "GB/s",
+                     "frac": round(bytes_ / (ms / 1e3) / 1e9 / hbm, 5), "alg_bytes": bytes_},
+        "launches": 2,
+        "cpu_baseline": {"value": round(R * W_prev * C * reps_cpu / el, 1), "unit": "candidates/s", "cores": 1,
+                         "kind": "oracle", "sample": f"the same inputs x{reps_cpu} in {el:.2f} s, numpy sort"},
     }
 
 
@@ -411,6 +474,7 @@ def run_ours(args):
     assert dec.status() == 0
 
     prefill = time_prefill(wl, device, stream, flush) if (wl.L_prompt > 0 and not args.no_prefill) else None
+    select = None if args.no_prefill else time_select(device, stream, flush, R=wl.R, W_prev=wl.W, C=256, W=wl.W)
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu:
@@ -435,7 +499,7 @@ def run_ours(args):
                        "programmatic_launch": not args.no_pdl},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "clocks": clk.summary(), "gpu_launches": launches * args.steps,
-            "prefill": prefill,
+            "prefill": prefill, "beam_select": select,
         }
         print(json.dumps(line))
     if ws > 1:
@@ -489,7 +553,7 @@ def main():
     ap.add_argument("--no-pdl", action="store_true",
                     help="launch every step only after the previous one has finished")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
-    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill timing")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill and beam-selection timings")
     ap.add_argument("--s0", choices=["prefill", "direct"], default="prefill",
                     help="S0 from the GDN recurrence over the synthetic prompt (default) or drawn "
                          "directly; the decode's work does not depend on the S0 values")

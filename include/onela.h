@@ -195,6 +195,32 @@ ONELA_API int onela_decode_step(onela_handle *h, int32_t W_prev, int32_t W,
                       const int32_t *parent_idx, float *o,
                       onela_stream stream);
 
+/* Beam selection on the device: the next beam set out of the children of
+ * the current one (the evolving beam tree of the abstract), so that the
+ * parent indices of the next decode step never leave the GPU.  For request r
+ * the candidate (b, c), b < W_prev, c < C, scores
+ *     s = beam_score[r][b] + logp[r][b][c]      (one fp32 addition)
+ * and the W candidates with the largest s are kept, best first; equal scores
+ * (+0 and -0 are equal) go to the smaller flat index b*C + c; NaN ranks below
+ * every number.  Outputs, DEVICE [R][W]:
+ *   parent_idx  int32, b of the candidate (the next step's parent_idx),
+ *   token       int32, c of the candidate,
+ *   score       fp32, s (the next step's beam_score).
+ *   beam_score  DEVICE fp32 [R][W_prev]; logp DEVICE fp32 [R][W_prev][C].
+ *   scratch     DEVICE buffer of at least onela_select_scratch_bytes(R,
+ *               W_prev, C, W) bytes, owned by the caller, borrowed for the
+ *               stream-ordered duration of the call.
+ * Sizes: R <= 65535, 1 <= W <= 2048, W <= W_prev * C < 2^32.  No host
+ * synchronisation; capturable in a CUDA graph.
+ * Errors: ONELA_ERR_ARG (null pointer, bad size), ONELA_ERR_SCRATCH (scratch
+ * too small), ONELA_ERR_CUDA. */
+ONELA_API size_t onela_select_scratch_bytes(int32_t R, int32_t W_prev, int32_t C, int32_t W);
+ONELA_API int onela_select_beams(int32_t R, int32_t W_prev, int32_t C, int32_t W,
+                                 const float *beam_score, const float *logp,
+                                 int32_t *parent_idx, int32_t *token, float *score,
+                                 void *scratch, size_t scratch_bytes, int32_t device,
+                                 onela_stream stream);
+
 /* Rewind to step 0 keeping S0 (records are logically dropped, nothing is
  * freed) and clear the error word.  Waits for `stream` first, so that no
  * step still in flight can set the word after it is cleared; not meant for

@@ -22,7 +22,8 @@ from ._lib import (  # noqa: F401
     ONELA_ERR_STATE, ONELA_ERR_UNSUPPORTED, ONELA_F32, ONELA_FLAG_PDL, ONELA_KERNEL_AUTO, ONELA_KERNEL_SIMT,
     ONELA_ERR_SCRATCH, ONELA_KERNEL_TC, ONELA_OK, Handle, OnelaError, error_string, onela_create,
     onela_decode_step, onela_decode_step_noalloc, onela_destroy, onela_kernel_kind, onela_prefill,
-    onela_read_ancestry, onela_read_prompt_state, onela_read_records, onela_reset, onela_set_prompt_state,
+    onela_read_ancestry, onela_read_prompt_state, onela_read_records, onela_reset, onela_select_beams,
+    onela_set_prompt_state,
     onela_status, onela_status_code, onela_steps_done,
 )
 

@@ -51,6 +51,9 @@ def _load() -> ctypes.CDLL:
         "onela_set_prompt_state": ([vp, vp, vp], ctypes.c_int),
         "onela_prefill": ([vp, i32, vp, vp, vp, vp, vp], ctypes.c_int),
         "onela_read_prompt_state": ([vp, vp, vp], ctypes.c_int),
+        "onela_select_scratch_bytes": ([i32, i32, i32, i32], ctypes.c_size_t),
+        "onela_select_beams": ([i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, i32, vp],
+                               ctypes.c_int),
         "onela_decode_step": ([vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         "onela_reset": ([vp, vp], ctypes.c_int),
         "onela_status": ([vp, ctypes.POINTER(i32)], ctypes.c_int),
@@ -151,6 +154,33 @@ def onela_prefill(h: Handle, k, v, g, beta, stream=None) -> None:
         _ptr(beta, "beta", torch.float32, (c.R, L, c.H), c.device),
     )
     _check(lib.onela_prefill(h.ptr, L, *args, _stream(stream)), "onela_prefill")
+
+
+def onela_select_beams(beam_score: torch.Tensor, logp: torch.Tensor, W: int, stream=None, out=None):
+    """beam_score fp32 [R][W_prev], logp fp32 [R][W_prev][C] on one CUDA device.
+    Returns (parent_idx int32 [R][W], token int32 [R][W], score fp32 [R][W]).
+    ``out`` = (parent_idx, token, score, scratch) reuses caller tensors (no
+    allocation, e.g. inside a captured CUDA graph); scratch is a uint8 tensor
+    of at least onela_select_scratch_bytes bytes."""
+    if not isinstance(logp, torch.Tensor) or logp.dim() != 3:
+        raise ValueError("logp must be a 3-D tensor [R][W_prev][C]")
+    R, W_prev, C = (int(x) for x in logp.shape)
+    dev = logp.device
+    args = (_ptr(beam_score, "beam_score", torch.float32, (R, W_prev), dev.index),
+            _ptr(logp, "logp", torch.float32, (R, W_prev, C), dev.index))
+    nbytes = int(lib.onela_select_scratch_bytes(R, W_prev, C, int(W)))
+    if out is None:
+        parent = torch.empty((R, W), dtype=torch.int32, device=dev)
+        token = torch.empty((R, W), dtype=torch.int32, device=dev)
+        score = torch.empty((R, W), dtype=torch.float32, device=dev)
+        scratch = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+    else:
+        parent, token, score, scratch = out
+        nbytes = scratch.numel()
+    _check(lib.onela_select_beams(R, W_prev, C, int(W), *args, _ptr(parent, "parent"), _ptr(token, "token"),
+                                  _ptr(score, "score"), _ptr(scratch, "scratch"), nbytes, dev.index,
+                                  _stream(stream)), "onela_select_beams")
+    return parent, token, score
 
 
 def onela_read_prompt_state(h: Handle, stream=None) -> torch.Tensor:

@@ -77,5 +77,9 @@ size_t s0_image_bytes(int R, int H, int dk, int dv, int planes);
 cudaError_t launch_prefill(const void *k, const void *v, const float *g, const float *beta, void *S0, int R, int L,
                            int H, int dk, int dv, int qkv_bf16, int s0_bf16, cudaStream_t s);
 bool tc_supports(int dk, int dv, int qkv_bf16, int T_max, int W_max);
+// Beam selection (select.cu): the W best of W_prev x C candidates per request.
+size_t select_scratch_bytes(int R, int W_prev, int C, int W);
+cudaError_t launch_select(const float *beam_score, const float *logp, int R, int W_prev, int C, int W,
+                          int32_t *parent, int32_t *token, float *score, void *scratch, cudaStream_t s);
 
 }  // namespace onela

@@ -211,6 +211,29 @@ int onela_prefill(onela_handle *h, int32_t L, const void *k, const void *v, cons
   return ONELA_OK;
 }
 
+size_t onela_select_scratch_bytes(int32_t R, int32_t W_prev, int32_t C, int32_t W) {
+  if (R < 1 || W_prev < 1 || C < 1 || W < 1) return 0;
+  return onela::select_scratch_bytes(R, W_prev, C, W);
+}
+
+int onela_select_beams(int32_t R, int32_t W_prev, int32_t C, int32_t W, const float *beam_score, const float *logp,
+                       int32_t *parent_idx, int32_t *token, float *score, void *scratch, size_t scratch_bytes,
+                       int32_t device, onela_stream stream) {
+  if (!beam_score || !logp || !parent_idx || !token || !score || !scratch) return ONELA_ERR_ARG;
+  const long long N = (long long)W_prev * C;
+  if (R < 1 || R > 65535 || W_prev < 1 || C < 1 || W < 1 || W > 2048 || N < W || N > 0xffffffffLL || device < 0)
+    return ONELA_ERR_ARG;
+  if (scratch_bytes < onela::select_scratch_bytes(R, W_prev, C, W)) return ONELA_ERR_SCRATCH;
+  DeviceGuard g(device);
+  if (!g.ok) return ONELA_ERR_CUDA;
+  if (onela::launch_select(beam_score, logp, R, W_prev, C, W, parent_idx, token, score, scratch,
+                           static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return ONELA_ERR_CUDA;
+  }
+  return ONELA_OK;
+}
+
 int onela_read_prompt_state(onela_handle *h, void *S0, onela_stream stream) {
   if (!h || !S0) return ONELA_ERR_ARG;
   if (!h->has_prompt) return ONELA_ERR_STATE;

@@ -11,6 +11,8 @@ gdn     numpy fp64 reference: prefill, full-state beam tree, replay
         formulation (for the replay == full-state identity), ancestry walk.
 cref    ctypes loader for ``c/gdn_fullstate.c``: the same full-state beam tree
         in plain C (fp64, OpenMP over beams), the timed CPU baseline.
+beam    beam selection: the W best children (fp32 scores, ties to the smaller
+        flat index), numpy sort.
 
 Parity pins (what each function is checked against, tests/test_oracle_*.py):
 closed form of one step in exact rational arithmetic; the textbook gated delta
@@ -18,6 +20,7 @@ rule written in its matrix form; the delta rule's exact-recall property;
 replay == full state; W = 1 == sequential GDN; alpha = 1, beta = 0 leaves S0
 unchanged; beta = 0 is a pure gate product; ancestry by brute-force tree
 construction; linearity in (S0, v); permutation equivariance of beam labels;
-a hand-worked scalar example (tests/golden/).
+a hand-worked scalar example (tests/golden/).  Beam selection: brute-force
+ordering of Python tuples, fp32 rounding ties, signed zeros, NaN and -inf.
 """
 from . import gdn  # noqa: F401

@@ -75,6 +75,20 @@ def test_null_arguments_are_rejected():
     assert lib.onela_prefill(None, 4, None, None, None, None, None) == L.ONELA_ERR_ARG
     assert lib.onela_read_prompt_state(None, None, None) == L.ONELA_ERR_ARG
     assert lib.onela_steps_done(None) == -1
+    assert lib.onela_select_beams(1, 4, 4, 2, *([None] * 6), 0, 0, None) == L.ONELA_ERR_ARG
+
+
+def test_select_rejects_bad_sizes_on_the_host():
+    import linear_attention_beam_shared_b200 as L
+    lib = L._lib.lib
+    p = ctypes.c_void_p(16)  # never dereferenced: the checks come first
+    args = (p, p, p, p, p, p)
+    assert lib.onela_select_beams(1, 4, 4, 2049, *args, 1 << 30, 0, None) == L.ONELA_ERR_ARG  # W > 2048
+    assert lib.onela_select_beams(1, 2, 2, 5, *args, 1 << 30, 0, None) == L.ONELA_ERR_ARG     # W > W_prev C
+    assert lib.onela_select_beams(0, 4, 4, 2, *args, 1 << 30, 0, None) == L.ONELA_ERR_ARG     # R = 0
+    need = lib.onela_select_scratch_bytes(2, 256, 256, 256)
+    assert need == 2 * 2 * 16 * 256 * 8
+    assert lib.onela_select_beams(2, 256, 256, 256, *args, need - 1, 0, None) == L.ONELA_ERR_SCRATCH
 
 
 def test_binding_refuses_cpu_tensors():
