@@ -14,9 +14,10 @@
 // Stage 1 (one CTA per chunk of kChunk candidates and request) finds the
 // chunk's K = W largest keys by radix selection: eight passes over the 64-bit
 // keys, 8 bits at a time from the top, each building a 256-bin histogram of
-// the keys that still match the prefix chosen so far (warp-aggregated
-// shared-memory atomics) and fixing the next 8 bits of the K-th largest key;
-// every key >= that key is kept.  Merge rounds select the W largest of
+// the keys that still match the prefix chosen so far (shared-memory
+// atomics) and fixing the next 8 bits of the K-th largest key, stopping early
+// once the chosen bin holds exactly the keys still wanted; every key >= the
+// threshold is kept.  Merge rounds select the W largest of
 // groups of survivor lists the same way, until one list per request is left;
 // the last round orders it (each key's rank is the number of larger keys)
 // and writes parent, token and score.
@@ -47,6 +48,7 @@ struct SelectSmem {
   uint64_t prefix;   // bits of the K-th largest key fixed so far
   int want;          // how many keys still to take at or below the prefix
   int count;         // keys written so far
+  int done;          // the chosen bin holds exactly the keys still wanted
 };
 
 // The K-th largest of the block's keys (kPer per thread in k[], absent ones
@@ -57,6 +59,7 @@ __device__ uint64_t kth_largest(const uint64_t (&k)[kPer], int K, SelectSmem &sm
   if (tid == 0) {
     sm.prefix = 0;
     sm.want = K;
+    sm.done = 0;
   }
 #pragma unroll 1
   for (int pass = 0; pass < 8; ++pass) {
@@ -69,11 +72,7 @@ __device__ uint64_t kth_largest(const uint64_t (&k)[kPer], int K, SelectSmem &sm
     for (int i = 0; i < kPer; ++i) {
       const bool act = (k[i] & hi_mask) == prefix;
       const uint32_t d = (uint32_t)(k[i] >> shift) & 255u;
-      const unsigned m = __ballot_sync(0xffffffffu, act);
-      if (act) {
-        const unsigned peers = __match_any_sync(m, d);
-        if (lane == __ffs(peers) - 1) atomicAdd(&sm.hist[d], (uint32_t)__popc(peers));
-      }
+      if (act) atomicAdd(&sm.hist[d], 1u);
     }
     __syncthreads();
     if (tid < 32) {
@@ -99,12 +98,16 @@ __device__ uint64_t kth_largest(const uint64_t (&k)[kPer], int K, SelectSmem &sm
           if (run < want && want <= run + c[q]) {
             sm.prefix = prefix | ((uint64_t)(255 - 8 * lane - q) << shift);
             sm.want = (int)(want - run);
+            // Every key of this bin is wanted: the threshold is the bin's
+            // lowest possible key (the remaining bits zero).
+            if (want == run + c[q]) sm.done = 1;
           }
           run += c[q];
         }
       }
     }
     __syncthreads();
+    if (sm.done) break;
   }
   return sm.prefix;
 }
