@@ -20,7 +20,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
-import glob
+
 import json
 import os
 import statistics
@@ -80,12 +80,14 @@ def measured_peaks():
     return 6650.0, 1590.0, 1400.0, "fallback"
 
 
-def kernel_source_hash():
-    """Hash of the kernel sources with comments and blank lines removed, so
-    that a change of wording alone keeps the recorded counters valid."""
+def kernel_source_hash(kind="tc"):
+    """Hash of the decode kernel's source file (step_tc.cu or step_simt.cu)
+    with comments and blank lines removed, so that a change of wording, or a
+    change to another kernel of the library, keeps the recorded counters
+    valid."""
     import re
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "linear_attention_beam_shared_b200", "csrc", "*"))):
+    for p in [os.path.join(ROOT, "linear_attention_beam_shared_b200", "csrc", f"step_{kind}.cu")]:
         with open(p, "r", encoding="utf-8", errors="replace") as f:
             text = f.read()
         text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
@@ -104,7 +106,7 @@ def ncu_traffic(kernel_kind):
     with open(path) as f:
         d = json.load(f)
     entry = d.get(kernel_kind)
-    if not entry or entry.get("source_hash") != kernel_source_hash():
+    if not entry or entry.get("source_hash") != kernel_source_hash(kernel_kind):
         return None
     return entry
 

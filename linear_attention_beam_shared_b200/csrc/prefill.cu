@@ -8,10 +8,12 @@
 // from S_0 = 0 over the L prompt tokens, in fp32.
 //
 // Row i of S evolves on its own: u_i = S[i,:] . k_l uses only row i, and
-// the update of row i needs only delta_i.  So one CTA takes 32 rows of one
-// (request, head); each row is held in the registers of 8 threads (EPT
-// consecutive elements each), and per token the 8 threads form their
-// partial dot product, sum it in 3 shuffles, and update their elements.  The tokens'
+// the update of row i needs only delta_i.  So one CTA takes 16 rows of one
+// (request, head) (small blocks spread the heads over every SM); each row is
+// held in the registers of 8 threads (EPT consecutive elements each), and
+// per token the 8 threads form their partial dot product, sum it in 3
+// shuffles, and update their elements, with the next token's operands
+// already on their way from shared memory.  The tokens'
 // k, v, gate and beta stream through shared memory in chunks of kTC tokens
 // (cp.async, double-buffered); the gates of a chunk become alpha = exp(g)
 // once per token, not once per thread.
@@ -23,7 +25,7 @@
 namespace onela {
 namespace {
 
-constexpr int kRB = 32;       // rows of S per CTA
+constexpr int kRB = 16;       // rows of S per CTA
 constexpr int kTPR = 8;       // threads per row
 constexpr int kPThreads = kRB * kTPR;
 constexpr int kTC = 32;       // tokens per staged chunk
@@ -152,25 +154,34 @@ __global__ void __launch_bounds__(kPThreads) prefill_kernel(const T *k, const T 
     __syncthreads();
     if (tid < n) cur.alpha[tid] = expf(cur.g[tid]);
     __syncthreads();
+    // The next token's operands are loaded while this token's sum is reduced.
+    float kk[EPT];
+    load_row_part<T, EPT>(kk, &cur.k[0][part * EPT]);
+    float a = cur.alpha[0], bt = cur.beta[0], vi = row < dv ? to_f(cur.v[0][rr]) : 0.f;
 #pragma unroll 1
     for (int tl = 0; tl < n; ++tl) {
-      float kk[EPT];
-      load_row_part<T, EPT>(kk, &cur.k[tl][part * EPT]);
-      float p0 = 0.f, p1 = 0.f;
+      float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
 #pragma unroll
-      for (int e = 0; e < EPT; e += 2) {
+      for (int e = 0; e < EPT; e += 4) {
         p0 = fmaf(s[e], kk[e], p0);
         p1 = fmaf(s[e + 1], kk[e + 1], p1);
+        p2 = fmaf(s[e + 2], kk[e + 2], p2);
+        p3 = fmaf(s[e + 3], kk[e + 3], p3);
       }
-      float u = p0 + p1;
+      float u = (p0 + p1) + (p2 + p3);
+      float kn[EPT];
+      const int tn = tl + 1 < n ? tl + 1 : tl;
+      load_row_part<T, EPT>(kn, &cur.k[tn][part * EPT]);
+      const float an = cur.alpha[tn], bn = cur.beta[tn], vn = row < dv ? to_f(cur.v[tn][rr]) : 0.f;
       u += __shfl_xor_sync(0xffffffffu, u, 1);
       u += __shfl_xor_sync(0xffffffffu, u, 2);
       u += __shfl_xor_sync(0xffffffffu, u, 4);
-      const float a = cur.alpha[tl];
-      const float vi = row < dv ? to_f(cur.v[tl][rr]) : 0.f;
-      const float delta = cur.beta[tl] * (vi - a * u);
+      const float delta = bt * (vi - a * u);
 #pragma unroll
       for (int e = 0; e < EPT; ++e) s[e] = fmaf(a, s[e], delta * kk[e]);
+#pragma unroll
+      for (int e = 0; e < EPT; ++e) kk[e] = kn[e];
+      a = an, bt = bn, vi = vn;
     }
     __syncthreads();  // this buffer is refilled by the next round's copies
   }
