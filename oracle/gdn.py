@@ -31,6 +31,10 @@ beam_decode_replay    the projection-replay formulation (records + ancestry),
                       in fp64; used only to check "replay == full state".
 ancestry_walk         pointer walk over the parent arrays (depth-ordered
                       ancestor beam indices of every beam).
+common_ancestor_depth the deepest depth whose ancestor every beam of a step
+                      shares (the folding extension).
+fold_state            the full state of that shared ancestor, taken from the
+                      full-state beam tree (the folding extension's result).
 
 Conventions: alpha = exp(g) in fp64 from the fp32 g the operator receives;
 every input is first converted exactly to fp64 (``to_f64``).
@@ -49,6 +53,8 @@ __all__ = [
     "beam_decode_fullstate",
     "beam_decode_replay",
     "ancestry_walk",
+    "common_ancestor_depth",
+    "fold_state",
 ]
 
 
@@ -113,17 +119,21 @@ def _step_inputs(step: Dict) -> tuple:
             to_f64(step["beta"]), np.asarray(step["parents"], dtype=np.int64))
 
 
-def beam_decode_fullstate(S0, steps: Sequence[Dict]) -> List[Dict[str, np.ndarray]]:
+def beam_decode_fullstate(S0, steps: Sequence[Dict], S_prev=None,
+                          keep_states: bool = False) -> List[Dict[str, np.ndarray]]:
     """The oracle: a full fp64 state per beam, copied from the parent.
 
     S0: [R][H][d_v][d_k] (any stored type; converted exactly to fp64).
     steps[t]: q, k [R][W][H][d_k]; v [R][W][H][d_v]; g (or alpha), beta
     [R][W][H]; parents [R][W] with values in [0, W_prev), W_prev = 1 at t = 1.
-    Returns per step: o, delta [R][W][H][d_v] and alpha [R][W][H] (fp64).
+    S_prev: optional [R][W_prev][H][d_v][d_k], the states of the beams the
+    first given step expands (default: S0 as the single root).
+    Returns per step: o, delta [R][W][H][d_v] and alpha [R][W][H] (fp64), and
+    with keep_states the states S_t [R][W][H][d_v][d_k] as "S".
     """
     S0 = to_f64(S0)
     R = S0.shape[0]
-    S_prev = S0[:, None]                     # [R][W_prev=1][H][d_v][d_k]
+    S_prev = S0[:, None] if S_prev is None else to_f64(S_prev)   # [R][W_prev][H][d_v][d_k]
     out = []
     for step in steps:
         q, k, v, alpha, beta, parents = _step_inputs(step)
@@ -137,6 +147,8 @@ def beam_decode_fullstate(S0, steps: Sequence[Dict]) -> List[Dict[str, np.ndarra
         S = a[..., None] * S + delta[..., :, None] * k[..., None, :]
         o = np.einsum("rwhij,rwhj->rwhi", S, q)                # S_t q_t
         out.append({"o": o, "delta": delta, "alpha": alpha})
+        if keep_states:
+            out[-1]["S"] = S
         S_prev = S
     return out
 
@@ -165,6 +177,52 @@ def ancestry_walk(parent_list: Sequence, t: int) -> np.ndarray:
             else:
                 node = np.take_along_axis(prev, node, axis=-1)
     return anc
+
+
+def common_ancestor_depth(parent_list: Sequence, t: int, max_depth: int):
+    """Per request, the deepest depth D <= max_depth at which every beam of
+    step t has the same ancestor, and that ancestor at each depth 1..D.
+
+    The beam of depth t itself counts as its own ancestor at depth t, so a
+    step that kept one beam shares depth t.  parent_list[s-1] holds the
+    parents [R][W_s] of step s.  Returns (D [R] int64, list of R int64 arrays
+    of length D_r with the shared ancestor at depths 1..D_r).
+    """
+    par = [np.asarray(p, dtype=np.int64) for p in parent_list]
+    R, W_t = par[t - 1].shape
+    # Path of every beam of step t, depth 1 .. t (its own index last).
+    paths = np.concatenate([ancestry_walk(par, t), np.broadcast_to(np.arange(W_t), (R, W_t))[..., None]],
+                           axis=-1)
+    D = np.zeros(R, dtype=np.int64)
+    shared = []
+    for r in range(R):
+        d = 0
+        while d < min(t, max_depth) and len(set(paths[r, :, d].tolist())) == 1:
+            d += 1
+        D[r] = d
+        shared.append(paths[r, 0, :d].copy())
+    return D, shared
+
+
+def fold_state(S0, steps: Sequence[Dict], D) -> np.ndarray:
+    """The state each request's decode replays from once depths 1..D[r] are
+    folded: the full state of the shared ancestor at depth D[r] (S0 where
+    D[r] = 0), read off the full-state beam tree.  [R][H][d_v][d_k] fp64."""
+    S0 = to_f64(S0)
+    D = np.asarray(D, dtype=np.int64)
+    out = S0.copy()
+    if D.max(initial=0) == 0:
+        return out
+    res = beam_decode_fullstate(S0, steps[:int(D.max())], keep_states=True)
+    t = len(steps)
+    _, shared = common_ancestor_depth([s["parents"] for s in steps], t, t)
+    for r in range(S0.shape[0]):
+        d = int(D[r])
+        if d > 0:
+            if len(shared[r]) < d:
+                raise ValueError("no shared ancestor at that depth")
+            out[r] = res[d - 1]["S"][r, shared[r][d - 1]]
+    return out
 
 
 def beam_decode_replay(S0, steps: Sequence[Dict]) -> List[Dict[str, np.ndarray]]:
