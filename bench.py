@@ -252,6 +252,119 @@ def time_select(device, stream, flush, R=1, W_prev=256, C=256, W=256, reps=20, w
     }
 
 
+def time_fold(wl, S0, kernel, device, stream, flush, T=16, every=4, reps=10, warmup=3, alone=True):
+    """Folding on a deeper decode: the workload's shapes over T steps, every
+    beam of steps every, 2 every, ... a child of one beam (the beam sets
+    narrow to one shared ancestor), decoded as one CUDA graph with a fold
+    right after each such step and, for comparison, without folds; then the
+    fold alone (after the first narrowing step, caches flushed).  The folded and unfolded outputs must agree to fp32 rounding.
+    Returns the JSON object for the bench line."""
+    import linear_attention_beam_shared_b200 as L
+    wd = wl.replace(name=wl.name + "_deep", T=T)
+    steps = synth.draw_decode(wd)
+    narrow = list(range(every - 1, T - 1, every))            # 0-based steps
+    for i in narrow:
+        steps[i]["parents"] = torch.zeros_like(steps[i]["parents"])
+    fold_after = {i + 1 for i in narrow}                     # fold after these steps (1-based)
+    dsteps = [{k: (v.to(device) if isinstance(v, torch.Tensor) else v) for k, v in st.items()} for st in steps]
+
+    def make(fold):
+        outs = [torch.empty((wd.R, st["W"], wd.H, wd.d_v), dtype=torch.float32, device=device) for st in steps]
+        dec = L.BeamDecoder(wd.R, wd.H, wd.d_k, wd.d_v, wd.W, T, wd.s0_dtype, wd.qkv_dtype, kernel=kernel,
+                            device=device.index, flags=L.ONELA_FLAG_PDL)
+        dec.set_prompt_state(S0.to(device))
+
+        def run():
+            for t, (st, o) in enumerate(zip(dsteps, outs), start=1):
+                dec.step(st["q"], st["k"], st["v"], st["g"], st["beta"], st["parents"], o=o, stream=stream)
+                if fold and t in fold_after:
+                    dec.fold(stream=stream)
+        with torch.cuda.stream(stream):
+            run()
+        stream.synchronize()
+        assert dec.status() == 0
+        depth = dec.fold_depth(stream).cpu().tolist()
+        dec.reset(stream)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            run()
+        dec.reset(stream)
+        return dec, g, outs, depth
+
+    def timed(graphs, pre=None):
+        for _ in range(warmup):
+            with torch.cuda.stream(stream):
+                if pre is not None:
+                    pre.replay()
+                flush.fill_(5)
+                graphs.replay()
+        stream.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        with torch.cuda.stream(stream):
+            for i, (e0, e1) in enumerate(ev):
+                if pre is not None:
+                    pre.replay()
+                flush.fill_(i & 0xFF)
+                e0.record(stream)
+                graphs.replay()
+                e1.record(stream)
+        stream.synchronize()
+        return max_over_ranks(sum(e0.elapsed_time(e1) for e0, e1 in ev) / reps, device)
+
+    res = {}
+    for fold in (True, False):
+        dec, g, outs, depth = make(fold)
+        ms = timed(g)
+        res[fold] = (ms, [o.clone() for o in outs], depth)
+        del g
+        dec.close()
+    diff = max(float((a - b).abs().max()) for a, b in zip(res[True][1], res[False][1]))
+    scale = max(float(b.abs().max()) for b in res[False][1])
+    assert diff <= 2e-5 * max(1.0, scale), f"folded decode differs from the unfolded one by {diff}"
+
+    out = {
+        "workload": f"{wl.name} shapes over T={T} steps (R={wd.R}, H={wd.H}, d={wd.d_k}, W={wd.W}), every beam of "
+                    f"steps {', '.join(str(i + 1) for i in narrow)} a child of beam 0; folds right after them",
+        "ms_per_decode": {"folded": round(res[True][0], 5), "unfolded": round(res[False][0], 5)},
+        "speedup": round(res[False][0] / res[True][0], 3),
+        "replayed_depths_max": {"folded": every, "unfolded": T - 1},
+        "fold_depth_at_end": res[True][2],
+        "max_abs_diff_folded_vs_unfolded": diff,
+    }
+    if not alone:
+        return out
+    # The fold alone: steps 1..every (one graph), then the fold (another).
+    dec = L.BeamDecoder(wd.R, wd.H, wd.d_k, wd.d_v, wd.W, T, wd.s0_dtype, wd.qkv_dtype, kernel=kernel,
+                        device=device.index, flags=L.ONELA_FLAG_PDL)
+    dec.set_prompt_state(S0.to(device))
+    outs = [torch.empty((wd.R, st["W"], wd.H, wd.d_v), dtype=torch.float32, device=device) for st in steps]
+    g_steps, g_fold = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_steps, stream=stream):
+        for st, o in zip(dsteps[:every], outs):
+            dec.step(st["q"], st["k"], st["v"], st["g"], st["beta"], st["parents"], o=o, stream=stream)
+    with torch.cuda.graph(g_fold, stream=stream):
+        dec.fold(stream=stream)
+    fold_ms = timed(g_fold, pre=g_steps)
+    D = dec.fold_depth(stream).cpu().tolist()
+    assert D == [every - 1] * wd.R, D
+    del g_steps, g_fold
+    dec.close()
+
+    s_b = 2 if wd.s0_dtype == "bf16" else 4
+    e_b = 2 if wd.qkv_dtype == "bf16" else 4
+    n_state = wd.R * wd.H * wd.d_v * wd.d_k
+    planes = 1 if wd.s0_dtype == "bf16" else 2
+    img = n_state * planes * 2 if kernel != L.ONELA_KERNEL_SIMT else 0
+    rec = (every - 1) * wd.R * wd.H * (4 + 4 * wd.d_v + e_b * wd.d_k)
+    fold_bytes = 2 * n_state * s_b + img + rec + wd.R * wd.W * (every - 1) * 4
+    hbm = measured_peaks()[0]
+    ach = fold_bytes / (fold_ms / 1e3) / 1e9
+    out["fold"] = {"us": round(fold_ms * 1e3, 3), "launches": 1 if img else 2, "depth": every - 1,
+                 "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s",
+                              "frac": round(ach / hbm, 5), "alg_bytes": int(fold_bytes)}}
+    return out
+
+
 def byte_model(wl, steps):
     """Algorithmic bytes of one whole decode (all T steps): every byte the
     method must move at least once, with each distinct ancestor record counted
@@ -477,6 +590,8 @@ def run_ours(args):
 
     prefill = time_prefill(wl, device, stream, flush) if (wl.L_prompt > 0 and not args.no_prefill) else None
     select = None if args.no_prefill else time_select(device, stream, flush, R=wl.R, W_prev=wl.W, C=256, W=wl.W)
+    fold = None if args.no_prefill else [time_fold(wl, S0, kernel, device, stream, flush, every=4),
+                                          time_fold(wl, S0, kernel, device, stream, flush, every=8, alone=False)]
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu:
@@ -501,7 +616,7 @@ def run_ours(args):
                        "programmatic_launch": not args.no_pdl},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "clocks": clk.summary(), "gpu_launches": launches * args.steps,
-            "prefill": prefill, "beam_select": select,
+            "prefill": prefill, "beam_select": select, "fold": fold,
         }
         print(json.dumps(line))
     if ws > 1:

@@ -221,12 +221,50 @@ ONELA_API int onela_select_beams(int32_t R, int32_t W_prev, int32_t C, int32_t W
                                  void *scratch, size_t scratch_bytes, int32_t device,
                                  onela_stream stream);
 
-/* Rewind to step 0 keeping S0 (records are logically dropped, nothing is
- * freed) and clear the error word.  Waits for `stream` first, so that no
+/* Rewind to step 0 keeping S0 (records and any fold are logically dropped,
+ * nothing is freed) and clear the error word.  Waits for `stream` first, so that no
  * step still in flight can set the word after it is cleared; not meant for
  * the inside of a captured region.
  * Errors: ONELA_ERR_ARG, ONELA_ERR_CUDA. */
 ONELA_API int onela_reset(onela_handle *h, onela_stream stream);
+
+/* Fold the shared ancestor prefix of every request into its root state, so
+ * that later steps replay only the records below it.  An extension of the
+ * method: the evolve.pub review's Summary and Weaknesses name the replay
+ * cost that grows with decode depth (every ancestor's record is replayed at
+ * every step).  For each request r, with t = steps done and W_t the beams of
+ * step t: D_r = the deepest depth <= max_depth at which all W_t beams have
+ * the same ancestor (D_r = t when W_t = 1; never below the depth already
+ * folded).  The root state becomes that ancestor's full state,
+ *     S <- alpha_d S + delta_d k_d^T   for the newly folded depths d,
+ * (the GDN recurrence of the review's section 3.2, equation 2) computed in
+ * fp32 from the records and stored in cfg.s0_dtype, and later steps replay
+ * depths D_r + 1 .. t' - 1 only.  The outputs stay those of the unfolded
+ * decode up to that one rounding of the folded state.  Records, ancestry
+ * rows (absolute depths) and the prompt state itself are unchanged;
+ * onela_reset, onela_set_prompt_state and onela_prefill return to the
+ * prompt state.  The depth limit of the decode stays T_max.
+ *   max_depth  >= 0; values above the steps done act as the steps done;
+ *              0 (or no step done yet) leaves everything as it is.
+ * Runs on the device only (no host synchronisation; capturable in a CUDA
+ * graph: the prompt state is never overwritten, so a captured decode that
+ * folds replays from the prompt each time); the next decode step is an
+ * ordinary launch even under ONELA_FLAG_PDL.  Memory: a second state buffer
+ * (and operand image, tensor-core kernel), allocated by onela_create.
+ * Errors: ONELA_ERR_ARG, ONELA_ERR_STATE (no prompt state), ONELA_ERR_PARENT
+ * (a bad parent index was seen: the ancestry is meaningless), ONELA_ERR_CUDA. */
+ONELA_API int onela_fold(onela_handle *h, int32_t max_depth, onela_stream stream);
+
+/* Copy the root state the decode replays from (the prompt state, or the
+ * folded state after onela_fold) into a caller DEVICE buffer on `stream`:
+ * [R][H][d_v][d_k] in cfg.s0_dtype.
+ * Errors: ONELA_ERR_ARG, ONELA_ERR_STATE, ONELA_ERR_CUDA. */
+ONELA_API int onela_read_root_state(onela_handle *h, void *S, onela_stream stream);
+
+/* Copy the folded depth D_r of every request into a caller DEVICE buffer of
+ * R int32 on `stream` (all 0 when nothing is folded).
+ * Errors: ONELA_ERR_ARG, ONELA_ERR_CUDA. */
+ONELA_API int onela_read_fold_depth(onela_handle *h, int32_t *depth, onela_stream stream);
 
 /* Wait for the handle's device (cudaDeviceSynchronize on it) and report the
  * error word in *device_err (0: none; bit 0: a bad parent index).

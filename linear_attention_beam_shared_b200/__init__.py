@@ -21,9 +21,9 @@ from ._lib import (  # noqa: F401
     ONELA_BF16, ONELA_ERR_ARG, ONELA_ERR_CAPACITY, ONELA_ERR_CUDA, ONELA_ERR_PARENT,
     ONELA_ERR_STATE, ONELA_ERR_UNSUPPORTED, ONELA_F32, ONELA_FLAG_PDL, ONELA_KERNEL_AUTO, ONELA_KERNEL_SIMT,
     ONELA_ERR_SCRATCH, ONELA_KERNEL_TC, ONELA_OK, Handle, OnelaError, error_string, onela_create,
-    onela_decode_step, onela_decode_step_noalloc, onela_destroy, onela_kernel_kind, onela_prefill,
-    onela_read_ancestry, onela_read_prompt_state, onela_read_records, onela_reset, onela_select_beams,
-    onela_set_prompt_state,
+    onela_decode_step, onela_decode_step_noalloc, onela_destroy, onela_fold, onela_kernel_kind, onela_prefill,
+    onela_read_ancestry, onela_read_fold_depth, onela_read_prompt_state, onela_read_records,
+    onela_read_root_state, onela_reset, onela_select_beams, onela_set_prompt_state,
     onela_status, onela_status_code, onela_steps_done,
 )
 
@@ -70,6 +70,17 @@ class BeamDecoder:
     def reset(self, stream=None):
         onela_reset(self.h, stream)
         self.W_prev, self.Ws = 1, []
+
+    def fold(self, max_depth=None, stream=None):
+        """Fold each request's shared ancestor prefix (down to max_depth,
+        default: as deep as it goes) into its root state (see onela_fold)."""
+        onela_fold(self.h, len(self.Ws) if max_depth is None else max_depth, stream)
+
+    def root_state(self, stream=None):
+        return onela_read_root_state(self.h, stream)
+
+    def fold_depth(self, stream=None):
+        return onela_read_fold_depth(self.h, stream)
 
     def status(self) -> int:
         return onela_status(self.h)

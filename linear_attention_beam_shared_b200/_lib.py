@@ -56,6 +56,9 @@ def _load() -> ctypes.CDLL:
                                ctypes.c_int),
         "onela_decode_step": ([vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         "onela_reset": ([vp, vp], ctypes.c_int),
+        "onela_fold": ([vp, i32, vp], ctypes.c_int),
+        "onela_read_root_state": ([vp, vp, vp], ctypes.c_int),
+        "onela_read_fold_depth": ([vp, vp, vp], ctypes.c_int),
         "onela_status": ([vp, ctypes.POINTER(i32)], ctypes.c_int),
         "onela_destroy": ([vp], ctypes.c_int),
         "onela_read_records": ([vp, i32, vp, vp, vp, vp], ctypes.c_int),
@@ -209,6 +212,24 @@ def onela_decode_step(h: Handle, W_prev: int, W: int, q, k, v, g, beta, parent_i
 
 def onela_reset(h: Handle, stream=None) -> None:
     _check(lib.onela_reset(h.ptr, _stream(stream)), "onela_reset")
+
+
+def onela_fold(h: Handle, max_depth: int, stream=None) -> None:
+    _check(lib.onela_fold(h.ptr, int(max_depth), _stream(stream)), "onela_fold")
+
+
+def onela_read_root_state(h: Handle, stream=None) -> torch.Tensor:
+    c = h.cfg
+    S = torch.empty((c.R, c.H, c.d_v, c.d_k), dtype=_DT[c.s0_dtype], device=torch.device("cuda", c.device))
+    _check(lib.onela_read_root_state(h.ptr, _ptr(S, "S"), _stream(stream)), "onela_read_root_state")
+    return S
+
+
+def onela_read_fold_depth(h: Handle, stream=None) -> torch.Tensor:
+    c = h.cfg
+    d = torch.empty((c.R,), dtype=torch.int32, device=torch.device("cuda", c.device))
+    _check(lib.onela_read_fold_depth(h.ptr, _ptr(d, "depth"), _stream(stream)), "onela_read_fold_depth")
+    return d
 
 
 def onela_status(h: Handle) -> int:

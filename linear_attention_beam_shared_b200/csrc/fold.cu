@@ -1,0 +1,289 @@
+// Folding a shared ancestor prefix into the root state: an extension of the
+// method.  The evolve.pub review's Summary counts a replay cost that grows
+// with depth among the limitations, and its Weaknesses list replay depth as
+// unanalysed beyond small T: every ancestor's record is replayed at every
+// step, so a beam at depth t replays t - 1 records.
+//
+// Once every beam of a request descends from one beam c at depth D, the
+// records of c's chain (depths 1..D) are replayed identically by all of them.
+// Folding replaces the root state by c's full state,
+//     S_c = alpha_D S_{D-1} + delta_D k_D^T,  S_0 = the prompt state,
+// (the recurrence of the review's section 3.2 equations), after which the
+// decode kernels replay only depths D+1..t-1.  Nothing else changes: the
+// record store, the ancestry rows (still absolute depths) and the outputs
+// stay those of the unfolded decode, up to the rounding of S_c to the
+// state's storage type.
+//
+// The folded depth of each request is double-buffered (d0_in is read, d0_out
+// written), so that every CTA of a launch sees the same previous depth.
+//
+// Tensor-core handles: one launch, fold_tc_kernel.  Each CTA takes a block
+// of state rows of one (request, head): it loads its part of the state the
+// fold starts from (before waiting on the previous kernel, under
+// programmatic launch), finds the shared depth D itself (every CTA of the
+// request reads the same ancestry rows and agrees), stages the newly folded
+// records (alpha, its rows of delta, k) in shared memory, runs the
+// recurrence and writes the folded state and its bf16 operand image for the
+// tensor-core decode kernel.
+//
+// General handles: two ordinary launches,
+//   fold_plan_kernel   one CTA per request: D and the ancestors of the newly
+//                      folded depths;
+//   fold_state_kernel  one thread per state element: the recurrence.
+// Both run the recurrence in fp32 as S <- fma(delta_i, k_j, alpha S).
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "internal.h"
+#include "sm100_ptx.h"
+
+namespace onela {
+namespace {
+
+constexpr int kPlanThreads = 256;
+constexpr int kFoldThreads = 256;
+constexpr int kFoldMaxT = 16;  // deepest decode of the one-launch fold
+constexpr int kImgRows = 128;  // rows of an operand image atom
+
+__device__ __forceinline__ float ldf(const float *p, int64_t i) { return p[i]; }
+__device__ __forceinline__ float ldf(const __nv_bfloat16 *p, int64_t i) { return __bfloat162float(p[i]); }
+__device__ __forceinline__ void stf(float *p, int64_t i, float x) { p[i] = x; }
+__device__ __forceinline__ void stf(__nv_bfloat16 *p, int64_t i, float x) { p[i] = __float2bfloat16_rn(x); }
+
+__global__ void __launch_bounds__(kPlanThreads) fold_plan_kernel(const StepParams p, int Wt, int max_depth, int first,
+                                                                 const int32_t *d0_in, int32_t *d0_out,
+                                                                 int32_t *anc_fold) {
+  __shared__ int s_split;  // smallest row index at which two beams differ
+  const int r = blockIdx.x, tid = threadIdx.x, t = p.t, TM = p.T_max;
+  const int old = first ? 0 : d0_in[r];
+  const int n = t - 1;  // ancestry entries of a step-t beam (depths 1..t-1)
+  if (tid == 0) s_split = n;
+  __syncthreads();
+  const int32_t *row0 = p.anc + anc_row(p, t, r, 0);
+  for (int e = tid; e < (Wt - 1) * n; e += kPlanThreads) {
+    const int b = 1 + e / n, j = e - (b - 1) * n;
+    if (p.anc[anc_row(p, t, r, b) + j] != row0[j]) atomicMin(&s_split, j);
+  }
+  __syncthreads();
+  // Sharing an ancestor at a depth implies sharing its ancestors, so the
+  // shared depths are 1..s_split; a step that kept one beam shares it too.
+  int D = s_split;
+  if (D == n && Wt == 1) D = t;
+  if (D > max_depth) D = max_depth;
+  if (D < old) D = old;
+  for (int j = old + tid; j < D; j += kPlanThreads) anc_fold[(int64_t)r * TM + j] = j < n ? row0[j] : 0;
+  if (tid == 0) d0_out[r] = D;
+}
+
+template <typename QT, typename ST>
+__global__ void __launch_bounds__(kFoldThreads) fold_state_kernel(const StepParams p, int first, ST *S_fold,
+                                                                  const int32_t *d0_in, const int32_t *d0_out,
+                                                                  const int32_t *anc_fold) {
+  const int h = blockIdx.y, r = blockIdx.z;
+  const int from = first ? 0 : d0_in[r], D = d0_out[r];
+  if (!first && from == D) return;  // unchanged: S_fold already holds it
+  const int dk = p.dk, dv = p.dv;
+  const int64_t e = (int64_t)blockIdx.x * kFoldThreads + threadIdx.x;
+  if (e >= (int64_t)dv * dk) return;
+  const int i = (int)(e / dk), j = (int)(e - (int64_t)i * dk);
+  const int64_t idx = ((int64_t)r * p.H + h) * dv * dk + e;
+  const ST *src = first ? static_cast<const ST *>(p.S0) : S_fold;
+  float s = ldf(src, idx);
+  const QT *rec_k = static_cast<const QT *>(p.rec_k);
+#pragma unroll 1
+  for (int d = from + 1; d <= D; ++d) {
+    const int64_t row = rec_row(p, d, r, h, anc_fold[(int64_t)r * p.T_max + d - 1]);
+    const float a = p.rec_alpha[row];
+    s = fmaf(p.rec_delta[row * dv + i], ldf(rec_k, row * dk + j), a * s);
+  }
+  stf(S_fold, idx, s);
+}
+
+template <typename QT, typename ST>
+cudaError_t launch_state(const StepParams &p, int first, void *S_fold, const int32_t *d0_in, const int32_t *d0_out,
+                         const int32_t *anc_fold, cudaStream_t s) {
+  const int64_t n = (int64_t)p.dv * p.dk;
+  const dim3 grid((unsigned)((n + kFoldThreads - 1) / kFoldThreads), p.H, p.R);
+  fold_state_kernel<QT, ST><<<grid, kFoldThreads, 0, s>>>(p, first, static_cast<ST *>(S_fold), d0_in, d0_out,
+                                                          anc_fold);
+  return cudaGetLastError();
+}
+
+// 8 consecutive state elements (16- or 32-byte aligned) to and from fp32.
+__device__ __forceinline__ void ld8(const float *p, float (&x)[8]) {
+  const float4 a = reinterpret_cast<const float4 *>(p)[0], b = reinterpret_cast<const float4 *>(p)[1];
+  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+__device__ __forceinline__ void ld8(const __nv_bfloat16 *p, float (&x)[8]) {
+  const uint4 a = *reinterpret_cast<const uint4 *>(p);
+  const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&a);
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const float2 f = __bfloat1622float2(h2[u]);
+    x[2 * u] = f.x;
+    x[2 * u + 1] = f.y;
+  }
+}
+// Stores x in the state's type; x becomes the stored value.
+__device__ __forceinline__ void st8(float *p, float (&x)[8]) {
+  reinterpret_cast<float4 *>(p)[0] = make_float4(x[0], x[1], x[2], x[3]);
+  reinterpret_cast<float4 *>(p)[1] = make_float4(x[4], x[5], x[6], x[7]);
+}
+__device__ __forceinline__ void st8(__nv_bfloat16 *p, float (&x)[8]) {
+  __align__(16) __nv_bfloat16 o[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    o[u] = __float2bfloat16_rn(x[u]);
+    x[u] = __bfloat162float(o[u]);
+  }
+  *reinterpret_cast<uint4 *>(p) = *reinterpret_cast<const uint4 *>(o);
+}
+
+// One launch: plan, recurrence, folded state and its operand image.  Block:
+// kFoldThreads threads, DK / 8 per state row (8 columns each), so RB rows.
+template <typename ST, int DK>
+__global__ void __launch_bounds__(kFoldThreads) fold_tc_kernel(const StepParams p, int Wt, int max_depth, int first,
+                                                               const int32_t *d0_in, int32_t *d0_out,
+                                                               int32_t *anc_fold, ST *S_fold, uint4 *img) {
+  constexpr int TPR = DK / 8, RB = kFoldThreads / TPR, NK = DK / 64;
+  __shared__ int s_split;
+  __shared__ int s_row0[kFoldMaxT];
+  __shared__ float s_a[kFoldMaxT];
+  __shared__ float s_d[kFoldMaxT][RB];
+  __shared__ float s_k[kFoldMaxT][DK];
+  const int h = blockIdx.y, r = blockIdx.z, tid = threadIdx.x;
+  const int dv = p.dv, t = p.t, n = t - 1;
+  const int i0 = blockIdx.x * RB, ir = tid / TPR, c = tid - ir * TPR, i = i0 + ir;
+  const bool valid = i < dv;
+  const int64_t rh = (int64_t)r * p.H + h;
+  const int64_t si = (rh * dv + i) * DK + c * 8;
+
+  // The state the fold starts from: the prompt state, or the folded state of
+  // an earlier fold (complete before the kernels this one follows began).
+  float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  if (valid) ld8((first ? static_cast<const ST *>(p.S0) : S_fold) + si, x);
+  const int old = first ? 0 : d0_in[r];
+  if (tid == 0) s_split = n;
+  // The ancestry rows and records of step t come from the previous kernel.
+  ptx::pdl_wait();
+  const int32_t *row0 = p.anc + anc_row(p, t, r, 0);
+  if (tid < n) s_row0[tid] = row0[tid];
+  __syncthreads();
+  // Each thread compares whole rows of its beams, all entries loaded at once.
+  const int jhi = min(n, max_depth);
+  for (int b = 1 + tid; b < Wt; b += kFoldThreads) {
+    const int32_t *row = p.anc + anc_row(p, t, r, b);
+    int v[kFoldMaxT];
+#pragma unroll
+    for (int j = 0; j < kFoldMaxT; ++j) v[j] = (j >= old && j < jhi) ? row[j] : 0;
+    int split = n;
+#pragma unroll
+    for (int j = kFoldMaxT - 1; j >= 0; --j)
+      if (j >= old && j < jhi && v[j] != s_row0[j]) split = j;
+    if (split < n) atomicMin(&s_split, split);
+  }
+  __syncthreads();
+  int D = s_split;
+  if (D == n && Wt == 1) D = t;
+  if (D > max_depth) D = max_depth;
+  if (D < old) D = old;
+  if (blockIdx.x == 0 && h == 0) {
+    for (int j = old + tid; j < D; j += kFoldThreads) anc_fold[(int64_t)r * p.T_max + j] = j < n ? s_row0[j] : 0;
+    if (tid == 0) d0_out[r] = D;
+  }
+  if (!first && D == old) return;  // unchanged: the folded state and image hold it
+
+  const int nd = D - old;
+  const __nv_bfloat16 *rec_k = static_cast<const __nv_bfloat16 *>(p.rec_k);
+  for (int e = tid; e < nd * (1 + RB + DK); e += kFoldThreads) {
+    const int dd = e / (1 + RB + DK), q = e - dd * (1 + RB + DK);
+    const int d = old + dd + 1;
+    const int64_t row = rec_row(p, d, r, h, d - 1 < n ? s_row0[d - 1] : 0);
+    if (q == 0)
+      s_a[dd] = p.rec_alpha[row];
+    else if (q <= RB)
+      s_d[dd][q - 1] = i0 + q - 1 < dv ? p.rec_delta[row * dv + i0 + q - 1] : 0.f;
+    else
+      s_k[dd][q - 1 - RB] = __bfloat162float(rec_k[row * DK + q - 1 - RB]);
+  }
+  __syncthreads();
+  if (!valid) return;
+#pragma unroll 1
+  for (int dd = 0; dd < nd; ++dd) {
+    const float a = s_a[dd], dl = s_d[dd][ir];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) x[u] = fmaf(dl, s_k[dd][c * 8 + u], a * x[u]);
+  }
+  st8(S_fold + si, x);
+  // The operand image: plane pl holds the bf16 term pl of the split of the
+  // stored value (hi, then the bf16 rounding of what is left, ...).
+  const int planes = p.s0_planes, ka = c >> 3, cc = c & 7;
+  float rest[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) rest[u] = x[u];
+  for (int pl = 0; pl < planes; ++pl) {
+    __align__(16) __nv_bfloat16 o[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      o[u] = __float2bfloat16_rn(rest[u]);
+      rest[u] = rest[u] - __bfloat162float(o[u]);
+    }
+    const int64_t off = ((rh * planes + pl) * NK + ka) * (kImgRows * 128) + ptx::swz128(i, cc);
+    img[off / 16] = *reinterpret_cast<const uint4 *>(o);
+  }
+}
+
+template <typename ST, int DK>
+cudaError_t launch_tc(const StepParams &p, int Wt, int max_depth, int first, const int32_t *d0_in, int32_t *d0_out,
+                      int32_t *anc_fold, void *S_fold, void *img, int pdl, cudaStream_t s) {
+  constexpr int RB = kFoldThreads / (DK / 8);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((p.dv + RB - 1) / RB, p.H, p.R);
+  cfg.blockDim = dim3(kFoldThreads, 1, 1);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, fold_tc_kernel<ST, DK>, p, Wt, max_depth, first, d0_in, d0_out, anc_fold,
+                            static_cast<ST *>(S_fold), static_cast<uint4 *>(img));
+}
+
+bool fold_args_ok(const StepParams &p, int Wt, int max_depth) {
+  return p.t >= 1 && Wt >= 1 && Wt <= p.W_max && max_depth >= 0 && max_depth <= p.t && p.R >= 1 && p.R <= 65535 &&
+         p.H <= 65535;
+}
+
+}  // namespace
+
+cudaError_t launch_fold(const StepParams &p, int Wt, int max_depth, int first, const int32_t *d0_in, int32_t *d0_out,
+                        int32_t *anc_fold, void *S_fold, int qkv_bf16, int s0_bf16, cudaStream_t s) {
+  if (!fold_args_ok(p, Wt, max_depth)) return cudaErrorInvalidValue;
+  fold_plan_kernel<<<p.R, kPlanThreads, 0, s>>>(p, Wt, max_depth, first, d0_in, d0_out, anc_fold);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (qkv_bf16)
+    return s0_bf16 ? launch_state<__nv_bfloat16, __nv_bfloat16>(p, first, S_fold, d0_in, d0_out, anc_fold, s)
+                   : launch_state<__nv_bfloat16, float>(p, first, S_fold, d0_in, d0_out, anc_fold, s);
+  return s0_bf16 ? launch_state<float, __nv_bfloat16>(p, first, S_fold, d0_in, d0_out, anc_fold, s)
+                 : launch_state<float, float>(p, first, S_fold, d0_in, d0_out, anc_fold, s);
+}
+
+cudaError_t launch_fold_tc(const StepParams &p, int Wt, int max_depth, int first, const int32_t *d0_in,
+                           int32_t *d0_out, int32_t *anc_fold, void *S_fold, void *img, int s0_bf16, int pdl,
+                           cudaStream_t s) {
+  if (!fold_args_ok(p, Wt, max_depth) || p.T_max > kFoldMaxT || p.dk != p.dv || p.s0_planes < 1 ||
+      p.s0_planes > 3)
+    return cudaErrorInvalidValue;
+  if (p.dk == 64)
+    return s0_bf16 ? launch_tc<__nv_bfloat16, 64>(p, Wt, max_depth, first, d0_in, d0_out, anc_fold, S_fold, img, pdl, s)
+                   : launch_tc<float, 64>(p, Wt, max_depth, first, d0_in, d0_out, anc_fold, S_fold, img, pdl, s);
+  if (p.dk == 128)
+    return s0_bf16 ? launch_tc<__nv_bfloat16, 128>(p, Wt, max_depth, first, d0_in, d0_out, anc_fold, S_fold, img, pdl, s)
+                   : launch_tc<float, 128>(p, Wt, max_depth, first, d0_in, d0_out, anc_fold, S_fold, img, pdl, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace onela

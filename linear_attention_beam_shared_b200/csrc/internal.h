@@ -45,6 +45,12 @@ struct StepParams {
   float *rec_delta;       // [T_max][R][H][W_max][dv]
   void *rec_k;            // [T_max][R][H][W_max][dk] in the qkv type
   int32_t *anc;           // [T_max][R][W_max][T_max]
+  // Folded prefix (onela_fold), per request: depths 1..d0[r] are folded into
+  // S0 (then the folded state), their ancestors are the same for every beam
+  // of the request, anc_fold[r][j] at depth j + 1 ([R][T_max]), and only
+  // depths d0[r] + 1 .. t - 1 are replayed.  d0 null: nothing folded.
+  const int32_t *d0;
+  const int32_t *anc_fold;
   int32_t *err;           // host-mapped error word (device view)
   // TMA descriptors of k, q and v (tensor-core kernel; encoded per call):
   // 4-D {d, H, W, R} bf16, box {64, 1, 32, 1}, 128-byte swizzle.
@@ -68,6 +74,24 @@ constexpr int32_t kErrParent = 1;
 // Kernel launchers (step_simt.cu, step_tc.cu).  Return a cudaError_t.
 cudaError_t launch_step_simt(const StepParams &p, int qkv_bf16, int s0_bf16, cudaStream_t s);
 cudaError_t launch_step_tc(const StepParams &p, int pdl, cudaStream_t s);
+// Folds, per request, the deepest ancestor at depth <= max_depth that every
+// beam of step p.t shares into the folded state S_fold: reads the previous
+// folded depth from d0_in (unless first), writes the new one to d0_out and
+// the newly shared ancestors to anc_fold; S_fold becomes the ancestor's full
+// state, from S_fold (or p.S0 when first) by S <- alpha S + delta k^T over
+// the newly folded depths, fp32 arithmetic, stored in the state's type.
+// When first, every request's S_fold is written.  General shapes: two
+// ordinary launches.
+cudaError_t launch_fold(const StepParams &p, int Wt, int max_depth, int first, const int32_t *d0_in, int32_t *d0_out,
+                        int32_t *anc_fold, void *S_fold, int qkv_bf16, int s0_bf16, cudaStream_t s);
+// The same for tensor-core handles (bf16 keys, d_k = d_v in {64, 128},
+// T_max <= 16) in one launch that also writes S_fold's operand image (with
+// p.s0_planes terms); programmatic launch when pdl (the kernel waits before
+// it reads the ancestry rows and records; it reads S_fold and d0_in before,
+// so the previous kernel must not be a fold).
+cudaError_t launch_fold_tc(const StepParams &p, int Wt, int max_depth, int first, const int32_t *d0_in,
+                           int32_t *d0_out, int32_t *anc_fold, void *S_fold, void *img, int s0_bf16, int pdl,
+                           cudaStream_t s);
 cudaError_t launch_s0_image(const void *S0, void *img, int R, int H, int dk, int dv,
                             int s0_bf16, int planes, cudaStream_t s);
 size_t s0_image_bytes(int R, int H, int dk, int dv, int planes);

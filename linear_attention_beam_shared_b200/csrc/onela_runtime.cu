@@ -19,6 +19,17 @@ struct onela_handle {
   std::vector<int> Ws;  // beams of each step done
   void *S0;
   void *S0img;
+  // Folded prefix (onela_fold): the root state the decode replays from once
+  // folded, its operand image (tensor-core kernel), and on the device the
+  // folded depths d0 [2][R] (double-buffered: a fold reads one and writes
+  // the other) and anc_fold [R][T_max].  The prompt state and its image stay
+  // as they are, so a rewind needs no device work.
+  void *S0f;
+  void *S0fimg;
+  int32_t *fold_buf;
+  int folded;      // S0f and fold_buf are in use since the last rewind
+  int fold_cur;    // which d0 buffer holds the current depths
+  int after_fold;  // the last call was a fold: the next kernel may not overlap it
   int32_t *par_store;         // each step's parents, written by the kernel
   // Every earlier call's k, gate and parent_idx (caller memory; read again
   // only under ONELA_FLAG_PDL).
@@ -56,6 +67,8 @@ struct DeviceGuard {
 void rewind_to_prompt(onela_handle *h) {
   h->has_prompt = 1;
   h->steps_done = 0;
+  h->folded = 0;
+  h->after_fold = 0;
   h->Ws.clear();
   h->hist_k.clear();
   h->hist_g.clear();
@@ -65,6 +78,9 @@ void rewind_to_prompt(onela_handle *h) {
 void free_all(onela_handle *h) {
   cudaFree(h->S0);
   cudaFree(h->S0img);
+  cudaFree(h->S0f);
+  cudaFree(h->S0fimg);
+  cudaFree(h->fold_buf);
   cudaFree(h->rec_alpha);
   cudaFree(h->par_store);
   cudaFree(h->rec_delta);
@@ -82,8 +98,10 @@ onela::StepParams base_params(const onela_handle *h) {
   p.dv = h->cfg.d_v;
   p.W_max = h->cfg.W_max;
   p.T_max = h->cfg.T_max;
-  p.S0 = h->S0;
-  p.S0img = h->S0img;
+  p.S0 = h->folded ? h->S0f : h->S0;
+  p.S0img = h->folded ? h->S0fimg : h->S0img;
+  p.d0 = h->folded ? h->fold_buf + h->fold_cur * h->cfg.R : nullptr;
+  p.anc_fold = h->fold_buf + 2 * h->cfg.R;
   p.s0_planes = h->planes;
   p.rec_alpha = h->rec_alpha;
   p.par_store = h->par_store;
@@ -146,8 +164,11 @@ int onela_create(const onela_config *cfg, onela_handle **out) {
   const size_t nS0 = (size_t)c.R * c.H * c.d_v * c.d_k;
   const size_t nrow = (size_t)c.T_max * c.R * c.H * c.W_max;
   bool ok = cudaMalloc(&h->S0, nS0 * esize(c.s0_dtype)) == cudaSuccess;
+  ok = ok && cudaMalloc(&h->S0f, nS0 * esize(c.s0_dtype)) == cudaSuccess;
+  ok = ok && cudaMalloc((void **)&h->fold_buf, (size_t)c.R * (2 + c.T_max) * sizeof(int32_t)) == cudaSuccess;
   if (ok && kernel == ONELA_KERNEL_TC)
-    ok = cudaMalloc(&h->S0img, onela::s0_image_bytes(c.R, c.H, c.d_k, c.d_v, h->planes)) == cudaSuccess;
+    ok = cudaMalloc(&h->S0img, onela::s0_image_bytes(c.R, c.H, c.d_k, c.d_v, h->planes)) == cudaSuccess &&
+         cudaMalloc(&h->S0fimg, onela::s0_image_bytes(c.R, c.H, c.d_k, c.d_v, h->planes)) == cudaSuccess;
   ok = ok && cudaMalloc((void **)&h->rec_alpha, nrow * sizeof(float)) == cudaSuccess;
   if (ok && kernel == ONELA_KERNEL_TC)
     ok = cudaMalloc((void **)&h->par_store, (size_t)c.T_max * c.R * c.W_max * sizeof(int32_t)) == cudaSuccess;
@@ -160,6 +181,8 @@ int onela_create(const onela_config *cfg, onela_handle **out) {
     *h->err_host = 0;
     // Zeroed so that nothing uninitialised is ever read, even after a bad parent.
     ok = cudaMemset(h->rec_alpha, 0, nrow * sizeof(float)) == cudaSuccess &&
+         (!h->S0fimg ||
+          cudaMemset(h->S0fimg, 0, onela::s0_image_bytes(c.R, c.H, c.d_k, c.d_v, h->planes)) == cudaSuccess) &&
          cudaMemset(h->anc, 0, (size_t)c.T_max * c.R * c.W_max * c.T_max * sizeof(int32_t)) == cudaSuccess &&
          cudaDeviceSynchronize() == cudaSuccess;
   }
@@ -273,7 +296,9 @@ int onela_decode_step(onela_handle *h, int32_t W_prev, int32_t W, const void *q,
   p.o = o;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
-  const bool pdl = (c.flags & ONELA_FLAG_PDL) && p.t >= 2;
+  // The step after a fold reads the folded state before its wait: it is an
+  // ordinary launch.
+  const bool pdl = (c.flags & ONELA_FLAG_PDL) && p.t >= 2 && !h->after_fold;
   if (h->kernel == ONELA_KERNEL_TC) {
     // The tensor-core kernel reads tiles of q, k, v and o with 16-byte accesses.
     const uintptr_t any = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
@@ -311,6 +336,7 @@ int onela_decode_step(onela_handle *h, int32_t W_prev, int32_t W, const void *q,
     return ONELA_ERR_CUDA;
   }
   h->steps_done += 1;
+  h->after_fold = 0;
   h->Ws.push_back(W);
   h->hist_k.push_back(k);
   h->hist_g.push_back(gate);
@@ -326,11 +352,74 @@ int onela_reset(onela_handle *h, onela_stream stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ONELA_ERR_CUDA;
   *reinterpret_cast<volatile int32_t *>(h->err_host) = 0;
   h->steps_done = 0;
+  h->folded = 0;
+  h->after_fold = 0;
   h->Ws.clear();
   h->hist_k.clear();
   h->hist_g.clear();
   h->hist_par.clear();
   return ONELA_OK;
+}
+
+int onela_fold(onela_handle *h, int32_t max_depth, onela_stream stream) {
+  if (!h || max_depth < 0) return ONELA_ERR_ARG;
+  if (*reinterpret_cast<volatile int32_t *>(h->err_host) & onela::kErrParent) return ONELA_ERR_PARENT;
+  if (!h->has_prompt) return ONELA_ERR_STATE;
+  if (h->steps_done == 0 || max_depth == 0) return ONELA_OK;  // nothing to fold
+  DeviceGuard g(h->cfg.device);
+  if (!g.ok) return ONELA_ERR_CUDA;
+  const onela_config &c = h->cfg;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  onela::StepParams p = base_params(h);
+  p.t = h->steps_done;
+  const int first = h->folded ? 0 : 1;
+  const int32_t *d0_in = h->fold_buf + h->fold_cur * c.R;
+  int32_t *d0_out = h->fold_buf + (1 - h->fold_cur) * c.R, *anc_fold = h->fold_buf + 2 * c.R;
+  const int depth = max_depth < h->steps_done ? max_depth : h->steps_done;
+  cudaError_t e;
+  if (h->kernel == ONELA_KERNEL_TC) {
+    // Overlaps the step before it (never another fold: it reads the folded
+    // state before its wait).
+    const int pdl = (c.flags & ONELA_FLAG_PDL) && !h->after_fold;
+    e = onela::launch_fold_tc(p, h->Ws.back(), depth, first, d0_in, d0_out, anc_fold, h->S0f, h->S0fimg,
+                              c.s0_dtype == ONELA_BF16, pdl, s);
+  } else {
+    e = onela::launch_fold(p, h->Ws.back(), depth, first, d0_in, d0_out, anc_fold, h->S0f,
+                           c.qkv_dtype == ONELA_BF16, c.s0_dtype == ONELA_BF16, s);
+  }
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return ONELA_ERR_CUDA;
+  }
+  h->fold_cur = 1 - h->fold_cur;
+  h->folded = 1;
+  h->after_fold = 1;
+  return ONELA_OK;
+}
+
+int onela_read_root_state(onela_handle *h, void *S, onela_stream stream) {
+  if (!h || !S) return ONELA_ERR_ARG;
+  if (!h->has_prompt) return ONELA_ERR_STATE;
+  DeviceGuard g(h->cfg.device);
+  if (!g.ok) return ONELA_ERR_CUDA;
+  const onela_config &c = h->cfg;
+  const size_t bytes = (size_t)c.R * c.H * c.d_v * c.d_k * esize(c.s0_dtype);
+  if (cudaMemcpyAsync(S, h->folded ? h->S0f : h->S0, bytes, cudaMemcpyDeviceToDevice,
+                      static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return ONELA_ERR_CUDA;
+  return ONELA_OK;
+}
+
+int onela_read_fold_depth(onela_handle *h, int32_t *depth, onela_stream stream) {
+  if (!h || !depth) return ONELA_ERR_ARG;
+  DeviceGuard g(h->cfg.device);
+  if (!g.ok) return ONELA_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t bytes = (size_t)h->cfg.R * sizeof(int32_t);
+  const cudaError_t e = h->folded ? cudaMemcpyAsync(depth, h->fold_buf + h->fold_cur * h->cfg.R, bytes,
+                                                    cudaMemcpyDeviceToDevice, s)
+                                  : cudaMemsetAsync(depth, 0, bytes, s);
+  return e == cudaSuccess ? ONELA_OK : ONELA_ERR_CUDA;
 }
 
 int onela_status(onela_handle *h, int32_t *device_err) {

@@ -37,7 +37,8 @@ __global__ void __launch_bounds__(kNT) step_simt_kernel(const StepParams p) {
   const int b0 = tile * kBT;
   const int nb = min(kBT, p.W - b0);
   const int dk = p.dk, dv = p.dv, H = p.H, t = p.t, TM = p.T_max;
-  const int nanc = t - 1;
+  const int d0 = p.d0 ? p.d0[r] : 0;  // depths 1..d0 are folded into S0
+  const int nanc = t - 1 - d0;  // replayed ancestors: chain index j is depth d0 + j + 1
 
   float *xk = smem;                        // [BT][dk]
   float *xq = xk + kBT * dk;               // [BT][dk]
@@ -82,21 +83,24 @@ __global__ void __launch_bounds__(kNT) step_simt_kernel(const StepParams p) {
         par = 0;
       }
       int *chain = s_chain + b * TM;
-      if (nanc >= 1) {
-        chain[nanc - 1] = par;
-        if (nanc >= 2) {
-          const int32_t *prow = p.anc + anc_row(p, t - 1, r, par);
-          for (int j = 0; j < nanc - 1; ++j) chain[j] = prow[j];
+      if (t >= 2) {
+        // The parent's ancestry row holds absolute depths 1..t-2 (the
+        // folded prefix included); the chain keeps the replayed ones.
+        const int32_t *prow = p.anc + anc_row(p, t - 1, r, par);
+        if (nanc >= 1) {
+          chain[nanc - 1] = par;
+          for (int j = 0; j < nanc - 1; ++j) chain[j] = prow[d0 + j];
         }
         if (h == 0) {
           int32_t *row = p.anc + anc_row(p, t, r, gb);
-          for (int j = 0; j < nanc; ++j) row[j] = chain[j];
+          for (int j = 0; j < t - 2; ++j) row[j] = prow[j];
+          row[t - 2] = par;
         }
       }
       float run = 1.f;
-      for (int j = nanc - 1; j >= 0; --j) {  // record at depth j + 1
+      for (int j = nanc - 1; j >= 0; --j) {  // record at depth d0 + j + 1
         s_w[b * TM + j] = run;
-        run *= p.rec_alpha[rec_row(p, j + 1, r, h, chain[j])];
+        run *= p.rec_alpha[rec_row(p, d0 + j + 1, r, h, chain[j])];
       }
       G = run;
       const int64_t si = (int64_t)(r * p.W + gb) * H + h;
@@ -118,7 +122,7 @@ __global__ void __launch_bounds__(kNT) step_simt_kernel(const StepParams p) {
       const int b = pi / per, jj = pi - b * per;
       float dkk = 0.f, dkq = 0.f;
       if (jj < nanc) {
-        const QT *kr = rec_k + rec_row(p, jj + 1, r, h, s_chain[b * TM + jj]) * dk;
+        const QT *kr = rec_k + rec_row(p, d0 + jj + 1, r, h, s_chain[b * TM + jj]) * dk;
         for (int l = lane; l < dk; l += 32) {
           const float kj = ld_f(kr, l);
           dkk += kj * xk[b * dk + l];
@@ -189,7 +193,7 @@ __global__ void __launch_bounds__(kNT) step_simt_kernel(const StepParams p) {
       float uk = s_G[b] * acck[m];
       float uq = s_G[b] * accq[m];
       for (int jj = 0; jj < nanc; ++jj) {
-        const float d = p.rec_delta[rec_row(p, jj + 1, r, h, s_chain[b * TM + jj]) * dv + i];
+        const float d = p.rec_delta[rec_row(p, d0 + jj + 1, r, h, s_chain[b * TM + jj]) * dv + i];
         uk = fmaf(s_ck[b * TM + jj], d, uk);
         uq = fmaf(s_cq[b * TM + jj], d, uq);
       }

@@ -92,19 +92,26 @@ __host__ __device__ inline Layout layout(int nk, int planes, int TM, int W_max, 
   // (the slot list 4 TM longer); a beam-index scratch [W_max]; the parents
   // of steps 2..t-1; the per-step table (3 pointers and 3 ints per step).
   L.total = L.book + 128u + 4u * kBT * 4u + (uint32_t)kBT * TM * 16u + (3u * kBT + 4u) * TM * 4u +
-            (uint32_t)((W_max + 3) & ~3) * 4u + (uint32_t)((hist_cap + 3) & ~3) * 4u + kTabBytes + 16u;
+            (uint32_t)((W_max + 3) & ~3) * 4u + (uint32_t)((hist_cap + 3) & ~3) * 2u + kTabBytes + 16u;
   return L;
 }
 
 // Copies n ints from global src to shared dst with cp.async, by the 32 lanes
 // of one warp: 16-byte pieces when both ends allow it, single ints otherwise.
-__device__ __forceinline__ void copy_ints_warp(int *dst, const int32_t *src, int n, int lane) {
+__device__ __forceinline__ void copy_parents16_warp(uint16_t *dst, const int32_t *src, int n, int lane) {
+  // dst is 8-byte aligned; parents are below 2^16 (anything else is out of
+  // range and is clamped where it is used).
   int done = 0;
-  if (((ptx::smem_u32(dst) | (uint32_t)reinterpret_cast<uintptr_t>(src)) & 15u) == 0) {
+  if ((reinterpret_cast<uintptr_t>(src) & 15u) == 0) {
     done = n & ~3;
-    for (int e = lane * 4; e < done; e += 128) ptx::cp_async16(dst + e, src + e, 16u);
+#pragma unroll 2
+    for (int e = lane * 4; e < done; e += 128) {
+      const int4 v = __ldg(reinterpret_cast<const int4 *>(src + e));
+      *reinterpret_cast<uint2 *>(dst + e) = make_uint2(((uint32_t)v.x & 0xffffu) | ((uint32_t)v.y << 16),
+                                                      ((uint32_t)v.z & 0xffffu) | ((uint32_t)v.w << 16));
+    }
   }
-  for (int e = done + lane; e < n; e += 32) ptx::cp_async4(dst + e, src + e);
+  for (int e = done + lane; e < n; e += 32) dst[e] = (uint16_t)__ldg(src + e);
 }
 
 // Four consecutive bf16 elements (packed in u, or at p, 8-byte aligned) as floats.
@@ -131,8 +138,9 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
   const int b0 = tile * kBT;
   const int nb = min(kBT, p.W - b0);
   const int H = p.H, t = p.t, TM = p.T_max, P = p.s0_planes;
-  const int nanc = t - 1;   // ancestors per beam (depths 1..t-1)
-  const int jp = nanc - 1;  // depth index of the parents (depth t-1)
+  const int d0 = p.d0 ? p.d0[r] : 0;  // depths 1..d0 are folded into S0
+  const int nanc = t - 1 - d0;  // ancestors per beam (depths d0+1..t-1); chain index j is depth d0+j+1
+  const int jp = nanc - 1;      // chain index of the parents (depth t-1)
   const bool hin = p.hist_inputs != 0;
 
   const Layout L = layout(NK, P, TM, p.W_max, p.hist_cap);
@@ -158,7 +166,7 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
   int *s_list = s_chain + kBT * TM;  // slot -> (beam << 5 | depth-1), [(32 + 4) TM]
   float *s_w = reinterpret_cast<float *>(s_list + (kBT + 4) * TM);  // [32][TM] gates along the chains
   int *s_seen = reinterpret_cast<int *>(s_w + kBT * TM);           // beam index -> a lane (scratch)
-  int *s_hist = s_seen + ((p.W_max + 3) & ~3);                      // parents of steps 2..t-1
+  uint16_t *s_hist = reinterpret_cast<uint16_t *>(s_seen + ((p.W_max + 3) & ~3));  // parents of steps 2..t-1
   // Per-step table (index = step j), filled by the ancestry warp before the
   // first barrier with one load per lane: loops then read shared memory
   // instead of indexing the parameters at run time.
@@ -202,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
   if (warp == kAncWarp) {
     // This tile's parents, gates and betas, and the per-step table.
     if (lane < nb) {
-      par = nanc >= 1 ? p.parents[r * p.W + b0 + lane] : 0;
+      par = t >= 2 ? p.parents[r * p.W + b0 + lane] : 0;
       const int64_t si = row0 + (int64_t)lane * H;
       g_alpha = p.g[si];
       g_beta = p.beta[si];
@@ -216,13 +224,13 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
       s_trs[lane] = p.hpar_rs[lane];
     }
   }
-  // The parents of steps 2..t-1 for this request, back to back, each array
-  // starting on a 16-byte boundary: beam warp w >= 1 copies steps w + 1,
-  // w + 8, w + 15.  Every thread waits for its own copies before the barrier.
+  // The parents of steps 2..t-1 for this request as 16-bit indices, back
+  // to back, each array starting on an 8-byte boundary: beam warp w >= 1
+  // copies steps w + 1, w + 8, w + 15.
   if (p.hist_cap > 0 && warp >= 1 && warp < kAncWarp)
-#pragma unroll 1
+#pragma unroll 2
     for (int j = warp + 1; j < t; j += kAncWarp - 1)
-      copy_ints_warp(s_hist + p.hoff[j], p.hpar[j] + (int64_t)r * p.hpar_rs[j], p.hW[j], lane);
+      copy_parents16_warp(s_hist + p.hoff[j], p.hpar[j] + (int64_t)r * p.hpar_rs[j], p.hW[j], lane);
   ptx::cp_async_commit();
   ptx::cp_async_wait_all();
   ptx::tc_fence_before();
@@ -250,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
     // the parent, at step j + 2, of a[j + 1]), the tile's distinct
     // ancestors and the replay weights.
     const int b = lane;
-    if (b < nb && nanc >= 1 && (par < 0 || par >= p.W_prev)) {
+    if (b < nb && t >= 2 && (par < 0 || par >= p.W_prev)) {
       *reinterpret_cast<volatile int32_t *>(p.err) = kErrParent;
       par = 0;
     }
@@ -263,8 +271,9 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
       s_chain[b * TM + jp] = a;
 #pragma unroll 1
       for (int j = jp - 1; j >= 0; --j) {
-        int pa = p.hist_cap > 0 ? s_hist[s_toff[j + 2] + a] : s_tpar[j + 2][(int64_t)r * s_trs[j + 2] + a];
-        if (pa < 0 || pa >= s_tW[j + 1]) pa = 0;  // reported by step j + 2
+        const int st = d0 + j + 2;  // the step whose parent array leads from depth st-1 to st
+        int pa = p.hist_cap > 0 ? s_hist[s_toff[st] + a] : s_tpar[st][(int64_t)r * s_trs[st] + a];
+        if (pa < 0 || pa >= s_tW[st - 1]) pa = 0;  // reported by step st
         a = pa;
         s_chain[b * TM + j] = a;
       }
@@ -276,8 +285,9 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
 #pragma unroll 1
       for (int j = 0; j <= jp; ++j) {
         const int a = s_chain[b * TM + j];
-        ptx::cp_async4(s_w + b * TM + j, hin ? s_tg[j + 1] + ((int64_t)r * s_tW[j + 1] + a) * H + h
-                                             : p.rec_alpha + rec_row(p, j + 1, r, h, a));
+        const int dj = d0 + j + 1;  // depth of the record
+        ptx::cp_async4(s_w + b * TM + j, hin ? s_tg[dj] + ((int64_t)r * s_tW[dj] + a) * H + h
+                                             : p.rec_alpha + rec_row(p, dj, r, h, a));
       }
     }
     ptx::cp_async_commit();
@@ -364,8 +374,9 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
         const int j = j0 + e;
         if (bval && j < nanc) {
           const int a = s_chain[bb * TM + j];
-          const __nv_bfloat16 *row = hin ? s_tk[j + 1] + ((int64_t)(r * s_tW[j + 1] + a) * H + h) * DK
-                                         : rec_k + rec_row(p, j + 1, r, h, a) * DK;
+          const int dj = d0 + j + 1;
+          const __nv_bfloat16 *row = hin ? s_tk[dj] + ((int64_t)(r * s_tW[dj] + a) * H + h) * DK
+                                         : rec_k + rec_row(p, dj, r, h, a) * DK;
           const uint8_t *rb = reinterpret_cast<const uint8_t *>(row) + l * 8;
 #pragma unroll
           for (int u = 0; u < NU; ++u) buf[e][u] = __ldg(reinterpret_cast<const uint2 *>(rb + (u ^ sx) * 64));
@@ -448,7 +459,9 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
       if (h == 0) {
         int32_t *row = p.anc + anc_row(p, t, r, gb);
 #pragma unroll 1
-        for (int j = 0; j < nanc; ++j) row[j] = s_chain[bb * TM + j];
+        for (int j = 0; j < d0; ++j) row[j] = p.anc_fold[r * TM + j];
+#pragma unroll 1
+        for (int j = 0; j < nanc; ++j) row[d0 + j] = s_chain[bb * TM + j];
         p.par_store[((int64_t)(t - 1) * p.R + r) * p.W_max + gb] = s_par[bb];
       }
     }
@@ -493,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
       const int rr = e / PD, c = e - rr * PD;
       const int packed = s_list[lo + rr];
       ptx::cp_async16(base + L.dst + (uint32_t)(rr * DV + c * 4) * 4u,
-                      p.rec_delta + rec_row(p, (packed & 31) + 1, r, h, packed >> 5) * DV + c * 4, 16u);
+                      p.rec_delta + rec_row(p, d0 + (packed & 31) + 1, r, h, packed >> 5) * DV + c * 4, 16u);
     }
     ptx::cp_async_commit();
     ptx::cp_async_wait_all();
@@ -515,15 +528,15 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
         }
 #pragma unroll
         for (int u = 0; u < NU; ++u) {
-          const float4 d0 = row[0][8 * (u ^ sx)], d1 = row[1][8 * (u ^ sx)];
-          acc_k[4 * u + 0] = fmaf(d1.x, ck[1], fmaf(d0.x, ck[0], acc_k[4 * u + 0]));
-          acc_k[4 * u + 1] = fmaf(d1.y, ck[1], fmaf(d0.y, ck[0], acc_k[4 * u + 1]));
-          acc_k[4 * u + 2] = fmaf(d1.z, ck[1], fmaf(d0.z, ck[0], acc_k[4 * u + 2]));
-          acc_k[4 * u + 3] = fmaf(d1.w, ck[1], fmaf(d0.w, ck[0], acc_k[4 * u + 3]));
-          acc_q[4 * u + 0] = fmaf(d1.x, cq[1], fmaf(d0.x, cq[0], acc_q[4 * u + 0]));
-          acc_q[4 * u + 1] = fmaf(d1.y, cq[1], fmaf(d0.y, cq[0], acc_q[4 * u + 1]));
-          acc_q[4 * u + 2] = fmaf(d1.z, cq[1], fmaf(d0.z, cq[0], acc_q[4 * u + 2]));
-          acc_q[4 * u + 3] = fmaf(d1.w, cq[1], fmaf(d0.w, cq[0], acc_q[4 * u + 3]));
+          const float4 e0 = row[0][8 * (u ^ sx)], e1 = row[1][8 * (u ^ sx)];
+          acc_k[4 * u + 0] = fmaf(e1.x, ck[1], fmaf(e0.x, ck[0], acc_k[4 * u + 0]));
+          acc_k[4 * u + 1] = fmaf(e1.y, ck[1], fmaf(e0.y, ck[0], acc_k[4 * u + 1]));
+          acc_k[4 * u + 2] = fmaf(e1.z, ck[1], fmaf(e0.z, ck[0], acc_k[4 * u + 2]));
+          acc_k[4 * u + 3] = fmaf(e1.w, ck[1], fmaf(e0.w, ck[0], acc_k[4 * u + 3]));
+          acc_q[4 * u + 0] = fmaf(e1.x, cq[1], fmaf(e0.x, cq[0], acc_q[4 * u + 0]));
+          acc_q[4 * u + 1] = fmaf(e1.y, cq[1], fmaf(e0.y, cq[0], acc_q[4 * u + 1]));
+          acc_q[4 * u + 2] = fmaf(e1.z, cq[1], fmaf(e0.z, cq[0], acc_q[4 * u + 2]));
+          acc_q[4 * u + 3] = fmaf(e1.w, cq[1], fmaf(e0.w, cq[0], acc_q[4 * u + 3]));
         }
       }
     }

@@ -24,7 +24,8 @@ def declared_symbols():
 def test_header_declares_the_decode_entry_points():
     names = declared_symbols()
     for n in ("onela_create", "onela_set_prompt_state", "onela_prefill", "onela_decode_step",
-              "onela_reset", "onela_status", "onela_destroy"):
+              "onela_reset", "onela_status", "onela_destroy", "onela_fold", "onela_read_root_state",
+              "onela_read_fold_depth"):
         assert n in names
 
 
@@ -74,6 +75,9 @@ def test_null_arguments_are_rejected():
     assert lib.onela_read_ancestry(None, 1, None, None) == L.ONELA_ERR_ARG
     assert lib.onela_prefill(None, 4, None, None, None, None, None) == L.ONELA_ERR_ARG
     assert lib.onela_read_prompt_state(None, None, None) == L.ONELA_ERR_ARG
+    assert lib.onela_fold(None, 3, None) == L.ONELA_ERR_ARG
+    assert lib.onela_read_root_state(None, None, None) == L.ONELA_ERR_ARG
+    assert lib.onela_read_fold_depth(None, None, None) == L.ONELA_ERR_ARG
     assert lib.onela_steps_done(None) == -1
     assert lib.onela_select_beams(1, 4, 4, 2, *([None] * 6), 0, 0, None) == L.ONELA_ERR_ARG
 
