@@ -142,16 +142,22 @@ __device__ __forceinline__ void st8(__nv_bfloat16 *p, float (&x)[8]) {
 
 // One launch: plan, recurrence, folded state and its operand image.  Block:
 // kFoldThreads threads, DK / 8 per state row (8 columns each), so RB rows.
+// After the wait on the previous kernel, two rounds of loads: the ancestry
+// rows (beam 0's and each thread's beams'), then the records of every depth
+// that may be folded (the shared depth is known only once the rows are
+// compared; records past it are loaded and not used).
 template <typename ST, int DK>
 __global__ void __launch_bounds__(kFoldThreads) fold_tc_kernel(const StepParams p, int Wt, int max_depth, int first,
                                                                const int32_t *d0_in, int32_t *d0_out,
                                                                int32_t *anc_fold, ST *S_fold, uint4 *img) {
   constexpr int TPR = DK / 8, RB = kFoldThreads / TPR, NK = DK / 64;
+  constexpr int KC = DK / 8, DC = RB / 4, PER = KC + DC + 1;  // 16-byte record pieces per depth
+  constexpr int MAXI = (kFoldMaxT * PER + kFoldThreads - 1) / kFoldThreads;
   __shared__ int s_split;
   __shared__ int s_row0[kFoldMaxT];
   __shared__ float s_a[kFoldMaxT];
-  __shared__ float s_d[kFoldMaxT][RB];
-  __shared__ float s_k[kFoldMaxT][DK];
+  __shared__ __align__(16) float s_d[kFoldMaxT][RB];
+  __shared__ __align__(16) __nv_bfloat16 s_k[kFoldMaxT][DK];
   const int h = blockIdx.y, r = blockIdx.z, tid = threadIdx.x;
   const int dv = p.dv, t = p.t, n = t - 1;
   const int i0 = blockIdx.x * RB, ir = tid / TPR, c = tid - ir * TPR, i = i0 + ir;
@@ -167,23 +173,72 @@ __global__ void __launch_bounds__(kFoldThreads) fold_tc_kernel(const StepParams 
   if (tid == 0) s_split = n;
   // The ancestry rows and records of step t come from the previous kernel.
   ptx::pdl_wait();
+  // Depths that can be folded: old + 1 .. Dmax (depth t only when step t
+  // kept a single beam, its own record).
+  const int jhi = min(n, max_depth);
+  const int Dmax = max(old, min(max_depth, Wt == 1 ? t : n));
   const int32_t *row0 = p.anc + anc_row(p, t, r, 0);
   if (tid < n) s_row0[tid] = row0[tid];
-  __syncthreads();
-  // Each thread compares whole rows of its beams, all entries loaded at once.
-  const int jhi = min(n, max_depth);
-  for (int b = 1 + tid; b < Wt; b += kFoldThreads) {
+  int v[kFoldMaxT], w0[kFoldMaxT];
+  const int b = 1 + tid;  // Wt <= kFoldThreads + 1 here; more beams: the loop below
+  if (b < Wt) {
     const int32_t *row = p.anc + anc_row(p, t, r, b);
-    int v[kFoldMaxT];
 #pragma unroll
-    for (int j = 0; j < kFoldMaxT; ++j) v[j] = (j >= old && j < jhi) ? row[j] : 0;
-    int split = n;
+    for (int j = 0; j < kFoldMaxT; ++j) {
+      v[j] = (j >= old && j < jhi) ? row[j] : 0;
+      w0[j] = (j >= old && j < jhi) ? row0[j] : 0;
+    }
+  }
+  __syncthreads();  // s_row0
+  // Round two, issued before the comparisons wait for round one.
+  uint4 piece[MAXI];
+  const int nitems = (Dmax - old) * PER;
+#pragma unroll
+  for (int m = 0; m < MAXI; ++m) {
+    const int e = tid + m * kFoldThreads;
+    piece[m] = make_uint4(0u, 0u, 0u, 0u);
+    if (e < nitems) {
+      const int dd = e / PER, q = e - dd * PER, d = old + dd + 1;
+      const int64_t row = rec_row(p, d, r, h, d - 1 < n ? s_row0[d - 1] : 0);
+      if (q < KC)
+        piece[m] = *reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.rec_k) + row * DK + q * 8);
+      else if (q < KC + DC)
+        piece[m] = *reinterpret_cast<const uint4 *>(p.rec_delta + row * dv + i0 + (q - KC) * 4);
+      else
+        piece[m].x = __float_as_uint(p.rec_alpha[row]);
+    }
+  }
+  int split = n;
+  if (b < Wt) {
 #pragma unroll
     for (int j = kFoldMaxT - 1; j >= 0; --j)
-      if (j >= old && j < jhi && v[j] != s_row0[j]) split = j;
-    if (split < n) atomicMin(&s_split, split);
+      if (j >= old && j < jhi && v[j] != w0[j]) split = j;
+  }
+  for (int bb = b + kFoldThreads; bb < Wt; bb += kFoldThreads) {
+    const int32_t *row = p.anc + anc_row(p, t, r, bb);
+    for (int j = old; j < jhi; ++j)
+      if (row[j] != s_row0[j]) {
+        split = min(split, j);
+        break;
+      }
+  }
+  if (split < n) atomicMin(&s_split, split);
+#pragma unroll
+  for (int m = 0; m < MAXI; ++m) {
+    const int e = tid + m * kFoldThreads;
+    if (e < nitems) {
+      const int dd = e / PER, q = e - dd * PER;
+      if (q < KC)
+        *reinterpret_cast<uint4 *>(&s_k[dd][q * 8]) = piece[m];
+      else if (q < KC + DC)
+        *reinterpret_cast<uint4 *>(&s_d[dd][(q - KC) * 4]) = piece[m];
+      else
+        s_a[dd] = __uint_as_float(piece[m].x);
+    }
   }
   __syncthreads();
+  // Sharing an ancestor at a depth implies sharing its ancestors, so the
+  // shared depths are 1..s_split; a step that kept one beam shares it too.
   int D = s_split;
   if (D == n && Wt == 1) D = t;
   if (D > max_depth) D = max_depth;
@@ -192,28 +247,18 @@ __global__ void __launch_bounds__(kFoldThreads) fold_tc_kernel(const StepParams 
     for (int j = old + tid; j < D; j += kFoldThreads) anc_fold[(int64_t)r * p.T_max + j] = j < n ? s_row0[j] : 0;
     if (tid == 0) d0_out[r] = D;
   }
-  if (!first && D == old) return;  // unchanged: the folded state and image hold it
-
-  const int nd = D - old;
-  const __nv_bfloat16 *rec_k = static_cast<const __nv_bfloat16 *>(p.rec_k);
-  for (int e = tid; e < nd * (1 + RB + DK); e += kFoldThreads) {
-    const int dd = e / (1 + RB + DK), q = e - dd * (1 + RB + DK);
-    const int d = old + dd + 1;
-    const int64_t row = rec_row(p, d, r, h, d - 1 < n ? s_row0[d - 1] : 0);
-    if (q == 0)
-      s_a[dd] = p.rec_alpha[row];
-    else if (q <= RB)
-      s_d[dd][q - 1] = i0 + q - 1 < dv ? p.rec_delta[row * dv + i0 + q - 1] : 0.f;
-    else
-      s_k[dd][q - 1 - RB] = __bfloat162float(rec_k[row * DK + q - 1 - RB]);
-  }
-  __syncthreads();
-  if (!valid) return;
+  if ((!first && D == old) || !valid) return;  // unchanged: the folded state and image hold it
 #pragma unroll 1
-  for (int dd = 0; dd < nd; ++dd) {
+  for (int dd = 0; dd < D - old; ++dd) {
     const float a = s_a[dd], dl = s_d[dd][ir];
+    const uint4 kq = *reinterpret_cast<const uint4 *>(&s_k[dd][c * 8]);
+    const __nv_bfloat162 *k2 = reinterpret_cast<const __nv_bfloat162 *>(&kq);
 #pragma unroll
-    for (int u = 0; u < 8; ++u) x[u] = fmaf(dl, s_k[dd][c * 8 + u], a * x[u]);
+    for (int u = 0; u < 4; ++u) {
+      const float2 kf = __bfloat1622float2(k2[u]);
+      x[2 * u] = fmaf(dl, kf.x, a * x[2 * u]);
+      x[2 * u + 1] = fmaf(dl, kf.y, a * x[2 * u + 1]);
+    }
   }
   st8(S_fold + si, x);
   // The operand image: plane pl holds the bf16 term pl of the split of the

@@ -8,7 +8,9 @@ imports nothing from it.
 Modules
 -------
 gdn     numpy fp64 reference: prefill, full-state beam tree, replay
-        formulation (for the replay == full-state identity), ancestry walk.
+        formulation (for the replay == full-state identity), ancestry walk,
+        and for the folding extension the shared-ancestor depth and the
+        shared ancestor's full state.
 cref    ctypes loader for ``c/gdn_fullstate.c``: the same full-state beam tree
         in plain C (fp64, OpenMP over beams), the timed CPU baseline.
 beam    beam selection: the W best children (fp32 scores, ties to the smaller
@@ -22,5 +24,8 @@ unchanged; beta = 0 is a pure gate product; ancestry by brute-force tree
 construction; linearity in (S0, v); permutation equivariance of beam labels;
 a hand-worked scalar example (tests/golden/).  Beam selection: brute-force
 ordering of Python tuples, fp32 rounding ties, signed zeros, NaN and -inf.
+Folding: hand-built trees and a brute-force path walk for the shared depth;
+the prefill recurrence for a single beam's folded state; decoding on from a
+folded state equals the unfolded decode.
 """
 from . import gdn  # noqa: F401
