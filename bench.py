@@ -365,6 +365,65 @@ def time_fold(wl, S0, kernel, device, stream, flush, T=16, every=4, reps=10, war
     return out
 
 
+def time_sweep(device, stream, flush, reps=10, warmup=3):
+    """The beam-width sweep (W = 64 .. 1024, T = 5, 1K-prompt shapes) and the
+    request sweep (R = 1, 8, 32 at H = 16, d = 128, W = 256, T = 7): one whole
+    decode per CUDA graph with programmatic launch between its steps, L2
+    flushed before each, CUDA events; algorithmic bytes from the byte model.
+    S0 is drawn directly (its values do not change the work).  Returns the
+    JSON object for the bench line."""
+    import linear_attention_beam_shared_b200 as L
+    cases = [synth.workload(f"wsweep{w}") for w in (64, 128, 256, 512, 1024)]
+    cases += [synth.shape_sweep_workload(R, 16, 128, 256, 7) for R in (1, 8, 32)]
+    hbm = measured_peaks()[0]
+    points = []
+    for wl in cases:
+        steps = synth.draw_decode(wl)
+        S0 = synth.cast_state(0.1 * np.random.default_rng(wl.seed_id).standard_normal(
+            (wl.R, wl.H, wl.d_v, wl.d_k)), wl.s0_dtype)
+        ds = [{k: (v.to(device) if isinstance(v, torch.Tensor) else v) for k, v in st.items()} for st in steps]
+        outs = [torch.empty((wl.R, st["W"], wl.H, wl.d_v), dtype=torch.float32, device=device) for st in steps]
+        dec = L.BeamDecoder(wl.R, wl.H, wl.d_k, wl.d_v, wl.W, wl.T, wl.s0_dtype, wl.qkv_dtype,
+                            device=device.index, flags=L.ONELA_FLAG_PDL)
+        kind = {L.ONELA_KERNEL_SIMT: "simt", L.ONELA_KERNEL_TC: "tc"}[dec.kernel]
+        dec.set_prompt_state(S0.to(device))
+
+        def run():
+            for st, o in zip(ds, outs):
+                dec.step(st["q"], st["k"], st["v"], st["g"], st["beta"], st["parents"], o=o, stream=stream)
+        with torch.cuda.stream(stream):
+            run()
+        stream.synchronize()
+        assert dec.status() == 0
+        dec.reset(stream)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            run()
+        dec.reset(stream)
+        for _ in range(warmup):
+            with torch.cuda.stream(stream):
+                flush.fill_(9)
+                g.replay()
+        stream.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        with torch.cuda.stream(stream):
+            for i, (e0, e1) in enumerate(ev):
+                flush.fill_(i & 0xFF)
+                e0.record(stream)
+                g.replay()
+                e1.record(stream)
+        stream.synchronize()
+        ms = max_over_ranks(sum(e0.elapsed_time(e1) for e0, e1 in ev) / reps, device)
+        del g
+        dec.close()
+        alg, _, _ = byte_model(wl, steps)
+        gbs = alg / (ms / 1e3) / 1e9
+        points.append({"R": wl.R, "H": wl.H, "d": wl.d_k, "W": wl.W, "T": wl.T, "kernel": kind,
+                       "ms_per_decode": round(ms, 5), "value": round(wl.units / (ms / 1e3), 1),
+                       "achieved_gbs": round(gbs, 1), "frac": round(gbs / hbm, 4)})
+    return {"unit": UNIT, "peak_gbs": hbm, "l2": "flushed before every decode", "points": points}
+
+
 def byte_model(wl, steps):
     """Algorithmic bytes of one whole decode (all T steps): every byte the
     method must move at least once, with each distinct ancestor record counted
@@ -626,6 +685,7 @@ def run_ours(args):
 
     prefill = time_prefill(wl, device, stream, flush) if (wl.L_prompt > 0 and not args.no_prefill) else None
     select = None if args.no_prefill else time_select(device, stream, flush, R=wl.R, W_prev=wl.W, C=256, W=wl.W)
+    sweep = None if (args.no_sweep or ws > 1) else time_sweep(device, stream, flush)
     fold = None if args.no_prefill else [time_fold(wl, S0, kernel, device, stream, flush, every=4),
                                           time_fold(wl, S0, kernel, device, stream, flush, every=8, alone=False)]
 
@@ -652,7 +712,7 @@ def run_ours(args):
                        "programmatic_launch": not args.no_pdl},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "clocks": clk.summary(), "gpu_launches": launches * args.steps,
-            "prefill": prefill, "beam_select": select, "fold": fold,
+            "prefill": prefill, "beam_select": select, "fold": fold, "sweep": sweep,
         }
         print(json.dumps(line))
     if ws > 1:
@@ -706,7 +766,8 @@ def main():
     ap.add_argument("--no-pdl", action="store_true",
                     help="launch every step only after the previous one has finished")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
-    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill and beam-selection timings")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill, beam-selection and fold timings")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the beam-width and request sweeps")
     ap.add_argument("--s0", choices=["prefill", "direct"], default="prefill",
                     help="S0 from the GDN recurrence over the synthetic prompt (default) or drawn "
                          "directly; the decode's work does not depend on the S0 values")
