@@ -188,6 +188,47 @@ def test_deterministic(kernel):
         assert torch.equal(x["o"], y["o"]) and torch.equal(x["delta"], y["delta"])
 
 
+@pytest.mark.parametrize("kernel", [1, 2])
+def test_permutation_equivariance(kernel):
+    """Relabelling the beams of one step (and remapping the next step's
+    parents to the new labels) permutes that step's outputs and delta
+    records and leaves every other output unchanged, bit for bit: a beam's
+    arithmetic does not depend on its neighbours, its tile or the order in
+    which the tile's distinct ancestors are found.  The tensor-core kernel
+    visits a beam's element groups in swapped order at odd positions, so
+    there the relabelling keeps each beam's parity."""
+    import linear_attention_beam_shared_b200 as L
+    _skip_unavailable(kernel, 128, 128, "bf16")
+    wl, S0, steps = P.custom_steps(13, 2, 2, 128, 128, (40, 70, 70, 50))
+    S0c = synth.cast_state(S0, "f32")
+    a, _ = P.run_gpu(S0c, steps, "bf16", kernel)
+    s = 1                                    # relabel the beams of step 2
+    W = steps[s]["W"]
+    rng = np.random.default_rng(5)
+    if kernel == L.ONELA_KERNEL_TC:
+        perm = np.arange(W)
+        for par in (0, 1):
+            idx = np.arange(par, W, 2)
+            perm[idx] = rng.permutation(idx)
+    else:
+        perm = rng.permutation(W)
+    perm = torch.from_numpy(perm)            # new beam i is old beam perm[i]
+    inv = torch.empty_like(perm)
+    inv[perm] = torch.arange(W)
+    steps2 = [dict(x) for x in steps]
+    for key in ("q", "k", "v", "g", "beta", "parents"):
+        steps2[s][key] = steps[s][key][:, perm].contiguous()
+    steps2[s + 1]["parents"] = inv[steps[s + 1]["parents"].long()].to(torch.int32)
+    b, _ = P.run_gpu(S0c, steps2, "bf16", kernel)
+    assert not torch.equal(perm, torch.arange(W))
+    for t, (x, y) in enumerate(zip(a, b)):
+        if t == s:
+            assert torch.equal(x["o"][:, perm], y["o"])
+            assert torch.equal(x["delta"][:, perm], y["delta"])
+        else:
+            assert torch.equal(x["o"], y["o"]) and torch.equal(x["delta"], y["delta"])
+
+
 @pytest.mark.parametrize("kernel,flags", [(1, 0), (2, 0), (2, 1)])
 def test_graph_replay_matches_eager(kernel, flags):
     import linear_attention_beam_shared_b200 as L
