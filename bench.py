@@ -366,8 +366,9 @@ def time_fold(wl, S0, kernel, device, stream, flush, T=16, every=4, reps=10, war
 
 
 def time_sweep(device, stream, flush, reps=10, warmup=3):
-    """The beam-width sweep (W = 64 .. 1024, T = 5, 1K-prompt shapes) and the
-    request sweep (R = 1, 8, 32 at H = 16, d = 128, W = 256, T = 7): one whole
+    """The beam-width sweep (W = 64 .. 1024, T = 5, 1K-prompt shapes), the
+    request sweep (R = 1, 8, 32 at H = 16, d = 128, W = 256, T = 7) and the
+    head sizes d = 64 and 256 at R = 1, H = 16, W = 256, T = 7: one whole
     decode per CUDA graph with programmatic launch between its steps, L2
     flushed before each, CUDA events; algorithmic bytes from the byte model.
     S0 is drawn directly (its values do not change the work).  Returns the
@@ -375,6 +376,9 @@ def time_sweep(device, stream, flush, reps=10, warmup=3):
     import linear_attention_beam_shared_b200 as L
     cases = [synth.workload(f"wsweep{w}") for w in (64, 128, 256, 512, 1024)]
     cases += [synth.shape_sweep_workload(R, 16, 128, 256, 7) for R in (1, 8, 32)]
+    # d = 64 (tensor-core kernel) and d = 256 (general kernel: the tensor-core
+    # one takes d <= 128) at the headline beam set.
+    cases += [synth.shape_sweep_workload(1, 16, d, 256, 7) for d in (64, 256)]
     hbm = measured_peaks()[0]
     points = []
     for wl in cases:
