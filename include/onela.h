@@ -63,7 +63,7 @@ enum {
   ONELA_OK = 0,
   ONELA_ERR_ARG = 1,         /* null pointer, bad size or dtype, bad W_prev  */
   ONELA_ERR_STATE = 2,       /* decode before onela_set_prompt_state         */
-  ONELA_ERR_CAPACITY = 3,    /* step beyond T_max, or W beyond W_max         */
+  ONELA_ERR_CAPACITY = 3,    /* W beyond W_max, or unfolded depths beyond T_max */
   ONELA_ERR_PARENT = 4,      /* the device saw a parent index outside
                                 [0, W_prev); reported by the next call or by
                                 onela_status                                 */
@@ -102,7 +102,10 @@ enum { ONELA_KERNEL_AUTO = 0, ONELA_KERNEL_SIMT = 1, ONELA_KERNEL_TC = 2 };
  *   R, H            requests and heads (each (request, head) pair has its own
  *                   S0 and its own records).
  *   d_k, d_v        key and value widths, 1 <= d <= 256.
- *   W_max, T_max    most beams per step and most decode steps per decode.
+ *   W_max           most beams per step.
+ *   T_max           depths the record store keeps: a decode may run T_max
+ *                   steps, and deeper when onela_fold keeps every step's
+ *                   unfolded depths (t - 1 - D_r) below T_max.
  *   s0_dtype        ONELA_F32 or ONELA_BF16: element type of S0.
  *   qkv_dtype       ONELA_F32 or ONELA_BF16: element type of q, k, v (and of
  *                   the k stored in the records).
@@ -130,6 +133,8 @@ typedef struct {
  * and the bf16 operand image of S0), the
  * ancestry index (int32 [T_max][R][W_max][T_max]) and an error word in
  * mapped, pinned host memory that the kernels write and the host reads.
+ * The store is a ring over depths: depth t uses slot (t - 1) mod T_max, and
+ * an ancestry row holds the ancestor at depth j + 1 in entry j mod T_max.
  * Host-side allocation only; no kernel runs.  *out receives the handle.
  * Errors: ONELA_ERR_ARG (null pointer or invalid field), ONELA_ERR_CUDA. */
 ONELA_API int onela_create(const onela_config *cfg, onela_handle **out);
@@ -186,7 +191,10 @@ ONELA_API int onela_read_prompt_state(onela_handle *h, void *S0, onela_stream st
  * A parent index outside [0, W_prev) is clamped to 0 on the device, recorded
  * in the device error word and reported as ONELA_ERR_PARENT by the next call
  * on the handle (or by onela_status); the outputs of that step are then
- * meaningless.
+ * meaningless.  Step t > T_max is refused (ONELA_ERR_CAPACITY) unless the
+ * handle has folded since the last rewind; then the device checks that
+ * t - 1 - D_r <= T_max - 1 for every request and otherwise reports
+ * ONELA_ERR_CAPACITY the same way (the step's outputs are meaningless).
  * Errors: ONELA_ERR_ARG, ONELA_ERR_STATE, ONELA_ERR_CAPACITY,
  * ONELA_ERR_PARENT, ONELA_ERR_UNSUPPORTED, ONELA_ERR_CUDA. */
 ONELA_API int onela_decode_step(onela_handle *h, int32_t W_prev, int32_t W,
@@ -241,9 +249,10 @@ ONELA_API int onela_reset(onela_handle *h, onela_stream stream);
  * fp32 from the records and stored in cfg.s0_dtype, and later steps replay
  * depths D_r + 1 .. t' - 1 only.  The outputs stay those of the unfolded
  * decode up to that one rounding of the folded state.  Records, ancestry
- * rows (absolute depths) and the prompt state itself are unchanged;
- * onela_reset, onela_set_prompt_state and onela_prefill return to the
- * prompt state.  The depth limit of the decode stays T_max.
+ * rows and the prompt state itself are unchanged; onela_reset,
+ * onela_set_prompt_state and onela_prefill return to the prompt state.
+ * Folding lets a decode go past T_max steps: the store keeps the last T_max
+ * depths, and only the unfolded ones are read.
  *   max_depth  >= 0; values above the steps done act as the steps done;
  *              0 (or no step done yet) leaves everything as it is.
  * Runs on the device only (no host synchronisation; capturable in a CUDA
@@ -267,8 +276,10 @@ ONELA_API int onela_read_root_state(onela_handle *h, void *S, onela_stream strea
 ONELA_API int onela_read_fold_depth(onela_handle *h, int32_t *depth, onela_stream stream);
 
 /* Wait for the handle's device (cudaDeviceSynchronize on it) and report the
- * error word in *device_err (0: none; bit 0: a bad parent index).
- * Returns ONELA_ERR_PARENT when bit 0 is set, ONELA_OK otherwise.
+ * error word in *device_err (0: none; bit 0: a bad parent index; bit 1: a
+ * bounded wait ran out in the tensor-core kernel; bit 2: a step's unfolded
+ * depths did not fit the store).  Returns ONELA_ERR_PARENT when bit 0 is
+ * set, ONELA_ERR_CAPACITY when bit 2 is, ONELA_OK otherwise.
  * Errors: ONELA_ERR_ARG, ONELA_ERR_CUDA. */
 ONELA_API int onela_status(onela_handle *h, int32_t *device_err);
 
@@ -276,14 +287,16 @@ ONELA_API int onela_status(onela_handle *h, int32_t *device_err);
  * Errors: ONELA_ERR_ARG. */
 ONELA_API int onela_destroy(onela_handle *h);
 
-/* Copy the records of depth t (1 <= t <= steps done) into caller DEVICE
+/* Copy the records of depth t (steps done - T_max < t <= steps done: the
+ * depths the store still holds) into caller DEVICE
  * buffers on `stream`: alpha fp32 [R][H][W_t], delta fp32 [R][H][W_t][d_v],
  * k [R][H][W_t][d_k] in qkv_dtype.  Any of the three may be NULL.
  * Errors: ONELA_ERR_ARG, ONELA_ERR_CUDA. */
 ONELA_API int onela_read_records(onela_handle *h, int32_t t, float *alpha, float *delta,
                        void *k, onela_stream stream);
 
-/* Copy the ancestry rows of depth t (1 <= t <= steps done) into a caller
+/* Copy the ancestry rows of depth t (1 <= t <= steps done, t <= T_max,
+ * and t still held: steps done - T_max < t) into a caller
  * DEVICE buffer on `stream`: int32 [R][W_t][t-1], entry [r][b][j] = index of
  * the beam at depth j+1 on the path from the root to beam b of step t.
  * Errors: ONELA_ERR_ARG, ONELA_ERR_CUDA. */

@@ -61,9 +61,12 @@ __global__ void __launch_bounds__(kPlanThreads) fold_plan_kernel(const StepParam
   if (tid == 0) s_split = n;
   __syncthreads();
   const int32_t *row0 = p.anc + anc_row(p, t, r, 0);
-  for (int e = tid; e < (Wt - 1) * n; e += kPlanThreads) {
-    const int b = 1 + e / n, j = e - (b - 1) * n;
-    if (p.anc[anc_row(p, t, r, b) + j] != row0[j]) atomicMin(&s_split, j);
+  // Depths old + 1 .. n can be newly shared; depth j + 1 sits in entry
+  // j mod T_max of the rows.
+  const int nw = n - old;
+  for (int e = tid; e < (Wt - 1) * nw; e += kPlanThreads) {
+    const int b = 1 + e / nw, j = old + e - (b - 1) * nw;
+    if (p.anc[anc_row(p, t, r, b) + j % TM] != row0[j % TM]) atomicMin(&s_split, j);
   }
   __syncthreads();
   // Sharing an ancestor at a depth implies sharing its ancestors, so the
@@ -72,7 +75,7 @@ __global__ void __launch_bounds__(kPlanThreads) fold_plan_kernel(const StepParam
   if (D == n && Wt == 1) D = t;
   if (D > max_depth) D = max_depth;
   if (D < old) D = old;
-  for (int j = old + tid; j < D; j += kPlanThreads) anc_fold[(int64_t)r * TM + j] = j < n ? row0[j] : 0;
+  for (int j = old + tid; j < D; j += kPlanThreads) anc_fold[(int64_t)r * TM + j % TM] = j < n ? row0[j % TM] : 0;
   if (tid == 0) d0_out[r] = D;
 }
 
@@ -93,7 +96,7 @@ __global__ void __launch_bounds__(kFoldThreads) fold_state_kernel(const StepPara
   const QT *rec_k = static_cast<const QT *>(p.rec_k);
 #pragma unroll 1
   for (int d = from + 1; d <= D; ++d) {
-    const int64_t row = rec_row(p, d, r, h, anc_fold[(int64_t)r * p.T_max + d - 1]);
+    const int64_t row = rec_row(p, d, r, h, anc_fold[(int64_t)r * p.T_max + (d - 1) % p.T_max]);
     const float a = p.rec_alpha[row];
     s = fmaf(p.rec_delta[row * dv + i], ldf(rec_k, row * dk + j), a * s);
   }
@@ -154,12 +157,12 @@ __global__ void __launch_bounds__(kFoldThreads) fold_tc_kernel(const StepParams 
   constexpr int KC = DK / 8, DC = RB / 4, PER = KC + DC + 1;  // 16-byte record pieces per depth
   constexpr int MAXI = (kFoldMaxT * PER + kFoldThreads - 1) / kFoldThreads;
   __shared__ int s_split;
-  __shared__ int s_row0[kFoldMaxT];
+  __shared__ int s_row0[kFoldMaxT];  // beam 0's ancestry row (entry j: depth j + 1 mod T_max)
   __shared__ float s_a[kFoldMaxT];
   __shared__ __align__(16) float s_d[kFoldMaxT][RB];
   __shared__ __align__(16) __nv_bfloat16 s_k[kFoldMaxT][DK];
   const int h = blockIdx.y, r = blockIdx.z, tid = threadIdx.x;
-  const int dv = p.dv, t = p.t, n = t - 1;
+  const int dv = p.dv, t = p.t, n = t - 1, TM = p.T_max;
   const int i0 = blockIdx.x * RB, ir = tid / TPR, c = tid - ir * TPR, i = i0 + ir;
   const bool valid = i < dv;
   const int64_t rh = (int64_t)r * p.H + h;
@@ -176,17 +179,21 @@ __global__ void __launch_bounds__(kFoldThreads) fold_tc_kernel(const StepParams 
   // Depths that can be folded: old + 1 .. Dmax (depth t only when step t
   // kept a single beam, its own record).
   const int jhi = min(n, max_depth);
-  const int Dmax = max(old, min(max_depth, Wt == 1 ? t : n));
+  // (at most T_max of them: more only after a step reported kErrWindow)
+  const int Dmax = max(old, min(min(max_depth, Wt == 1 ? t : n), old + TM));
   const int32_t *row0 = p.anc + anc_row(p, t, r, 0);
-  if (tid < n) s_row0[tid] = row0[tid];
+  if (tid < min(n, TM)) s_row0[tid] = row0[tid];
+  // Entry w of v and w0: depth old + w + 1 (at most T_max - 1 depths can be
+  // newly shared, as the step replayed them).
   int v[kFoldMaxT], w0[kFoldMaxT];
   const int b = 1 + tid;  // Wt <= kFoldThreads + 1 here; more beams: the loop below
   if (b < Wt) {
     const int32_t *row = p.anc + anc_row(p, t, r, b);
 #pragma unroll
-    for (int j = 0; j < kFoldMaxT; ++j) {
-      v[j] = (j >= old && j < jhi) ? row[j] : 0;
-      w0[j] = (j >= old && j < jhi) ? row0[j] : 0;
+    for (int w = 0; w < kFoldMaxT; ++w) {
+      const int j = old + w;
+      v[w] = j < jhi ? row[j % TM] : 0;
+      w0[w] = j < jhi ? row0[j % TM] : 0;
     }
   }
   __syncthreads();  // s_row0
@@ -199,7 +206,7 @@ __global__ void __launch_bounds__(kFoldThreads) fold_tc_kernel(const StepParams 
     piece[m] = make_uint4(0u, 0u, 0u, 0u);
     if (e < nitems) {
       const int dd = e / PER, q = e - dd * PER, d = old + dd + 1;
-      const int64_t row = rec_row(p, d, r, h, d - 1 < n ? s_row0[d - 1] : 0);
+      const int64_t row = rec_row(p, d, r, h, d - 1 < n ? s_row0[(d - 1) % TM] : 0);
       if (q < KC)
         piece[m] = *reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.rec_k) + row * DK + q * 8);
       else if (q < KC + DC)
@@ -211,13 +218,13 @@ __global__ void __launch_bounds__(kFoldThreads) fold_tc_kernel(const StepParams 
   int split = n;
   if (b < Wt) {
 #pragma unroll
-    for (int j = kFoldMaxT - 1; j >= 0; --j)
-      if (j >= old && j < jhi && v[j] != w0[j]) split = j;
+    for (int w = kFoldMaxT - 1; w >= 0; --w)
+      if (old + w < jhi && v[w] != w0[w]) split = old + w;
   }
   for (int bb = b + kFoldThreads; bb < Wt; bb += kFoldThreads) {
     const int32_t *row = p.anc + anc_row(p, t, r, bb);
     for (int j = old; j < jhi; ++j)
-      if (row[j] != s_row0[j]) {
+      if (row[j % TM] != s_row0[j % TM]) {
         split = min(split, j);
         break;
       }
@@ -242,9 +249,10 @@ __global__ void __launch_bounds__(kFoldThreads) fold_tc_kernel(const StepParams 
   int D = s_split;
   if (D == n && Wt == 1) D = t;
   if (D > max_depth) D = max_depth;
+  if (D > Dmax) D = Dmax;
   if (D < old) D = old;
   if (blockIdx.x == 0 && h == 0) {
-    for (int j = old + tid; j < D; j += kFoldThreads) anc_fold[(int64_t)r * p.T_max + j] = j < n ? s_row0[j] : 0;
+    for (int j = old + tid; j < D; j += kFoldThreads) anc_fold[(int64_t)r * TM + j % TM] = j < n ? s_row0[j % TM] : 0;
     if (tid == 0) d0_out[r] = D;
   }
   if ((!first && D == old) || !valid) return;  // unchanged: the folded state and image hold it

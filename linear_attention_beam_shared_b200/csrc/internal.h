@@ -7,7 +7,7 @@
 
 namespace onela {
 
-constexpr int kHistSteps = 17;     // steps 1..16: the deepest tensor-core decode
+constexpr int kHistSteps = 17;     // steps of history the tensor-core kernel can see (its window is <= 16)
 constexpr int kHistMaxInts = 4096;  // parents of earlier steps the tensor-core kernel
                                     // keeps in shared memory (more: read from global memory)
 
@@ -21,34 +21,43 @@ struct StepParams {
   const void *q, *k, *v;  // [R][W][H][d] in the qkv type
   const float *g, *beta;  // [R][W][H]
   const int32_t *parents; // [R][W]
-  int32_t *par_store;     // [T_max][R][W_max]: each step's parents (tensor-core kernel)
-  // History of the decode for the tensor-core kernel, indexed by step j
-  // (1 <= j < t): keys, gates and parents of every earlier step.
-  // hist_inputs = 1: the callers' own arrays of step j, valid under
-  // ONELA_FLAG_PDL -- hk[j] [R][W_j][H][d_k], hg[j] [R][W_j][H] (the gate
-  // before exp), hpar[j] [R][W_j].  hist_inputs = 0: the record store
-  // (rec_k, rec_alpha) and the par_store row of step j.  Parents of request r
-  // start at hpar[j] + r * hpar_rs[j]; hW[j] = W_j.
+  int32_t *par_store;     // [T_max slots][R][W_max]: each step's parents (tensor-core kernel)
+  // History of the decode for the tensor-core kernel: entry i describes step
+  // j = hbase + i (hbase <= j < t, at most kHistSteps steps back): keys,
+  // gates and parents.  hist_inputs = 1: the callers' own arrays of step j,
+  // valid under ONELA_FLAG_PDL -- hk[i] [R][W_j][H][d_k], hg[i] [R][W_j][H]
+  // (the gate before exp), hpar[i] [R][W_j].  hist_inputs = 0: the record
+  // store (rec_k, rec_alpha) and the par_store row of step j.  Parents of
+  // request r start at hpar[i] + r * hpar_rs[i]; hW[i] = W_j.  The kernel
+  // copies the parents of steps hcopy .. t - 1 to shared memory.
   int hist_inputs;
+  int hbase, hcopy;
   const void *hk[kHistSteps];
   const float *hg[kHistSteps];
   const int32_t *hpar[kHistSteps];
   int hpar_rs[kHistSteps];
   int hW[kHistSteps];
-  int hoff[kHistSteps];  // where step j's parents start in the kernel's shared copy (ints)
-  int hist_cap;  // ints of shared memory for the parents of steps 2..t-1 (0: read them from global memory)
+  int hoff[kHistSteps];  // where step j's parents start in the kernel's shared copy (entries)
+  int hist_cap;  // entries of shared memory for the parents of steps hcopy..t-1 (0: read them from global memory)
   float *o;               // [R][W][H][dv]
   const void *S0;         // [R][H][dv][dk] in the S0 type
   const void *S0img;      // tensor-core operand image of S0 (see step_tc.cu)
   int s0_planes;          // bf16 terms in S0img (1 for bf16 S0)
-  float *rec_alpha;       // [T_max][R][H][W_max]
-  float *rec_delta;       // [T_max][R][H][W_max][dv]
-  void *rec_k;            // [T_max][R][H][W_max][dk] in the qkv type
-  int32_t *anc;           // [T_max][R][W_max][T_max]
+  // The record store keeps the last T_max depths: depth s sits in slot
+  // (s - 1) mod T_max (rec_slot).  A step replays depths d0 + 1 .. t - 1,
+  // which must fit: t - 1 - d0 <= T_max - 1 (else kErrWindow).
+  float *rec_alpha;       // [T_max slots][R][H][W_max]
+  float *rec_delta;       // [T_max slots][R][H][W_max][dv]
+  void *rec_k;            // [T_max slots][R][H][W_max][dk] in the qkv type
+  // Ancestry rows [T_max slots][R][W_max][T_max]: the row of a beam of depth
+  // s holds its ancestor at depth j + 1 in entry j mod T_max, for the last
+  // T_max - 1 depths before s.
+  int32_t *anc;
   // Folded prefix (onela_fold), per request: depths 1..d0[r] are folded into
   // S0 (then the folded state), their ancestors are the same for every beam
-  // of the request, anc_fold[r][j] at depth j + 1 ([R][T_max]), and only
-  // depths d0[r] + 1 .. t - 1 are replayed.  d0 null: nothing folded.
+  // of the request, anc_fold[r][j mod T_max] at depth j + 1 ([R][T_max], the
+  // last T_max depths), and only depths d0[r] + 1 .. t - 1 are replayed.
+  // d0 null: nothing folded.
   const int32_t *d0;
   const int32_t *anc_fold;
   int32_t *err;           // host-mapped error word (device view)
@@ -59,17 +68,26 @@ struct StepParams {
   alignas(64) CUtensorMap tm_v;
 };
 
+// Slot of depth s (1-based) in the record store, the parents store and the
+// ancestry rows.
+__host__ __device__ __forceinline__ int rec_slot(const StepParams &p, int s) { return (s - 1) % p.T_max; }
+// Row index of the record of beam b, head h, request r in a slot.
+__host__ __device__ __forceinline__ int64_t rec_row_slot(const StepParams &p, int slot, int r, int h, int b) {
+  return ((int64_t)(slot * p.R + r) * p.H + h) * p.W_max + b;
+}
 // Row index of the record of beam b, head h, request r at depth s (1-based).
 __host__ __device__ __forceinline__ int64_t rec_row(const StepParams &p, int s, int r, int h, int b) {
-  return ((int64_t)((s - 1) * p.R + r) * p.H + h) * p.W_max + b;
+  return rec_row_slot(p, rec_slot(p, s), r, h, b);
 }
 // First entry of the ancestry row of beam b, request r, at depth s (1-based).
 __host__ __device__ __forceinline__ int64_t anc_row(const StepParams &p, int s, int r, int b) {
-  return ((int64_t)((s - 1) * p.R + r) * p.W_max + b) * p.T_max;
+  return ((int64_t)(rec_slot(p, s) * p.R + r) * p.W_max + b) * p.T_max;
 }
 
 // Device error word bits.
 constexpr int32_t kErrParent = 1;
+// (bit 1: a bounded wait ran out, tensor-core kernel)
+constexpr int32_t kErrWindow = 4;  // a step's unfolded depths did not fit the record store
 
 // Kernel launchers (step_simt.cu, step_tc.cu).  Return a cudaError_t.
 cudaError_t launch_step_simt(const StepParams &p, int qkv_bf16, int s0_bf16, cudaStream_t s);

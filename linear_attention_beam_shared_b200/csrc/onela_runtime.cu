@@ -273,11 +273,16 @@ int onela_decode_step(onela_handle *h, int32_t W_prev, int32_t W, const void *q,
                       const float *gate, const float *beta, const int32_t *parent_idx, float *o,
                       onela_stream stream) {
   if (!h || !q || !k || !v || !gate || !beta || !parent_idx || !o) return ONELA_ERR_ARG;
-  if (*reinterpret_cast<volatile int32_t *>(h->err_host) & onela::kErrParent) return ONELA_ERR_PARENT;
+  const int32_t word = *reinterpret_cast<volatile int32_t *>(h->err_host);
+  if (word & onela::kErrParent) return ONELA_ERR_PARENT;
+  if (word & onela::kErrWindow) return ONELA_ERR_CAPACITY;
   if (!h->has_prompt) return ONELA_ERR_STATE;
   const onela_config &c = h->cfg;
   if (W < 1) return ONELA_ERR_ARG;
-  if (W > c.W_max || h->steps_done >= c.T_max) return ONELA_ERR_CAPACITY;
+  // Past T_max steps only with a fold: the device checks that each step's
+  // unfolded depths fit the store (kErrWindow otherwise).
+  if (W > c.W_max || (h->steps_done >= c.T_max && !h->folded) || h->steps_done >= (1 << 30))
+    return ONELA_ERR_CAPACITY;
   const int expect_prev = h->steps_done == 0 ? 1 : h->Ws.back();
   if (W_prev != expect_prev) return ONELA_ERR_ARG;
   DeviceGuard g(c.device);
@@ -308,20 +313,27 @@ int onela_decode_step(onela_handle *h, int32_t W_prev, int32_t W, const void *q,
     // ONELA_FLAG_PDL (still valid by its contract), else the record store
     // and the parents the earlier kernels stored (they have completed).
     p.hist_inputs = pdl ? 1 : 0;
+    // The table covers steps hbase .. t-1 (the kernel replays at most
+    // T_max - 1 <= 15 of them); the parents of steps hcopy .. t-1 go to
+    // shared memory.
+    p.hbase = p.t - onela::kHistSteps + 1 > 1 ? p.t - onela::kHistSteps + 1 : 1;
+    p.hcopy = p.t - c.T_max + 1 > 2 ? p.t - c.T_max + 1 : 2;
+    if (p.hcopy < p.hbase + 1) p.hcopy = p.hbase + 1;
     int hist = 0;
-    for (int j = 1; j < p.t; ++j) {
-      p.hW[j] = h->Ws[j - 1];
+    for (int j = p.hbase; j < p.t; ++j) {
+      const int i = j - p.hbase;
+      p.hW[i] = h->Ws[j - 1];
       if (pdl) {
-        p.hk[j] = h->hist_k[j - 1];
-        p.hg[j] = h->hist_g[j - 1];
-        p.hpar[j] = h->hist_par[j - 1];
-        p.hpar_rs[j] = h->Ws[j - 1];
+        p.hk[i] = h->hist_k[j - 1];
+        p.hg[i] = h->hist_g[j - 1];
+        p.hpar[i] = h->hist_par[j - 1];
+        p.hpar_rs[i] = h->Ws[j - 1];
       } else {
-        p.hpar[j] = h->par_store + (size_t)(j - 1) * c.R * c.W_max;
-        p.hpar_rs[j] = c.W_max;
+        p.hpar[i] = h->par_store + (size_t)((j - 1) % c.T_max) * c.R * c.W_max;
+        p.hpar_rs[i] = c.W_max;
       }
-      if (j >= 2) {
-        p.hoff[j] = hist;
+      if (j >= p.hcopy) {
+        p.hoff[i] = hist;
         hist += (h->Ws[j - 1] + 3) & ~3;
       }
     }
@@ -363,7 +375,9 @@ int onela_reset(onela_handle *h, onela_stream stream) {
 
 int onela_fold(onela_handle *h, int32_t max_depth, onela_stream stream) {
   if (!h || max_depth < 0) return ONELA_ERR_ARG;
-  if (*reinterpret_cast<volatile int32_t *>(h->err_host) & onela::kErrParent) return ONELA_ERR_PARENT;
+  const int32_t word = *reinterpret_cast<volatile int32_t *>(h->err_host);
+  if (word & onela::kErrParent) return ONELA_ERR_PARENT;
+  if (word & onela::kErrWindow) return ONELA_ERR_CAPACITY;
   if (!h->has_prompt) return ONELA_ERR_STATE;
   if (h->steps_done == 0 || max_depth == 0) return ONELA_OK;  // nothing to fold
   DeviceGuard g(h->cfg.device);
@@ -429,7 +443,8 @@ int onela_status(onela_handle *h, int32_t *device_err) {
   if (cudaDeviceSynchronize() != cudaSuccess) return ONELA_ERR_CUDA;
   const int32_t e = *reinterpret_cast<volatile int32_t *>(h->err_host);
   if (device_err) *device_err = e;
-  return (e & onela::kErrParent) ? ONELA_ERR_PARENT : ONELA_OK;
+  if (e & onela::kErrParent) return ONELA_ERR_PARENT;
+  return (e & onela::kErrWindow) ? ONELA_ERR_CAPACITY : ONELA_OK;
 }
 
 int onela_destroy(onela_handle *h) {
@@ -444,7 +459,7 @@ int onela_destroy(onela_handle *h) {
 }
 
 int onela_read_records(onela_handle *h, int32_t t, float *alpha, float *delta, void *k, onela_stream stream) {
-  if (!h || t < 1 || t > h->steps_done) return ONELA_ERR_ARG;
+  if (!h || t < 1 || t > h->steps_done || t <= h->steps_done - h->cfg.T_max) return ONELA_ERR_ARG;
   DeviceGuard g(h->cfg.device);
   if (!g.ok) return ONELA_ERR_CUDA;
   const onela_config &c = h->cfg;
@@ -453,7 +468,7 @@ int onela_read_records(onela_handle *h, int32_t t, float *alpha, float *delta, v
   const size_t ks = esize(c.qkv_dtype);
   // Rows are [R][H][W_max]: copy the first W_t rows of each (r, h) block.
   const size_t nblk = (size_t)c.R * c.H;
-  const size_t base = (size_t)(t - 1) * nblk * c.W_max;
+  const size_t base = (size_t)((t - 1) % c.T_max) * nblk * c.W_max;
   bool ok = true;
   if (alpha)
     ok = ok && cudaMemcpy2DAsync(alpha, Wt * sizeof(float), h->rec_alpha + base, (size_t)c.W_max * sizeof(float),
@@ -470,7 +485,9 @@ int onela_read_records(onela_handle *h, int32_t t, float *alpha, float *delta, v
 }
 
 int onela_read_ancestry(onela_handle *h, int32_t t, int32_t *anc, onela_stream stream) {
-  if (!h || !anc || t < 1 || t > h->steps_done) return ONELA_ERR_ARG;
+  // Whole rows exist only while the depths 1..t-1 fit the row (t <= T_max).
+  if (!h || !anc || t < 1 || t > h->steps_done || t > h->cfg.T_max || t <= h->steps_done - h->cfg.T_max)
+    return ONELA_ERR_ARG;
   if (t == 1) return ONELA_OK;  // the chain of a depth-1 beam is empty
   DeviceGuard g(h->cfg.device);
   if (!g.ok) return ONELA_ERR_CUDA;

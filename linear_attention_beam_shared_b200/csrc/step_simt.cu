@@ -50,7 +50,13 @@ __global__ void __launch_bounds__(kNT) step_simt_kernel(const StepParams p) {
   const int b0 = tile * kBT;
   const int nb = min(kBT, p.W - b0);
   const int dk = p.dk, dv = p.dv, H = p.H, t = p.t, TM = p.T_max;
-  const int d0 = p.d0 ? p.d0[r] : 0;  // depths 1..d0 are folded into S0
+  // Depths 1..d0 are folded into S0; the beams replay depths d0+1..t-1,
+  // which must fit the record store's T_max slots.
+  int d0 = p.d0 ? p.d0[r] : 0;
+  if (t - 1 - d0 > TM - 1) {
+    if (tid == 0) *reinterpret_cast<volatile int32_t *>(p.err) = kErrWindow;
+    d0 = t - TM;  // keeps every access inside the store; the results are void
+  }
   const int nanc = t - 1 - d0;  // replayed ancestors: chain index j is depth d0 + j + 1
 
   const int XS = dk + 1;                   // row stride of xk, xq
@@ -99,17 +105,18 @@ __global__ void __launch_bounds__(kNT) step_simt_kernel(const StepParams p) {
       }
       int *chain = s_chain + b * TM;
       if (t >= 2) {
-        // The parent's ancestry row holds absolute depths 1..t-2 (the
-        // folded prefix included); the chain keeps the replayed ones.
+        // The parent's ancestry row holds the ancestor at depth dd in
+        // entry (dd - 1) mod T_max for its last T_max - 1 depths (the folded
+        // prefix included); the chain keeps the replayed ones.
         const int32_t *prow = p.anc + anc_row(p, t - 1, r, par);
         if (nanc >= 1) {
           chain[nanc - 1] = par;
-          for (int j = 0; j < nanc - 1; ++j) chain[j] = prow[d0 + j];
+          for (int j = 0; j < nanc - 1; ++j) chain[j] = prow[(d0 + j) % TM];
         }
         if (h == 0) {
           int32_t *row = p.anc + anc_row(p, t, r, gb);
-          for (int j = 0; j < t - 2; ++j) row[j] = prow[j];
-          row[t - 2] = par;
+          for (int dd = max(1, t - TM + 1); dd < t - 1; ++dd) row[(dd - 1) % TM] = prow[(dd - 1) % TM];
+          row[(t - 2) % TM] = par;
         }
       }
       float run = 1.f;

@@ -138,9 +138,18 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
   const int b0 = tile * kBT;
   const int nb = min(kBT, p.W - b0);
   const int H = p.H, t = p.t, TM = p.T_max, P = p.s0_planes;
-  const int d0 = p.d0 ? p.d0[r] : 0;  // depths 1..d0 are folded into S0
-  const int nanc = t - 1 - d0;  // ancestors per beam (depths d0+1..t-1); chain index j is depth d0+j+1
+  // Depths 1..d0 are folded into S0; the beams replay depths d0+1..t-1,
+  // which must fit the record store's T_max slots.
+  int d0 = p.d0 ? p.d0[r] : 0;
+  if (t - 1 - d0 > TM - 1) {
+    if (tid == 0) *reinterpret_cast<volatile int32_t *>(p.err) = kErrWindow;
+    d0 = t - TM;  // keeps every access inside the store; the results are void
+  }
+  const int nanc = t - 1 - d0;  // ancestors per beam; chain index j is depth d0+j+1
   const int jp = nanc - 1;      // chain index of the parents (depth t-1)
+  const int soff = d0 % TM;     // slot of depth d0 + 1
+  const int tslot = (t - 1) % TM;  // slot of depth t
+  const int hb = p.hbase;       // step of the history table's entry 0
   const bool hin = p.hist_inputs != 0;
 
   const Layout L = layout(NK, P, TM, p.W_max, p.hist_cap);
@@ -229,8 +238,9 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
   // copies steps w + 1, w + 8, w + 15.
   if (p.hist_cap > 0 && warp >= 1 && warp < kAncWarp)
 #pragma unroll 2
-    for (int j = warp + 1; j < t; j += kAncWarp - 1)
-      copy_parents16_warp(s_hist + p.hoff[j], p.hpar[j] + (int64_t)r * p.hpar_rs[j], p.hW[j], lane);
+    for (int j = p.hcopy + warp - 1; j < t; j += kAncWarp - 1)
+      copy_parents16_warp(s_hist + p.hoff[j - hb], p.hpar[j - hb] + (int64_t)r * p.hpar_rs[j - hb], p.hW[j - hb],
+                          lane);
   ptx::cp_async_commit();
   ptx::cp_async_wait_all();
   ptx::tc_fence_before();
@@ -272,8 +282,9 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
 #pragma unroll 1
       for (int j = jp - 1; j >= 0; --j) {
         const int st = d0 + j + 2;  // the step whose parent array leads from depth st-1 to st
-        int pa = p.hist_cap > 0 ? s_hist[s_toff[st] + a] : s_tpar[st][(int64_t)r * s_trs[st] + a];
-        if (pa < 0 || pa >= s_tW[st - 1]) pa = 0;  // reported by step st
+        const int si = st - hb;
+        int pa = p.hist_cap > 0 ? s_hist[s_toff[si] + a] : s_tpar[si][(int64_t)r * s_trs[si] + a];
+        if (pa < 0 || pa >= s_tW[si - 1]) pa = 0;  // reported by step st
         a = pa;
         s_chain[b * TM + j] = a;
       }
@@ -285,9 +296,10 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
 #pragma unroll 1
       for (int j = 0; j <= jp; ++j) {
         const int a = s_chain[b * TM + j];
-        const int dj = d0 + j + 1;  // depth of the record
-        ptx::cp_async4(s_w + b * TM + j, hin ? s_tg[dj] + ((int64_t)r * s_tW[dj] + a) * H + h
-                                             : p.rec_alpha + rec_row(p, dj, r, h, a));
+        const int di = d0 + j + 1 - hb;  // history entry of the record's depth
+        const int sl = soff + j < TM ? soff + j : soff + j - TM;
+        ptx::cp_async4(s_w + b * TM + j, hin ? s_tg[di] + ((int64_t)r * s_tW[di] + a) * H + h
+                                             : p.rec_alpha + rec_row_slot(p, sl, r, h, a));
       }
     }
     ptx::cp_async_commit();
@@ -374,9 +386,10 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
         const int j = j0 + e;
         if (bval && j < nanc) {
           const int a = s_chain[bb * TM + j];
-          const int dj = d0 + j + 1;
-          const __nv_bfloat16 *row = hin ? s_tk[dj] + ((int64_t)(r * s_tW[dj] + a) * H + h) * DK
-                                         : rec_k + rec_row(p, dj, r, h, a) * DK;
+          const int di = d0 + j + 1 - hb;
+          const int sl = soff + j < TM ? soff + j : soff + j - TM;
+          const __nv_bfloat16 *row = hin ? s_tk[di] + ((int64_t)(r * s_tW[di] + a) * H + h) * DK
+                                         : rec_k + rec_row_slot(p, sl, r, h, a) * DK;
           const uint8_t *rb = reinterpret_cast<const uint8_t *>(row) + l * 8;
 #pragma unroll
           for (int u = 0; u < NU; ++u) buf[e][u] = __ldg(reinterpret_cast<const uint2 *>(rb + (u ^ sx) * 64));
@@ -448,21 +461,28 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
       for (int e = tid; e < kBT * NK * 8; e += 128) {
         const int n = e / (NK * 8), cc = e - n * (NK * 8);
         if (n < nb)
-          reinterpret_cast<uint4 *>(rec_k + rec_row(p, t, r, h, b0 + n) * DK)[cc] =
+          reinterpret_cast<uint4 *>(rec_k + rec_row_slot(p, tslot, r, h, b0 + n) * DK)[cc] =
               *reinterpret_cast<const uint4 *>(s_x + (cc >> 3) * XA + ptx::swz128(n, cc & 7));
       }
     }
     // alpha, the ancestry row and the parent of the beam.
     if (bval && l == 0) {
       const int gb = b0 + bb;
-      p.rec_alpha[rec_row(p, t, r, h, gb)] = s_alpha[bb];
+      p.rec_alpha[rec_row_slot(p, tslot, r, h, gb)] = s_alpha[bb];
       if (h == 0) {
-        int32_t *row = p.anc + anc_row(p, t, r, gb);
+        // Entry (depth - 1) mod T_max for the last T_max - 1 depths before t:
+        // the folded ones from the shared ancestors, the others from the chain.
+        int32_t *row = p.anc + ((int64_t)(tslot * p.R + r) * p.W_max + gb) * TM;
+        // dlo - 1 = t - T_max past the first T_max steps, whose entry
+        // follows the slot of depth t; stepped with a wrap.
+        const int dlo = max(1, t - TM + 1);
+        int e = t > TM ? (tslot + 1 < TM ? tslot + 1 : 0) : 0;
 #pragma unroll 1
-        for (int j = 0; j < d0; ++j) row[j] = p.anc_fold[r * TM + j];
-#pragma unroll 1
-        for (int j = 0; j < nanc; ++j) row[d0 + j] = s_chain[bb * TM + j];
-        p.par_store[((int64_t)(t - 1) * p.R + r) * p.W_max + gb] = s_par[bb];
+        for (int dd = dlo; dd < t; ++dd) {
+          row[e] = dd <= d0 ? p.anc_fold[r * TM + e] : s_chain[bb * TM + dd - 1 - d0];
+          e = e + 1 < TM ? e + 1 : 0;
+        }
+        p.par_store[((int64_t)tslot * p.R + r) * p.W_max + gb] = s_par[bb];
       }
     }
   }
@@ -505,8 +525,9 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
     for (int e = tid; e < nrows * PD; e += kThreads) {
       const int rr = e / PD, c = e - rr * PD;
       const int packed = s_list[lo + rr];
+      const int j = packed & 31, sl = soff + j < TM ? soff + j : soff + j - TM;
       ptx::cp_async16(base + L.dst + (uint32_t)(rr * DV + c * 4) * 4u,
-                      p.rec_delta + rec_row(p, d0 + (packed & 31) + 1, r, h, packed >> 5) * DV + c * 4, 16u);
+                      p.rec_delta + rec_row_slot(p, sl, r, h, packed >> 5) * DV + c * 4, 16u);
     }
     ptx::cp_async_commit();
     ptx::cp_async_wait_all();
@@ -546,7 +567,7 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
   if (!ok) *reinterpret_cast<volatile int32_t *>(p.err) = kErrTimeout;
   if (bval && ok) {
     float4 *op = reinterpret_cast<float4 *>(p.o + (row0 + (int64_t)bb * H) * DV) + l;
-    float4 *dp = reinterpret_cast<float4 *>(p.rec_delta + rec_row(p, t, r, h, b0 + bb) * DV) + l;
+    float4 *dp = reinterpret_cast<float4 *>(p.rec_delta + rec_row_slot(p, tslot, r, h, b0 + bb) * DV) + l;
 #pragma unroll
     for (int u = 0; u < NU; ++u) {
       float4 d, o;

@@ -42,8 +42,9 @@ def narrow(steps, at, beam):
 
 def run_with_folds(S0, steps, qkv, kernel, folds, flags=0, T_max=None):
     """Decode all steps on the GPU; after step t (1-based) in `folds`, fold
-    with max_depth folds[t].  Returns per-step outputs/records/ancestry and,
-    per fold, (t, fold depth [R], root state)."""
+    with max_depth folds[t].  Returns per-step outputs, records and ancestry
+    (records only for the depths the store still holds, ancestry only while
+    t <= T_max) and, per fold, (t, fold depth [R], root state)."""
     import linear_attention_beam_shared_b200 as L
     R, H, dv, dk = S0.shape
     s0_dtype = "bf16" if S0.dtype == torch.bfloat16 else "f32"
@@ -61,11 +62,17 @@ def run_with_folds(S0, steps, qkv, kernel, folds, flags=0, T_max=None):
                 fold_info.append((t, dec.fold_depth().cpu().numpy(), dec.root_state().cpu()))
         assert dec.status() == 0
         res = []
+        T, TM = len(steps), T_max or len(steps)
         for t, o in enumerate(outs, start=1):
-            a, d, kr = dec.records(t)
-            res.append({"o": o.cpu(), "alpha": a.cpu().permute(0, 2, 1).contiguous(),
-                        "delta": d.cpu().permute(0, 2, 1, 3).contiguous(),
-                        "k": kr.cpu().permute(0, 2, 1, 3).contiguous(), "anc": dec.ancestry(t).cpu()})
+            r = {"o": o.cpu()}
+            if t > T - TM:
+                a, d, kr = dec.records(t)
+                r.update({"alpha": a.cpu().permute(0, 2, 1).contiguous(),
+                          "delta": d.cpu().permute(0, 2, 1, 3).contiguous(),
+                          "k": kr.cpu().permute(0, 2, 1, 3).contiguous()})
+            if t <= TM and t > T - TM:
+                r["anc"] = dec.ancestry(t).cpu()
+            res.append(r)
         return res, fold_info, dec.kernel
     finally:
         dec.close()
@@ -264,3 +271,72 @@ def test_fold_full_size(name):
     assert D.tolist() == want.tolist() and (D >= 2).all()
     check_state(S, gdn.fold_state(S0t, steps[:4], want))
     P.compare(gpu, P.oracle(S0t, steps), steps, wl.s0_dtype)
+
+
+@pytest.mark.parametrize("kind", ["simt", "tc"])
+@pytest.mark.parametrize("pdl", [0, 1])
+def test_decode_deeper_than_the_record_store(kind, pdl):
+    """A store of T_max = 6 depths and a 26-step decode: every beam of steps
+    4, 8, ..., 24 is a child of one beam and a fold follows each of them, so
+    no step replays more than 5 depths while the records wrap around the
+    store.  Every output, and the delta records the store still holds,
+    against the fp64 oracle of the whole 26-step tree."""
+    import linear_attention_beam_shared_b200 as L
+    T, TM = 26, 6
+    dk = dv = 128 if kind == "tc" else 32
+    Ws = [12, 20, 16, 20, 24, 16, 20, 12] * 3 + [16, 20]
+    wl, S0, steps = P.custom_steps(40, R=2, H=2, dk=dk, dv=dv, Ws=Ws, parents="uniform")
+    for at in range(3, T - 1, 4):
+        steps = narrow(steps, at, [at % 5, (at + 2) % 7])
+    folds = {at + 1: T for at in range(3, T - 1, 4)}
+    S0t = synth.cast_state(S0, "f32")
+    gpu, info, used = run_with_folds(S0t, steps, "bf16", kernel_id(kind), folds,
+                                     flags=L.ONELA_FLAG_PDL if pdl else 0, T_max=TM)
+    assert used == kernel_id(kind)
+    for t, D, _ in info:
+        assert D.tolist() == [t - 1, t - 1]
+    ref = P.oracle(S0t, steps)
+    for t, (g, r) in enumerate(zip(gpu, ref), start=1):
+        err = float(np.abs(g["o"].double().numpy() - r["o"]).max())
+        assert err <= P.TOL["f32"], (t, err)
+        if "delta" in g:
+            err = float(np.abs(g["delta"].double().numpy() - r["delta"]).max())
+            assert err <= P.TOL["f32"], (t, err)
+            assert torch.equal(g["k"], steps[t - 1]["k"])
+
+
+@pytest.mark.parametrize("kind", ["simt", "tc"])
+def test_unfolded_window_overflow_is_reported(kind):
+    """With nothing shared to fold, a decode that goes past T_max unfolded
+    depths is stopped: the host refuses step T_max + 1 without a fold, and
+    after a fold that folded nothing the device reports the overflow
+    (ONELA_ERR_CAPACITY) instead of replaying overwritten records.  Records
+    of depths that left the store cannot be read back."""
+    import linear_attention_beam_shared_b200 as L
+    TM = 4
+    dk = dv = 128 if kind == "tc" else 32
+    wl, S0, steps = P.custom_steps(41, R=1, H=2, dk=dk, dv=dv, Ws=[8] * 6, parents="uniform")
+    for t in range(1, 6):
+        steps[t]["parents"] = torch.arange(8, dtype=torch.int32)[None]
+    dec = L.BeamDecoder(1, 2, dk, dv, 8, TM, "f32", "bf16", kernel=kernel_id(kind))
+    try:
+        ds = P.to_dev(steps)
+        dec.set_prompt_state(synth.cast_state(S0, "f32").cuda())
+        for s in ds[:TM]:
+            dec.step(s["q"], s["k"], s["v"], s["g"], s["beta"], s["parents"])
+        s = ds[TM]
+        with pytest.raises(L.OnelaError) as e:
+            dec.step(s["q"], s["k"], s["v"], s["g"], s["beta"], s["parents"])
+        assert e.value.code == L.ONELA_ERR_CAPACITY
+        dec.fold()
+        assert dec.fold_depth().cpu().tolist() == [0]
+        dec.step(s["q"], s["k"], s["v"], s["g"], s["beta"], s["parents"])
+        with pytest.raises(L.OnelaError) as e:
+            dec.status()
+        assert e.value.code == L.ONELA_ERR_CAPACITY
+        with pytest.raises(L.OnelaError):
+            L.onela_read_records(dec.h, 1, 8)
+        dec.reset()
+        assert dec.status() == 0
+    finally:
+        dec.close()
