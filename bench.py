@@ -252,12 +252,14 @@ def time_select(device, stream, flush, R=1, W_prev=256, C=256, W=256, reps=20, w
     }
 
 
-def time_fold(wl, S0, kernel, device, stream, flush, T=16, every=4, reps=10, warmup=3, alone=True):
+def time_fold(wl, S0, kernel, device, stream, flush, T=16, every=4, reps=10, warmup=3, alone=True, tmax=None):
     """Folding on a deeper decode: the workload's shapes over T steps, every
     beam of steps every, 2 every, ... a child of one beam (the beam sets
     narrow to one shared ancestor), decoded as one CUDA graph with a fold
     right after each such step and, for comparison, without folds; then the
-    fold alone (after the first narrowing step, caches flushed).  The folded and unfolded outputs must agree to fp32 rounding.
+    fold alone (after the first narrowing step, caches flushed).  The folded
+    and unfolded outputs must agree to fp32 rounding.  tmax < T: a record
+    store of tmax depths, which only the folded decode can run through.
     Returns the JSON object for the bench line."""
     import linear_attention_beam_shared_b200 as L
     wd = wl.replace(name=wl.name + "_deep", T=T)
@@ -270,8 +272,8 @@ def time_fold(wl, S0, kernel, device, stream, flush, T=16, every=4, reps=10, war
 
     def make(fold):
         outs = [torch.empty((wd.R, st["W"], wd.H, wd.d_v), dtype=torch.float32, device=device) for st in steps]
-        dec = L.BeamDecoder(wd.R, wd.H, wd.d_k, wd.d_v, wd.W, T, wd.s0_dtype, wd.qkv_dtype, kernel=kernel,
-                            device=device.index, flags=L.ONELA_FLAG_PDL)
+        dec = L.BeamDecoder(wd.R, wd.H, wd.d_k, wd.d_v, wd.W, tmax or T, wd.s0_dtype, wd.qkv_dtype,
+                            kernel=kernel, device=device.index, flags=L.ONELA_FLAG_PDL)
         dec.set_prompt_state(S0.to(device))
 
         def run():
@@ -312,12 +314,21 @@ def time_fold(wl, S0, kernel, device, stream, flush, T=16, every=4, reps=10, war
         return max_over_ranks(sum(e0.elapsed_time(e1) for e0, e1 in ev) / reps, device)
 
     res = {}
-    for fold in (True, False):
+    for fold in ((True,) if tmax and tmax < T else (True, False)):
         dec, g, outs, depth = make(fold)
         ms = timed(g)
         res[fold] = (ms, [o.clone() for o in outs], depth)
         del g
         dec.close()
+    if False not in res:
+        return {
+            "workload": f"{wl.name} shapes over T={T} steps through a record store of {tmax} depths "
+                        f"(R={wd.R}, H={wd.H}, d={wd.d_k}, W={wd.W}), every beam of steps "
+                        f"{', '.join(str(i + 1) for i in narrow)} a child of beam 0; folds right after them",
+            "ms_per_decode": {"folded": round(res[True][0], 5), "unfolded": None},
+            "us_per_step": round(res[True][0] * 1e3 / T, 3),
+            "fold_depth_at_end": res[True][2],
+        }
     diff = max(float((a - b).abs().max()) for a, b in zip(res[True][1], res[False][1]))
     scale = max(float(b.abs().max()) for b in res[False][1])
     assert diff <= 2e-5 * max(1.0, scale), f"folded decode differs from the unfolded one by {diff}"
@@ -691,7 +702,9 @@ def run_ours(args):
     select = None if args.no_prefill else time_select(device, stream, flush, R=wl.R, W_prev=wl.W, C=256, W=wl.W)
     sweep = None if (args.no_sweep or ws > 1) else time_sweep(device, stream, flush)
     fold = None if args.no_prefill else [time_fold(wl, S0, kernel, device, stream, flush, every=4),
-                                          time_fold(wl, S0, kernel, device, stream, flush, every=8, alone=False)]
+                                          time_fold(wl, S0, kernel, device, stream, flush, every=8, alone=False),
+                                          time_fold(wl, S0, kernel, device, stream, flush, T=32, every=8, alone=False,
+                                                    tmax=16)]
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu:
