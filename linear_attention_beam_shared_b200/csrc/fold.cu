@@ -10,9 +10,10 @@
 //     S_c = alpha_D S_{D-1} + delta_D k_D^T,  S_0 = the prompt state,
 // (the recurrence of the review's section 3.2 equations), after which the
 // decode kernels replay only depths D+1..t-1.  Nothing else changes: the
-// record store, the ancestry rows (still absolute depths) and the outputs
-// stay those of the unfolded decode, up to the rounding of S_c to the
-// state's storage type.
+// record store, the ancestry rows and the outputs stay those of the
+// unfolded decode, up to the rounding of S_c to the state's storage type.
+// Since only the unfolded depths are read, a decode that keeps folding can
+// run past the T_max depths the record store keeps.
 //
 // The folded depth of each request is double-buffered (d0_in is read, d0_out
 // written), so that every CTA of a launch sees the same previous depth.

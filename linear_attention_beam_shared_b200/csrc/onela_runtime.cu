@@ -493,7 +493,8 @@ int onela_read_ancestry(onela_handle *h, int32_t t, int32_t *anc, onela_stream s
   if (!g.ok) return ONELA_ERR_CUDA;
   const onela_config &c = h->cfg;
   const int Wt = h->Ws[t - 1];
-  // Source rows [R][W_max][T_max] -> dest [R][W_t][t-1].
+  // Source rows [R][W_max][T_max] (t <= T_max: entry j is depth j + 1) ->
+  // dest [R][W_t][t-1].
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   for (int r = 0; r < c.R; ++r) {
     const int32_t *src = h->anc + ((size_t)(t - 1) * c.R + r) * c.W_max * c.T_max;

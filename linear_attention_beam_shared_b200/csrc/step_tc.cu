@@ -44,6 +44,13 @@
 // ancestors' delta rows arrive in one round of 16-byte copies, every beam
 // thread replays and writes o and delta.  No kernel reads a depth-t entry
 // before step t has completed, so the early writes race with nothing.
+//
+// With a folded prefix (onela_fold) S0 is the folded state and the chain
+// starts at depth d0 + 1.  The record store is a ring over the last T_max
+// depths, so depth t's early writes replace the entries of depth t - T_max:
+// the steps that may still run then read only deltas from the store (keys,
+// gates and parents come from the callers' arrays under programmatic
+// launch), and deltas are written after the wait.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cudaTypedefs.h>
@@ -90,14 +97,16 @@ __host__ __device__ inline Layout layout(int nk, int planes, int TM, int W_max, 
   // 128 B of barriers and counters; 4 per-beam scalars; per (beam, depth)
   // the replay coefficients (float4), the chain, slot-list ints and gates
   // (the slot list 4 TM longer); a beam-index scratch [W_max]; the parents
-  // of steps 2..t-1; the per-step table (3 pointers and 3 ints per step).
+  // of the last steps before t; the per-step table (3 pointers and 3 ints per
+  // step).
   L.total = L.book + 128u + 4u * kBT * 4u + (uint32_t)kBT * TM * 16u + (3u * kBT + 4u) * TM * 4u +
             (uint32_t)((W_max + 3) & ~3) * 4u + (uint32_t)((hist_cap + 3) & ~3) * 2u + kTabBytes + 16u;
   return L;
 }
 
-// Copies n ints from global src to shared dst with cp.async, by the 32 lanes
-// of one warp: 16-byte pieces when both ends allow it, single ints otherwise.
+// Copies n parent indices (int32, global) to shared memory as 16-bit
+// indices, by the 32 lanes of one warp: 16-byte loads when the source allows
+// it, single ints otherwise.
 __device__ __forceinline__ void copy_parents16_warp(uint16_t *dst, const int32_t *src, int n, int lane) {
   // dst is 8-byte aligned; parents are below 2^16 (anything else is out of
   // range and is clamped where it is used).
@@ -175,7 +184,7 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
   int *s_list = s_chain + kBT * TM;  // slot -> (beam << 5 | depth-1), [(32 + 4) TM]
   float *s_w = reinterpret_cast<float *>(s_list + (kBT + 4) * TM);  // [32][TM] gates along the chains
   int *s_seen = reinterpret_cast<int *>(s_w + kBT * TM);           // beam index -> a lane (scratch)
-  uint16_t *s_hist = reinterpret_cast<uint16_t *>(s_seen + ((p.W_max + 3) & ~3));  // parents of steps 2..t-1
+  uint16_t *s_hist = reinterpret_cast<uint16_t *>(s_seen + ((p.W_max + 3) & ~3));  // parents of steps hcopy..t-1
   // Per-step table (index = step j), filled by the ancestry warp before the
   // first barrier with one load per lane: loops then read shared memory
   // instead of indexing the parameters at run time.
@@ -233,9 +242,9 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
       s_trs[lane] = p.hpar_rs[lane];
     }
   }
-  // The parents of steps 2..t-1 for this request as 16-bit indices, back
-  // to back, each array starting on an 8-byte boundary: beam warp w >= 1
-  // copies steps w + 1, w + 8, w + 15.
+  // The parents of steps hcopy..t-1 for this request as 16-bit indices,
+  // back to back, each array starting on an 8-byte boundary: beam warp w >= 1
+  // copies steps hcopy + w - 1, hcopy + w + 6, ...
   if (p.hist_cap > 0 && warp >= 1 && warp < kAncWarp)
 #pragma unroll 2
     for (int j = p.hcopy + warp - 1; j < t; j += kAncWarp - 1)
@@ -264,9 +273,9 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
 
   if (warp == kAncWarp) {
     // ------------------------------------------------ the ancestry warp
-    // Beam b's ancestors a[j] at depth j + 1 (a[t-2] = its parent; a[j] is
-    // the parent, at step j + 2, of a[j + 1]), the tile's distinct
-    // ancestors and the replay weights.
+    // Beam b's replayed ancestors a[j] at depth d0 + j + 1 (a[nanc-1] = its
+    // parent; a[j] is the parent, at step d0 + j + 2, of a[j + 1]), the
+    // tile's distinct ancestors and the replay weights.
     const int b = lane;
     if (b < nb && t >= 2 && (par < 0 || par >= p.W_prev)) {
       *reinterpret_cast<volatile int32_t *>(p.err) = kErrParent;
