@@ -340,3 +340,40 @@ def test_unfolded_window_overflow_is_reported(kind):
         assert dec.status() == 0
     finally:
         dec.close()
+
+
+@pytest.mark.parametrize("kind", ["simt", "tc"])
+def test_fold_with_more_beams_than_threads(kind):
+    """600 beams: the tensor-core fold compares the ancestry rows of beams
+    past its 256 threads in a second loop.  Request 0 narrows to one beam at
+    step 2, request 1 does not."""
+    dk = dv = 128 if kind == "tc" else 32
+    wl, S0, steps = P.custom_steps(42, R=2, H=2, dk=dk, dv=dv, Ws=[300, 600, 600, 500], parents="uniform")
+    par = steps[1]["parents"].clone()
+    par[0] = 17
+    par[1] = torch.arange(600, dtype=torch.int32) % 300
+    steps[1]["parents"] = par
+    S0t = synth.cast_state(S0, "f32")
+    gpu, info, _ = run_with_folds(S0t, steps, "bf16", kernel_id(kind), {3: 3})
+    (_, D, S), = info
+    want = expected_depths(steps, {3: 3})[3]
+    assert D.tolist() == want.tolist() and D.tolist()[0] >= 1
+    check_state(S, gdn.fold_state(S0t, steps[:3], want))
+    P.compare(gpu, P.oracle(S0t, steps), steps, "f32")
+
+
+@pytest.mark.parametrize("kind", ["simt", "tc"])
+def test_single_beam_decode_through_a_small_store(kind):
+    """W = 1 for 20 steps through a 4-depth store, folded after every step
+    (each fold takes the step's own depth): the sequential GDN recurrence's
+    outputs, while the store wraps five times."""
+    T, TM = 20, 4
+    dk = dv = 128 if kind == "tc" else 32
+    wl, S0, steps = P.custom_steps(43, R=2, H=2, dk=dk, dv=dv, Ws=[1] * T, parents="uniform")
+    S0t = synth.cast_state(S0, "f32")
+    gpu, info, _ = run_with_folds(S0t, steps, "bf16", kernel_id(kind), {t: T for t in range(1, T)}, T_max=TM)
+    for t, D, _ in info:
+        assert D.tolist() == [t, t]
+    ref = P.oracle(S0t, steps)
+    for t, (g, r) in enumerate(zip(gpu, ref), start=1):
+        assert float(np.abs(g["o"].double().numpy() - r["o"]).max()) <= P.TOL["f32"], t
