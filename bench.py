@@ -390,6 +390,7 @@ def time_sweep(device, stream, flush, reps=10, warmup=3):
     # d = 64 (tensor-core kernel) and d = 256 (general kernel: the tensor-core
     # one takes d <= 128) at the headline beam set.
     cases += [synth.shape_sweep_workload(1, 16, d, 256, 7) for d in (64, 256)]
+    cases += [synth.workload("long5k_bf16")]  # the headline shapes with a bf16 S0
     hbm = measured_peaks()[0]
     points = []
     for wl in cases:
@@ -433,7 +434,7 @@ def time_sweep(device, stream, flush, reps=10, warmup=3):
         dec.close()
         alg, _, _ = byte_model(wl, steps)
         gbs = alg / (ms / 1e3) / 1e9
-        points.append({"R": wl.R, "H": wl.H, "d": wl.d_k, "W": wl.W, "T": wl.T, "kernel": kind,
+        points.append({"R": wl.R, "H": wl.H, "d": wl.d_k, "W": wl.W, "T": wl.T, "s0": wl.s0_dtype, "kernel": kind,
                        "ms_per_decode": round(ms, 5), "value": round(wl.units / (ms / 1e3), 1),
                        "achieved_gbs": round(gbs, 1), "frac": round(gbs / hbm, 4)})
     return {"unit": UNIT, "peak_gbs": hbm, "l2": "flushed before every decode", "points": points}
