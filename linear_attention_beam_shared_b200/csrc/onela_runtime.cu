@@ -121,7 +121,8 @@ const char *onela_error_string(int code) {
     case ONELA_OK: return "ok";
     case ONELA_ERR_ARG: return "invalid argument";
     case ONELA_ERR_STATE: return "no prompt state installed";
-    case ONELA_ERR_CAPACITY: return "step or beam count beyond the handle's capacity";
+    case ONELA_ERR_CAPACITY:
+      return "beam count beyond W_max, or unfolded depths beyond the T_max the record store keeps";
     case ONELA_ERR_PARENT: return "parent index outside [0, W_prev) seen on the device";
     case ONELA_ERR_CUDA: return "CUDA call failed";
     case ONELA_ERR_UNSUPPORTED: return "kernel does not support this shape";
