@@ -26,6 +26,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -470,8 +471,9 @@ class ClockSampler:
     def __init__(self, gpu_index):
         self.proc = None
         self.gpu = gpu_index
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv") if os.path.isdir(
-            os.path.join(ROOT, "gpurun_out")) else f"/tmp/onela_clocks_{os.getpid()}.csv"
+        # The raw samples go to ONELA_CLOCKS_CSV when set, else a temporary file.
+        self.path = os.environ.get("ONELA_CLOCKS_CSV") or os.path.join(
+            tempfile.gettempdir(), f"onela_clocks_{os.getpid()}_{gpu_index}.csv")
 
     def __enter__(self):
         q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"

@@ -183,7 +183,7 @@ __global__ void __launch_bounds__(kPThreads) prefill_kernel(const T *k, const T 
       for (int e = 0; e < EPT; ++e) kk[e] = kn[e];
       a = an, bt = bn, vi = vn;
     }
-    __syncthreads();  // this buffer is refilled by the next round's copies
+    __syncthreads();  // this buffer is refilled by the copies of the chunk after next
   }
   if (row < dv) {
     TS *out = S0 + ((int64_t)(r * H + h) * dv + row) * dk;
