@@ -81,11 +81,12 @@ enum {
  *                   (S0 products, ancestry, key products, gate weights), and
  *                   waits for step t-1 only before it stages the ancestors'
  *                   deltas.  For that it reads the k, gate and parent_idx
- *                   arrays of every earlier step of the decode again.  Set
+ *                   arrays of the earlier steps of the decode again (at
+ *                   most the last 16).  Set
  *                   it only when (a) the kernel before step t in the stream
  *                   produces no input of step t (q, k, v, g, beta,
  *                   parent_idx), and (b) the k, gate and parent_idx arrays of
- *                   every earlier step of the decode stay unchanged and
+ *                   the last 16 steps before t stay unchanged and
  *                   allocated until step t has completed -- e.g. back-to-back
  *                   decode steps whose inputs were all written before the
  *                   first of them, as in a CUDA graph of a whole decode, or
