@@ -69,8 +69,12 @@ enum {
                                 onela_status                                 */
   ONELA_ERR_CUDA = 5,        /* a CUDA call failed (allocation, launch ...)  */
   ONELA_ERR_UNSUPPORTED = 6, /* the requested kernel cannot run this shape   */
-  ONELA_ERR_SCRATCH = 7      /* onela_decode_step_noalloc: the decode does not
+  ONELA_ERR_SCRATCH = 7,     /* onela_decode_step_noalloc: the decode does not
                                 fit in its fixed 32 MiB device array         */
+  ONELA_ERR_TIMEOUT = 8      /* a bounded wait inside a kernel ran out (bit 1
+                                of the error word): the outputs of that call
+                                are void; reported by the next call or by
+                                onela_status                                 */
 };
 
 /* onela_config.flags bits.
@@ -197,7 +201,7 @@ ONELA_API int onela_read_prompt_state(onela_handle *h, void *S0, onela_stream st
  * t - 1 - D_r <= T_max - 1 for every request and otherwise reports
  * ONELA_ERR_CAPACITY the same way (the step's outputs are meaningless).
  * Errors: ONELA_ERR_ARG, ONELA_ERR_STATE, ONELA_ERR_CAPACITY,
- * ONELA_ERR_PARENT, ONELA_ERR_UNSUPPORTED, ONELA_ERR_CUDA. */
+ * ONELA_ERR_PARENT, ONELA_ERR_TIMEOUT, ONELA_ERR_UNSUPPORTED, ONELA_ERR_CUDA. */
 ONELA_API int onela_decode_step(onela_handle *h, int32_t W_prev, int32_t W,
                       const void *q, const void *k, const void *v,
                       const float *g, const float *beta,
@@ -262,7 +266,8 @@ ONELA_API int onela_reset(onela_handle *h, onela_stream stream);
  * ordinary launch even under ONELA_FLAG_PDL.  Memory: a second state buffer
  * (and operand image, tensor-core kernel), allocated by onela_create.
  * Errors: ONELA_ERR_ARG, ONELA_ERR_STATE (no prompt state), ONELA_ERR_PARENT
- * (a bad parent index was seen: the ancestry is meaningless), ONELA_ERR_CUDA. */
+ * (a bad parent index was seen: the ancestry is meaningless), ONELA_ERR_TIMEOUT,
+ * ONELA_ERR_CAPACITY, ONELA_ERR_CUDA. */
 ONELA_API int onela_fold(onela_handle *h, int32_t max_depth, onela_stream stream);
 
 /* Copy the root state the decode replays from (the prompt state, or the
@@ -278,9 +283,12 @@ ONELA_API int onela_read_fold_depth(onela_handle *h, int32_t *depth, onela_strea
 
 /* Wait for the handle's device (cudaDeviceSynchronize on it) and report the
  * error word in *device_err (0: none; bit 0: a bad parent index; bit 1: a
- * bounded wait ran out in the tensor-core kernel; bit 2: a step's unfolded
- * depths did not fit the store).  Returns ONELA_ERR_PARENT when bit 0 is
- * set, ONELA_ERR_CAPACITY when bit 2 is, ONELA_OK otherwise.
+ * bounded wait ran out in a tensor-core kernel, whose outputs are then void;
+ * bit 2: a step's unfolded depths did not fit the store; several bits may be
+ * set).  Returns ONELA_ERR_PARENT when bit 0 is set, else ONELA_ERR_TIMEOUT
+ * when bit 1 is, else ONELA_ERR_CAPACITY when bit 2 is, else ONELA_OK.  The
+ * decode calls and onela_fold return the same code, without waiting, for
+ * what earlier calls left in the word.
  * Errors: ONELA_ERR_ARG, ONELA_ERR_CUDA. */
 ONELA_API int onela_status(onela_handle *h, int32_t *device_err);
 
@@ -328,6 +336,10 @@ ONELA_API int onela_kernel_kind(const onela_handle *h);
  *              A call with t = 1 starts a new decode and clears the error
  *              word.
  *   W_prev, W  beams of the previous step (1 at t = 1) and of this one.
+ *              W_prev must be the previous call's W: the array keeps no
+ *              host-side record of it, so this is not verified, and a larger
+ *              W_prev would let parent indices reach rows an earlier decode
+ *              left in the array (silently wrong outputs).
  *   S0         [R][H][d_v][d_k] in s0_dtype, read directly at every step.
  *   q, k, v, g, beta, parent_idx, o   as for onela_decode_step.
  *   status     DEVICE pointer to one int32, written on `stream` with the

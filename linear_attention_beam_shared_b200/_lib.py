@@ -20,6 +20,7 @@ LIB_PATH = os.path.join(_PKG, "libonela_b200.so")
 ONELA_F32, ONELA_BF16 = 0, 1
 ONELA_OK, ONELA_ERR_ARG, ONELA_ERR_STATE, ONELA_ERR_CAPACITY = 0, 1, 2, 3
 ONELA_ERR_PARENT, ONELA_ERR_CUDA, ONELA_ERR_UNSUPPORTED, ONELA_ERR_SCRATCH = 4, 5, 6, 7
+ONELA_ERR_TIMEOUT = 8
 ONELA_KERNEL_AUTO, ONELA_KERNEL_SIMT, ONELA_KERNEL_TC = 0, 1, 2
 ONELA_FLAG_PDL = 1
 

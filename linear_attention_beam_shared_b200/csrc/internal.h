@@ -84,10 +84,29 @@ __host__ __device__ __forceinline__ int64_t anc_row(const StepParams &p, int s, 
   return ((int64_t)(rec_slot(p, s) * p.R + r) * p.W_max + b) * p.T_max;
 }
 
-// Device error word bits.
-constexpr int32_t kErrParent = 1;
-// (bit 1: a bounded wait ran out, tensor-core kernel)
-constexpr int32_t kErrWindow = 4;  // a step's unfolded depths did not fit the record store
+// Device error word.  Each condition owns one byte of the word, which a
+// kernel sets to 1 with a plain byte store, so that two conditions seen in one
+// launch never overwrite each other (the word may be host-mapped memory, where
+// a read-modify-write from the device is not atomic).  The host turns the raw
+// word into the documented bits with err_bits.
+constexpr int kErrByteParent = 0;   // a parent index outside [0, W_prev)
+constexpr int kErrByteTimeout = 1;  // a bounded wait ran out: that launch's outputs are void
+constexpr int kErrByteWindow = 2;   // a step's unfolded depths did not fit the record store
+constexpr int32_t kErrParent = 1, kErrTimeout = 2, kErrWindow = 4;  // documented bits
+__device__ __forceinline__ void set_err(int32_t *err, int byte) {
+  reinterpret_cast<volatile uint8_t *>(err)[byte] = 1;
+}
+inline int32_t err_bits(int32_t raw) {
+  const uint32_t u = (uint32_t)raw;
+  return ((u & 0xffu) ? kErrParent : 0) | (((u >> 8) & 0xffu) ? kErrTimeout : 0) |
+         (((u >> 16) & 0xffu) ? kErrWindow : 0);
+}
+
+// Raises the dynamic shared-memory limit of kernel `func` on the current
+// device to at least `smem` bytes.  The attribute is set once per (kernel,
+// device, larger size): it is not a stream operation, so it must not be
+// repeated inside a captured region.  Safe to call from several host threads.
+cudaError_t ensure_smem_limit(const void *func, size_t smem);
 
 // Kernel launchers (step_simt.cu, step_tc.cu).  Return a cudaError_t.
 cudaError_t launch_step_simt(const StepParams &p, int qkv_bf16, int s0_bf16, cudaStream_t s);

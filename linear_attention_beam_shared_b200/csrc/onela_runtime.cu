@@ -4,7 +4,10 @@
 
 #include <cstdlib>
 #include <cstring>
+#include <map>
+#include <mutex>
 #include <new>
+#include <utility>
 #include <vector>
 
 #include "../../include/onela.h"
@@ -89,6 +92,15 @@ void free_all(onela_handle *h) {
   if (h->err_host) cudaFreeHost(h->err_host);
 }
 
+// The return code for what the device error word holds (ONELA_OK if nothing).
+int word_code(const onela_handle *h) {
+  const int32_t bits = onela::err_bits(*reinterpret_cast<volatile int32_t *>(h->err_host));
+  if (bits & onela::kErrParent) return ONELA_ERR_PARENT;
+  if (bits & onela::kErrTimeout) return ONELA_ERR_TIMEOUT;
+  if (bits & onela::kErrWindow) return ONELA_ERR_CAPACITY;
+  return ONELA_OK;
+}
+
 onela::StepParams base_params(const onela_handle *h) {
   onela::StepParams p;
   std::memset(&p, 0, sizeof(p));
@@ -114,6 +126,24 @@ onela::StepParams base_params(const onela_handle *h) {
 
 }  // namespace
 
+namespace onela {
+
+cudaError_t ensure_smem_limit(const void *func, size_t smem) {
+  static std::mutex mu;
+  static std::map<std::pair<const void *, int>, size_t> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  size_t &have = done[{func, dev}];
+  if (smem <= have) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e == cudaSuccess) have = smem;
+  return e;
+}
+
+}  // namespace onela
+
 extern "C" {
 
 const char *onela_error_string(int code) {
@@ -127,6 +157,7 @@ const char *onela_error_string(int code) {
     case ONELA_ERR_CUDA: return "CUDA call failed";
     case ONELA_ERR_UNSUPPORTED: return "kernel does not support this shape";
     case ONELA_ERR_SCRATCH: return "decode does not fit in the 32 MiB array of onela_decode_step_noalloc";
+    case ONELA_ERR_TIMEOUT: return "a bounded wait inside a kernel ran out; the outputs since the last check are void";
     default: return "unknown error";
   }
 }
@@ -274,9 +305,8 @@ int onela_decode_step(onela_handle *h, int32_t W_prev, int32_t W, const void *q,
                       const float *gate, const float *beta, const int32_t *parent_idx, float *o,
                       onela_stream stream) {
   if (!h || !q || !k || !v || !gate || !beta || !parent_idx || !o) return ONELA_ERR_ARG;
-  const int32_t word = *reinterpret_cast<volatile int32_t *>(h->err_host);
-  if (word & onela::kErrParent) return ONELA_ERR_PARENT;
-  if (word & onela::kErrWindow) return ONELA_ERR_CAPACITY;
+  const int rc = word_code(h);
+  if (rc != ONELA_OK) return rc;
   if (!h->has_prompt) return ONELA_ERR_STATE;
   const onela_config &c = h->cfg;
   if (W < 1) return ONELA_ERR_ARG;
@@ -376,9 +406,8 @@ int onela_reset(onela_handle *h, onela_stream stream) {
 
 int onela_fold(onela_handle *h, int32_t max_depth, onela_stream stream) {
   if (!h || max_depth < 0) return ONELA_ERR_ARG;
-  const int32_t word = *reinterpret_cast<volatile int32_t *>(h->err_host);
-  if (word & onela::kErrParent) return ONELA_ERR_PARENT;
-  if (word & onela::kErrWindow) return ONELA_ERR_CAPACITY;
+  const int rc = word_code(h);
+  if (rc != ONELA_OK) return rc;
   if (!h->has_prompt) return ONELA_ERR_STATE;
   if (h->steps_done == 0 || max_depth == 0) return ONELA_OK;  // nothing to fold
   DeviceGuard g(h->cfg.device);
@@ -442,10 +471,8 @@ int onela_status(onela_handle *h, int32_t *device_err) {
   DeviceGuard g(h->cfg.device);
   if (!g.ok) return ONELA_ERR_CUDA;
   if (cudaDeviceSynchronize() != cudaSuccess) return ONELA_ERR_CUDA;
-  const int32_t e = *reinterpret_cast<volatile int32_t *>(h->err_host);
-  if (device_err) *device_err = e;
-  if (e & onela::kErrParent) return ONELA_ERR_PARENT;
-  return (e & onela::kErrWindow) ? ONELA_ERR_CAPACITY : ONELA_OK;
+  if (device_err) *device_err = onela::err_bits(*reinterpret_cast<volatile int32_t *>(h->err_host));
+  return word_code(h);
 }
 
 int onela_destroy(onela_handle *h) {

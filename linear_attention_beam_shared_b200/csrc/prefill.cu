@@ -206,16 +206,8 @@ cudaError_t launch_prefill_t(const void *k, const void *v, const float *g, const
   constexpr int DKP = EPT * kTPR;
   const size_t smem = 2 * sizeof(ChunkBuf<T, DKP>);
   auto kern = prefill_kernel<T, TS, EPT>;
-  static size_t configured[64] = {0};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  cudaError_t e = smem > 48 * 1024 ? ensure_smem_limit((const void *)kern, smem) : cudaSuccess;
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (smem > 48 * 1024 && smem > configured[dev]) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    configured[dev] = smem;
-  }
   dim3 grid((dv + kRB - 1) / kRB, H, R);
   kern<<<grid, kPThreads, smem, s>>>(static_cast<const T *>(k), static_cast<const T *>(v), g, beta,
                                      static_cast<TS *>(S0), R, L, H, dk, dv);

@@ -54,7 +54,7 @@ __global__ void __launch_bounds__(kNT) step_simt_kernel(const StepParams p) {
   // which must fit the record store's T_max slots.
   int d0 = p.d0 ? p.d0[r] : 0;
   if (t - 1 - d0 > TM - 1) {
-    if (tid == 0) *reinterpret_cast<volatile int32_t *>(p.err) = kErrWindow;
+    if (tid == 0) set_err(p.err, kErrByteWindow);
     d0 = t - TM;  // keeps every access inside the store; the results are void
   }
   const int nanc = t - 1 - d0;  // replayed ancestors: chain index j is depth d0 + j + 1
@@ -100,7 +100,7 @@ __global__ void __launch_bounds__(kNT) step_simt_kernel(const StepParams p) {
       const int gb = b0 + b;
       int par = p.parents[r * p.W + gb];
       if (par < 0 || par >= p.W_prev) {
-        *reinterpret_cast<volatile int32_t *>(p.err) = kErrParent;
+        set_err(p.err, kErrByteParent);
         par = 0;
       }
       int *chain = s_chain + b * TM;
@@ -294,16 +294,8 @@ cudaError_t launch_typed(const StepParams &p, cudaStream_t s) {
   auto kern = step_simt_kernel<QT, ST>;
   // Raise the dynamic shared-memory limit once per device (not a stream
   // operation, so it must not be repeated inside a captured region).
-  static size_t configured[64] = {0};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  cudaError_t e = ensure_smem_limit((const void *)kern, smem);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (smem > configured[dev]) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    configured[dev] = smem;
-  }
   dim3 grid((p.W + kBT - 1) / kBT, p.H, p.R);
   kern<<<grid, kNT, smem, s>>>(p);
   return cudaGetLastError();

@@ -73,7 +73,6 @@ constexpr uint32_t kTabBytes = 3u * 8u * kHistSteps + 3u * 4u * kHistSteps;  // 
 constexpr int kMaxT = 16;           // deepest decode the kernel serves
 constexpr int kMaxW = 1024;         // widest beam set the kernel serves
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far beyond any legal wait
-constexpr int32_t kErrTimeout = 2;
 
 struct Layout {
   uint32_t x;     // X [NK][64 rows][128 B]: k rows, then q rows
@@ -151,7 +150,7 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
   // which must fit the record store's T_max slots.
   int d0 = p.d0 ? p.d0[r] : 0;
   if (t - 1 - d0 > TM - 1) {
-    if (tid == 0) *reinterpret_cast<volatile int32_t *>(p.err) = kErrWindow;
+    if (tid == 0) set_err(p.err, kErrByteWindow);
     d0 = t - TM;  // keeps every access inside the store; the results are void
   }
   const int nanc = t - 1 - d0;  // ancestors per beam; chain index j is depth d0+j+1
@@ -278,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
     // tile's distinct ancestors and the replay weights.
     const int b = lane;
     if (b < nb && t >= 2 && (par < 0 || par >= p.W_prev)) {
-      *reinterpret_cast<volatile int32_t *>(p.err) = kErrParent;
+      set_err(p.err, kErrByteParent);
       par = 0;
     }
     const float alpha_b = b < nb ? expf(g_alpha) : 0.f;
@@ -573,7 +572,7 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
   }
 
   // --------------------------------------------------------- epilogue
-  if (!ok) *reinterpret_cast<volatile int32_t *>(p.err) = kErrTimeout;
+  if (!ok) set_err(p.err, kErrByteTimeout);
   if (bval && ok) {
     float4 *op = reinterpret_cast<float4 *>(p.o + (row0 + (int64_t)bb * H) * DV) + l;
     float4 *dp = reinterpret_cast<float4 *>(p.rec_delta + rec_row_slot(p, tslot, r, h, b0 + bb) * DV) + l;
@@ -666,16 +665,8 @@ cudaError_t launch_dk(const StepParams &p_in, bool pdl, cudaStream_t s) {
     return cudaErrorInvalidValue;
   const Layout L = layout(DK / 64, p.s0_planes, p.T_max, p.W_max, p.hist_cap);
   const size_t smem = L.total + 1024;
-  static size_t configured[64] = {0};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  cudaError_t e = ensure_smem_limit((const void *)step_tc_kernel<DK>, smem);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (smem > configured[dev]) {
-    e = cudaFuncSetAttribute(step_tc_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    configured[dev] = smem;
-  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((p.W + kBT - 1) / kBT, p.H, p.R);
   cfg.blockDim = dim3(kThreads, 1, 1);

@@ -43,8 +43,8 @@ def test_library_exports_every_declared_symbol():
 
 def test_error_strings():
     import linear_attention_beam_shared_b200 as L
-    for code in range(0, 7):
-        assert L.error_string(code)
+    for code in range(0, 9):
+        assert L.error_string(code) != "unknown error"
     assert L.error_string(99) == "unknown error"
 
 
