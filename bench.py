@@ -81,6 +81,9 @@ def measured_peaks():
     return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+KERNEL_SOURCES = {"tc": "step_tc.cu", "simt": "step_simt.cu"}
+
+
 def kernel_source_hash(kind="tc"):
     """Hash of the decode kernel's source file (step_tc.cu or step_simt.cu)
     with comments and blank lines removed, so that a change of wording, or a
@@ -88,7 +91,7 @@ def kernel_source_hash(kind="tc"):
     valid."""
     import re
     h = hashlib.sha256()
-    for p in [os.path.join(ROOT, "linear_attention_beam_shared_b200", "csrc", f"step_{kind}.cu")]:
+    for p in [os.path.join(ROOT, "linear_attention_beam_shared_b200", "csrc", KERNEL_SOURCES[kind])]:
         with open(p, "r", encoding="utf-8", errors="replace") as f:
             text = f.read()
         text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
@@ -381,15 +384,13 @@ def time_sweep(device, stream, flush, reps=10, warmup=3):
     """The beam-width sweep (W = 64 .. 1024, T = 5, 1K-prompt shapes), the
     request sweep (R = 1, 8, 32 at H = 16, d = 128, W = 256, T = 7) and the
     head sizes d = 64 and 256 at R = 1, H = 16, W = 256, T = 7: one whole
-    decode per CUDA graph with programmatic launch between its steps, L2
-    flushed before each, CUDA events; algorithmic bytes from the byte model.
-    S0 is drawn directly (its values do not change the work).  Returns the
-    JSON object for the bench line."""
+    decode (one onela_decode_steps call) per CUDA graph, L2 flushed before
+    each, CUDA events; algorithmic bytes from the byte model.  S0 is drawn
+    directly (its values do not change the work).  Returns the JSON object
+    for the bench line."""
     import linear_attention_beam_shared_b200 as L
     cases = [synth.workload(f"wsweep{w}") for w in (64, 128, 256, 512, 1024)]
     cases += [synth.shape_sweep_workload(R, 16, 128, 256, 7) for R in (1, 8, 32)]
-    # d = 64 (tensor-core kernel) and d = 256 (general kernel: the tensor-core
-    # one takes d <= 128) at the headline beam set.
     cases += [synth.shape_sweep_workload(1, 16, d, 256, 7) for d in (64, 256)]
     cases += [synth.workload("long5k_bf16")]  # the headline shapes with a bf16 S0
     hbm = measured_peaks()[0]
@@ -401,44 +402,63 @@ def time_sweep(device, stream, flush, reps=10, warmup=3):
         ds = [{k: (v.to(device) if isinstance(v, torch.Tensor) else v) for k, v in st.items()} for st in steps]
         outs = [torch.empty((wl.R, st["W"], wl.H, wl.d_v), dtype=torch.float32, device=device) for st in steps]
         dec = L.BeamDecoder(wl.R, wl.H, wl.d_k, wl.d_v, wl.W, wl.T, wl.s0_dtype, wl.qkv_dtype,
-                            device=device.index, flags=L.ONELA_FLAG_PDL)
-        kind = {L.ONELA_KERNEL_SIMT: "simt", L.ONELA_KERNEL_TC: "tc"}[dec.kernel]
+                            device=device.index)
         dec.set_prompt_state(S0.to(device))
-
-        def run():
-            for st, o in zip(ds, outs):
-                dec.step(st["q"], st["k"], st["v"], st["g"], st["beta"], st["parents"], o=o, stream=stream)
-        with torch.cuda.stream(stream):
-            run()
-        stream.synchronize()
-        assert dec.status() == 0
-        dec.reset(stream)
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            run()
-        dec.reset(stream)
-        for _ in range(warmup):
-            with torch.cuda.stream(stream):
-                flush.fill_(9)
-                g.replay()
-        stream.synchronize()
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
-        with torch.cuda.stream(stream):
-            for i, (e0, e1) in enumerate(ev):
-                flush.fill_(i & 0xFF)
-                e0.record(stream)
-                g.replay()
-                e1.record(stream)
-        stream.synchronize()
-        ms = max_over_ranks(sum(e0.elapsed_time(e1) for e0, e1 in ev) / reps, device)
+        g, launches = decode_graph(dec, ds, outs, stream)
+        kind = {L.ONELA_KERNEL_SIMT: "simt", L.ONELA_KERNEL_TC: "tc"}[dec.kernel]
+        ms = time_graph(g, stream, flush, reps, warmup)
         del g
+        assert dec.status() == 0
         dec.close()
         alg, _, _ = byte_model(wl, steps)
         gbs = alg / (ms / 1e3) / 1e9
         points.append({"R": wl.R, "H": wl.H, "d": wl.d_k, "W": wl.W, "T": wl.T, "s0": wl.s0_dtype, "kernel": kind,
-                       "ms_per_decode": round(ms, 5), "value": round(wl.units / (ms / 1e3), 1),
+                       "launches": launches, "ms_per_decode": round(ms, 5), "value": round(wl.units / (ms / 1e3), 1),
                        "achieved_gbs": round(gbs, 1), "frac": round(gbs / hbm, 4)})
+        del ds, outs
     return {"unit": UNIT, "peak_gbs": hbm, "l2": "flushed before every decode", "points": points}
+
+
+def decode_graph(dec, dsteps, outs, stream, per_step=False):
+    """One whole decode through the public API captured in a CUDA graph: one
+    onela_decode_steps call, or (per_step) one onela_decode_step call per
+    step.  Returns (graph, kernel launches per decode)."""
+    def run():
+        if per_step:
+            for st, o in zip(dsteps, outs):
+                dec.step(st["q"], st["k"], st["v"], st["g"], st["beta"], st["parents"], o=o, stream=stream)
+        else:
+            dec.steps(dsteps, outs, stream=stream)
+    with torch.cuda.stream(stream):
+        run()
+    stream.synchronize()
+    assert dec.status() == 0
+    launches = len(dsteps) if per_step else dec.last_launches()
+    dec.reset(stream)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        run()
+    dec.reset(stream)
+    return graph, launches
+
+
+def time_graph(graph, stream, flush, reps, warmup):
+    """Mean device time (ms, max over ranks) of graph replays, each after a
+    512 MiB write that flushes L2, timed with CUDA events on the stream."""
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            flush.fill_(9)
+            graph.replay()
+    stream.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    with torch.cuda.stream(stream):
+        for i, (e0, e1) in enumerate(ev):
+            flush.fill_(i & 0xFF)
+            e0.record(stream)
+            graph.replay()
+            e1.record(stream)
+    stream.synchronize()
+    return max_over_ranks(sum(e0.elapsed_time(e1) for e0, e1 in ev) / reps, stream.device)
 
 
 def byte_model(wl, steps):
@@ -558,29 +578,19 @@ def run_ours(args):
             (wl.R, wl.H, wl.d_v, wl.d_k)), wl.s0_dtype)
     steps = synth.draw_decode(wl)
     kernel = {"auto": L.ONELA_KERNEL_AUTO, "simt": L.ONELA_KERNEL_SIMT, "tc": L.ONELA_KERNEL_TC}[args.kernel]
-    # Inputs are resident before the graph runs and the steps follow one
-    # another directly, so steps 2..T may start while the previous one ends.
-    flags = 0 if args.no_pdl else L.ONELA_FLAG_PDL
+    # One whole decode = one onela_decode_steps call with every step's inputs
+    # resident (each step after the first overlaps the one before it; no
+    # handle flag and no contract across calls).
     dec = L.BeamDecoder(wl.R, wl.H, wl.d_k, wl.d_v, wl.W, wl.T, wl.s0_dtype, wl.qkv_dtype,
-                        kernel=kernel, device=device.index, flags=flags)
-    kind = {L.ONELA_KERNEL_SIMT: "simt", L.ONELA_KERNEL_TC: "tc"}[dec.kernel]
+                        kernel=kernel, device=device.index)
     dec.set_prompt_state(S0.to(device))
     dsteps = [{k: (v.to(device) if isinstance(v, torch.Tensor) else v) for k, v in s.items()} for s in steps]
     outs = [torch.empty((wl.R, s["W"], wl.H, wl.d_v), dtype=torch.float32, device=device) for s in steps]
 
     stream = torch.cuda.Stream(device=device)
     # Eager warm-up of the API (also loads the module), then capture.
-    with torch.cuda.stream(stream):
-        for s, o in zip(dsteps, outs):
-            dec.step(s["q"], s["k"], s["v"], s["g"], s["beta"], s["parents"], o=o, stream=stream)
-    stream.synchronize()
-    assert dec.status() == 0
-    dec.reset(stream)
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
-        for s, o in zip(dsteps, outs):
-            dec.step(s["q"], s["k"], s["v"], s["g"], s["beta"], s["parents"], o=o, stream=stream)
-    dec.reset(stream)
+    graph, launches = decode_graph(dec, dsteps, outs, stream)
+    kind = {L.ONELA_KERNEL_SIMT: "simt", L.ONELA_KERNEL_TC: "tc"}[dec.kernel]
 
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=device)
     for _ in range(args.warmup):
@@ -609,25 +619,45 @@ def run_ours(args):
     assert dec.status() == 0
     ms_per_step = total_ms / args.steps
     value = whole_job_value(wl.units, ws, ms_per_step)
+    del graph
+    dec.close()
 
     # Roofline of the decode kernel (the only kernel in the step).
     alg_bytes, upper_bytes, _ = byte_model(wl, steps)
-    launches = wl.T
     hbm, bf16_tf, bf16_sus, src = measured_peaks()
-    achieved = alg_bytes / (ms_per_step / 1e3) / 1e9
+    achieved = alg_bytes / launches / (ms_per_step / launches / 1e3) / 1e9
     traffic = ncu_traffic(kind)
     roofline = {
         "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
         "frac": round(achieved / hbm, 4),
         "traffic": traffic["bytes_per_launch"] if traffic else None,
         "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else "fallback",
-        "kernel": f"onela step kernel ({kind})",
+        "kernel": {"tc": "tensor-core step kernel", "simt": "SIMT step kernel"}[kind],
+        "launches_per_decode": launches,
         "alg_bytes_per_launch": round(alg_bytes / launches),
         "upper_bound_bytes_per_launch": round(upper_bytes / launches),
         "avg_launch_us": round(ms_per_step * 1e3 / launches, 3),
     }
     flops = 4 * wl.d_k * wl.d_v * wl.W * wl.H * wl.R * wl.T
     roofline["tensor_frac_of_sustained_bf16"] = round(flops / (ms_per_step / 1e3) / 1e12 / bf16_sus, 5) if bf16_sus else None
+
+    # The same decode as one onela_decode_step call per step: under
+    # ONELA_FLAG_PDL (steps overlap by its contract across calls), and with
+    # ordinary launches (each step waits for the one before it).
+    variants = None
+    if not args.no_variants and kind == "tc":
+        variants = {}
+        for name, fl in (("per_step_calls_pdl_flag", L.ONELA_FLAG_PDL), ("per_step_calls", 0)):
+            d2 = L.BeamDecoder(wl.R, wl.H, wl.d_k, wl.d_v, wl.W, wl.T, wl.s0_dtype, wl.qkv_dtype,
+                               kernel=kernel, device=device.index, flags=fl)
+            d2.set_prompt_state(S0.to(device))
+            g2, n2 = decode_graph(d2, dsteps, outs, stream, per_step=True)
+            ms2 = time_graph(g2, stream, flush, reps=20, warmup=3)
+            del g2
+            assert d2.status() == 0
+            d2.close()
+            variants[name] = {"ms_per_decode": round(ms2, 5), "launches": n2,
+                              "frac": round(alg_bytes / (ms2 / 1e3) / 1e9 / hbm, 4)}
 
     # End to end through the public API with host buffers: per step the H2D
     # copy of that step's inputs from pinned memory, the decode call, and the
@@ -637,8 +667,6 @@ def run_ours(args):
     # downloads of different steps overlap (the two copy directions run on
     # separate engines).  A handle without the programmatic-launch flag: a
     # copy, not the previous step, is what each step waits for.
-    del graph
-    dec.close()
     dec = L.BeamDecoder(wl.R, wl.H, wl.d_k, wl.d_v, wl.W, wl.T, wl.s0_dtype, wl.qkv_dtype,
                         kernel=kernel, device=device.index)
     dec.set_prompt_state(S0.to(device))
@@ -728,10 +756,11 @@ def run_ours(args):
                                    f"q/k/v {wl.qkv_dtype}, parents Zipf(1.1)",
                        "global_batch": wl.R * ws, "seq_len": wl.T, "parallelism": f"replicas{ws}",
                        "l2": "flushed (512 MiB write) before every timed step", "kernel": kind,
-                       "step": f"one whole {wl.T}-step decode in a CUDA graph",
-                       "programmatic_launch": not args.no_pdl},
+                       "step": f"one whole {wl.T}-step decode (one onela_decode_steps call) in a CUDA graph",
+                       "launches_per_decode": launches},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "clocks": clk.summary(), "gpu_launches": launches * args.steps,
+            "variants": variants,
             "prefill": prefill, "beam_select": select, "fold": fold, "sweep": sweep,
         }
         print(json.dumps(line))
@@ -783,8 +812,8 @@ def main():
     ap.add_argument("--workload", default="long5k")
     ap.add_argument("--kernel", choices=["auto", "simt", "tc"], default="auto")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline leg")
-    ap.add_argument("--no-pdl", action="store_true",
-                    help="launch every step only after the previous one has finished")
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip timing the one-launch-per-step variants of the headline decode")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill, beam-selection and fold timings")
     ap.add_argument("--no-sweep", action="store_true", help="skip the beam-width and request sweeps")

@@ -98,6 +98,7 @@ enum {
  *                   never overlaps. */
 enum { ONELA_FLAG_PDL = 1 };
 
+
 /* Which decode kernel runs.  AUTO picks the tensor-core kernel when the
  * shape allows it (bf16 q/k/v, d_k = d_v in {64, 128}, T_max <= 16,
  * W_max <= 1024) and the SIMT kernel otherwise. */
@@ -208,6 +209,48 @@ ONELA_API int onela_decode_step(onela_handle *h, int32_t W_prev, int32_t W,
                       const int32_t *parent_idx, float *o,
                       onela_stream stream);
 
+/* Several consecutive decode steps in one call, with every step's inputs
+ * given at once: steps t = T + 1 .. T + n, T = steps done before the call.
+ * Computes exactly what n calls of onela_decode_step compute (the same
+ * kernel, launch by launch), with step i's W_prev the previous step's W (1 at
+ * t = 1).
+ *   n           1 <= n; the step count.
+ *   W           HOST array of n beam counts, 1 <= W[i] <= W_max.
+ *   q, k, v, g, beta, parent_idx, o
+ *               HOST arrays of n DEVICE pointers: step i's tensors, laid out
+ *               as for onela_decode_step with W = W[i].  They are borrowed for
+ *               the stream-ordered duration of the call: none may change or
+ *               be freed before the call's last step has completed.
+ * Because all of a call's inputs exist before its first step runs, the
+ * tensor-core kernel launches each step after the first as a programmatic
+ * dependent of the step before it (the work that needs no earlier delta runs
+ * while the previous step finishes, as with ONELA_FLAG_PDL, but without its
+ * contract across calls): only a step whose early record writes would replace
+ * a depth stored before the call (possible past T_max steps, with folds) is an
+ * ordinary launch.  The first step of a call is always an ordinary launch.
+ * Capacity: T + n <= T_max unless the handle has folded since the last
+ * rewind.  q, k, v and o must start on 16-byte boundaries on a tensor-core
+ * handle.  Every check that can be made on the host is made before the first
+ * launch, so a host-side error leaves no work enqueued.
+ * Errors: ONELA_ERR_ARG, ONELA_ERR_STATE, ONELA_ERR_CAPACITY,
+ * ONELA_ERR_PARENT, ONELA_ERR_TIMEOUT, ONELA_ERR_UNSUPPORTED, ONELA_ERR_CUDA. */
+ONELA_API int onela_decode_steps(onela_handle *h, int32_t n, const int32_t *W,
+                                 const void *const *q, const void *const *k, const void *const *v,
+                                 const float *const *g, const float *const *beta,
+                                 const int32_t *const *parent_idx, float *const *o,
+                                 onela_stream stream);
+
+/* Bound of every wait inside the tensor-core step kernel on another of its
+ * warp roles (the S0 products, the ancestor chains): limit_ns in [1e3, 1e10]
+ * nanoseconds, default 2e9.  A wait that runs out sets bit 1 of the error
+ * word (ONELA_ERR_TIMEOUT); the kernel then finishes without the missing
+ * data (its outputs are void) instead of waiting longer.  stall != 0 is a
+ * testing aid: in later tensor-core steps the wait for the ancestor chains
+ * then expects one arrival that never comes, so that it runs out at the bound
+ * (nothing faults or hangs); stall = 0 restores normal operation.
+ * Errors: ONELA_ERR_ARG. */
+ONELA_API int onela_set_wait_policy(onela_handle *h, uint64_t limit_ns, int32_t stall);
+
 /* Beam selection on the device: the next beam set out of the children of
  * the current one (the evolving beam tree of the abstract), so that the
  * parent indices of the next decode step never leave the GPU.  For request r
@@ -316,6 +359,9 @@ ONELA_API int onela_read_ancestry(onela_handle *h, int32_t t, int32_t *anc,
  * the handle runs (ONELA_KERNEL_SIMT or ONELA_KERNEL_TC). */
 ONELA_API int onela_steps_done(const onela_handle *h);
 ONELA_API int onela_kernel_kind(const onela_handle *h);
+/* Query: kernel launches the last successful decode call enqueued
+ * (onela_decode_step: 1; onela_decode_steps: n; 0 before any call). */
+ONELA_API int onela_last_call_launches(const onela_handle *h);
 
 /* Decode step without any device allocation.
  *

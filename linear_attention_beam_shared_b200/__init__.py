@@ -21,7 +21,7 @@ from ._lib import (  # noqa: F401
     ONELA_BF16, ONELA_ERR_ARG, ONELA_ERR_CAPACITY, ONELA_ERR_CUDA, ONELA_ERR_PARENT,
     ONELA_ERR_STATE, ONELA_ERR_UNSUPPORTED, ONELA_F32, ONELA_FLAG_PDL, ONELA_KERNEL_AUTO, ONELA_KERNEL_SIMT,
     ONELA_ERR_SCRATCH, ONELA_ERR_TIMEOUT, ONELA_KERNEL_TC, ONELA_OK, Handle, OnelaError, error_string, onela_create,
-    onela_decode_step, onela_decode_step_noalloc, onela_destroy, onela_fold, onela_kernel_kind, onela_prefill,
+    onela_decode_step, onela_decode_step_noalloc, onela_decode_steps, onela_set_wait_policy, onela_destroy, onela_fold, onela_kernel_kind, onela_last_call_launches, onela_prefill,
     onela_read_ancestry, onela_read_fold_depth, onela_read_prompt_state, onela_read_records,
     onela_read_root_state, onela_reset, onela_select_beams, onela_set_prompt_state,
     onela_status, onela_status_code, onela_steps_done,
@@ -66,6 +66,24 @@ class BeamDecoder:
         self.W_prev = W
         self.Ws.append(W)
         return o
+
+    def steps(self, steps, outs=None, stream=None):
+        """Several consecutive steps in one call (see onela_decode_steps):
+        steps is a list of dicts with q, k, v, g, beta, parents."""
+        c = self.h.cfg
+        if outs is None:
+            outs = [torch.empty((c.R, int(s["parents"].shape[-1]), c.H, c.d_v), dtype=torch.float32,
+                                device=self.device) for s in steps]
+        onela_decode_steps(self.h, steps, outs, stream)
+        for s in steps:
+            W = int(s["parents"].shape[-1])
+            self.W_prev = W
+            self.Ws.append(W)
+        return outs
+
+    def last_launches(self) -> int:
+        """Kernel launches of the last decode call."""
+        return onela_last_call_launches(self.h)
 
     def reset(self, stream=None):
         onela_reset(self.h, stream)

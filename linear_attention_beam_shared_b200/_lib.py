@@ -56,6 +56,8 @@ def _load() -> ctypes.CDLL:
         "onela_select_beams": ([i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, i32, vp],
                                ctypes.c_int),
         "onela_decode_step": ([vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
+        "onela_decode_steps": ([vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
+        "onela_set_wait_policy": ([vp, ctypes.c_uint64, i32], ctypes.c_int),
         "onela_reset": ([vp, vp], ctypes.c_int),
         "onela_fold": ([vp, i32, vp], ctypes.c_int),
         "onela_read_root_state": ([vp, vp, vp], ctypes.c_int),
@@ -66,6 +68,7 @@ def _load() -> ctypes.CDLL:
         "onela_read_ancestry": ([vp, i32, vp, vp], ctypes.c_int),
         "onela_steps_done": ([vp], ctypes.c_int),
         "onela_kernel_kind": ([vp], ctypes.c_int),
+        "onela_last_call_launches": ([vp], ctypes.c_int),
         "onela_error_string": ([ctypes.c_int], ctypes.c_char_p),
         "onela_decode_step_noalloc": ([ctypes.POINTER(onela_config), i32, i32, i32, vp, vp, vp, vp, vp,
                                        vp, vp, vp, vp, vp], ctypes.c_int),
@@ -211,6 +214,34 @@ def onela_decode_step(h: Handle, W_prev: int, W: int, q, k, v, g, beta, parent_i
            "onela_decode_step")
 
 
+def onela_decode_steps(h: Handle, steps, outs, stream=None) -> None:
+    """Several consecutive steps in one call.  steps: list of dicts with the
+    step tensors q, k, v, g, beta, parents (the layouts of onela_decode_step);
+    outs: list of o tensors (each step's W is its parents' length)."""
+    c = h.cfg
+    dt = _DT[c.qkv_dtype]
+    n = len(steps)
+    if n < 1 or len(outs) != n:
+        raise ValueError("steps and outs must be non-empty lists of the same length")
+    Ws = [int(s["parents"].shape[-1]) for s in steps]
+    arrs = {name: (ctypes.c_void_p * n)() for name in ("q", "k", "v", "g", "beta", "parents", "o")}
+    for i, (s, o, W) in enumerate(zip(steps, outs, Ws)):
+        arrs["q"][i] = _ptr(s["q"], "q", dt, (c.R, W, c.H, c.d_k), c.device).value
+        arrs["k"][i] = _ptr(s["k"], "k", dt, (c.R, W, c.H, c.d_k), c.device).value
+        arrs["v"][i] = _ptr(s["v"], "v", dt, (c.R, W, c.H, c.d_v), c.device).value
+        arrs["g"][i] = _ptr(s["g"], "g", torch.float32, (c.R, W, c.H), c.device).value
+        arrs["beta"][i] = _ptr(s["beta"], "beta", torch.float32, (c.R, W, c.H), c.device).value
+        arrs["parents"][i] = _ptr(s["parents"], "parent_idx", torch.int32, (c.R, W), c.device).value
+        arrs["o"][i] = _ptr(o, "o", torch.float32, (c.R, W, c.H, c.d_v), c.device).value
+    Wa = (ctypes.c_int32 * n)(*Ws)
+    _check(lib.onela_decode_steps(h.ptr, n, Wa, arrs["q"], arrs["k"], arrs["v"], arrs["g"], arrs["beta"],
+                                  arrs["parents"], arrs["o"], _stream(stream)), "onela_decode_steps")
+
+
+def onela_set_wait_policy(h: Handle, limit_ns: int, stall: bool = False) -> None:
+    _check(lib.onela_set_wait_policy(h.ptr, int(limit_ns), 1 if stall else 0), "onela_set_wait_policy")
+
+
 def onela_reset(h: Handle, stream=None) -> None:
     _check(lib.onela_reset(h.ptr, _stream(stream)), "onela_reset")
 
@@ -282,6 +313,10 @@ def onela_steps_done(h: Handle) -> int:
 
 def onela_kernel_kind(h: Handle) -> int:
     return int(lib.onela_kernel_kind(h.ptr))
+
+
+def onela_last_call_launches(h: Handle) -> int:
+    return int(lib.onela_last_call_launches(h.ptr))
 
 
 def onela_decode_step_noalloc(R: int, H: int, d_k: int, d_v: int, W_max: int, T_max: int,

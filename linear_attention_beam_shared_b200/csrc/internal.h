@@ -24,13 +24,14 @@ struct StepParams {
   int32_t *par_store;     // [T_max slots][R][W_max]: each step's parents (tensor-core kernel)
   // History of the decode for the tensor-core kernel: entry i describes step
   // j = hbase + i (hbase <= j < t, at most kHistSteps steps back): keys,
-  // gates and parents.  hist_inputs = 1: the callers' own arrays of step j,
-  // valid under ONELA_FLAG_PDL -- hk[i] [R][W_j][H][d_k], hg[i] [R][W_j][H]
-  // (the gate before exp), hpar[i] [R][W_j].  hist_inputs = 0: the record
-  // store (rec_k, rec_alpha) and the par_store row of step j.  Parents of
-  // request r start at hpar[i] + r * hpar_rs[i]; hW[i] = W_j.  The kernel
-  // copies the parents of steps hcopy .. t - 1 to shared memory.
-  int hist_inputs;
+  // gates and parents.  Bit i of hist_inputs set: the callers' own arrays of
+  // step j (still valid: under ONELA_FLAG_PDL, or a step of the same
+  // onela_decode_steps call) -- hk[i] [R][W_j][H][d_k], hg[i] [R][W_j][H]
+  // (the gate before exp), hpar[i] [R][W_j].  Bit clear: the record store
+  // (rec_k, rec_alpha) and the par_store row of step j.  Parents of request r
+  // start at hpar[i] + r * hpar_rs[i]; hW[i] = W_j.  The kernel copies the
+  // parents of steps hcopy .. t - 1 to shared memory.
+  uint32_t hist_inputs;
   int hbase, hcopy;
   const void *hk[kHistSteps];
   const float *hg[kHistSteps];
@@ -61,6 +62,11 @@ struct StepParams {
   const int32_t *d0;
   const int32_t *anc_fold;
   int32_t *err;           // host-mapped error word (device view)
+  // Bound of every wait of the tensor-core kernel on another warp role
+  // (nanoseconds); stall = 1 (tests only) makes the wait for the ancestry
+  // warp run out at that bound.
+  unsigned long long wait_limit_ns;
+  int stall;
   // TMA descriptors of k, q and v (tensor-core kernel; encoded per call):
   // 4-D {d, H, W, R} bf16, box {64, 1, 32, 1}, 128-byte swizzle.
   alignas(64) CUtensorMap tm_k;
@@ -138,6 +144,7 @@ size_t s0_image_bytes(int R, int H, int dk, int dv, int planes);
 cudaError_t launch_prefill(const void *k, const void *v, const float *g, const float *beta, void *S0, int R, int L,
                            int H, int dk, int dv, int qkv_bf16, int s0_bf16, cudaStream_t s);
 bool tc_supports(int dk, int dv, int qkv_bf16, int T_max, int W_max);
+
 // Beam selection (select.cu): the W best of W_prev x C candidates per request.
 size_t select_scratch_bytes(int R, int W_prev, int C, int W);
 cudaError_t launch_select(const float *beam_score, const float *logp, int R, int W_prev, int C, int W,

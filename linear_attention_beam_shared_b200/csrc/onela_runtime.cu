@@ -45,6 +45,11 @@ struct onela_handle {
   int32_t *anc;
   int32_t *err_host;  // host-mapped error word
   int32_t *err_dev;   // its device view
+  // Bound of every wait inside the tensor-core step kernel, and the testing
+  // aid of onela_set_wait_policy.
+  unsigned long long wait_limit_ns;
+  int stall;
+  int last_launches;  // kernel launches of the last decode call
 };
 
 namespace {
@@ -121,6 +126,8 @@ onela::StepParams base_params(const onela_handle *h) {
   p.rec_k = h->rec_k;
   p.anc = h->anc;
   p.err = h->err_dev;
+  p.wait_limit_ns = h->wait_limit_ns;
+  p.stall = h->stall;
   return p;
 }
 
@@ -169,7 +176,8 @@ int onela_create(const onela_config *cfg, onela_handle **out) {
   if (c.R < 1 || c.H < 1 || c.d_k < 1 || c.d_k > 256 || c.d_v < 1 || c.d_v > 256 || c.W_max < 1 ||
       c.T_max < 1 || c.T_max > 64 || !valid_dtype(c.s0_dtype) || !valid_dtype(c.qkv_dtype) ||
       c.kernel < ONELA_KERNEL_AUTO || c.kernel > ONELA_KERNEL_TC || c.device < 0 ||
-      !(c.s0_split == 0 || c.s0_split == 2 || c.s0_split == 3) || (c.flags & ~ONELA_FLAG_PDL) != 0)
+      !(c.s0_split == 0 || c.s0_split == 2 || c.s0_split == 3) ||
+      (c.flags & ~ONELA_FLAG_PDL) != 0)
     return ONELA_ERR_ARG;
   // Sizes must stay addressable with 64-bit offsets and the kernels' int grid.
   const double rows = (double)c.T_max * c.R * c.H * c.W_max;
@@ -193,6 +201,8 @@ int onela_create(const onela_config *cfg, onela_handle **out) {
   h->planes = c.s0_dtype == ONELA_BF16 ? 1 : (c.s0_split == 0 ? 2 : c.s0_split);
   h->steps_done = 0;
   h->has_prompt = 0;
+  h->wait_limit_ns = 2000000000ull;
+  h->stall = 0;
   const size_t nS0 = (size_t)c.R * c.H * c.d_v * c.d_k;
   const size_t nrow = (size_t)c.T_max * c.R * c.H * c.W_max;
   bool ok = cudaMalloc(&h->S0, nS0 * esize(c.s0_dtype)) == cudaSuccess;
@@ -301,9 +311,17 @@ int onela_read_prompt_state(onela_handle *h, void *S0, onela_stream stream) {
   return ONELA_OK;
 }
 
-int onela_decode_step(onela_handle *h, int32_t W_prev, int32_t W, const void *q, const void *k, const void *v,
-                      const float *gate, const float *beta, const int32_t *parent_idx, float *o,
-                      onela_stream stream) {
+}  // extern "C"
+
+namespace {
+
+// One decode step.  call_t0 > 0: the step belongs to an onela_decode_steps
+// call whose first step is depth call_t0, so the callers' arrays of steps
+// call_t0 .. t-1 are still valid, and a later step of the call may overlap
+// the step before it (programmatic launch).
+int decode_one(onela_handle *h, int32_t W_prev, int32_t W, const void *q, const void *k, const void *v,
+               const float *gate, const float *beta, const int32_t *parent_idx, float *o, cudaStream_t s,
+               int call_t0) {
   if (!h || !q || !k || !v || !gate || !beta || !parent_idx || !o) return ONELA_ERR_ARG;
   const int rc = word_code(h);
   if (rc != ONELA_OK) return rc;
@@ -330,31 +348,37 @@ int onela_decode_step(onela_handle *h, int32_t W_prev, int32_t W, const void *q,
   p.beta = beta;
   p.parents = parent_idx;
   p.o = o;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
+  const bool contract = (c.flags & ONELA_FLAG_PDL) != 0;
   // The step after a fold reads the folded state before its wait: it is an
-  // ordinary launch.
-  const bool pdl = (c.flags & ONELA_FLAG_PDL) && p.t >= 2 && !h->after_fold;
+  // ordinary launch.  Otherwise a step overlaps the step before it under
+  // ONELA_FLAG_PDL, or inside one onela_decode_steps call when the depth its
+  // early writes replace (t - T_max) is none, or of the same call (then no
+  // step still running reads it from the store).
+  const int tr = p.t - c.T_max;
+  const bool in_call = call_t0 > 0 && p.t > call_t0 && (tr < 1 || tr >= call_t0);
+  const bool pdl = p.t >= 2 && !h->after_fold && (contract || in_call);
   if (h->kernel == ONELA_KERNEL_TC) {
     // The tensor-core kernel reads tiles of q, k, v and o with 16-byte accesses.
     const uintptr_t any = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
                           reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(o);
     if (any & 15u) return ONELA_ERR_ARG;
-    // Keys, gates and parents of the earlier steps: the callers' arrays under
-    // ONELA_FLAG_PDL (still valid by its contract), else the record store
-    // and the parents the earlier kernels stored (they have completed).
-    p.hist_inputs = pdl ? 1 : 0;
     // The table covers steps hbase .. t-1 (the kernel replays at most
     // T_max - 1 <= 15 of them); the parents of steps hcopy .. t-1 go to
-    // shared memory.
+    // shared memory.  Keys, gates and parents of a step come from the
+    // caller's arrays while they are valid (ONELA_FLAG_PDL, or a step of
+    // this call), else from the record store and the stored parents (those
+    // steps have completed).
     p.hbase = p.t - onela::kHistSteps + 1 > 1 ? p.t - onela::kHistSteps + 1 : 1;
     p.hcopy = p.t - c.T_max + 1 > 2 ? p.t - c.T_max + 1 : 2;
     if (p.hcopy < p.hbase + 1) p.hcopy = p.hbase + 1;
+    p.hist_inputs = 0;
     int hist = 0;
     for (int j = p.hbase; j < p.t; ++j) {
       const int i = j - p.hbase;
       p.hW[i] = h->Ws[j - 1];
-      if (pdl) {
+      if (contract || (call_t0 > 0 && j >= call_t0)) {
+        p.hist_inputs |= 1u << i;
         p.hk[i] = h->hist_k[j - 1];
         p.hg[i] = h->hist_g[j - 1];
         p.hpar[i] = h->hist_par[j - 1];
@@ -380,10 +404,62 @@ int onela_decode_step(onela_handle *h, int32_t W_prev, int32_t W, const void *q,
   }
   h->steps_done += 1;
   h->after_fold = 0;
+  h->last_launches = 1;
   h->Ws.push_back(W);
   h->hist_k.push_back(k);
   h->hist_g.push_back(gate);
   h->hist_par.push_back(parent_idx);
+  return ONELA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int onela_decode_step(onela_handle *h, int32_t W_prev, int32_t W, const void *q, const void *k, const void *v,
+                      const float *gate, const float *beta, const int32_t *parent_idx, float *o,
+                      onela_stream stream) {
+  return decode_one(h, W_prev, W, q, k, v, gate, beta, parent_idx, o, static_cast<cudaStream_t>(stream), 0);
+}
+
+int onela_decode_steps(onela_handle *h, int32_t n, const int32_t *W, const void *const *q, const void *const *k,
+                       const void *const *v, const float *const *gate, const float *const *beta,
+                       const int32_t *const *parent_idx, float *const *o, onela_stream stream) {
+  if (!h || n < 1 || !W || !q || !k || !v || !gate || !beta || !parent_idx || !o) return ONELA_ERR_ARG;
+  for (int i = 0; i < n; ++i)
+    if (!q[i] || !k[i] || !v[i] || !gate[i] || !beta[i] || !parent_idx[i] || !o[i]) return ONELA_ERR_ARG;
+  const int rc = word_code(h);
+  if (rc != ONELA_OK) return rc;
+  if (!h->has_prompt) return ONELA_ERR_STATE;
+  const onela_config &c = h->cfg;
+  // Everything that can be checked on the host is checked before the first
+  // launch, so an error leaves no work enqueued.
+  for (int i = 0; i < n; ++i) {
+    if (W[i] < 1) return ONELA_ERR_ARG;
+    if (W[i] > c.W_max) return ONELA_ERR_CAPACITY;
+  }
+  if (((long long)h->steps_done + n > c.T_max && !h->folded) || (long long)h->steps_done + n >= (1 << 30))
+    return ONELA_ERR_CAPACITY;
+  if (h->kernel == ONELA_KERNEL_TC)
+    for (int i = 0; i < n; ++i)
+      if ((reinterpret_cast<uintptr_t>(q[i]) | reinterpret_cast<uintptr_t>(k[i]) | reinterpret_cast<uintptr_t>(v[i]) |
+           reinterpret_cast<uintptr_t>(o[i])) & 15u)
+        return ONELA_ERR_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int call_t0 = h->steps_done + 1;
+  for (int i = 0; i < n; ++i) {
+    const int Wp = h->steps_done == 0 ? 1 : h->Ws.back();
+    const int e = decode_one(h, Wp, W[i], q[i], k[i], v[i], gate[i], beta[i], parent_idx[i], o[i], s, call_t0);
+    if (e != ONELA_OK) return e;
+  }
+  h->last_launches = n;
+  return ONELA_OK;
+}
+
+int onela_set_wait_policy(onela_handle *h, uint64_t limit_ns, int32_t stall) {
+  if (!h || limit_ns < 1000 || limit_ns > 10000000000ull) return ONELA_ERR_ARG;
+  h->wait_limit_ns = limit_ns;
+  h->stall = stall != 0;
   return ONELA_OK;
 }
 
@@ -536,5 +612,7 @@ int onela_read_ancestry(onela_handle *h, int32_t t, int32_t *anc, onela_stream s
 int onela_steps_done(const onela_handle *h) { return h ? h->steps_done : -1; }
 
 int onela_kernel_kind(const onela_handle *h) { return h ? h->kernel : -1; }
+
+int onela_last_call_launches(const onela_handle *h) { return h ? h->last_launches : -1; }
 
 }  // extern "C"

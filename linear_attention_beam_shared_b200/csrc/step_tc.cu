@@ -34,8 +34,10 @@
 // of every step), their keys and their gates are inputs.  So each kernel
 // lets its dependent launch start at once, and before its
 // griddepcontrol.wait it reads inputs only: the callers' arrays of the
-// earlier steps under ONELA_FLAG_PDL, the record store otherwise (then the
-// earlier steps have completed).  Before the wait: the ancestry warp builds
+// earlier steps where they are still valid (under ONELA_FLAG_PDL, or steps of
+// the same onela_decode_steps call), the record store otherwise (a step that
+// overlaps its predecessor never reads from the store a depth that a step
+// still running may replace).  Before the wait: the ancestry warp builds
 // each beam's ancestor chain (parent indices only; records never move,
 // abstract), then the tile's distinct ancestors and the replay weights; the
 // MMA warp issues D1 as soon as the image is in; the beam warps form the key
@@ -57,6 +59,7 @@
 
 #include "internal.h"
 #include "sm100_ptx.h"
+#include "tc_common.h"
 
 namespace onela {
 namespace {
@@ -72,7 +75,6 @@ constexpr int kTmemCols = 64;       // D1
 constexpr uint32_t kTabBytes = 3u * 8u * kHistSteps + 3u * 4u * kHistSteps;  // per-step table
 constexpr int kMaxT = 16;           // deepest decode the kernel serves
 constexpr int kMaxW = 1024;         // widest beam set the kernel serves
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far beyond any legal wait
 
 struct Layout {
   uint32_t x;     // X [NK][64 rows][128 B]: k rows, then q rows
@@ -103,33 +105,6 @@ __host__ __device__ inline Layout layout(int nk, int planes, int TM, int W_max, 
   return L;
 }
 
-// Copies n parent indices (int32, global) to shared memory as 16-bit
-// indices, by the 32 lanes of one warp: 16-byte loads when the source allows
-// it, single ints otherwise.
-__device__ __forceinline__ void copy_parents16_warp(uint16_t *dst, const int32_t *src, int n, int lane) {
-  // dst is 8-byte aligned; parents are below 2^16 (anything else is out of
-  // range and is clamped where it is used).
-  int done = 0;
-  if ((reinterpret_cast<uintptr_t>(src) & 15u) == 0) {
-    done = n & ~3;
-#pragma unroll 2
-    for (int e = lane * 4; e < done; e += 128) {
-      const int4 v = __ldg(reinterpret_cast<const int4 *>(src + e));
-      *reinterpret_cast<uint2 *>(dst + e) = make_uint2(((uint32_t)v.x & 0xffffu) | ((uint32_t)v.y << 16),
-                                                      ((uint32_t)v.z & 0xffffu) | ((uint32_t)v.w << 16));
-    }
-  }
-  for (int e = done + lane; e < n; e += 32) dst[e] = (uint16_t)__ldg(src + e);
-}
-
-// Four consecutive bf16 elements (packed in u, or at p, 8-byte aligned) as floats.
-__device__ __forceinline__ float4 bf16x4(uint2 u) {
-  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
-  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
-  return make_float4(a.x, a.y, b.x, b.y);
-}
-__device__ __forceinline__ float4 bf16x4(const uint8_t *p) { return bf16x4(*reinterpret_cast<const uint2 *>(p)); }
-
 template <int DK>
 __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_constant__ StepParams p) {
   constexpr int NK = DK / 64;        // 128-byte K atoms per key row
@@ -158,7 +133,7 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
   const int soff = d0 % TM;     // slot of depth d0 + 1
   const int tslot = (t - 1) % TM;  // slot of depth t
   const int hb = p.hbase;       // step of the history table's entry 0
-  const bool hin = p.hist_inputs != 0;
+  const uint32_t hmask = p.hist_inputs;  // bit i: history entry i from the callers' arrays
 
   const Layout L = layout(NK, P, TM, p.W_max, p.hist_cap);
   uint8_t *s_x = base + L.x;
@@ -202,7 +177,7 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
   if (tid == 0) {
     ptx::mbar_init(bar_s0, 1);
     ptx::mbar_init(bar1, 1);
-    ptx::mbar_init(bar_chain, 32);
+    ptx::mbar_init(bar_chain, 32 + (p.stall ? 1 : 0));  // stall (tests): an arrival that never comes
     ptx::mbar_fence_init();
     // S0 image (bulk copy); k, q, v tiles by TMA, beams past W read as zeros.
     ptx::mbar_arrive_expect_tx(bar_s0, s0_bytes + NK * (XA + VA));
@@ -306,8 +281,8 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
         const int a = s_chain[b * TM + j];
         const int di = d0 + j + 1 - hb;  // history entry of the record's depth
         const int sl = soff + j < TM ? soff + j : soff + j - TM;
-        ptx::cp_async4(s_w + b * TM + j, hin ? s_tg[di] + ((int64_t)r * s_tW[di] + a) * H + h
-                                             : p.rec_alpha + rec_row_slot(p, sl, r, h, a));
+        ptx::cp_async4(s_w + b * TM + j, (hmask >> di) & 1u ? s_tg[di] + ((int64_t)r * s_tW[di] + a) * H + h
+                                                           : p.rec_alpha + rec_row_slot(p, sl, r, h, a));
       }
     }
     ptx::cp_async_commit();
@@ -338,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
       for (int j = jp; j >= 0; --j) {
         const float gj = s_w[b * TM + j];
         reinterpret_cast<float *>(s_c + b * TM + j)[3] = w;
-        w *= hin ? expf(gj) : gj;
+        w *= (hmask >> (d0 + j + 1 - hb)) & 1u ? expf(gj) : gj;
       }
     }
     s_Gp[b] = w;
@@ -347,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
     // D1 = S0 . X^T on the tensor cores, issued by lane 0 once the image is
     // here.
     if (lane == 0) {
-      ok = ptx::mbar_wait(bar_s0, 0, kWaitLimitNs);
+      ok = ptx::mbar_wait(bar_s0, 0, p.wait_limit_ns);
       ptx::tc_fence_after();
       constexpr uint32_t idesc1 = ptx::idesc_bf16_f32(kM, kN);
       int acc = 0;
@@ -365,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
     }
   } else {
     // ------------------------------------------------ the beam warps
-    if (!ptx::mbar_wait(bar_s0, 0, kWaitLimitNs)) ok = false;  // X and v visible to this thread
+    if (!ptx::mbar_wait(bar_s0, 0, p.wait_limit_ns)) ok = false;  // X and v visible to this thread
     // This thread's elements of k_b and q_b, and k_b . q_b.
 #pragma unroll
     for (int u = 0; u < NU; ++u) {
@@ -387,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
     // thread's pieces of each ancestor's key row come straight from global
     // memory (step j's own k input, or the key records), two depths per
     // pass, the next pass's loads in flight during this pass's arithmetic.
-    if (!ptx::mbar_wait(bar_chain, 0, kWaitLimitNs)) ok = false;
+    if (!ptx::mbar_wait(bar_chain, 0, p.wait_limit_ns)) ok = false;
     auto issue = [&](uint2 (&buf)[2][NU], int j0) {
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
@@ -396,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
           const int a = s_chain[bb * TM + j];
           const int di = d0 + j + 1 - hb;
           const int sl = soff + j < TM ? soff + j : soff + j - TM;
-          const __nv_bfloat16 *row = hin ? s_tk[di] + ((int64_t)(r * s_tW[di] + a) * H + h) * DK
+          const __nv_bfloat16 *row = (hmask >> di) & 1u ? s_tk[di] + ((int64_t)(r * s_tW[di] + a) * H + h) * DK
                                          : rec_k + rec_row_slot(p, sl, r, h, a) * DK;
           const uint8_t *rb = reinterpret_cast<const uint8_t *>(row) + l * 8;
 #pragma unroll
@@ -453,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
     if (warp >= 4) {
       // D1^T into shared memory (region A: the image is consumed).
       const int ei = wq * 32 + lane;  // TMEM lane: output element of D1
-      if (!ptx::mbar_wait(bar1, 0, kWaitLimitNs)) ok = false;
+      if (!ptx::mbar_wait(bar1, 0, p.wait_limit_ns)) ok = false;
       ptx::tc_fence_after();
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
@@ -630,32 +605,35 @@ __global__ void s0_image_kernel(const void *S0, uint4 *img, int R, int H, int dk
   }
 }
 
-// cuTensorMapEncodeTiled, fetched once from the driver.
+// cuTensorMapEncodeTiled, fetched once from the driver (thread-safe static
+// initialisation).
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
     void *ptr = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
+      return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    return nullptr;
+  }();
   return fn;
 }
 
-// 4-D map over a [R][W][H][d] bf16 tensor: {d, H, W, R}, box {64, 1, 32, 1},
-// 128-byte swizzle (the K-major operand layout), zeros outside the tensor.
-bool encode_rows(CUtensorMap *m, const void *base, int d, int H, int W, int R) {
+}  // namespace
+
+bool encode_rows(CUtensorMap *m, const void *base, int d, int H, int W, int R, int box_rows) {
   PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)W, (cuuint64_t)R};
   const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, (cuuint64_t)W * H * d * 2};
-  const cuuint32_t box[4] = {64, 1, (cuuint32_t)kBT, 1};
+  const cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
   const cuuint32_t es[4] = {1, 1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+namespace {
 
 template <int DK>
 cudaError_t launch_dk(const StepParams &p_in, bool pdl, cudaStream_t s) {

@@ -44,7 +44,11 @@ def to_dev(steps, device="cuda"):
 
 def run_gpu(S0: torch.Tensor, steps: List[Dict], qkv_dtype: str, kernel: int,
             T_max: Optional[int] = None, W_max: Optional[int] = None, read_back=True,
-            s0_split: int = 0, flags: int = 0):
+            s0_split: int = 0, flags: int = 0, chunks: Optional[List[int]] = None):
+    """Decode on the GPU through the C ABI.  chunks = None: one
+    onela_decode_step call per step; else onela_decode_steps calls over
+    consecutive runs of chunks[0], chunks[1], ... steps (a chunk of 1 is a
+    onela_decode_step call)."""
     import linear_attention_beam_shared_b200 as L
     R, H, dv, dk = S0.shape
     s0_dtype = "bf16" if S0.dtype == torch.bfloat16 else "f32"
@@ -56,9 +60,20 @@ def run_gpu(S0: torch.Tensor, steps: List[Dict], qkv_dtype: str, kernel: int,
         dsteps = to_dev(steps)          # every input resident before the first step
         dec.set_prompt_state(S0.cuda())
         outs = []
-        for s in dsteps:
-            o = dec.step(s["q"], s["k"], s["v"], s["g"], s["beta"], s["parents"])
-            outs.append(o)
+        if chunks is None:
+            for s in dsteps:
+                o = dec.step(s["q"], s["k"], s["v"], s["g"], s["beta"], s["parents"])
+                outs.append(o)
+        else:
+            assert sum(chunks) == T
+            i = 0
+            for c in chunks:
+                if c == 1:
+                    s = dsteps[i]
+                    outs.append(dec.step(s["q"], s["k"], s["v"], s["g"], s["beta"], s["parents"]))
+                else:
+                    outs += dec.steps(dsteps[i:i + c])
+                i += c
         assert dec.status() == 0
         res = []
         for t, o in enumerate(outs, start=1):

@@ -40,11 +40,13 @@ def narrow(steps, at, beam):
     return steps
 
 
-def run_with_folds(S0, steps, qkv, kernel, folds, flags=0, T_max=None):
+def run_with_folds(S0, steps, qkv, kernel, folds, flags=0, T_max=None, chunked=False):
     """Decode all steps on the GPU; after step t (1-based) in `folds`, fold
-    with max_depth folds[t].  Returns per-step outputs, records and ancestry
-    (records only for the depths the store still holds, ancestry only while
-    t <= T_max) and, per fold, (t, fold depth [R], root state)."""
+    with max_depth folds[t].  chunked: the steps between two folds go in one
+    onela_decode_steps call instead of one onela_decode_step call each.
+    Returns per-step outputs, records and ancestry (records only for the
+    depths the store still holds, ancestry only while t <= T_max) and, per
+    fold, (t, fold depth [R], root state)."""
     import linear_attention_beam_shared_b200 as L
     R, H, dv, dk = S0.shape
     s0_dtype = "bf16" if S0.dtype == torch.bfloat16 else "f32"
@@ -54,8 +56,16 @@ def run_with_folds(S0, steps, qkv, kernel, folds, flags=0, T_max=None):
         ds = P.to_dev(steps)
         dec.set_prompt_state(S0.cuda())
         outs, fold_info = [], []
+        pending = []
         for t, s in enumerate(ds, start=1):
-            outs.append(dec.step(s["q"], s["k"], s["v"], s["g"], s["beta"], s["parents"]))
+            if chunked:
+                pending.append(s)
+                if t not in folds and t < len(ds):
+                    continue
+                outs += dec.steps(pending)
+                pending = []
+            else:
+                outs.append(dec.step(s["q"], s["k"], s["v"], s["g"], s["beta"], s["parents"]))
             for md in as_list(folds.get(t, [])):
                 dec.fold(md)
             if t in folds:
