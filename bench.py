@@ -414,9 +414,92 @@ def time_sweep(device, stream, flush, reps=10, warmup=3):
         gbs = alg / (ms / 1e3) / 1e9
         points.append({"R": wl.R, "H": wl.H, "d": wl.d_k, "W": wl.W, "T": wl.T, "s0": wl.s0_dtype, "kernel": kind,
                        "launches": launches, "ms_per_decode": round(ms, 5), "value": round(wl.units / (ms / 1e3), 1),
-                       "achieved_gbs": round(gbs, 1), "frac": round(gbs / hbm, 4)})
+                       "achieved_gbs": round(gbs, 1), "frac": round(gbs / hbm, 4),
+                       "capacity_ratio": capacity(wl)["ratio"]})
         del ds, outs
     return {"unit": UNIT, "peak_gbs": hbm, "l2": "flushed before every decode", "points": points}
+
+
+def grid_inputs(R, H, d, W, T, device, seed):
+    """Timing inputs for one shape of the multi-request grid, made on the
+    device with the workload recipe (q, k unit-norm Gaussian, v Gaussian,
+    alpha ~ U(0.85, 0.999) passed as log, beta = sigmoid(Gaussian), bf16
+    q/k/v; parents uniform for even requests and truncated Zipf(1.1) over the
+    previous beam rank for odd ones (Zipf when R = 1); S0 Gaussian 0.1).  The
+    values do not change the work; the parents fix the ancestors replayed.
+    Returns (S0, device steps, the same steps with CPU parents)."""
+    g = torch.Generator(device=device).manual_seed(seed)
+    S0 = 0.1 * torch.randn((R, H, d, d), generator=g, device=device)
+    zipf = torch.tensor(synth.zipf_probs(W, 1.1), device=device, dtype=torch.float32)
+    steps, cpu_steps = [], []
+    for t in range(1, T + 1):
+        q = torch.nn.functional.normalize(torch.randn((R, W, H, d), generator=g, device=device), dim=-1)
+        k = torch.nn.functional.normalize(torch.randn((R, W, H, d), generator=g, device=device), dim=-1)
+        v = torch.randn((R, W, H, d), generator=g, device=device)
+        alpha = 0.85 + 0.149 * torch.rand((R, W, H), generator=g, device=device)
+        beta = torch.sigmoid(torch.randn((R, W, H), generator=g, device=device))
+        if t == 1:
+            par = torch.zeros((R, W), dtype=torch.int32, device=device)
+        else:
+            rows = []
+            for r in range(R):
+                if R > 1 and r % 2 == 0:
+                    rows.append(torch.randint(0, W, (W,), generator=g, device=device))
+                else:
+                    rows.append(torch.multinomial(zipf, W, replacement=True, generator=g))
+            par = torch.stack(rows).to(torch.int32)
+        st = {"q": q.to(torch.bfloat16), "k": k.to(torch.bfloat16), "v": v.to(torch.bfloat16),
+              "g": torch.log(alpha).float(), "beta": beta.float(), "parents": par, "W": W, "W_prev": 1 if t == 1 else W}
+        steps.append(st)
+        cpu_steps.append({"parents": par.cpu(), "W": W})
+    return S0, steps, cpu_steps
+
+
+def time_grid(device, stream, flush, reps=3, warmup=1, full=True):
+    """The multi-request operator-shape grid: R in {1, 8, 32}, H in {8, 16, 32},
+    d_k = d_v in {64, 128, 256}, W in {128, 256, 512}, T in {1, 3, 5, 7} (fp32
+    S0, bf16 q/k/v), each shape one onela_decode_steps call per CUDA graph, L2
+    flushed before every decode.  full = False: R = 1 only.  Returns the JSON
+    object for the bench line (a row per shape and a summary)."""
+    import linear_attention_beam_shared_b200 as L
+    hbm = measured_peaks()[0]
+    rows, fracs = [], {}
+    for R in ((1, 8, 32) if full else (1,)):
+        for H in (8, 16, 32):
+            for d in (64, 128, 256):
+                for W in (128, 256, 512):
+                    for T in (1, 3, 5, 7):
+                        wl = synth.shape_sweep_workload(R, H, d, W, T)
+                        free, _ = torch.cuda.mem_get_info(device)
+                        need = (T * R * H * W * (4 + 4 * d + 2 * d) + T * R * W * H * d * (3 * 2 + 4)) * 1.3
+                        if need > free * 0.8:
+                            rows.append([R, H, d, W, T, None, None, "skipped: does not fit"])
+                            continue
+                        S0, ds, cpu_steps = grid_inputs(R, H, d, W, T, device, seed=R * 1000 + H * 37 + d + W + T)
+                        outs = [torch.empty((R, W, H, d), dtype=torch.float32, device=device) for _ in ds]
+                        dec = L.BeamDecoder(R, H, d, d, W, T, "f32", "bf16", device=device.index)
+                        dec.set_prompt_state(S0)
+                        g, launches = decode_graph(dec, ds, outs, stream)
+                        kind = {L.ONELA_KERNEL_SIMT: "simt", L.ONELA_KERNEL_TC: "tc"}[dec.kernel]
+                        ms = time_graph(g, stream, flush, reps, warmup)
+                        del g
+                        assert dec.status() == 0
+                        dec.close()
+                        alg, _, _ = byte_model(wl, cpu_steps)
+                        frac = alg / (ms / 1e3) / 1e9 / hbm
+                        fracs.setdefault(kind, []).append(frac)
+                        rows.append([R, H, d, W, T, round(ms, 5), round(frac, 4), kind])
+                        del ds, outs, S0
+                        torch.cuda.empty_cache()
+    allf = sorted(f for v in fracs.values() for f in v)
+    summary = {"shapes": len(rows), "timed": len(allf),
+               "median_frac": round(statistics.median(allf), 4) if allf else None,
+               "worst_frac": round(allf[0], 4) if allf else None, "best_frac": round(allf[-1], 4) if allf else None,
+               "by_kernel": {k: {"shapes": len(v), "median_frac": round(statistics.median(v), 4),
+                                 "worst_frac": round(min(v), 4)} for k, v in fracs.items()}}
+    return {"unit": "fraction of measured HBM bandwidth (algorithmic bytes)", "peak_gbs": hbm,
+            "l2": "flushed before every decode", "columns": ["R", "H", "d", "W", "T", "ms_per_decode", "frac", "kernel"],
+            "summary": summary, "rows": rows}
 
 
 def decode_graph(dec, dsteps, outs, stream, per_step=False):
@@ -483,6 +566,21 @@ def byte_model(wl, steps):
         total += b_t
         upper += u_t
     return total, upper, per_step
+
+
+def capacity(wl):
+    """State memory per (request, head) at the end of a T-step decode: this
+    library's (S0 in its dtype, the T depths of records (alpha fp32, delta fp32,
+    k in the q/k/v dtype), the ancestry rows and parents shared by the
+    request's heads) against a full-state beam decode that keeps one fp32
+    d_v x d_k state per beam (the pages' FullState)."""
+    s = 2 if wl.s0_dtype == "bf16" else 4
+    e = 2 if wl.qkv_dtype == "bf16" else 4
+    T, W, dk, dv, H = wl.T, wl.W, wl.d_k, wl.d_v, wl.H
+    onela = dk * dv * s + T * W * (4 + 4 * dv + e * dk) + T * W * (T + 1) * 4 / H
+    full = W * dk * dv * 4
+    return {"bytes_per_request_head": int(round(onela)), "fullstate_fp32_bytes_per_request_head": int(full),
+            "ratio": round(full / onela, 2)}
 
 
 class ClockSampler:
@@ -732,6 +830,7 @@ def run_ours(args):
     prefill = time_prefill(wl, device, stream, flush) if (wl.L_prompt > 0 and not args.no_prefill) else None
     select = None if args.no_prefill else time_select(device, stream, flush, R=wl.R, W_prev=wl.W, C=256, W=wl.W)
     sweep = None if (args.no_sweep or ws > 1) else time_sweep(device, stream, flush)
+    grid = None if (args.no_grid or ws > 1) else time_grid(device, stream, flush, full=not args.grid_r1)
     fold = None if args.no_prefill else [time_fold(wl, S0, kernel, device, stream, flush, every=4),
                                           time_fold(wl, S0, kernel, device, stream, flush, every=8, alone=False),
                                           time_fold(wl, S0, kernel, device, stream, flush, T=32, every=8, alone=False,
@@ -760,8 +859,8 @@ def run_ours(args):
                        "launches_per_decode": launches},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "clocks": clk.summary(), "gpu_launches": launches * args.steps,
-            "variants": variants,
-            "prefill": prefill, "beam_select": select, "fold": fold, "sweep": sweep,
+            "variants": variants, "capacity": capacity(wl),
+            "prefill": prefill, "beam_select": select, "fold": fold, "sweep": sweep, "grid": grid,
         }
         print(json.dumps(line))
     if ws > 1:
@@ -817,6 +916,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill, beam-selection and fold timings")
     ap.add_argument("--no-sweep", action="store_true", help="skip the beam-width and request sweeps")
+    ap.add_argument("--no-grid", action="store_true", help="skip the multi-request shape grid")
+    ap.add_argument("--grid-r1", action="store_true", help="the shape grid at R = 1 only")
     ap.add_argument("--s0", choices=["prefill", "direct"], default="prefill",
                     help="S0 from the GDN recurrence over the synthetic prompt (default) or drawn "
                          "directly; the decode's work does not depend on the S0 values")

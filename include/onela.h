@@ -97,6 +97,11 @@ enum {
  *                   the verification of a tree of drafted tokens.  Step 1
  *                   never overlaps. */
 enum { ONELA_FLAG_PDL = 1 };
+/*   ONELA_FLAG_NVTX  mark every decode step, fold and prefill call on the
+ *                   host with an NVTX range ("onela step t", ...) for
+ *                   timeline profilers; off by default (the ranges cost a
+ *                   little host time per call, nothing on the device). */
+enum { ONELA_FLAG_NVTX = 4 };
 
 
 /* Which decode kernel runs.  AUTO picks the tensor-core kernel when the
@@ -120,7 +125,8 @@ enum { ONELA_KERNEL_AUTO = 0, ONELA_KERNEL_SIMT = 1, ONELA_KERNEL_TC = 2 };
  *                   terms S0 is split into (2 or 3; 0 means 2).  Ignored
  *                   otherwise.
  *   device          CUDA device ordinal the handle lives on.
- *   flags           ONELA_FLAG_* bits (0: none).
+ *   flags           ONELA_FLAG_* bits (0: none): ONELA_FLAG_PDL,
+ *                   ONELA_FLAG_NVTX.
  */
 typedef struct {
   int32_t R, H, d_k, d_v, W_max, T_max;

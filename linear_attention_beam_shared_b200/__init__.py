@@ -19,7 +19,7 @@ import torch
 from . import _lib
 from ._lib import (  # noqa: F401
     ONELA_BF16, ONELA_ERR_ARG, ONELA_ERR_CAPACITY, ONELA_ERR_CUDA, ONELA_ERR_PARENT,
-    ONELA_ERR_STATE, ONELA_ERR_UNSUPPORTED, ONELA_F32, ONELA_FLAG_PDL, ONELA_KERNEL_AUTO, ONELA_KERNEL_SIMT,
+    ONELA_ERR_STATE, ONELA_ERR_UNSUPPORTED, ONELA_F32, ONELA_FLAG_NVTX, ONELA_FLAG_PDL, ONELA_KERNEL_AUTO, ONELA_KERNEL_SIMT,
     ONELA_ERR_SCRATCH, ONELA_ERR_TIMEOUT, ONELA_KERNEL_TC, ONELA_OK, Handle, OnelaError, error_string, onela_create,
     onela_decode_step, onela_decode_step_noalloc, onela_decode_steps, onela_set_wait_policy, onela_destroy, onela_fold, onela_kernel_kind, onela_last_call_launches, onela_prefill,
     onela_read_ancestry, onela_read_fold_depth, onela_read_prompt_state, onela_read_records,

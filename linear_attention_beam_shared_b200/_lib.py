@@ -23,6 +23,7 @@ ONELA_ERR_PARENT, ONELA_ERR_CUDA, ONELA_ERR_UNSUPPORTED, ONELA_ERR_SCRATCH = 4, 
 ONELA_ERR_TIMEOUT = 8
 ONELA_KERNEL_AUTO, ONELA_KERNEL_SIMT, ONELA_KERNEL_TC = 0, 1, 2
 ONELA_FLAG_PDL = 1
+ONELA_FLAG_NVTX = 4
 
 _DT = {ONELA_F32: torch.float32, ONELA_BF16: torch.bfloat16}
 _DT_CODE = {"f32": ONELA_F32, "bf16": ONELA_BF16, torch.float32: ONELA_F32, torch.bfloat16: ONELA_BF16}

@@ -143,7 +143,7 @@ size_t s0_image_bytes(int R, int H, int dk, int dv, int planes);
 // fp32), g and beta [R][L][H] fp32 -> S0 [R][H][dv][dk] (bf16 if s0_bf16).
 cudaError_t launch_prefill(const void *k, const void *v, const float *g, const float *beta, void *S0, int R, int L,
                            int H, int dk, int dv, int qkv_bf16, int s0_bf16, cudaStream_t s);
-bool tc_supports(int dk, int dv, int qkv_bf16, int T_max, int W_max);
+bool tc_supports(int dk, int dv, int qkv_bf16, int T_max, int W_max, int planes);
 
 // Beam selection (select.cu): the W best of W_prev x C candidates per request.
 size_t select_scratch_bytes(int R, int W_prev, int C, int W);

@@ -1,7 +1,9 @@
 // Host runtime of the decode library: handle, validation, record store,
 // ancestry index, error word, and the C ABI declared in include/onela.h.
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
+#include <cstdio>
 #include <cstdlib>
 #include <cstring>
 #include <map>
@@ -57,6 +59,21 @@ namespace {
 size_t esize(int dtype) { return dtype == ONELA_BF16 ? 2 : 4; }
 
 bool valid_dtype(int d) { return d == ONELA_F32 || d == ONELA_BF16; }
+
+// An NVTX range on the host for the duration of a call, when the handle
+// asks for them (ONELA_FLAG_NVTX).
+struct NvtxRange {
+  bool on;
+  NvtxRange(const onela_config &c, const char *what, int t) : on((c.flags & ONELA_FLAG_NVTX) != 0) {
+    if (!on) return;
+    char name[48];
+    std::snprintf(name, sizeof(name), t > 0 ? "onela %s %d" : "onela %s", what, t);
+    nvtxRangePushA(name);
+  }
+  ~NvtxRange() {
+    if (on) nvtxRangePop();
+  }
+};
 
 // Switch to the handle's device for the duration of a call.
 struct DeviceGuard {
@@ -177,7 +194,7 @@ int onela_create(const onela_config *cfg, onela_handle **out) {
       c.T_max < 1 || c.T_max > 64 || !valid_dtype(c.s0_dtype) || !valid_dtype(c.qkv_dtype) ||
       c.kernel < ONELA_KERNEL_AUTO || c.kernel > ONELA_KERNEL_TC || c.device < 0 ||
       !(c.s0_split == 0 || c.s0_split == 2 || c.s0_split == 3) ||
-      (c.flags & ~ONELA_FLAG_PDL) != 0)
+      (c.flags & ~(ONELA_FLAG_PDL | ONELA_FLAG_NVTX)) != 0)
     return ONELA_ERR_ARG;
   // Sizes must stay addressable with 64-bit offsets and the kernels' int grid.
   const double rows = (double)c.T_max * c.R * c.H * c.W_max;
@@ -185,9 +202,11 @@ int onela_create(const onela_config *cfg, onela_handle **out) {
   if ((double)c.R * c.W_max * c.H * (c.d_k > c.d_v ? c.d_k : c.d_v) > 2.0e9) return ONELA_ERR_ARG;
 
   const int qkv_bf16 = c.qkv_dtype == ONELA_BF16;
+  const int planes = c.s0_dtype == ONELA_BF16 ? 1 : (c.s0_split == 0 ? 2 : c.s0_split);
   int kernel = c.kernel;
-  if (kernel == ONELA_KERNEL_AUTO) kernel = onela::tc_supports(c.d_k, c.d_v, qkv_bf16, c.T_max, c.W_max) ? ONELA_KERNEL_TC : ONELA_KERNEL_SIMT;
-  if (kernel == ONELA_KERNEL_TC && !onela::tc_supports(c.d_k, c.d_v, qkv_bf16, c.T_max, c.W_max)) return ONELA_ERR_UNSUPPORTED;
+  const bool tc_ok = onela::tc_supports(c.d_k, c.d_v, qkv_bf16, c.T_max, c.W_max, planes);
+  if (kernel == ONELA_KERNEL_AUTO) kernel = tc_ok ? ONELA_KERNEL_TC : ONELA_KERNEL_SIMT;
+  if (kernel == ONELA_KERNEL_TC && !tc_ok) return ONELA_ERR_UNSUPPORTED;
 
   int ndev = 0;
   if (cudaGetDeviceCount(&ndev) != cudaSuccess || c.device >= ndev) return ONELA_ERR_CUDA;
@@ -198,7 +217,7 @@ int onela_create(const onela_config *cfg, onela_handle **out) {
   if (!h) return ONELA_ERR_CUDA;
   h->cfg = c;
   h->kernel = kernel;
-  h->planes = c.s0_dtype == ONELA_BF16 ? 1 : (c.s0_split == 0 ? 2 : c.s0_split);
+  h->planes = planes;
   h->steps_done = 0;
   h->has_prompt = 0;
   h->wait_limit_ns = 2000000000ull;
@@ -262,6 +281,7 @@ int onela_prefill(onela_handle *h, int32_t L, const void *k, const void *v, cons
   if (!g.ok) return ONELA_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const onela_config &c = h->cfg;
+  NvtxRange nvtx(c, "prefill", 0);
   if (onela::launch_prefill(k, v, gate, beta, h->S0, c.R, L, c.H, c.d_k, c.d_v, c.qkv_dtype == ONELA_BF16,
                             c.s0_dtype == ONELA_BF16, s) != cudaSuccess) {
     cudaGetLastError();
@@ -337,6 +357,7 @@ int decode_one(onela_handle *h, int32_t W_prev, int32_t W, const void *q, const 
   DeviceGuard g(c.device);
   if (!g.ok) return ONELA_ERR_CUDA;
 
+  NvtxRange nvtx(c, "step", h->steps_done + 1);
   onela::StepParams p = base_params(h);
   p.W = W;
   p.W_prev = W_prev;
@@ -496,13 +517,20 @@ int onela_fold(onela_handle *h, int32_t max_depth, onela_stream stream) {
   const int32_t *d0_in = h->fold_buf + h->fold_cur * c.R;
   int32_t *d0_out = h->fold_buf + (1 - h->fold_cur) * c.R, *anc_fold = h->fold_buf + 2 * c.R;
   const int depth = max_depth < h->steps_done ? max_depth : h->steps_done;
+  NvtxRange nvtx(c, "fold after step", h->steps_done);
   cudaError_t e;
-  if (h->kernel == ONELA_KERNEL_TC) {
+  if (h->kernel == ONELA_KERNEL_TC && c.d_k <= 128) {
     // Overlaps the step before it (never another fold: it reads the folded
     // state before its wait).
     const int pdl = (c.flags & ONELA_FLAG_PDL) && !h->after_fold;
     e = onela::launch_fold_tc(p, h->Ws.back(), depth, first, d0_in, d0_out, anc_fold, h->S0f, h->S0fimg,
                               c.s0_dtype == ONELA_BF16, pdl, s);
+  } else if (h->kernel == ONELA_KERNEL_TC) {
+    // d = 256: the general fold, then the folded state's operand image.
+    e = onela::launch_fold(p, h->Ws.back(), depth, first, d0_in, d0_out, anc_fold, h->S0f,
+                           c.qkv_dtype == ONELA_BF16, c.s0_dtype == ONELA_BF16, s);
+    if (e == cudaSuccess)
+      e = onela::launch_s0_image(h->S0f, h->S0fimg, c.R, c.H, c.d_k, c.d_v, c.s0_dtype == ONELA_BF16, h->planes, s);
   } else {
     e = onela::launch_fold(p, h->Ws.back(), depth, first, d0_in, d0_out, anc_fold, h->S0f,
                            c.qkv_dtype == ONELA_BF16, c.s0_dtype == ONELA_BF16, s);

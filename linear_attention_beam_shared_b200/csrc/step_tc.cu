@@ -78,22 +78,23 @@ constexpr int kMaxW = 1024;         // widest beam set the kernel serves
 
 struct Layout {
   uint32_t x;     // X [NK][64 rows][128 B]: k rows, then q rows
-  uint32_t v;     // v [NK][32 rows][128 B]
+  uint32_t v;     // v [NV][32 rows][128 B]: this CTA's d_v columns
   uint32_t a;     // region A: the S0 image; then D1^T; then the deltas
-  uint32_t d1;    // D1^T [64 vectors][d_v] fp32
-  uint32_t dst;   // ancestor deltas [kDRows][d_v] fp32
+  uint32_t d1;    // D1^T [64 vectors][this CTA's d_v rows] fp32
+  uint32_t dst;   // ancestor deltas [kDRows][this CTA's d_v rows] fp32
   uint32_t book;  // barriers and bookkeeping
   uint32_t total;
 };
 
-__host__ __device__ inline Layout layout(int nk, int planes, int TM, int W_max, int hist_cap) {
+// nk: 64-element K atoms of a key row; nv: 64-row atoms of this CTA's d_v rows.
+__host__ __device__ inline Layout layout(int nk, int nv, int planes, int TM, int W_max, int hist_cap) {
   Layout L;
   L.x = 0;
   L.v = (uint32_t)nk * 8192u;
-  L.a = (uint32_t)nk * 12288u;
-  L.d1 = L.a + (uint32_t)nk * 16384u;
+  L.a = L.v + (uint32_t)nv * 4096u;
+  L.d1 = L.a + (uint32_t)nv * 16384u;
   L.dst = L.a;
-  const uint32_t s0 = (uint32_t)planes * nk * 16384u, ops = (uint32_t)nk * 32768u;
+  const uint32_t s0 = (uint32_t)planes * nk * 16384u, ops = (uint32_t)nv * 32768u;
   L.book = L.a + (s0 > ops ? s0 : ops);
   // 128 B of barriers and counters; 4 per-beam scalars; per (beam, depth)
   // the replay coefficients (float4), the chain, slot-list ints and gates
@@ -105,18 +106,25 @@ __host__ __device__ inline Layout layout(int nk, int planes, int TM, int W_max, 
   return L;
 }
 
-template <int DK>
-__global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_constant__ StepParams p) {
+// DK: d_k; DV: the d_v rows of S (and columns of v, o, delta) one CTA
+// handles -- all of them for d <= 128, one half of them for d = 256 (the two
+// halves of a beam tile are two CTAs; both form the full key products).
+template <int DK, int DV>
+__global__ void __launch_bounds__(kThreads, DK <= 128 ? 2 : 1) step_tc_kernel(const __grid_constant__ StepParams p) {
   constexpr int NK = DK / 64;        // 128-byte K atoms per key row
-  constexpr int DV = DK;
+  constexpr int NV = DV / 64;        // 64-column atoms of this CTA's part of v
   constexpr uint32_t XA = kN * 128;  // bytes of one K atom of X (64 rows)
-  constexpr uint32_t VA = kBT * 128; // bytes of one K atom of v (32 rows)
-  constexpr int NU = DV / 32;        // 4-element groups per thread, beam-major phase
+  constexpr uint32_t VA = kBT * 128; // bytes of one atom of v (32 rows)
+  constexpr int NU = DV / 32;        // 4-element groups per thread of a value row, beam-major phase
+  constexpr int NUK = DK / 32;       // the same for a key row
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = ptx::smem_u32(smem_raw);
   uint8_t *base = smem_raw + ((1024u - (raw_u32 & 1023u)) & 1023u);
 
-  const int tile = blockIdx.x, h = blockIdx.y, r = blockIdx.z;
+  const int nmt = p.dv / DV;         // CTAs per beam tile (row halves of S)
+  const int tile = blockIdx.x, h = blockIdx.y, r = blockIdx.z / nmt, mt = blockIdx.z - r * nmt;
+  const int e_off = mt * DV;         // first d_v row of this CTA
+  const int DVT = p.dv;              // full d_v: the row stride of o and the delta records
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int b0 = tile * kBT;
   const int nb = min(kBT, p.W - b0);
@@ -135,7 +143,7 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
   const int hb = p.hbase;       // step of the history table's entry 0
   const uint32_t hmask = p.hist_inputs;  // bit i: history entry i from the callers' arrays
 
-  const Layout L = layout(NK, P, TM, p.W_max, p.hist_cap);
+  const Layout L = layout(NK, NV, P, TM, p.W_max, p.hist_cap);
   uint8_t *s_x = base + L.x;
   const uint8_t *s_v = base + L.v;
   float *s_d1 = reinterpret_cast<float *>(base + L.d1);
@@ -180,16 +188,17 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
     ptx::mbar_init(bar_chain, 32 + (p.stall ? 1 : 0));  // stall (tests): an arrival that never comes
     ptx::mbar_fence_init();
     // S0 image (bulk copy); k, q, v tiles by TMA, beams past W read as zeros.
-    ptx::mbar_arrive_expect_tx(bar_s0, s0_bytes + NK * (XA + VA));
-    const uint8_t *src = static_cast<const uint8_t *>(p.S0img) + (size_t)(r * H + h) * s0_bytes;
+    ptx::mbar_arrive_expect_tx(bar_s0, s0_bytes + NK * XA + NV * VA);
+    const uint8_t *src = static_cast<const uint8_t *>(p.S0img) + ((size_t)(r * H + h) * nmt + mt) * s0_bytes;
     for (uint32_t off = 0; off < s0_bytes; off += 16384u)
       ptx::bulk_g2s(base + L.a + off, src + off, 16384u, bar_s0);
 #pragma unroll
     for (int ka = 0; ka < NK; ++ka) {
       ptx::tma_load_4d(s_x + ka * XA, &p.tm_k, ka * 64, h, b0, r, bar_s0);
       ptx::tma_load_4d(s_x + ka * XA + kBT * 128, &p.tm_q, ka * 64, h, b0, r, bar_s0);
-      ptx::tma_load_4d(base + L.v + ka * VA, &p.tm_v, ka * 64, h, b0, r, bar_s0);
     }
+#pragma unroll
+    for (int ka = 0; ka < NV; ++ka) ptx::tma_load_4d(base + L.v + ka * VA, &p.tm_v, e_off + ka * 64, h, b0, r, bar_s0);
   }
   if (warp == kMmaWarp) {
     ptx::tmem_alloc(s_tmem, kTmemCols);
@@ -242,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
   // reading rows at the same step cover all 32 banks.
   const int bb = tid >> 3, l = tid & 7, sx = bb & 1;
   const bool bval = bb < nb;  // false in the ancestry warp (bb >= 32)
-  uint2 kb2[NU], qb2[NU];  // this thread's elements of k_b and q_b, bf16
+  uint2 kb2[NUK], qb2[NUK];  // this thread's elements of k_b and q_b, bf16
   float kq = 0.f;
 
   if (warp == kAncWarp) {
@@ -343,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
     if (!ptx::mbar_wait(bar_s0, 0, p.wait_limit_ns)) ok = false;  // X and v visible to this thread
     // This thread's elements of k_b and q_b, and k_b . q_b.
 #pragma unroll
-    for (int u = 0; u < NU; ++u) {
+    for (int u = 0; u < NUK; ++u) {
       const int uu = u ^ sx;
       const uint32_t off = (uint32_t)(uu >> 1) * XA + (uint32_t)(l & 1) * 8u;
       const int c = 4 * (uu & 1) + (l >> 1);
@@ -363,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
     // memory (step j's own k input, or the key records), two depths per
     // pass, the next pass's loads in flight during this pass's arithmetic.
     if (!ptx::mbar_wait(bar_chain, 0, p.wait_limit_ns)) ok = false;
-    auto issue = [&](uint2 (&buf)[2][NU], int j0) {
+    auto issue = [&](uint2 (&buf)[2][NUK], int j0) {
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int j = j0 + e;
@@ -375,19 +384,19 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
                                          : rec_k + rec_row_slot(p, sl, r, h, a) * DK;
           const uint8_t *rb = reinterpret_cast<const uint8_t *>(row) + l * 8;
 #pragma unroll
-          for (int u = 0; u < NU; ++u) buf[e][u] = __ldg(reinterpret_cast<const uint2 *>(rb + (u ^ sx) * 64));
+          for (int u = 0; u < NUK; ++u) buf[e][u] = __ldg(reinterpret_cast<const uint2 *>(rb + (u ^ sx) * 64));
         } else {
 #pragma unroll
-          for (int u = 0; u < NU; ++u) buf[e][u] = make_uint2(0u, 0u);
+          for (int u = 0; u < NUK; ++u) buf[e][u] = make_uint2(0u, 0u);
         }
       }
     };
-    auto dots = [&](const uint2 (&buf)[2][NU], int j0) {
+    auto dots = [&](const uint2 (&buf)[2][NUK], int j0) {
       float dk[2], dq[2];
 #pragma unroll
       for (int e = 0; e < 2; ++e) dk[e] = 0.f, dq[e] = 0.f;
 #pragma unroll
-      for (int u = 0; u < NU; ++u) {
+      for (int u = 0; u < NUK; ++u) {
         const float4 kbu = bf16x4(kb2[u]), qbu = bf16x4(qb2[u]);
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
@@ -415,7 +424,7 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
       const int j = j0 + (int)b2;
       if ((l & 1) == 0 && bval && j < nanc) reinterpret_cast<float *>(s_c + bb * TM + j)[b1] = x;
     };
-    uint2 kA[2][NU], kB[2][NU];
+    uint2 kA[2][NUK], kB[2][NUK];
     if (nanc > 0) issue(kA, 0);
 #pragma unroll 1
     for (int j0 = 0; j0 < nanc; j0 += 4) {
@@ -439,8 +448,8 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
 #pragma unroll
           for (int n = 0; n < 32; ++n) s_d1[(half * 32 + n) * DV + ei] = d[n];
       }
-    } else {
-      // The key records of depth t, from X.
+    } else if (mt == 0) {
+      // The key records of depth t, from X (once per beam tile).
       for (int e = tid; e < kBT * NK * 8; e += 128) {
         const int n = e / (NK * 8), cc = e - n * (NK * 8);
         if (n < nb)
@@ -448,8 +457,8 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
               *reinterpret_cast<const uint4 *>(s_x + (cc >> 3) * XA + ptx::swz128(n, cc & 7));
       }
     }
-    // alpha, the ancestry row and the parent of the beam.
-    if (bval && l == 0) {
+    // alpha, the ancestry row and the parent of the beam (once per beam tile).
+    if (bval && l == 0 && mt == 0) {
       const int gb = b0 + bb;
       p.rec_alpha[rec_row_slot(p, tslot, r, h, gb)] = s_alpha[bb];
       if (h == 0) {
@@ -510,7 +519,7 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
       const int packed = s_list[lo + rr];
       const int j = packed & 31, sl = soff + j < TM ? soff + j : soff + j - TM;
       ptx::cp_async16(base + L.dst + (uint32_t)(rr * DV + c * 4) * 4u,
-                      p.rec_delta + rec_row_slot(p, sl, r, h, packed >> 5) * DV + c * 4, 16u);
+                      p.rec_delta + rec_row_slot(p, sl, r, h, packed >> 5) * DVT + e_off + c * 4, 16u);
     }
     ptx::cp_async_commit();
     ptx::cp_async_wait_all();
@@ -549,8 +558,8 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
   // --------------------------------------------------------- epilogue
   if (!ok) set_err(p.err, kErrByteTimeout);
   if (bval && ok) {
-    float4 *op = reinterpret_cast<float4 *>(p.o + (row0 + (int64_t)bb * H) * DV) + l;
-    float4 *dp = reinterpret_cast<float4 *>(p.rec_delta + rec_row_slot(p, tslot, r, h, b0 + bb) * DV) + l;
+    float4 *op = reinterpret_cast<float4 *>(p.o + (row0 + (int64_t)bb * H) * DVT + e_off) + l;
+    float4 *dp = reinterpret_cast<float4 *>(p.rec_delta + rec_row_slot(p, tslot, r, h, b0 + bb) * DVT + e_off) + l;
 #pragma unroll
     for (int u = 0; u < NU; ++u) {
       float4 d, o;
@@ -570,9 +579,10 @@ __global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_const
 
 __global__ void s0_image_kernel(const void *S0, uint4 *img, int R, int H, int dk, int dv, int s0_bf16,
                                 int planes) {
-  // One thread per (r, h, plane, K atom, row < 128, 16-byte chunk).
-  const int nk = dk / 64;
-  const int64_t total = (int64_t)R * H * planes * nk * kM * 8;
+  // Layout [r][h][M tile of 128 rows][plane][K atom][128 rows][128 B]; one
+  // thread per 16-byte chunk.  Rows past d_v are zero.
+  const int nk = dk / 64, nmt = (dv + kM - 1) / kM;
+  const int64_t total = (int64_t)R * H * nmt * planes * nk * kM * 8;
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
        e += (int64_t)gridDim.x * blockDim.x) {
     int64_t x = e;
@@ -580,13 +590,15 @@ __global__ void s0_image_kernel(const void *S0, uint4 *img, int R, int H, int dk
     const int row = (int)(x % kM); x /= kM;
     const int ka = (int)(x % nk); x /= nk;
     const int pl = (int)(x % planes); x /= planes;
+    const int mt = (int)(x % nmt); x /= nmt;
     const int64_t rh = x;
+    const int srow = mt * kM + row;
     __align__(16) __nv_bfloat16 out[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       float s = 0.f;
-      if (row < dv) {
-        const int64_t si = (rh * dv + row) * dk + ka * 64 + c * 8 + u;
+      if (srow < dv) {
+        const int64_t si = (rh * dv + srow) * dk + ka * 64 + c * 8 + u;
         s = s0_bf16 ? __bfloat162float(static_cast<const __nv_bfloat16 *>(S0)[si])
                     : static_cast<const float *>(S0)[si];
       }
@@ -600,7 +612,7 @@ __global__ void s0_image_kernel(const void *S0, uint4 *img, int R, int H, int dk
       }
       out[u] = term;
     }
-    const int64_t off = ((rh * planes + pl) * nk + ka) * (kM * 128) + ptx::swz128(row, c);
+    const int64_t off = (((rh * nmt + mt) * planes + pl) * nk + ka) * (kM * 128) + ptx::swz128(row, c);
     img[off / 16] = *reinterpret_cast<const uint4 *>(out);
   }
 }
@@ -635,18 +647,18 @@ bool encode_rows(CUtensorMap *m, const void *base, int d, int H, int W, int R, i
 
 namespace {
 
-template <int DK>
+template <int DK, int DV>
 cudaError_t launch_dk(const StepParams &p_in, bool pdl, cudaStream_t s) {
   StepParams p = p_in;
   if (!encode_rows(&p.tm_k, p.k, DK, p.H, p.W, p.R) || !encode_rows(&p.tm_q, p.q, DK, p.H, p.W, p.R) ||
       !encode_rows(&p.tm_v, p.v, DK, p.H, p.W, p.R))
     return cudaErrorInvalidValue;
-  const Layout L = layout(DK / 64, p.s0_planes, p.T_max, p.W_max, p.hist_cap);
+  const Layout L = layout(DK / 64, DV / 64, p.s0_planes, p.T_max, p.W_max, p.hist_cap);
   const size_t smem = L.total + 1024;
-  cudaError_t e = ensure_smem_limit((const void *)step_tc_kernel<DK>, smem);
+  cudaError_t e = ensure_smem_limit((const void *)step_tc_kernel<DK, DV>, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((p.W + kBT - 1) / kBT, p.H, p.R);
+  cfg.gridDim = dim3((p.W + kBT - 1) / kBT, p.H, p.R * (p.dv / DV));
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
@@ -655,23 +667,25 @@ cudaError_t launch_dk(const StepParams &p_in, bool pdl, cudaStream_t s) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, step_tc_kernel<DK>, p);
+  return cudaLaunchKernelEx(&cfg, step_tc_kernel<DK, DV>, p);
 }
 
 }  // namespace
 
-bool tc_supports(int dk, int dv, int qkv_bf16, int T_max, int W_max) {
-  return qkv_bf16 && dk == dv && (dk == 64 || dk == 128) && T_max <= kMaxT && W_max <= kMaxW;
+bool tc_supports(int dk, int dv, int qkv_bf16, int T_max, int W_max, int planes) {
+  // d = 256: one CTA per half of the rows of S keeps a 128 KB image (two
+  // bf16 terms at most).
+  return qkv_bf16 && dk == dv && (dk == 64 || dk == 128 || (dk == 256 && planes <= 2)) && T_max <= kMaxT &&
+         W_max <= kMaxW;
 }
 
 size_t s0_image_bytes(int R, int H, int dk, int dv, int planes) {
-  (void)dv;
-  return (size_t)R * H * planes * (dk / 64) * 16384u;
+  return (size_t)R * H * ((dv + kM - 1) / kM) * planes * (dk / 64) * 16384u;
 }
 
 cudaError_t launch_s0_image(const void *S0, void *img, int R, int H, int dk, int dv, int s0_bf16, int planes,
                             cudaStream_t s) {
-  const int64_t total = (int64_t)R * H * planes * (dk / 64) * kM * 8;
+  const int64_t total = (int64_t)R * H * ((dv + kM - 1) / kM) * planes * (dk / 64) * kM * 8;
   const int threads = 256;
   const int64_t want = (total + threads - 1) / threads;
   const int blocks = (int)(want < 148 * 16 ? want : 148 * 16);
@@ -682,8 +696,9 @@ cudaError_t launch_s0_image(const void *S0, void *img, int R, int H, int dk, int
 cudaError_t launch_step_tc(const StepParams &p, int pdl, cudaStream_t s) {
   if (p.T_max > kMaxT || p.W_max > kMaxW || p.s0_planes < 1 || p.s0_planes > 3 || p.hist_cap > kHistMaxInts)
     return cudaErrorNotSupported;
-  if (p.dk == 64 && p.dv == 64) return launch_dk<64>(p, pdl != 0, s);
-  if (p.dk == 128 && p.dv == 128) return launch_dk<128>(p, pdl != 0, s);
+  if (p.dk == 64 && p.dv == 64) return launch_dk<64, 64>(p, pdl != 0, s);
+  if (p.dk == 128 && p.dv == 128) return launch_dk<128, 128>(p, pdl != 0, s);
+  if (p.dk == 256 && p.dv == 256 && p.s0_planes <= 2) return launch_dk<256, 128>(p, pdl != 0, s);
   return cudaErrorNotSupported;
 }
 

@@ -15,7 +15,7 @@ pytestmark = pytest.mark.gpu
 def kernels_for(dk, dv, qkv):
     import linear_attention_beam_shared_b200 as L
     ks = [L.ONELA_KERNEL_SIMT]
-    if qkv == "bf16" and dk == dv and dk in (64, 128) and _tc_available():
+    if qkv == "bf16" and dk == dv and dk in (64, 128, 256) and _tc_available():
         ks.append(L.ONELA_KERNEL_TC)
     return ks
 
@@ -316,3 +316,28 @@ def test_host_side_errors():
         assert dec.status() == 0
     finally:
         dec.close()
+
+
+@pytest.mark.parametrize("s0_dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("W,T,R,H", [(256, 7, 1, 4), (129, 4, 2, 3), (32, 1, 1, 2)])
+def test_tc_d256(s0_dtype, W, T, R, H):
+    """d_k = d_v = 256 on the tensor cores (two CTAs per beam tile, one per
+    half of the rows of S), whole decodes against the fp64 oracle."""
+    import linear_attention_beam_shared_b200 as L
+    wl, S0, steps = P.custom_steps(60 + W + T, R, H, 256, 256, (W,) * T, parents="mixed" if R > 1 else "zipf")
+    S0c = synth.cast_state(S0, s0_dtype)
+    gpu, kind = P.run_gpu(S0c, steps, "bf16", L.ONELA_KERNEL_TC)
+    assert kind == L.ONELA_KERNEL_TC
+    P.compare(gpu, P.oracle(S0c, steps), steps, s0_dtype)
+
+
+def test_tc_d256_three_terms_are_refused():
+    """A three-term split of an fp32 S0 does not fit one CTA at d = 256: the
+    tensor-core kernel refuses it and AUTO picks the general kernel."""
+    import linear_attention_beam_shared_b200 as L
+    with pytest.raises(L.OnelaError) as e:
+        L.onela_create(1, 2, 256, 256, 32, 3, "f32", "bf16", L.ONELA_KERNEL_TC, s0_split=3)
+    assert e.value.code == L.ONELA_ERR_UNSUPPORTED
+    h = L.onela_create(1, 2, 256, 256, 32, 3, "f32", "bf16", L.ONELA_KERNEL_AUTO, s0_split=3)
+    assert L.onela_kernel_kind(h) == L.ONELA_KERNEL_SIMT
+    L.onela_destroy(h)

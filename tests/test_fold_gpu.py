@@ -387,3 +387,21 @@ def test_single_beam_decode_through_a_small_store(kind):
     ref = P.oracle(S0t, steps)
     for t, (g, r) in enumerate(zip(gpu, ref), start=1):
         assert float(np.abs(g["o"].double().numpy() - r["o"]).max()) <= P.TOL["f32"], t
+
+
+def test_fold_tc_d256():
+    """Folding on a d = 256 tensor-core handle (the general fold, then the
+    folded state's operand image): outputs against the unfolded oracle."""
+    import linear_attention_beam_shared_b200 as L
+    wl, S0, steps = P.custom_steps(33, R=1, H=2, dk=256, dv=256, Ws=[40, 64, 33, 64, 50], parents="uniform")
+    steps = narrow(steps, 1, [5])
+    steps = narrow(steps, 3, [7])
+    folds = {3: 8, 5: 8}
+    S0t = synth.cast_state(S0, "f32")
+    gpu, info, used = run_with_folds(S0t, steps, "bf16", L.ONELA_KERNEL_TC, folds)
+    assert used == L.ONELA_KERNEL_TC
+    want = expected_depths(steps, folds)
+    for t, D, S in info:
+        assert D.tolist() == want[t].tolist()
+        check_state(S, gdn.fold_state(S0t, steps[:t], want[t]))
+    P.compare(gpu, P.oracle(S0t, steps), steps, "f32")
