@@ -404,9 +404,9 @@ def time_sweep(device, stream, flush, reps=10, warmup=3):
         dec = L.BeamDecoder(wl.R, wl.H, wl.d_k, wl.d_v, wl.W, wl.T, wl.s0_dtype, wl.qkv_dtype,
                             device=device.index)
         dec.set_prompt_state(S0.to(device))
-        g, launches = decode_graph(dec, ds, outs, stream)
+        g, launches, ev = decode_graph(dec, ds, outs, stream, flush=flush)
         kind = {L.ONELA_KERNEL_SIMT: "simt", L.ONELA_KERNEL_TC: "tc"}[dec.kernel]
-        ms = time_graph(g, stream, flush, reps, warmup)
+        ms = time_graph(g, stream, flush, reps, warmup, ev=ev)
         del g
         assert dec.status() == 0
         dec.close()
@@ -417,7 +417,7 @@ def time_sweep(device, stream, flush, reps=10, warmup=3):
                        "achieved_gbs": round(gbs, 1), "frac": round(gbs / hbm, 4),
                        "capacity_ratio": capacity(wl)["ratio"]})
         del ds, outs
-    return {"unit": UNIT, "peak_gbs": hbm, "l2": "flushed before every decode", "points": points}
+    return {"unit": UNIT, "peak_gbs": hbm, "l2": "flushed (512 MiB write) before every decode; decode timed by events inside its graph", "points": points}
 
 
 def grid_inputs(R, H, d, W, T, device, seed):
@@ -479,9 +479,9 @@ def time_grid(device, stream, flush, reps=3, warmup=1, full=True):
                         outs = [torch.empty((R, W, H, d), dtype=torch.float32, device=device) for _ in ds]
                         dec = L.BeamDecoder(R, H, d, d, W, T, "f32", "bf16", device=device.index)
                         dec.set_prompt_state(S0)
-                        g, launches = decode_graph(dec, ds, outs, stream)
+                        g, launches, ev = decode_graph(dec, ds, outs, stream, flush=flush)
                         kind = {L.ONELA_KERNEL_SIMT: "simt", L.ONELA_KERNEL_TC: "tc"}[dec.kernel]
-                        ms = time_graph(g, stream, flush, reps, warmup)
+                        ms = time_graph(g, stream, flush, reps, warmup, ev=ev)
                         del g
                         assert dec.status() == 0
                         dec.close()
@@ -502,10 +502,13 @@ def time_grid(device, stream, flush, reps=3, warmup=1, full=True):
             "summary": summary, "rows": rows}
 
 
-def decode_graph(dec, dsteps, outs, stream, per_step=False):
+def decode_graph(dec, dsteps, outs, stream, per_step=False, flush=None):
     """One whole decode through the public API captured in a CUDA graph: one
     onela_decode_steps call, or (per_step) one onela_decode_step call per
-    step.  Returns (graph, kernel launches per decode)."""
+    step.  With flush: the graph is [512 MiB write that flushes L2] [start
+    event] [the decode] [end event], so that the events time the decode's
+    kernels on the device and not the launch of the graph.  Returns (graph,
+    kernel launches per decode, (start, end) events or None)."""
     def run():
         if per_step:
             for st, o in zip(dsteps, outs):
@@ -519,29 +522,50 @@ def decode_graph(dec, dsteps, outs, stream, per_step=False):
     launches = len(dsteps) if per_step else dec.last_launches()
     dec.reset(stream)
     graph = torch.cuda.CUDAGraph()
+    ev = None
     with torch.cuda.graph(graph, stream=stream):
+        if flush is not None:
+            # External events: real event-record nodes in the graph (not the
+            # capture's internal dependencies), readable after each replay.
+            ev = (torch.cuda.Event(enable_timing=True, external=True),
+                  torch.cuda.Event(enable_timing=True, external=True))
+            flush.fill_(1)
+            ev[0].record(stream)
         run()
+        if flush is not None:
+            ev[1].record(stream)
     dec.reset(stream)
-    return graph, launches
+    return graph, launches, ev
 
 
-def time_graph(graph, stream, flush, reps, warmup):
-    """Mean device time (ms, max over ranks) of graph replays, each after a
-    512 MiB write that flushes L2, timed with CUDA events on the stream."""
+def time_graph(graph, stream, flush, reps, warmup, ev=None):
+    """Mean device time (ms, max over ranks) of a decode.  ev given (a graph
+    from decode_graph with flush): each replay writes 512 MiB and times the
+    decode between its own events.  Otherwise each replay follows a 512 MiB
+    write and is timed from outside, graph launch included."""
     with torch.cuda.stream(stream):
         for _ in range(warmup):
-            flush.fill_(9)
+            if ev is None:
+                flush.fill_(9)
             graph.replay()
     stream.synchronize()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    total = 0.0
+    if ev is not None:
+        for _ in range(reps):
+            with torch.cuda.stream(stream):
+                graph.replay()
+            stream.synchronize()
+            total += ev[0].elapsed_time(ev[1])
+        return max_over_ranks(total / reps, stream.device)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
     with torch.cuda.stream(stream):
-        for i, (e0, e1) in enumerate(ev):
+        for i, (e0, e1) in enumerate(evs):
             flush.fill_(i & 0xFF)
             e0.record(stream)
             graph.replay()
             e1.record(stream)
     stream.synchronize()
-    return max_over_ranks(sum(e0.elapsed_time(e1) for e0, e1 in ev) / reps, stream.device)
+    return max_over_ranks(sum(e0.elapsed_time(e1) for e0, e1 in evs) / reps, stream.device)
 
 
 def byte_model(wl, steps):
@@ -686,38 +710,39 @@ def run_ours(args):
     outs = [torch.empty((wl.R, s["W"], wl.H, wl.d_v), dtype=torch.float32, device=device) for s in steps]
 
     stream = torch.cuda.Stream(device=device)
-    # Eager warm-up of the API (also loads the module), then capture.
-    graph, launches = decode_graph(dec, dsteps, outs, stream)
-    kind = {L.ONELA_KERNEL_SIMT: "simt", L.ONELA_KERNEL_TC: "tc"}[dec.kernel]
-
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=device)
-    for _ in range(args.warmup):
-        with torch.cuda.stream(stream):
-            flush.fill_(1)
+    # Eager warm-up of the API (also loads the module), then capture: each
+    # replay writes 512 MiB (flushing L2), then the decode runs between two
+    # events recorded inside the graph.
+    graph, launches, ev = decode_graph(dec, dsteps, outs, stream, flush=flush)
+    kind = {L.ONELA_KERNEL_SIMT: "simt", L.ONELA_KERNEL_TC: "tc"}[dec.kernel]
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
             graph.replay()
     stream.synchronize()
 
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     if ws > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
+    times_ms = []
     with ClockSampler(device.index) as clk:
-        with torch.cuda.stream(stream):
-            for i in range(args.steps):
-                flush.fill_(i & 0xFF)
-                starts[i].record(stream)
+        for i in range(args.steps):
+            with torch.cuda.stream(stream):
                 graph.replay()
-                ends[i].record(stream)
+            stream.synchronize()
+            times_ms.append(ev[0].elapsed_time(ev[1]))
         torch.cuda.synchronize()
     if ws > 1:
         torch.distributed.barrier()
-    times_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = max_over_ranks(sum(times_ms), device)
     assert dec.status() == 0
     ms_per_step = total_ms / args.steps
     value = whole_job_value(wl.units, ws, ms_per_step)
     del graph
+    # The same decode timed from outside its graph (graph launch included).
+    graph2, _, _ = decode_graph(dec, dsteps, outs, stream)
+    ms_incl_launch = time_graph(graph2, stream, flush, reps=min(args.steps, 50), warmup=3)
+    del graph2
     dec.close()
 
     # Roofline of the decode kernel (the only kernel in the step).
@@ -749,8 +774,8 @@ def run_ours(args):
             d2 = L.BeamDecoder(wl.R, wl.H, wl.d_k, wl.d_v, wl.W, wl.T, wl.s0_dtype, wl.qkv_dtype,
                                kernel=kernel, device=device.index, flags=fl)
             d2.set_prompt_state(S0.to(device))
-            g2, n2 = decode_graph(d2, dsteps, outs, stream, per_step=True)
-            ms2 = time_graph(g2, stream, flush, reps=20, warmup=3)
+            g2, n2, ev2 = decode_graph(d2, dsteps, outs, stream, per_step=True, flush=flush)
+            ms2 = time_graph(g2, stream, flush, reps=20, warmup=3, ev=ev2)
             del g2
             assert d2.status() == 0
             d2.close()
@@ -854,12 +879,13 @@ def run_ours(args):
                                    f"W={wl.W}, T={wl.T}, L_prompt={wl.L_prompt}, S0 {wl.s0_dtype}, "
                                    f"q/k/v {wl.qkv_dtype}, parents Zipf(1.1)",
                        "global_batch": wl.R * ws, "seq_len": wl.T, "parallelism": f"replicas{ws}",
-                       "l2": "flushed (512 MiB write) before every timed step", "kernel": kind,
+                       "l2": "flushed (512 MiB write inside the graph, before the start event) before every timed step", "kernel": kind,
                        "step": f"one whole {wl.T}-step decode (one onela_decode_steps call) in a CUDA graph",
                        "launches_per_decode": launches},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "clocks": clk.summary(), "gpu_launches": launches * args.steps,
             "variants": variants, "capacity": capacity(wl),
+            "ms_per_step_graph_launch_included": round(ms_incl_launch, 6),
             "prefill": prefill, "beam_select": select, "fold": fold, "sweep": sweep, "grid": grid,
         }
         print(json.dumps(line))
@@ -917,7 +943,7 @@ def main():
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill, beam-selection and fold timings")
     ap.add_argument("--no-sweep", action="store_true", help="skip the beam-width and request sweeps")
     ap.add_argument("--no-grid", action="store_true", help="skip the multi-request shape grid")
-    ap.add_argument("--grid-r1", action="store_true", help="the shape grid at R = 1 only")
+    ap.add_argument("--grid-r1", action="store_true", help="the shape grid at R = 1 only (the default runs R = 1, 8, 32)")
     ap.add_argument("--s0", choices=["prefill", "direct"], default="prefill",
                     help="S0 from the GDN recurrence over the synthetic prompt (default) or drawn "
                          "directly; the decode's work does not depend on the S0 values")

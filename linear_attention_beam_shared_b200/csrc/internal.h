@@ -72,6 +72,7 @@ struct StepParams {
   alignas(64) CUtensorMap tm_k;
   alignas(64) CUtensorMap tm_q;
   alignas(64) CUtensorMap tm_v;
+
 };
 
 // Slot of depth s (1-based) in the record store, the parents store and the

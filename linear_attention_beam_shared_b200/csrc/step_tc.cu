@@ -206,6 +206,7 @@ __global__ void __launch_bounds__(kThreads, DK <= 128 ? 2 : 1) step_tc_kernel(co
   }
   // Before its wait this kernel reads inputs only, so the next step may start.
   ptx::pdl_launch_dependents();
+
   int par = 0;
   float g_alpha = 0.f, g_beta = 0.f;
   if (warp == kAncWarp) {
@@ -653,6 +654,7 @@ cudaError_t launch_dk(const StepParams &p_in, bool pdl, cudaStream_t s) {
   if (!encode_rows(&p.tm_k, p.k, DK, p.H, p.W, p.R) || !encode_rows(&p.tm_q, p.q, DK, p.H, p.W, p.R) ||
       !encode_rows(&p.tm_v, p.v, DK, p.H, p.W, p.R))
     return cudaErrorInvalidValue;
+
   const Layout L = layout(DK / 64, DV / 64, p.s0_planes, p.T_max, p.W_max, p.hist_cap);
   const size_t smem = L.total + 1024;
   cudaError_t e = ensure_smem_limit((const void *)step_tc_kernel<DK, DV>, smem);
