@@ -174,6 +174,18 @@ ONELA_API int onela_set_prompt_state(onela_handle *h, const void *S0, onela_stre
  *   beta     [R][L][H] fp32.
  * Rewinds the decode to step 0.  The inputs may be freed once the stream has
  * passed the call.
+ * Tensor-core handles with bf16 k and v, d_k = d_v in {64, 128} and k, v on
+ * 16-byte boundaries take the prompt in chunks of 64 tokens: per chunk the
+ * intra-chunk system (I + A) Delta = Z of the delta rule is solved once from
+ * the keys and gates, and the state advances by three tensor-core products
+ * (operands split into bf16 terms, fp32 accumulation: the same result as
+ * the token-by-token recurrence up to rounding order); the prompt is cut
+ * into segments that run side by side and are combined through their
+ * transition matrices (onela_set_prefill_segments).  This path keeps a
+ * workspace of about 25 KB per (request, head, chunk) on the handle, which
+ * the first call that needs more allocates (cudaMalloc, synchronous: not
+ * inside a stream capture).  Every other handle runs the recurrence token by
+ * token.
  * Errors: ONELA_ERR_ARG, ONELA_ERR_CUDA. */
 ONELA_API int onela_prefill(onela_handle *h, int32_t L, const void *k, const void *v,
                             const float *g, const float *beta, onela_stream stream);
@@ -256,6 +268,15 @@ ONELA_API int onela_decode_steps(onela_handle *h, int32_t n, const int32_t *W,
  * (nothing faults or hangs); stall = 0 restores normal operation.
  * Errors: ONELA_ERR_ARG. */
 ONELA_API int onela_set_wait_policy(onela_handle *h, uint64_t limit_ns, int32_t stall);
+
+/* Number of segments the chunked tensor-core prefill cuts a prompt into
+ * (1 .. 16; 0, the default, chooses one CTA per segment chain on every SM, at
+ * least 4 chunks per segment).  A segment of n chunks costs one chain of n
+ * sequential chunk updates; segments after the first also run the chain of
+ * their transition matrix, and the combine costs one d x d x d product per
+ * later segment.  Fewer segments than asked are used when the prompt has
+ * fewer chunks.  Errors: ONELA_ERR_ARG. */
+ONELA_API int onela_set_prefill_segments(onela_handle *h, int32_t segments);
 
 /* Beam selection on the device: the next beam set out of the children of
  * the current one (the evolving beam tree of the abstract), so that the
@@ -365,8 +386,11 @@ ONELA_API int onela_read_ancestry(onela_handle *h, int32_t t, int32_t *anc,
  * the handle runs (ONELA_KERNEL_SIMT or ONELA_KERNEL_TC). */
 ONELA_API int onela_steps_done(const onela_handle *h);
 ONELA_API int onela_kernel_kind(const onela_handle *h);
-/* Query: kernel launches the last successful decode call enqueued
- * (onela_decode_step: 1; onela_decode_steps: n; 0 before any call). */
+/* Query: kernel launches the last successful decode or prefill call enqueued
+ * (onela_decode_step: 1; onela_decode_steps: n; onela_prefill: 4 on the
+ * chunked tensor-core path, 2 on the token-by-token path of a tensor-core
+ * handle (the recurrence, then the S0 operand image), 1 otherwise; 0 before
+ * any call). */
 ONELA_API int onela_last_call_launches(const onela_handle *h);
 
 /* Decode step without any device allocation.

@@ -21,7 +21,7 @@ from ._lib import (  # noqa: F401
     ONELA_BF16, ONELA_ERR_ARG, ONELA_ERR_CAPACITY, ONELA_ERR_CUDA, ONELA_ERR_PARENT,
     ONELA_ERR_STATE, ONELA_ERR_UNSUPPORTED, ONELA_F32, ONELA_FLAG_NVTX, ONELA_FLAG_PDL, ONELA_KERNEL_AUTO, ONELA_KERNEL_SIMT,
     ONELA_ERR_SCRATCH, ONELA_ERR_TIMEOUT, ONELA_KERNEL_TC, ONELA_OK, Handle, OnelaError, error_string, onela_create,
-    onela_decode_step, onela_decode_step_noalloc, onela_decode_steps, onela_set_wait_policy, onela_destroy, onela_fold, onela_kernel_kind, onela_last_call_launches, onela_prefill,
+    onela_decode_step, onela_decode_step_noalloc, onela_decode_steps, onela_set_wait_policy, onela_set_prefill_segments, onela_destroy, onela_fold, onela_kernel_kind, onela_last_call_launches, onela_prefill,
     onela_read_ancestry, onela_read_fold_depth, onela_read_prompt_state, onela_read_records,
     onela_read_root_state, onela_reset, onela_select_beams, onela_set_prompt_state,
     onela_status, onela_status_code, onela_steps_done,
@@ -81,8 +81,12 @@ class BeamDecoder:
             self.Ws.append(W)
         return outs
 
+    def prefill_segments(self, segments: int) -> None:
+        """Segments of the chunked tensor-core prefill (0: automatic)."""
+        onela_set_prefill_segments(self.h, segments)
+
     def last_launches(self) -> int:
-        """Kernel launches of the last decode call."""
+        """Kernel launches of the last decode or prefill call."""
         return onela_last_call_launches(self.h)
 
     def reset(self, stream=None):

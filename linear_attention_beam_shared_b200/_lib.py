@@ -59,6 +59,7 @@ def _load() -> ctypes.CDLL:
         "onela_decode_step": ([vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         "onela_decode_steps": ([vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         "onela_set_wait_policy": ([vp, ctypes.c_uint64, i32], ctypes.c_int),
+        "onela_set_prefill_segments": ([vp, i32], ctypes.c_int),
         "onela_reset": ([vp, vp], ctypes.c_int),
         "onela_fold": ([vp, i32, vp], ctypes.c_int),
         "onela_read_root_state": ([vp, vp, vp], ctypes.c_int),
@@ -241,6 +242,10 @@ def onela_decode_steps(h: Handle, steps, outs, stream=None) -> None:
 
 def onela_set_wait_policy(h: Handle, limit_ns: int, stall: bool = False) -> None:
     _check(lib.onela_set_wait_policy(h.ptr, int(limit_ns), 1 if stall else 0), "onela_set_wait_policy")
+
+
+def onela_set_prefill_segments(h: Handle, segments: int) -> None:
+    _check(lib.onela_set_prefill_segments(h.ptr, int(segments)), "onela_set_prefill_segments")
 
 
 def onela_reset(h: Handle, stream=None) -> None:

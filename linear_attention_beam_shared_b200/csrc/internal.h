@@ -145,6 +145,21 @@ size_t s0_image_bytes(int R, int H, int dk, int dv, int planes);
 cudaError_t launch_prefill(const void *k, const void *v, const float *g, const float *beta, void *S0, int R, int L,
                            int H, int dk, int dv, int qkv_bf16, int s0_bf16, cudaStream_t s);
 bool tc_supports(int dk, int dv, int qkv_bf16, int T_max, int W_max, int planes);
+// The same recurrence in 64-token chunks on the tensor cores (prefill_tc.cu)
+// for bf16 k and v with d_k = d_v = d in {64, 128}, k and v 16-byte aligned:
+// the prompt is cut into nseg segments whose chains run side by side (one CTA
+// per segment for the values, one more per later segment for its transition
+// matrix) and are then combined.  ws holds prefill_tc_ws_bytes(R, L, H, d,
+// nseg) bytes, 16-byte aligned; a wait that runs out sets the timeout byte of
+// err.  Three launches.
+constexpr int kMaxPrefillSegments = 16;
+bool prefill_tc_supports(int dk, int dv, int qkv_bf16);
+int prefill_tc_segments(int R, int L, int H, int want);  // want <= 0: chosen for the SM count
+size_t prefill_tc_prep_bytes(int R, int L, int H);
+size_t prefill_tc_ws_bytes(int R, int L, int H, int d, int nseg);
+cudaError_t launch_prefill_tc(const void *k, const void *v, const float *g, const float *beta, void *S0, int R, int L,
+                              int H, int d, int s0_bf16, int nseg, void *ws, unsigned long long wait_ns, int32_t *err,
+                              cudaStream_t s);
 
 // Beam selection (select.cu): the W best of W_prev x C candidates per request.
 size_t select_scratch_bytes(int R, int W_prev, int C, int W);

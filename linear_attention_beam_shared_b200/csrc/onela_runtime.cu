@@ -51,7 +51,12 @@ struct onela_handle {
   // aid of onela_set_wait_policy.
   unsigned long long wait_limit_ns;
   int stall;
-  int last_launches;  // kernel launches of the last decode call
+  int last_launches;  // kernel launches of the last decode or prefill call
+  // Chunked tensor-core prefill: its workspace (grown on demand) and the
+  // number of prompt segments asked for (0: chosen from the SM count).
+  void *pf_ws;
+  size_t pf_ws_bytes;
+  int pf_segments;
 };
 
 namespace {
@@ -111,6 +116,7 @@ void free_all(onela_handle *h) {
   cudaFree(h->rec_delta);
   cudaFree(h->rec_k);
   cudaFree(h->anc);
+  cudaFree(h->pf_ws);
   if (h->err_host) cudaFreeHost(h->err_host);
 }
 
@@ -282,11 +288,37 @@ int onela_prefill(onela_handle *h, int32_t L, const void *k, const void *v, cons
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const onela_config &c = h->cfg;
   NvtxRange nvtx(c, "prefill", 0);
-  if (onela::launch_prefill(k, v, gate, beta, h->S0, c.R, L, c.H, c.d_k, c.d_v, c.qkv_dtype == ONELA_BF16,
-                            c.s0_dtype == ONELA_BF16, s) != cudaSuccess) {
+  const bool aligned = ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v)) & 15u) == 0;
+  int launches = 1;
+  if (h->kernel == ONELA_KERNEL_TC && aligned &&
+      onela::prefill_tc_supports(c.d_k, c.d_v, c.qkv_dtype == ONELA_BF16)) {
+    // Chunked on the tensor cores.
+    const int nseg = onela::prefill_tc_segments(c.R, L, c.H, h->pf_segments);
+    const size_t need = onela::prefill_tc_ws_bytes(c.R, L, c.H, c.d_k, nseg);
+    if (need > h->pf_ws_bytes) {
+      // The old workspace may still be in use by work queued earlier.
+      if (h->pf_ws && cudaStreamSynchronize(s) != cudaSuccess) return ONELA_ERR_CUDA;
+      cudaFree(h->pf_ws);
+      h->pf_ws = nullptr;
+      h->pf_ws_bytes = 0;
+      if (cudaMalloc(&h->pf_ws, need) != cudaSuccess) {
+        cudaGetLastError();
+        return ONELA_ERR_CUDA;
+      }
+      h->pf_ws_bytes = need;
+    }
+    if (onela::launch_prefill_tc(k, v, gate, beta, h->S0, c.R, L, c.H, c.d_k, c.s0_dtype == ONELA_BF16, nseg,
+                                 h->pf_ws, h->wait_limit_ns, h->err_dev, s) != cudaSuccess) {
+      cudaGetLastError();
+      return ONELA_ERR_CUDA;
+    }
+    launches = 3;
+  } else if (onela::launch_prefill(k, v, gate, beta, h->S0, c.R, L, c.H, c.d_k, c.d_v, c.qkv_dtype == ONELA_BF16,
+                                   c.s0_dtype == ONELA_BF16, s) != cudaSuccess) {
     cudaGetLastError();
     return ONELA_ERR_CUDA;
   }
+  h->last_launches = launches + (h->kernel == ONELA_KERNEL_TC ? 1 : 0);
   if (h->kernel == ONELA_KERNEL_TC) {
     if (onela::launch_s0_image(h->S0, h->S0img, c.R, c.H, c.d_k, c.d_v, c.s0_dtype == ONELA_BF16, h->planes, s) !=
         cudaSuccess)
@@ -481,6 +513,12 @@ int onela_set_wait_policy(onela_handle *h, uint64_t limit_ns, int32_t stall) {
   if (!h || limit_ns < 1000 || limit_ns > 10000000000ull) return ONELA_ERR_ARG;
   h->wait_limit_ns = limit_ns;
   h->stall = stall != 0;
+  return ONELA_OK;
+}
+
+int onela_set_prefill_segments(onela_handle *h, int32_t segments) {
+  if (!h || segments < 0 || segments > onela::kMaxPrefillSegments) return ONELA_ERR_ARG;
+  h->pf_segments = segments;
   return ONELA_OK;
 }
 

@@ -219,6 +219,7 @@ __device__ __forceinline__ void mma_commit(uint64_t *bar) {
 }
 
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // Shared-memory matrix descriptor, K-major, 128-byte swizzle: rows of 128 B
 // (64 bf16 of K), 8-row atoms of 1024 B stacked densely (stride 1024 B).

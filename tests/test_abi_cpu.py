@@ -78,6 +78,8 @@ def test_null_arguments_are_rejected():
     assert lib.onela_fold(None, 3, None) == L.ONELA_ERR_ARG
     assert lib.onela_read_root_state(None, None, None) == L.ONELA_ERR_ARG
     assert lib.onela_read_fold_depth(None, None, None) == L.ONELA_ERR_ARG
+    assert lib.onela_set_prefill_segments(None, 0) == L.ONELA_ERR_ARG
+    assert lib.onela_set_wait_policy(None, 10**9, 0) == L.ONELA_ERR_ARG
     assert lib.onela_steps_done(None) == -1
     assert lib.onela_select_beams(1, 4, 4, 2, *([None] * 6), 0, 0, None) == L.ONELA_ERR_ARG
 

@@ -12,6 +12,13 @@ error stays near sqrt(1000) x 2^-24 x max|S|, about 2e-6 x max|S|.  The test
 allows 1e-5 x max(1, max|S|) (five times that) as max-abs error; a bf16 S0
 is the fp32 result rounded once, so it may differ from the rounded oracle by
 one bf16 unit where the fp32 value lies next to a rounding boundary.
+
+Tensor-core handles (bf16 k and v, d_k = d_v in {64, 128}) take the prompt in
+chunks of 64 tokens.  There every tensor-core operand that is not a bf16
+value enters as three bf16 terms (relative residual about 2^-24, as fp32
+rounding) with fp32 accumulation, and the segments are combined in fp32, so
+the same tolerance holds; the tests below check that this path ran (its
+launch count) and hold it to the oracle at that tolerance.
 """
 import numpy as np
 import pytest
@@ -106,6 +113,7 @@ def test_prefill_full_size_then_decode(name):
     dev, ref = prompt_inputs(wl)
     S, h = gpu_prefill(wl, dev)
     try:
+        assert h.last_launches() == 4  # the chunked tensor-core path
         check_state(S, gdn.prefill(ref["k"], ref["v"], ref["a"], ref["b"]), wl.s0_dtype)
         steps = synth.draw_decode(wl)
         ds = P.to_dev(steps)
@@ -132,5 +140,84 @@ def test_prefill_rewinds_the_decode():
         h.prefill(dev["k"], dev["v"], dev["g"], dev["beta"])
         assert L.onela_steps_done(h.h) == 0
         torch.testing.assert_close(h.prompt_state().cpu(), S, rtol=0, atol=0)
+    finally:
+        h.close()
+
+
+def _tc_prefill(wl, dev, segments):
+    import linear_attention_beam_shared_b200 as L
+    h = L.BeamDecoder(wl.R, wl.H, wl.d_k, wl.d_v, wl.W, wl.T, wl.s0_dtype, wl.qkv_dtype, kernel=L.ONELA_KERNEL_TC)
+    try:
+        h.prefill_segments(segments)
+        h.prefill(dev["k"], dev["v"], dev["g"], dev["beta"])
+        launches = h.last_launches()
+        S = h.prompt_state()
+        torch.cuda.synchronize()
+        assert h.status() == 0
+        return S.cpu(), launches
+    finally:
+        h.close()
+
+
+@pytest.mark.parametrize("s0", ["f32", "bf16"])
+@pytest.mark.parametrize("shape,segments", [
+    ((1, 2, 128, 1), 0), ((1, 2, 128, 63), 0), ((1, 2, 128, 64), 1), ((2, 3, 128, 65), 2),
+    ((1, 1, 64, 200), 3), ((2, 2, 64, 130), 0), ((1, 2, 128, 1000), 16), ((1, 3, 128, 777), 5),
+])
+def test_prefill_tc_chunked(shape, segments, s0):
+    """The chunked tensor-core prefill (four launches: the per-chunk solve,
+    the segment chains, their combination, the S0 image): a single token, a
+    ragged last chunk, one exact chunk, one token past it, several requests
+    and heads, d = 64 (rows past d_v zero in the 128-row MMA), more segments
+    asked for than the prompt has chunks, an uneven split into segments."""
+    R, H, d, Lp = shape
+    wl = synth.Workload("pftc", R=R, H=H, d_k=d, d_v=d, W=8, T=3, L_prompt=Lp, s0_dtype=s0, qkv_dtype="bf16",
+                        parents="uniform", seed_id=13)
+    dev, ref = prompt_inputs(wl)
+    S, launches = _tc_prefill(wl, dev, segments)
+    assert launches == 4
+    check_state(S, gdn.prefill(ref["k"], ref["v"], ref["a"], ref["b"]), s0)
+
+
+def test_prefill_tc_segments_agree():
+    """Every way of cutting the prompt into segments gives the state within
+    the fp32 tolerance of the others (the combination through the transition
+    matrices is exact up to rounding)."""
+    wl = synth.Workload("pftc2", R=1, H=2, d_k=128, d_v=128, W=8, T=3, L_prompt=1500, s0_dtype="f32",
+                        qkv_dtype="bf16", parents="uniform", seed_id=14)
+    dev, ref = prompt_inputs(wl)
+    S_ref = gdn.prefill(ref["k"], ref["v"], ref["a"], ref["b"])
+    base, _ = _tc_prefill(wl, dev, 1)
+    scale = max(1.0, float(np.abs(S_ref).max()))
+    for segs in (2, 4, 7, 12):
+        S, _ = _tc_prefill(wl, dev, segs)
+        check_state(S, S_ref, "f32")
+        assert float((S - base).abs().max()) <= 2 * REL_TOL * scale
+
+
+def test_prefill_tc_matches_token_path():
+    """The chunked path and the token-by-token path of a SIMT handle build
+    the same state up to rounding."""
+    import linear_attention_beam_shared_b200 as L
+    wl = synth.Workload("pftc3", R=2, H=2, d_k=64, d_v=64, W=8, T=3, L_prompt=300, s0_dtype="f32",
+                        qkv_dtype="bf16", parents="uniform", seed_id=15)
+    dev, ref = prompt_inputs(wl)
+    S_tc, _ = _tc_prefill(wl, dev, 0)
+    S_tok, h = gpu_prefill(wl, dev, kernel=L.ONELA_KERNEL_SIMT)
+    try:
+        assert h.last_launches() == 1
+    finally:
+        h.close()
+    scale = max(1.0, float(S_tok.abs().max()))
+    assert float((S_tc - S_tok).abs().max()) <= 2 * REL_TOL * scale
+
+
+def test_prefill_tc_bad_segments():
+    import linear_attention_beam_shared_b200 as L
+    h = L.BeamDecoder(1, 1, 64, 64, 8, 3, "f32", "bf16")
+    try:
+        for bad in (-1, 17):
+            with pytest.raises(L.OnelaError):
+                h.prefill_segments(bad)
     finally:
         h.close()
