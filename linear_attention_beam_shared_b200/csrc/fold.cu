@@ -153,7 +153,7 @@ __device__ __forceinline__ void st8(__nv_bfloat16 *p, float (&x)[8]) {
 template <typename ST, int DK>
 __global__ void __launch_bounds__(kFoldThreads) fold_tc_kernel(const StepParams p, int Wt, int max_depth, int first,
                                                                const int32_t *d0_in, int32_t *d0_out,
-                                                               int32_t *anc_fold, ST *S_fold, uint4 *img) {
+                                                               int32_t *anc_fold, ST *S_fold, uint4 *img, int *done) {
   constexpr int TPR = DK / 8, RB = kFoldThreads / TPR, NK = DK / 64;
   constexpr int KC = DK / 8, DC = RB / 4, PER = KC + DC + 1;  // 16-byte record pieces per depth
   constexpr int MAXI = (kFoldMaxT * PER + kFoldThreads - 1) / kFoldThreads;
@@ -169,14 +169,19 @@ __global__ void __launch_bounds__(kFoldThreads) fold_tc_kernel(const StepParams 
   const int64_t rh = (int64_t)r * p.H + h;
   const int64_t si = (rh * dv + i) * DK + c * 8;
 
-  // The state the fold starts from: the prompt state, or the folded state of
-  // an earlier fold (complete before the kernels this one follows began).
+  // The state the fold starts from: the prompt state (read before the wait
+  // on the previous kernel), or the folded state of an earlier fold, which
+  // may still be running until the kernel before this one is complete.
   float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  if (valid) ld8((first ? static_cast<const ST *>(p.S0) : S_fold) + si, x);
-  const int old = first ? 0 : d0_in[r];
+  if (valid && first) ld8(static_cast<const ST *>(p.S0) + si, x);
   if (tid == 0) s_split = n;
   // The ancestry rows and records of step t come from the previous kernel.
   ptx::pdl_wait();
+  // The next step may start: it reads what this kernel writes only once the
+  // fold's CTAs have counted themselves done (StepParams::fold_done).
+  ptx::pdl_launch_dependents();
+  if (valid && !first) ld8(S_fold + si, x);
+  const int old = first ? 0 : d0_in[r];
   // Depths that can be folded: old + 1 .. Dmax (depth t only when step t
   // kept a single beam, its own record).
   const int jhi = min(n, max_depth);
@@ -256,41 +261,50 @@ __global__ void __launch_bounds__(kFoldThreads) fold_tc_kernel(const StepParams 
     for (int j = old + tid; j < D; j += kFoldThreads) anc_fold[(int64_t)r * TM + j % TM] = j < n ? s_row0[j % TM] : 0;
     if (tid == 0) d0_out[r] = D;
   }
-  if ((!first && D == old) || !valid) return;  // unchanged: the folded state and image hold it
+  // Unchanged (D == old) the state is stored back as it is: its image goes
+  // to the other image buffer all the same.
+  if (valid) {
 #pragma unroll 1
-  for (int dd = 0; dd < D - old; ++dd) {
-    const float a = s_a[dd], dl = s_d[dd][ir];
-    const uint4 kq = *reinterpret_cast<const uint4 *>(&s_k[dd][c * 8]);
-    const __nv_bfloat162 *k2 = reinterpret_cast<const __nv_bfloat162 *>(&kq);
+    for (int dd = 0; dd < D - old; ++dd) {
+      const float a = s_a[dd], dl = s_d[dd][ir];
+      const uint4 kq = *reinterpret_cast<const uint4 *>(&s_k[dd][c * 8]);
+      const __nv_bfloat162 *k2 = reinterpret_cast<const __nv_bfloat162 *>(&kq);
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float2 kf = __bfloat1622float2(k2[u]);
-      x[2 * u] = fmaf(dl, kf.x, a * x[2 * u]);
-      x[2 * u + 1] = fmaf(dl, kf.y, a * x[2 * u + 1]);
+      for (int u = 0; u < 4; ++u) {
+        const float2 kf = __bfloat1622float2(k2[u]);
+        x[2 * u] = fmaf(dl, kf.x, a * x[2 * u]);
+        x[2 * u + 1] = fmaf(dl, kf.y, a * x[2 * u + 1]);
+      }
+    }
+    st8(S_fold + si, x);
+    // The operand image: plane pl holds the bf16 term pl of the split of the
+    // stored value (hi, then the bf16 rounding of what is left, ...).
+    const int planes = p.s0_planes, ka = c >> 3, cc = c & 7;
+    float rest[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) rest[u] = x[u];
+    for (int pl = 0; pl < planes; ++pl) {
+      __align__(16) __nv_bfloat16 o[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        o[u] = __float2bfloat16_rn(rest[u]);
+        rest[u] = rest[u] - __bfloat162float(o[u]);
+      }
+      const int64_t off = ((rh * planes + pl) * NK + ka) * (kImgRows * 128) + ptx::swz128(i, cc);
+      img[off / 16] = *reinterpret_cast<const uint4 *>(o);
     }
   }
-  st8(S_fold + si, x);
-  // The operand image: plane pl holds the bf16 term pl of the split of the
-  // stored value (hi, then the bf16 rounding of what is left, ...).
-  const int planes = p.s0_planes, ka = c >> 3, cc = c & 7;
-  float rest[8];
-#pragma unroll
-  for (int u = 0; u < 8; ++u) rest[u] = x[u];
-  for (int pl = 0; pl < planes; ++pl) {
-    __align__(16) __nv_bfloat16 o[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      o[u] = __float2bfloat16_rn(rest[u]);
-      rest[u] = rest[u] - __bfloat162float(o[u]);
-    }
-    const int64_t off = ((rh * planes + pl) * NK + ka) * (kImgRows * 128) + ptx::swz128(i, cc);
-    img[off / 16] = *reinterpret_cast<const uint4 *>(o);
+  // This CTA's part of request r is written.
+  __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    ptx::red_release_add_gpu(done + r, 1);
   }
 }
 
 template <typename ST, int DK>
 cudaError_t launch_tc(const StepParams &p, int Wt, int max_depth, int first, const int32_t *d0_in, int32_t *d0_out,
-                      int32_t *anc_fold, void *S_fold, void *img, int pdl, cudaStream_t s) {
+                      int32_t *anc_fold, void *S_fold, void *img, int pdl, int *done, cudaStream_t s) {
   constexpr int RB = kFoldThreads / (DK / 8);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((p.dv + RB - 1) / RB, p.H, p.R);
@@ -302,7 +316,7 @@ cudaError_t launch_tc(const StepParams &p, int Wt, int max_depth, int first, con
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, fold_tc_kernel<ST, DK>, p, Wt, max_depth, first, d0_in, d0_out, anc_fold,
-                            static_cast<ST *>(S_fold), static_cast<uint4 *>(img));
+                            static_cast<ST *>(S_fold), static_cast<uint4 *>(img), done);
 }
 
 bool fold_args_ok(const StepParams &p, int Wt, int max_depth) {
@@ -325,18 +339,23 @@ cudaError_t launch_fold(const StepParams &p, int Wt, int max_depth, int first, c
                  : launch_state<float, float>(p, first, S_fold, d0_in, d0_out, anc_fold, s);
 }
 
+int fold_tc_ctas(const StepParams &p) {
+  const int RB = kFoldThreads / (p.dk / 8);
+  return (p.dv + RB - 1) / RB * p.H;
+}
+
 cudaError_t launch_fold_tc(const StepParams &p, int Wt, int max_depth, int first, const int32_t *d0_in,
                            int32_t *d0_out, int32_t *anc_fold, void *S_fold, void *img, int s0_bf16, int pdl,
-                           cudaStream_t s) {
+                           int *done, cudaStream_t s) {
   if (!fold_args_ok(p, Wt, max_depth) || p.T_max > kFoldMaxT || p.dk != p.dv || p.s0_planes < 1 ||
       p.s0_planes > 3)
     return cudaErrorInvalidValue;
   if (p.dk == 64)
-    return s0_bf16 ? launch_tc<__nv_bfloat16, 64>(p, Wt, max_depth, first, d0_in, d0_out, anc_fold, S_fold, img, pdl, s)
-                   : launch_tc<float, 64>(p, Wt, max_depth, first, d0_in, d0_out, anc_fold, S_fold, img, pdl, s);
+    return s0_bf16 ? launch_tc<__nv_bfloat16, 64>(p, Wt, max_depth, first, d0_in, d0_out, anc_fold, S_fold, img, pdl, done, s)
+                   : launch_tc<float, 64>(p, Wt, max_depth, first, d0_in, d0_out, anc_fold, S_fold, img, pdl, done, s);
   if (p.dk == 128)
-    return s0_bf16 ? launch_tc<__nv_bfloat16, 128>(p, Wt, max_depth, first, d0_in, d0_out, anc_fold, S_fold, img, pdl, s)
-                   : launch_tc<float, 128>(p, Wt, max_depth, first, d0_in, d0_out, anc_fold, S_fold, img, pdl, s);
+    return s0_bf16 ? launch_tc<__nv_bfloat16, 128>(p, Wt, max_depth, first, d0_in, d0_out, anc_fold, S_fold, img, pdl, done, s)
+                   : launch_tc<float, 128>(p, Wt, max_depth, first, d0_in, d0_out, anc_fold, S_fold, img, pdl, done, s);
   return cudaErrorInvalidValue;
 }
 

@@ -67,6 +67,25 @@ struct StepParams {
   // warp run out at that bound.
   unsigned long long wait_limit_ns;
   int stall;
+  // After a one-launch tensor-core fold (and until the next fold or
+  // rewind), for the tensor-core kernel: each CTA of that fold adds 1 to
+  // fold_done[r] (release at GPU scope) once its part of request r's folded
+  // state is written, so fold_done[r] >= fold_target means the fold is
+  // complete.  A CTA that sees it complete (acquire) replays from d0 and
+  // S0img.  Else, where the folded depth before that fold, d0_old[r] (0 if
+  // d0_old is null), still fits the record store (t - 1 - d0_old <= T_max -
+  // 1), it replays from it and its image S0img_old, which the fold does not
+  // write; else it waits for the kernel before it (whose completion implies
+  // the fold's) and replays from d0 and S0img.  fold_pending 0: d0 and S0img.
+  // The counts restart with every decode: step 1 zeroes fold_reset[r]
+  // (the same counters; null where the handle has none), and fold_target
+  // counts the CTAs of the folds since then.
+  int fold_pending;
+  const int *fold_done;
+  int fold_target;
+  int *fold_reset;
+  const int32_t *d0_old;
+  const void *S0img_old;
   // TMA descriptors of k, q and v (tensor-core kernel; encoded per call):
   // 4-D {d, H, W, R} bf16, box {64, 1, 32, 1}, 128-byte swizzle.
   alignas(64) CUtensorMap tm_k;
@@ -133,9 +152,12 @@ cudaError_t launch_fold(const StepParams &p, int Wt, int max_depth, int first, c
 // p.s0_planes terms); programmatic launch when pdl (the kernel waits before
 // it reads the ancestry rows and records; it reads S_fold and d0_in before,
 // so the previous kernel must not be a fold).
+// Each CTA adds 1 to done[r] (release) when its part of request r is
+// written; fold_tc_ctas(p) CTAs per request.
 cudaError_t launch_fold_tc(const StepParams &p, int Wt, int max_depth, int first, const int32_t *d0_in,
                            int32_t *d0_out, int32_t *anc_fold, void *S_fold, void *img, int s0_bf16, int pdl,
-                           cudaStream_t s);
+                           int *done, cudaStream_t s);
+int fold_tc_ctas(const StepParams &p);
 cudaError_t launch_s0_image(const void *S0, void *img, int R, int H, int dk, int dv,
                             int s0_bf16, int planes, cudaStream_t s);
 size_t s0_image_bytes(int R, int H, int dk, int dv, int planes);

@@ -30,11 +30,18 @@ struct onela_handle {
   // the other) and anc_fold [R][T_max].  The prompt state and its image stay
   // as they are, so a rewind needs no device work.
   void *S0f;
-  void *S0fimg;
+  void *S0fimg[2];  // its operand images: [fold_cur] the current one, the other the one before
   int32_t *fold_buf;
   int folded;      // S0f and fold_buf are in use since the last rewind
   int fold_cur;    // which d0 buffer holds the current depths
-  int after_fold;  // the last call was a fold: the next kernel may not overlap it
+  int after_fold;  // the last call was a fold
+  int fold_prev;   // a fold came before the last one since the rewind (its depth and image are the old ones)
+  // The last fold was the one-launch tensor-core fold, whose CTAs count
+  // themselves done in fold_buf's done counters ([R], zeroed by step 1 of
+  // each decode); fold_target: the count each request's counter reaches once
+  // the last fold is complete.
+  int fold_pending;
+  int fold_target;
   int32_t *par_store;         // each step's parents, written by the kernel
   // Every earlier call's k, gate and parent_idx (caller memory; read again
   // only under ONELA_FLAG_PDL).
@@ -99,6 +106,8 @@ void rewind_to_prompt(onela_handle *h) {
   h->steps_done = 0;
   h->folded = 0;
   h->after_fold = 0;
+  h->fold_pending = 0;
+  h->fold_target = 0;
   h->Ws.clear();
   h->hist_k.clear();
   h->hist_g.clear();
@@ -109,7 +118,8 @@ void free_all(onela_handle *h) {
   cudaFree(h->S0);
   cudaFree(h->S0img);
   cudaFree(h->S0f);
-  cudaFree(h->S0fimg);
+  cudaFree(h->S0fimg[0]);
+  cudaFree(h->S0fimg[1]);
   cudaFree(h->fold_buf);
   cudaFree(h->rec_alpha);
   cudaFree(h->par_store);
@@ -139,7 +149,7 @@ onela::StepParams base_params(const onela_handle *h) {
   p.W_max = h->cfg.W_max;
   p.T_max = h->cfg.T_max;
   p.S0 = h->folded ? h->S0f : h->S0;
-  p.S0img = h->folded ? h->S0fimg : h->S0img;
+  p.S0img = h->folded ? h->S0fimg[h->fold_cur] : h->S0img;
   p.d0 = h->folded ? h->fold_buf + h->fold_cur * h->cfg.R : nullptr;
   p.anc_fold = h->fold_buf + 2 * h->cfg.R;
   p.s0_planes = h->planes;
@@ -232,10 +242,12 @@ int onela_create(const onela_config *cfg, onela_handle **out) {
   const size_t nrow = (size_t)c.T_max * c.R * c.H * c.W_max;
   bool ok = cudaMalloc(&h->S0, nS0 * esize(c.s0_dtype)) == cudaSuccess;
   ok = ok && cudaMalloc(&h->S0f, nS0 * esize(c.s0_dtype)) == cudaSuccess;
-  ok = ok && cudaMalloc((void **)&h->fold_buf, (size_t)c.R * (2 + c.T_max) * sizeof(int32_t)) == cudaSuccess;
+  // d0 [2][R], anc_fold [R][T_max], the fold done counters [R].
+  ok = ok && cudaMalloc((void **)&h->fold_buf, (size_t)c.R * (3 + c.T_max) * sizeof(int32_t)) == cudaSuccess;
   if (ok && kernel == ONELA_KERNEL_TC)
     ok = cudaMalloc(&h->S0img, onela::s0_image_bytes(c.R, c.H, c.d_k, c.d_v, h->planes)) == cudaSuccess &&
-         cudaMalloc(&h->S0fimg, onela::s0_image_bytes(c.R, c.H, c.d_k, c.d_v, h->planes)) == cudaSuccess;
+         cudaMalloc(&h->S0fimg[0], onela::s0_image_bytes(c.R, c.H, c.d_k, c.d_v, h->planes)) == cudaSuccess &&
+         cudaMalloc(&h->S0fimg[1], onela::s0_image_bytes(c.R, c.H, c.d_k, c.d_v, h->planes)) == cudaSuccess;
   ok = ok && cudaMalloc((void **)&h->rec_alpha, nrow * sizeof(float)) == cudaSuccess;
   if (ok && kernel == ONELA_KERNEL_TC)
     ok = cudaMalloc((void **)&h->par_store, (size_t)c.T_max * c.R * c.W_max * sizeof(int32_t)) == cudaSuccess;
@@ -248,9 +260,11 @@ int onela_create(const onela_config *cfg, onela_handle **out) {
     *h->err_host = 0;
     // Zeroed so that nothing uninitialised is ever read, even after a bad parent.
     ok = cudaMemset(h->rec_alpha, 0, nrow * sizeof(float)) == cudaSuccess &&
-         (!h->S0fimg ||
-          cudaMemset(h->S0fimg, 0, onela::s0_image_bytes(c.R, c.H, c.d_k, c.d_v, h->planes)) == cudaSuccess) &&
+         (!h->S0fimg[0] ||
+          (cudaMemset(h->S0fimg[0], 0, onela::s0_image_bytes(c.R, c.H, c.d_k, c.d_v, h->planes)) == cudaSuccess &&
+           cudaMemset(h->S0fimg[1], 0, onela::s0_image_bytes(c.R, c.H, c.d_k, c.d_v, h->planes)) == cudaSuccess)) &&
          cudaMemset(h->anc, 0, (size_t)c.T_max * c.R * c.W_max * c.T_max * sizeof(int32_t)) == cudaSuccess &&
+         cudaMemset(h->fold_buf, 0, (size_t)c.R * (3 + c.T_max) * sizeof(int32_t)) == cudaSuccess &&
          cudaDeviceSynchronize() == cudaSuccess;
   }
   if (!ok) {
@@ -403,14 +417,25 @@ int decode_one(onela_handle *h, int32_t W_prev, int32_t W, const void *q, const 
   p.o = o;
   cudaError_t e;
   const bool contract = (c.flags & ONELA_FLAG_PDL) != 0;
-  // The step after a fold reads the folded state before its wait: it is an
-  // ordinary launch.  Otherwise a step overlaps the step before it under
-  // ONELA_FLAG_PDL, or inside one onela_decode_steps call when the depth its
-  // early writes replace (t - T_max) is none, or of the same call (then no
-  // step still running reads it from the store).
+  // A step overlaps the step before it under ONELA_FLAG_PDL, or inside one
+  // onela_decode_steps call when the depth its early writes replace
+  // (t - T_max) is none, or of the same call (then no step still running
+  // reads it from the store).  The tensor-core step right after a fold
+  // overlaps the fold: it replays from the folded state before that fold
+  // (which the fold does not write) where that still fits the record store,
+  // and waits for the fold elsewhere (StepParams::after_fold).
   const int tr = p.t - c.T_max;
   const bool in_call = call_t0 > 0 && p.t > call_t0 && (tr < 1 || tr >= call_t0);
-  const bool pdl = p.t >= 2 && !h->after_fold && (contract || in_call);
+  const bool after_fold = h->after_fold && h->fold_pending;  // after the one-launch tensor-core fold
+  const bool pdl = p.t >= 2 && (after_fold || (!h->after_fold && (contract || in_call)));
+  if (p.t == 1 && h->kernel == ONELA_KERNEL_TC) p.fold_reset = h->fold_buf + (2 + c.T_max) * c.R;
+  if (h->fold_pending && h->kernel == ONELA_KERNEL_TC) {
+    p.fold_pending = 1;
+    p.fold_done = h->fold_buf + (2 + c.T_max) * c.R;
+    p.fold_target = h->fold_target;
+    p.d0_old = h->fold_prev ? h->fold_buf + (1 - h->fold_cur) * c.R : nullptr;
+    p.S0img_old = h->fold_prev ? h->S0fimg[1 - h->fold_cur] : h->S0img;
+  }
   if (h->kernel == ONELA_KERNEL_TC) {
     // The tensor-core kernel reads tiles of q, k, v and o with 16-byte accesses.
     const uintptr_t any = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
@@ -532,6 +557,8 @@ int onela_reset(onela_handle *h, onela_stream stream) {
   h->steps_done = 0;
   h->folded = 0;
   h->after_fold = 0;
+  h->fold_pending = 0;
+  h->fold_target = 0;
   h->Ws.clear();
   h->hist_k.clear();
   h->hist_g.clear();
@@ -557,18 +584,25 @@ int onela_fold(onela_handle *h, int32_t max_depth, onela_stream stream) {
   const int depth = max_depth < h->steps_done ? max_depth : h->steps_done;
   NvtxRange nvtx(c, "fold after step", h->steps_done);
   cudaError_t e;
+  int pending = 0;
   if (h->kernel == ONELA_KERNEL_TC && c.d_k <= 128) {
-    // Overlaps the step before it (never another fold: it reads the folded
-    // state before its wait).
-    const int pdl = (c.flags & ONELA_FLAG_PDL) && !h->after_fold;
-    e = onela::launch_fold_tc(p, h->Ws.back(), depth, first, d0_in, d0_out, anc_fold, h->S0f, h->S0fimg,
-                              c.s0_dtype == ONELA_BF16, pdl, s);
+    // Overlaps the step before it, which writes nothing it reads before its
+    // wait (never another fold: it reads the folded state before its wait).
+    // The new image goes to the other image buffer: the next step may still
+    // read the current one.
+    const int pdl = !h->after_fold;
+    e = onela::launch_fold_tc(p, h->Ws.back(), depth, first, d0_in, d0_out, anc_fold, h->S0f,
+                              h->S0fimg[1 - h->fold_cur], c.s0_dtype == ONELA_BF16, pdl,
+                              h->fold_buf + (2 + c.T_max) * c.R, s);
+    h->fold_target += onela::fold_tc_ctas(p);
+    pending = 1;
   } else if (h->kernel == ONELA_KERNEL_TC) {
     // d = 256: the general fold, then the folded state's operand image.
     e = onela::launch_fold(p, h->Ws.back(), depth, first, d0_in, d0_out, anc_fold, h->S0f,
                            c.qkv_dtype == ONELA_BF16, c.s0_dtype == ONELA_BF16, s);
     if (e == cudaSuccess)
-      e = onela::launch_s0_image(h->S0f, h->S0fimg, c.R, c.H, c.d_k, c.d_v, c.s0_dtype == ONELA_BF16, h->planes, s);
+      e = onela::launch_s0_image(h->S0f, h->S0fimg[1 - h->fold_cur], c.R, c.H, c.d_k, c.d_v,
+                                 c.s0_dtype == ONELA_BF16, h->planes, s);
   } else {
     e = onela::launch_fold(p, h->Ws.back(), depth, first, d0_in, d0_out, anc_fold, h->S0f,
                            c.qkv_dtype == ONELA_BF16, c.s0_dtype == ONELA_BF16, s);
@@ -578,8 +612,10 @@ int onela_fold(onela_handle *h, int32_t max_depth, onela_stream stream) {
     return ONELA_ERR_CUDA;
   }
   h->fold_cur = 1 - h->fold_cur;
+  h->fold_prev = h->folded;
   h->folded = 1;
   h->after_fold = 1;
+  h->fold_pending = pending;
   return ONELA_OK;
 }
 

@@ -129,16 +129,6 @@ __global__ void __launch_bounds__(kThreads, DK <= 128 ? 2 : 1) step_tc_kernel(co
   const int b0 = tile * kBT;
   const int nb = min(kBT, p.W - b0);
   const int H = p.H, t = p.t, TM = p.T_max, P = p.s0_planes;
-  // Depths 1..d0 are folded into S0; the beams replay depths d0+1..t-1,
-  // which must fit the record store's T_max slots.
-  int d0 = p.d0 ? p.d0[r] : 0;
-  if (t - 1 - d0 > TM - 1) {
-    if (tid == 0) set_err(p.err, kErrByteWindow);
-    d0 = t - TM;  // keeps every access inside the store; the results are void
-  }
-  const int nanc = t - 1 - d0;  // ancestors per beam; chain index j is depth d0+j+1
-  const int jp = nanc - 1;      // chain index of the parents (depth t-1)
-  const int soff = d0 % TM;     // slot of depth d0 + 1
   const int tslot = (t - 1) % TM;  // slot of depth t
   const int hb = p.hbase;       // step of the history table's entry 0
   const uint32_t hmask = p.hist_inputs;  // bit i: history entry i from the callers' arrays
@@ -154,6 +144,7 @@ __global__ void __launch_bounds__(kThreads, DK <= 128 ? 2 : 1) step_tc_kernel(co
   uint64_t *bar_chain = bars + 2;  // ancestry warp: every beam's chain in s_chain
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(base + L.book + 64);
   int *s_U = reinterpret_cast<int *>(s_tmem + 1);
+  int *s_mode = s_U + 1;  // the CTA's root: [0] its folded depth, [1] how it was chosen
   int *s_par = reinterpret_cast<int *>(base + L.book + 128);
   float *s_alpha = reinterpret_cast<float *>(s_par + kBT);
   float *s_beta = s_alpha + kBT;
@@ -187,9 +178,26 @@ __global__ void __launch_bounds__(kThreads, DK <= 128 ? 2 : 1) step_tc_kernel(co
     ptx::mbar_init(bar1, 1);
     ptx::mbar_init(bar_chain, 32 + (p.stall ? 1 : 0));  // stall (tests): an arrival that never comes
     ptx::mbar_fence_init();
+    // The root this step replays from: the current folded state, or, while
+    // the last fold is not complete, the one before it (where its depths fit
+    // the record store; else this step waits for the kernel before it, whose
+    // completion implies the fold's).  Decided once for the CTA.
+    int mode = 0, d0s = 0;  // 0: current, 1: the one before the last fold, 2: current after the wait
+    if (p.fold_pending && ptx::ld_acquire_gpu(p.fold_done + r) < p.fold_target) {
+      d0s = p.d0_old ? p.d0_old[r] : 0;
+      mode = t - 1 - d0s <= TM - 1 ? 1 : 2;
+      if (mode == 2) ptx::pdl_wait();
+    }
+    if (mode != 1 && p.d0) d0s = p.d0[r];
+    s_mode[0] = d0s;
+    s_mode[1] = mode;
+    // A new decode: its folds count from zero (no fold of an earlier decode
+    // runs any more: step 1 is an ordinary launch).
+    if (t == 1 && p.fold_reset && tile == 0 && h == 0 && mt == 0) p.fold_reset[r] = 0;
     // S0 image (bulk copy); k, q, v tiles by TMA, beams past W read as zeros.
     ptx::mbar_arrive_expect_tx(bar_s0, s0_bytes + NK * XA + NV * VA);
-    const uint8_t *src = static_cast<const uint8_t *>(p.S0img) + ((size_t)(r * H + h) * nmt + mt) * s0_bytes;
+    const uint8_t *src =
+        static_cast<const uint8_t *>(mode == 1 ? p.S0img_old : p.S0img) + ((size_t)(r * H + h) * nmt + mt) * s0_bytes;
     for (uint32_t off = 0; off < s0_bytes; off += 16384u)
       ptx::bulk_g2s(base + L.a + off, src + off, 16384u, bar_s0);
 #pragma unroll
@@ -240,6 +248,17 @@ __global__ void __launch_bounds__(kThreads, DK <= 128 ? 2 : 1) step_tc_kernel(co
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *s_tmem;
+  if (s_mode[1] == 2) ptx::pdl_wait();
+  // Depths 1..d0 are folded into the root; the beams replay depths
+  // d0+1..t-1, which must fit the record store's T_max slots.
+  int d0 = s_mode[0];
+  if (t - 1 - d0 > TM - 1) {
+    if (tid == 0) set_err(p.err, kErrByteWindow);
+    d0 = t - TM;  // keeps every access inside the store; the results are void
+  }
+  const int nanc = t - 1 - d0;  // ancestors per beam; chain index j is depth d0+j+1
+  const int jp = nanc - 1;      // chain index of the parents (depth t-1)
+  const int soff = d0 % TM;     // slot of depth d0 + 1
 
   bool ok = true;
   const uint32_t x_u32 = ptx::smem_u32(s_x), a_u32 = ptx::smem_u32(base + L.a);

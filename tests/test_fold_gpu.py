@@ -315,6 +315,36 @@ def test_decode_deeper_than_the_record_store(kind, pdl):
             assert torch.equal(g["k"], steps[t - 1]["k"])
 
 
+@pytest.mark.parametrize("TM", [5, 6, 8])
+@pytest.mark.parametrize("pdl", [0, 1])
+def test_step_after_a_fold_lags_or_waits(TM, pdl):
+    """The tensor-core step right after a fold replays from the folded state
+    before that fold while its depths still fit the record store, and waits
+    for the fold otherwise.  With a fold after every fourth step (steps
+    4k replay 4 depths, so the store needs at least 5), the step after the
+    fold at 4k replays 5 depths from the fold before (4 after the first
+    fold): a 5-depth store takes that only after the first fold and waits
+    after the others, 6 and 8 never wait.  Outputs of every step and the
+    folded depths against the fp64 oracle."""
+    import linear_attention_beam_shared_b200 as L
+    T = 18
+    Ws = [8, 24, 16, 20, 12, 24, 16, 8, 20] * 2
+    wl, S0, steps = P.custom_steps(47 + TM, R=2, H=3, dk=64, dv=64, Ws=Ws, parents="zipf")
+    for at in range(3, T - 1, 4):
+        steps = narrow(steps, at, [at % 3, (at + 1) % 5])
+    folds = {at + 1: T for at in range(3, T - 1, 4)}
+    S0t = synth.cast_state(S0, "f32")
+    gpu, info, used = run_with_folds(S0t, steps, "bf16", kernel_id("tc"), folds,
+                                     flags=L.ONELA_FLAG_PDL if pdl else 0, T_max=TM)
+    assert used == kernel_id("tc")
+    for t, D, _ in info:
+        assert D.tolist() == [t - 1, t - 1]
+    ref = P.oracle(S0t, steps)
+    for t, (g, r) in enumerate(zip(gpu, ref), start=1):
+        err = float(np.abs(g["o"].double().numpy() - r["o"]).max())
+        assert err <= P.TOL["f32"], (t, err)
+
+
 @pytest.mark.parametrize("kind", ["simt", "tc"])
 def test_unfolded_window_overflow_is_reported(kind):
     """With nothing shared to fold, a decode that goes past T_max unfolded
