@@ -276,8 +276,11 @@ def time_fold(wl, S0, kernel, device, stream, flush, T=16, every=4, reps=10, war
 
     def make(fold):
         outs = [torch.empty((wd.R, st["W"], wd.H, wd.d_v), dtype=torch.float32, device=device) for st in steps]
-        dec = L.BeamDecoder(wd.R, wd.H, wd.d_k, wd.d_v, wd.W, tmax or T, wd.s0_dtype, wd.qkv_dtype,
+        # The folded decode runs through the record store of tmax depths; the
+        # unfolded one needs all T of them.
+        dec = L.BeamDecoder(wd.R, wd.H, wd.d_k, wd.d_v, wd.W, (tmax or T) if fold else T, wd.s0_dtype, wd.qkv_dtype,
                             kernel=kernel, device=device.index, flags=L.ONELA_FLAG_PDL)
+        kernels[fold] = dec.kernel
         dec.set_prompt_state(S0.to(device))
 
         def run():
@@ -317,25 +320,30 @@ def time_fold(wl, S0, kernel, device, stream, flush, T=16, every=4, reps=10, war
         stream.synchronize()
         return max_over_ranks(sum(e0.elapsed_time(e1) for e0, e1 in ev) / reps, device)
 
-    res = {}
-    for fold in ((True,) if tmax and tmax < T else (True, False)):
+    res, kernels = {}, {}
+    for fold in (True, False):
         dec, g, outs, depth = make(fold)
         ms = timed(g)
         res[fold] = (ms, [o.clone() for o in outs], depth)
         del g
         dec.close()
-    if False not in res:
-        return {
-            "workload": f"{wl.name} shapes over T={T} steps through a record store of {tmax} depths "
-                        f"(R={wd.R}, H={wd.H}, d={wd.d_k}, W={wd.W}), every beam of steps "
-                        f"{', '.join(str(i + 1) for i in narrow)} a child of beam 0; folds right after them",
-            "ms_per_decode": {"folded": round(res[True][0], 5), "unfolded": None},
-            "us_per_step": round(res[True][0] * 1e3 / T, 3),
-            "fold_depth_at_end": res[True][2],
-        }
     diff = max(float((a - b).abs().max()) for a, b in zip(res[True][1], res[False][1]))
     scale = max(float(b.abs().max()) for b in res[False][1])
     assert diff <= 2e-5 * max(1.0, scale), f"folded decode differs from the unfolded one by {diff}"
+    if tmax and tmax < T:
+        names = {L.ONELA_KERNEL_TC: "tc", L.ONELA_KERNEL_SIMT: "simt"}
+        return {
+            "workload": f"{wl.name} shapes over T={T} steps (R={wd.R}, H={wd.H}, d={wd.d_k}, W={wd.W}), every beam of "
+                        f"steps {', '.join(str(i + 1) for i in narrow)} a child of beam 0; folded: folds right after "
+                        f"them through a record store of {tmax} depths; unfolded: a store of {T} depths",
+            "ms_per_decode": {"folded": round(res[True][0], 5), "unfolded": round(res[False][0], 5)},
+            "speedup": round(res[False][0] / res[True][0], 3),
+            "record_store_depths": {"folded": tmax, "unfolded": T},
+            "kernel": {"folded": names.get(kernels[True]), "unfolded": names.get(kernels[False])},
+            "us_per_step": {"folded": round(res[True][0] * 1e3 / T, 3), "unfolded": round(res[False][0] * 1e3 / T, 3)},
+            "fold_depth_at_end": res[True][2],
+            "max_abs_diff_folded_vs_unfolded": diff,
+        }
 
     out = {
         "workload": f"{wl.name} shapes over T={T} steps (R={wd.R}, H={wd.H}, d={wd.d_k}, W={wd.W}), every beam of "

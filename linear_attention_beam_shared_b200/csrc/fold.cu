@@ -44,7 +44,7 @@ namespace {
 
 constexpr int kPlanThreads = 256;
 constexpr int kFoldThreads = 256;
-constexpr int kFoldMaxT = 16;  // deepest decode of the one-launch fold
+constexpr int kFoldMaxT = kFoldTcMaxT;  // deepest decode of the one-launch fold
 constexpr int kImgRows = 128;  // rows of an operand image atom
 
 __device__ __forceinline__ float ldf(const float *p, int64_t i) { return p[i]; }

@@ -7,7 +7,7 @@
 
 namespace onela {
 
-constexpr int kHistSteps = 17;     // steps of history the tensor-core kernel can see (its window is <= 16)
+constexpr int kHistSteps = 33;     // steps of history the tensor-core kernel can see (its window is <= 32)
 constexpr int kHistMaxInts = 4096;  // parents of earlier steps the tensor-core kernel
                                     // keeps in shared memory (more: read from global memory)
 
@@ -31,7 +31,7 @@ struct StepParams {
   // (rec_k, rec_alpha) and the par_store row of step j.  Parents of request r
   // start at hpar[i] + r * hpar_rs[i]; hW[i] = W_j.  The kernel copies the
   // parents of steps hcopy .. t - 1 to shared memory.
-  uint32_t hist_inputs;
+  uint64_t hist_inputs;
   int hbase, hcopy;
   const void *hk[kHistSteps];
   const float *hg[kHistSteps];
@@ -152,6 +152,7 @@ cudaError_t launch_fold(const StepParams &p, int Wt, int max_depth, int first, c
 // p.s0_planes terms); programmatic launch when pdl (the kernel waits before
 // it reads the ancestry rows and records; it reads S_fold and d0_in before,
 // so the previous kernel must not be a fold).
+constexpr int kFoldTcMaxT = 16;  // deepest record store of the one-launch tensor-core fold
 // Each CTA adds 1 to done[r] (release) when its part of request r is
 // written; fold_tc_ctas(p) CTAs per request.
 cudaError_t launch_fold_tc(const StepParams &p, int Wt, int max_depth, int first, const int32_t *d0_in,

@@ -442,12 +442,14 @@ int decode_one(onela_handle *h, int32_t W_prev, int32_t W, const void *q, const 
                           reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(o);
     if (any & 15u) return ONELA_ERR_ARG;
     // The table covers steps hbase .. t-1 (the kernel replays at most
-    // T_max - 1 <= 15 of them); the parents of steps hcopy .. t-1 go to
+    // T_max - 1 <= 31 of them); the parents of steps hcopy .. t-1 go to
     // shared memory.  Keys, gates and parents of a step come from the
     // caller's arrays while they are valid (ONELA_FLAG_PDL, or a step of
     // this call), else from the record store and the stored parents (those
     // steps have completed).
-    p.hbase = p.t - onela::kHistSteps + 1 > 1 ? p.t - onela::kHistSteps + 1 : 1;
+    // (T_max + 1 <= kHistSteps entries: a step replays at most T_max - 1
+    // depths, from depth t - T_max + 1 on)
+    p.hbase = p.t - c.T_max > 1 ? p.t - c.T_max : 1;
     p.hcopy = p.t - c.T_max + 1 > 2 ? p.t - c.T_max + 1 : 2;
     if (p.hcopy < p.hbase + 1) p.hcopy = p.hbase + 1;
     p.hist_inputs = 0;
@@ -456,7 +458,7 @@ int decode_one(onela_handle *h, int32_t W_prev, int32_t W, const void *q, const 
       const int i = j - p.hbase;
       p.hW[i] = h->Ws[j - 1];
       if (contract || (call_t0 > 0 && j >= call_t0)) {
-        p.hist_inputs |= 1u << i;
+        p.hist_inputs |= 1ull << i;
         p.hk[i] = h->hist_k[j - 1];
         p.hg[i] = h->hist_g[j - 1];
         p.hpar[i] = h->hist_par[j - 1];
@@ -585,7 +587,7 @@ int onela_fold(onela_handle *h, int32_t max_depth, onela_stream stream) {
   NvtxRange nvtx(c, "fold after step", h->steps_done);
   cudaError_t e;
   int pending = 0;
-  if (h->kernel == ONELA_KERNEL_TC && c.d_k <= 128) {
+  if (h->kernel == ONELA_KERNEL_TC && c.d_k <= 128 && c.T_max <= onela::kFoldTcMaxT) {
     // Overlaps the step before it, which writes nothing it reads before its
     // wait (never another fold: it reads the folded state before its wait).
     // The new image goes to the other image buffer: the next step may still
@@ -597,7 +599,8 @@ int onela_fold(onela_handle *h, int32_t max_depth, onela_stream stream) {
     h->fold_target += onela::fold_tc_ctas(p);
     pending = 1;
   } else if (h->kernel == ONELA_KERNEL_TC) {
-    // d = 256: the general fold, then the folded state's operand image.
+    // d = 256, or a store of more than kFoldTcMaxT depths: the general
+    // fold, then the folded state's operand image.
     e = onela::launch_fold(p, h->Ws.back(), depth, first, d0_in, d0_out, anc_fold, h->S0f,
                            c.qkv_dtype == ONELA_BF16, c.s0_dtype == ONELA_BF16, s);
     if (e == cudaSuccess)

@@ -72,8 +72,10 @@ constexpr int kN = 2 * kBT;         // vectors: k rows 0..31, q rows 32..63
 constexpr int kM = 128;             // MMA M
 constexpr int kDRows = 128;         // ancestor deltas per staging round after the wait
 constexpr int kTmemCols = 64;       // D1
-constexpr uint32_t kTabBytes = 3u * 8u * kHistSteps + 3u * 4u * kHistSteps;  // per-step table
-constexpr int kMaxT = 16;           // deepest decode the kernel serves
+// The per-step table: 3 pointers and 3 ints for each of nhist = T_max + 1
+// steps (at most kHistSteps).
+__host__ __device__ inline uint32_t tab_bytes(int nhist) { return (3u * 8u + 3u * 4u) * (uint32_t)nhist; }
+constexpr int kMaxT = 32;           // deepest decode the kernel serves
 constexpr int kMaxW = 1024;         // widest beam set the kernel serves
 
 struct Layout {
@@ -102,7 +104,7 @@ __host__ __device__ inline Layout layout(int nk, int nv, int planes, int TM, int
   // of the last steps before t; the per-step table (3 pointers and 3 ints per
   // step).
   L.total = L.book + 128u + 4u * kBT * 4u + (uint32_t)kBT * TM * 16u + (3u * kBT + 4u) * TM * 4u +
-            (uint32_t)((W_max + 3) & ~3) * 4u + (uint32_t)((hist_cap + 3) & ~3) * 2u + kTabBytes + 16u;
+            (uint32_t)((W_max + 3) & ~3) * 4u + (uint32_t)((hist_cap + 3) & ~3) * 2u + tab_bytes(TM + 1) + 16u;
   return L;
 }
 
@@ -131,7 +133,7 @@ __global__ void __launch_bounds__(kThreads, DK <= 128 ? 2 : 1) step_tc_kernel(co
   const int H = p.H, t = p.t, TM = p.T_max, P = p.s0_planes;
   const int tslot = (t - 1) % TM;  // slot of depth t
   const int hb = p.hbase;       // step of the history table's entry 0
-  const uint32_t hmask = p.hist_inputs;  // bit i: history entry i from the callers' arrays
+  const uint64_t hmask = p.hist_inputs;  // bit i: history entry i from the callers' arrays
 
   const Layout L = layout(NK, NV, P, TM, p.W_max, p.hist_cap);
   uint8_t *s_x = base + L.x;
@@ -162,11 +164,12 @@ __global__ void __launch_bounds__(kThreads, DK <= 128 ? 2 : 1) step_tc_kernel(co
   // first barrier with one load per lane: loops then read shared memory
   // instead of indexing the parameters at run time.
   const int32_t **s_tpar = reinterpret_cast<const int32_t **>(s_hist + ((p.hist_cap + 3) & ~3));
-  const float **s_tg = reinterpret_cast<const float **>(s_tpar + kHistSteps);
-  const __nv_bfloat16 **s_tk = reinterpret_cast<const __nv_bfloat16 **>(s_tg + kHistSteps);
-  int *s_toff = reinterpret_cast<int *>(s_tk + kHistSteps);
-  int *s_tW = s_toff + kHistSteps;
-  int *s_trs = s_tW + kHistSteps;
+  const int NH = TM + 1;  // table entries: steps t - T_max .. t - 1 (hbase = t - T_max at most)
+  const float **s_tg = reinterpret_cast<const float **>(s_tpar + NH);
+  const __nv_bfloat16 **s_tk = reinterpret_cast<const __nv_bfloat16 **>(s_tg + NH);
+  int *s_toff = reinterpret_cast<int *>(s_tk + NH);
+  int *s_tW = s_toff + NH;
+  int *s_trs = s_tW + NH;
 
   __nv_bfloat16 *rec_k = static_cast<__nv_bfloat16 *>(p.rec_k);
   const int64_t row0 = (int64_t)(r * p.W + b0) * H + h;  // (r, b0, h) row of [R][W][H][d]
@@ -225,13 +228,13 @@ __global__ void __launch_bounds__(kThreads, DK <= 128 ? 2 : 1) step_tc_kernel(co
       g_alpha = p.g[si];
       g_beta = p.beta[si];
     }
-    if (lane < kHistSteps) {
-      s_tpar[lane] = p.hpar[lane];
-      s_tg[lane] = p.hg[lane];
-      s_tk[lane] = static_cast<const __nv_bfloat16 *>(p.hk[lane]);
-      s_toff[lane] = p.hoff[lane];
-      s_tW[lane] = p.hW[lane];
-      s_trs[lane] = p.hpar_rs[lane];
+    for (int e = lane; e < NH; e += 32) {
+      s_tpar[e] = p.hpar[e];
+      s_tg[e] = p.hg[e];
+      s_tk[e] = static_cast<const __nv_bfloat16 *>(p.hk[e]);
+      s_toff[e] = p.hoff[e];
+      s_tW[e] = p.hW[e];
+      s_trs[e] = p.hpar_rs[e];
     }
   }
   // The parents of steps hcopy..t-1 for this request as 16-bit indices,
@@ -310,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, DK <= 128 ? 2 : 1) step_tc_kernel(co
         const int a = s_chain[b * TM + j];
         const int di = d0 + j + 1 - hb;  // history entry of the record's depth
         const int sl = soff + j < TM ? soff + j : soff + j - TM;
-        ptx::cp_async4(s_w + b * TM + j, (hmask >> di) & 1u ? s_tg[di] + ((int64_t)r * s_tW[di] + a) * H + h
+        ptx::cp_async4(s_w + b * TM + j, (hmask >> di) & 1ull ? s_tg[di] + ((int64_t)r * s_tW[di] + a) * H + h
                                                            : p.rec_alpha + rec_row_slot(p, sl, r, h, a));
       }
     }
@@ -342,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, DK <= 128 ? 2 : 1) step_tc_kernel(co
       for (int j = jp; j >= 0; --j) {
         const float gj = s_w[b * TM + j];
         reinterpret_cast<float *>(s_c + b * TM + j)[3] = w;
-        w *= (hmask >> (d0 + j + 1 - hb)) & 1u ? expf(gj) : gj;
+        w *= (hmask >> (d0 + j + 1 - hb)) & 1ull ? expf(gj) : gj;
       }
     }
     s_Gp[b] = w;
@@ -400,7 +403,7 @@ __global__ void __launch_bounds__(kThreads, DK <= 128 ? 2 : 1) step_tc_kernel(co
           const int a = s_chain[bb * TM + j];
           const int di = d0 + j + 1 - hb;
           const int sl = soff + j < TM ? soff + j : soff + j - TM;
-          const __nv_bfloat16 *row = (hmask >> di) & 1u ? s_tk[di] + ((int64_t)(r * s_tW[di] + a) * H + h) * DK
+          const __nv_bfloat16 *row = (hmask >> di) & 1ull ? s_tk[di] + ((int64_t)(r * s_tW[di] + a) * H + h) * DK
                                          : rec_k + rec_row_slot(p, sl, r, h, a) * DK;
           const uint8_t *rb = reinterpret_cast<const uint8_t *>(row) + l * 8;
 #pragma unroll

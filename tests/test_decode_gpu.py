@@ -144,6 +144,23 @@ def test_deep_decode(kernel):
     P.compare(gpu, P.oracle(S0c, steps), steps, "f32")
 
 
+@pytest.mark.parametrize("T,W,d,R,H", [(24, 40, 64, 2, 3), (32, 256, 128, 1, 4), (20, 33, 128, 1, 2)])
+def test_tc_store_deeper_than_16(T, W, d, R, H):
+    """A record store of up to 32 depths on the tensor-core kernel (one CTA
+    per SM past 16 depths at d = 128): every step replays up to T - 1
+    ancestors, through both the callers' arrays (one onela_decode_steps
+    call) and the record store (one call per step)."""
+    import linear_attention_beam_shared_b200 as L
+    _skip_unavailable(2, d, d, "bf16")
+    wl, S0, steps = P.custom_steps(60 + T, R, H, d, d, (W,) * T, parents="zipf")
+    S0c = synth.cast_state(S0, "f32")
+    ref = P.oracle(S0c, steps)
+    for chunks in (None, [T]):
+        gpu, used = P.run_gpu(S0c, steps, "bf16", L.ONELA_KERNEL_TC, chunks=chunks)
+        assert used == L.ONELA_KERNEL_TC
+        P.compare(gpu, ref, steps, "f32")
+
+
 @pytest.mark.parametrize("kernel", [1, 2])
 def test_identity_gate_keeps_s0(kernel):
     """alpha = 1 (g = 0), beta = 0: delta is exactly zero and o = S0 q."""

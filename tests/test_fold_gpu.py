@@ -345,6 +345,27 @@ def test_step_after_a_fold_lags_or_waits(TM, pdl):
         assert err <= P.TOL["f32"], (t, err)
 
 
+def test_fold_tc_store_of_20_depths():
+    """A tensor-core handle whose record store is deeper than the one-launch
+    fold serves (20 depths): folds take the general path, then the folded
+    state's operand image; a 40-step decode through it against the oracle."""
+    import linear_attention_beam_shared_b200 as L
+    T, TM = 40, 20
+    Ws = [16, 24, 20, 12, 24, 16, 20, 28] * 5
+    wl, S0, steps = P.custom_steps(52, R=1, H=2, dk=128, dv=128, Ws=Ws, parents="uniform")
+    for at in range(9, T - 1, 10):
+        steps = narrow(steps, at, [at % 7])
+    folds = {at + 1: T for at in range(9, T - 1, 10)}
+    S0t = synth.cast_state(S0, "f32")
+    gpu, info, used = run_with_folds(S0t, steps, "bf16", kernel_id("tc"), folds, flags=L.ONELA_FLAG_PDL, T_max=TM)
+    assert used == kernel_id("tc")
+    for t, D, _ in info:
+        assert D.tolist() == [t - 1]
+    ref = P.oracle(S0t, steps)
+    for t, (g, r) in enumerate(zip(gpu, ref), start=1):
+        assert float(np.abs(g["o"].double().numpy() - r["o"]).max()) <= P.TOL["f32"], t
+
+
 @pytest.mark.parametrize("kind", ["simt", "tc"])
 def test_unfolded_window_overflow_is_reported(kind):
     """With nothing shared to fold, a decode that goes past T_max unfolded
