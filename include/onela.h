@@ -86,11 +86,11 @@ enum {
  *                   waits for step t-1 only before it stages the ancestors'
  *                   deltas.  For that it reads the k, gate and parent_idx
  *                   arrays of the earlier steps of the decode again (at
- *                   most the last 16).  Set
+ *                   most the last T_max).  Set
  *                   it only when (a) the kernel before step t in the stream
  *                   produces no input of step t (q, k, v, g, beta,
  *                   parent_idx), and (b) the k, gate and parent_idx arrays of
- *                   the last 16 steps before t stay unchanged and
+ *                   the last T_max steps before t stay unchanged and
  *                   allocated until step t has completed -- e.g. back-to-back
  *                   decode steps whose inputs were all written before the
  *                   first of them, as in a CUDA graph of a whole decode, or
@@ -105,8 +105,8 @@ enum { ONELA_FLAG_NVTX = 4 };
 
 
 /* Which decode kernel runs.  AUTO picks the tensor-core kernel when the
- * shape allows it (bf16 q/k/v, d_k = d_v in {64, 128}, T_max <= 16,
- * W_max <= 1024) and the SIMT kernel otherwise. */
+ * shape allows it (bf16 q/k/v, d_k = d_v in {64, 128}, or 256 with at most
+ * two S0 terms; T_max <= 32, W_max <= 1024) and the SIMT kernel otherwise. */
 enum { ONELA_KERNEL_AUTO = 0, ONELA_KERNEL_SIMT = 1, ONELA_KERNEL_TC = 2 };
 
 /* Handle configuration.
@@ -332,9 +332,15 @@ ONELA_API int onela_reset(onela_handle *h, onela_stream stream);
  *              0 (or no step done yet) leaves everything as it is.
  * Runs on the device only (no host synchronisation; capturable in a CUDA
  * graph: the prompt state is never overwritten, so a captured decode that
- * folds replays from the prompt each time); the next decode step is an
- * ordinary launch even under ONELA_FLAG_PDL.  Memory: a second state buffer
- * (and operand image, tensor-core kernel), allocated by onela_create.
+ * folds replays from the prompt each time).  Tensor-core handles with
+ * d_k = d_v <= 128 and T_max <= 16 fold in one launch that overlaps the
+ * steps around it: it starts once the step before it is complete, and a
+ * step launched while it runs replays from the root state before the fold
+ * (which the fold leaves alone) where those depths still fit the record
+ * store, else it waits for the fold; the outputs are the same either way up
+ * to rounding.  Other handles fold in ordinary launches, and the next step
+ * is an ordinary launch too.  Memory: a second state buffer and, tensor-core
+ * kernel, two operand images of it, allocated by onela_create.
  * Errors: ONELA_ERR_ARG, ONELA_ERR_STATE (no prompt state), ONELA_ERR_PARENT
  * (a bad parent index was seen: the ancestry is meaningless), ONELA_ERR_TIMEOUT,
  * ONELA_ERR_CAPACITY, ONELA_ERR_CUDA. */

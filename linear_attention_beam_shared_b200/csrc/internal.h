@@ -148,7 +148,7 @@ cudaError_t launch_step_tc(const StepParams &p, int pdl, cudaStream_t s);
 cudaError_t launch_fold(const StepParams &p, int Wt, int max_depth, int first, const int32_t *d0_in, int32_t *d0_out,
                         int32_t *anc_fold, void *S_fold, int qkv_bf16, int s0_bf16, cudaStream_t s);
 // The same for tensor-core handles (bf16 keys, d_k = d_v in {64, 128},
-// T_max <= 16) in one launch that also writes S_fold's operand image (with
+// T_max <= kFoldTcMaxT) in one launch that also writes S_fold's operand image (with
 // p.s0_planes terms); programmatic launch when pdl (the kernel waits before
 // it reads the ancestry rows and records; it reads S_fold and d0_in before,
 // so the previous kernel must not be a fold).
