@@ -417,8 +417,9 @@ def time_fold(wl, S0, kernel, device, stream, flush, T=16, every=4, reps=10, war
 
 def time_sweep(device, stream, flush, reps=10, warmup=3):
     """The beam-width sweep (W = 64 .. 1024, T = 5, 1K-prompt shapes), the
-    request sweep (R = 1, 8, 32 at H = 16, d = 128, W = 256, T = 7) and the
-    head sizes d = 64 and 256 at R = 1, H = 16, W = 256, T = 7: one whole
+    request sweep (R = 1, 8, 32 at H = 16, d = 128, W = 256, T = 7), the
+    head sizes d = 64 and 256 at R = 1, H = 16, W = 256, T = 7, the headline
+    shapes with a bf16 S0 and the op1k workload (T = 3): one whole
     decode (one onela_decode_steps call) per CUDA graph, L2 flushed before
     each, CUDA events; algorithmic bytes from the byte model.  S0 is drawn
     directly (its values do not change the work).  Returns the JSON object
@@ -428,6 +429,7 @@ def time_sweep(device, stream, flush, reps=10, warmup=3):
     cases += [synth.shape_sweep_workload(R, 16, 128, 256, 7) for R in (1, 8, 32)]
     cases += [synth.shape_sweep_workload(1, 16, d, 256, 7) for d in (64, 256)]
     cases += [synth.workload("long5k_bf16")]  # the headline shapes with a bf16 S0
+    cases += [synth.workload("op1k")]         # the 1K-prompt workload: T = 3
     hbm = measured_peaks()[0]
     points = []
     for wl in cases:
@@ -447,7 +449,8 @@ def time_sweep(device, stream, flush, reps=10, warmup=3):
         dec.close()
         alg, _, _ = byte_model(wl, steps)
         gbs = alg / (ms / 1e3) / 1e9
-        points.append({"R": wl.R, "H": wl.H, "d": wl.d_k, "W": wl.W, "T": wl.T, "s0": wl.s0_dtype, "kernel": kind,
+        points.append({"workload": wl.name, "R": wl.R, "H": wl.H, "d": wl.d_k, "W": wl.W, "T": wl.T, "s0": wl.s0_dtype,
+                       "kernel": kind,
                        "launches": launches, "ms_per_decode": round(ms, 5), "value": round(wl.units / (ms / 1e3), 1),
                        "achieved_gbs": round(gbs, 1), "frac": round(gbs / hbm, 4),
                        "capacity_ratio": capacity(wl)["ratio"]})

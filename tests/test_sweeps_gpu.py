@@ -63,6 +63,10 @@ def _slice(steps, r, h):
     (8, 32, 128, 512, 5, False),
     (1, 32, 256, 512, 7, False),
     (32, 32, 256, 512, 2, True),
+    (1, 16, 128, 128, 1, False),
+    (8, 16, 64, 256, 3, False),
+    (4, 8, 256, 256, 5, True),
+    (2, 16, 128, 128, 3, False),
 ])
 def test_shape_grid_sampled(R, H, d, W, T, direct):
     """direct: S0 drawn directly (N(0, 0.1^2)) instead of the 1K-token
