@@ -349,7 +349,8 @@ struct ChainLayout {
   static constexpr int NK = DK / 64;
   static constexpr uint32_t kt = 0;                           // K tile [NK][64 tokens][128 B]
   static constexpr uint32_t ktt = kt + NK * 8192u;            // K^T [DK rows][128 B]
-  static constexpr uint32_t vt = ktt + DK * 128u;             // v tile [NK][64 tokens][128 B]
+  static constexpr uint32_t vtt = ktt + DK * 128u;            // v^T [DK rows][128 B]
+  static constexpr uint32_t vt = vtt + DK * 128u;             // v tile [NK][64 tokens][128 B]
   static constexpr uint32_t tp = vt + NK * 8192u;             // T terms [3][64][128 B]
   static constexpr uint32_t gt = tp + 3u * kTPlane;           // gates, two buffers
   static constexpr uint32_t bar = gt + 2u * kGateBytes;       // 4 barriers and the TMEM address
@@ -559,10 +560,11 @@ __global__ void __launch_bounds__(kChainThreads, 1) prefill_chain_kernel(const _
     arrive();
     bool ok = true;
     uint32_t mph = 0;
-    // K^T by 8x8 tiles: a warp moves 4 token tiles of one 8-column block of
-    // the keys per step (a transposing load, a plain store).
+    // K^T (and v^T) by 8x8 tiles: a warp moves 4 token tiles of one 8-column
+    // block per step (a transposing load, a plain store).
     constexpr int KTS = DK / 64;  // steps per warp: (DK / 8) blocks x 2 token halves / 16 warps
     const uint32_t kt_u32e = ptx::smem_u32(base + LY::kt), ktt_u32e = ptx::smem_u32(base + LY::ktt);
+    const uint32_t vt_u32e = ptx::smem_u32(base + LY::vt), vtt_u32e = ptx::smem_u32(base + LY::vtt);
 #pragma unroll 1
     for (int c = c0; c < c1; ++c) {
       const uint32_t it = (uint32_t)(c - c0);
@@ -574,7 +576,16 @@ __global__ void __launch_bounds__(kChainThreads, 1) prefill_chain_kernel(const _
         uint32_t frag[4];
         ldsm_x4_trans(kt_u32e + (nb >> 3) * 8192 + ptx::swz128(ih * 32 + 8 * tk + tr, nb & 7), frag);
         stsm_x4(ktt_u32e + ptx::swz128(8 * nb + tr, ih * 4 + tk), frag);
+        if (!amode) {
+          ldsm_x4_trans(vt_u32e + (nb >> 3) * 8192 + ptx::swz128(ih * 32 + 8 * tk + tr, nb & 7), frag);
+          stsm_x4(vtt_u32e + ptx::swz128(8 * nb + tr, ih * 4 + tk), frag);
+        }
       }
+      // v^T rows are read by the other epilogue warps: all 16 meet here (named
+      // barrier 1; the load and MMA warp does not take part).  The next
+      // chunk's transposes come only after every warp has arrived from its
+      // Z^T stage, so nothing is overwritten while it is read.
+      if (!amode) ptx::bar_sync(1, kEpiThreads);
       const float *gts = reinterpret_cast<const float *>(base + LY::gt + (it & 1) * kGateBytes);
       const int i0 = part * TT;
       // Z^T = (v - gamma . Y) beta, token-wise
@@ -585,14 +596,28 @@ __global__ void __launch_bounds__(kChainThreads, 1) prefill_chain_kernel(const _
       float y[TT];
       ptx::tmem_ld16(tmem + lb + i0, y);
       ptx::tmem_ld_wait();
+      {
+        // v of row e for tokens i0 .. i0 + 15 from v^T (two 16-byte loads),
+        // beta and gamma as float4.
+        uint4 vv[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
+        if (!amode && live) {
+          vv[0] = *reinterpret_cast<const uint4 *>(base + LY::vtt + ptx::swz128(e, i0 >> 3));
+          vv[1] = *reinterpret_cast<const uint4 *>(base + LY::vtt + ptx::swz128(e, (i0 >> 3) + 1));
+        }
+        const uint32_t vw[8] = {vv[0].x, vv[0].y, vv[0].z, vv[0].w, vv[1].x, vv[1].y, vv[1].z, vv[1].w};
 #pragma unroll
-      for (int x = 0; x < TT; ++x) {
-        const int i = i0 + x;
-        float v = 0.f;
-        if (!amode && live)
-          v = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(
-              base + LY::vt + (e >> 6) * 8192 + ptx::swz128(i, (e & 63) >> 3) + ((e & 7) << 1)));
-        y[x] = gts[i] * fmaf(-gts[kC + i], y[x], v);
+        for (int x4 = 0; x4 < TT / 4; ++x4) {
+          const float4 bq = reinterpret_cast<const float4 *>(gts + i0)[x4];
+          const float4 gq = reinterpret_cast<const float4 *>(gts + kC + i0)[x4];
+          const float bs[4] = {bq.x, bq.y, bq.z, bq.w}, gs[4] = {gq.x, gq.y, gq.z, gq.w};
+#pragma unroll
+          for (int z = 0; z < 4; ++z) {
+            const int x = 4 * x4 + z;
+            const uint32_t w = vw[x >> 1];
+            const float v = __uint_as_float((x & 1) ? (w & 0xffff0000u) : (w << 16));
+            y[x] = bs[z] * fmaf(-gs[z], y[x], v);
+          }
+        }
       }
       store_tokens(y);
       arrive();
@@ -603,7 +628,13 @@ __global__ void __launch_bounds__(kChainThreads, 1) prefill_chain_kernel(const _
       ptx::tmem_ld16(tmem + lb + 64 + i0, y);
       ptx::tmem_ld_wait();
 #pragma unroll
-      for (int x = 0; x < TT; ++x) y[x] *= gts[2 * kC + i0 + x];
+      for (int x4 = 0; x4 < TT / 4; ++x4) {
+        const float4 rq = reinterpret_cast<const float4 *>(gts + 2 * kC + i0)[x4];
+        y[4 * x4] *= rq.x;
+        y[4 * x4 + 1] *= rq.y;
+        y[4 * x4 + 2] *= rq.z;
+        y[4 * x4 + 3] *= rq.w;
+      }
       store_tokens(y);
       arrive();
       // S <- gamma_{C-1} S + dS
