@@ -1,5 +1,6 @@
-// Thin inline-PTX wrappers for the sm_100a features the tensor-core decode
-// kernel uses: mbarriers, bulk (TMA) copies, tcgen05 MMA / TMEM, fences.
+// Thin inline-PTX wrappers for the sm_100a features the tensor-core kernels
+// use: mbarriers, bulk (TMA) copies, tcgen05 MMA / TMEM, fences, GPU-scope
+// acquire and release.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -53,30 +54,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64
   return true;
 }
 
-// Spin on an mbarrier phase with acquire semantics at cluster scope (the
-// arrivals come from other CTAs of the cluster, released at cluster scope),
-// for at most limit_ns; false on timeout.
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.b32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait_cluster(bar, parity)) {
-    if (globaltimer_ns() - t0 > limit_ns) return false;
-  }
-  return true;
-}
-
 // ------------------------------------------------- global-memory counters
+// *p with acquire semantics at GPU scope.
 __device__ __forceinline__ int ld_acquire_gpu(const int *p) {
   int v;
   asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -86,48 +65,7 @@ __device__ __forceinline__ int ld_acquire_gpu(const int *p) {
 __device__ __forceinline__ void red_release_add_gpu(int *p, int v) {
   asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
-// Spin until *p >= target (acquire), for at most limit_ns; false on timeout.
-__device__ __forceinline__ bool wait_count_gpu(const int *p, int target, uint64_t limit_ns) {
-  if (ld_acquire_gpu(p) >= target) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (ld_acquire_gpu(p) < target) {
-    if (globaltimer_ns() - t0 > limit_ns) return false;
-  }
-  return true;
-}
-
-// ----------------------------------------------------------------- clusters
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-// The shared::cluster address of the variable at shared::cta address saddr
-// in the CTA of the cluster with the given rank.
-__device__ __forceinline__ uint32_t mapa(uint32_t saddr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
-  return r;
-}
-// 16-byte load from the shared memory of a CTA of the cluster.
-__device__ __forceinline__ float4 ld_dsmem_f4(uint32_t caddr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(caddr)
-               : "memory");
-  return v;
-}
-// Arrive on an mbarrier in the shared memory of a CTA of the cluster, with
-// release semantics at cluster scope.
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t caddr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(caddr) : "memory");
-}
-__device__ __forceinline__ void fence_acq_rel_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
-// Every thread of every CTA of the cluster (all threads of a warp together).
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
+// ------------------------------------------------------- named barriers
 // Named barrier id over n threads (n a multiple of 32).
 __device__ __forceinline__ void bar_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
 
@@ -150,13 +88,6 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const void *tmap, int c0,
       "[%6];" ::"r"(smem_u32(dst)),
       "l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
       : "memory");
-}
-
-// Prefetch of a 4-D tensor-map box into L2 (no shared-memory destination).
-__device__ __forceinline__ void tma_prefetch_4d(const void *tmap, int c0, int c1, int c2, int c3) {
-  asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(tmap), "r"(c0),
-               "r"(c1), "r"(c2), "r"(c3)
-               : "memory");
 }
 
 // 16-byte asynchronous copy global -> shared (L2 only); src_bytes = 0 writes

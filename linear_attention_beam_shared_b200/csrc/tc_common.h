@@ -1,4 +1,4 @@
-// Helpers shared by the tensor-core decode kernels (step_tc.cu, decode_tc.cu).
+// Helpers shared by the tensor-core kernels (step_tc.cu, prefill_tc.cu).
 #pragma once
 
 #include <cuda.h>
