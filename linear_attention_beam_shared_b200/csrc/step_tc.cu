@@ -1,8 +1,10 @@
 // Tensor-core decode-step kernel (tcgen05, sm_100a) for bf16 q/k/v and
-// d_k = d_v in {64, 128}.
+// d_k = d_v in {64, 128, 256}.
 //
-// One CTA per (request r, head h, tile of 32 beams); 320 threads (8 beam
-// warps, an ancestry warp and an MMA warp); two CTAs fit on an SM.  The step
+// One CTA per (request r, head h, tile of 32 beams) -- at d = 256 two, one
+// per half of the rows of S, each streaming its half of the S0 image through
+// a ring of shared-memory slots; 320 threads (8 beam warps, an ancestry warp
+// and an MMA warp); two CTAs fit on an SM.  The step
 // of the shared-state GDN beam decode (OneLA, evolve.pub review, key claims
 // on section 3.2, equations 2-4).  For beam b with ancestors a_1 .. a_{t-1}
 // (a_{t-1} = p, its parent) and P(a) the product of the gates on the path
@@ -71,6 +73,7 @@ constexpr int kBT = 32;             // beams per CTA
 constexpr int kN = 2 * kBT;         // vectors: k rows 0..31, q rows 32..63
 constexpr int kM = 128;             // MMA M
 constexpr int kDRows = 128;         // ancestor deltas per staging round after the wait
+constexpr int kRing = 3;            // 16 KB slots of the image ring (d_k = 256)
 constexpr int kTmemCols = 64;       // D1
 // The per-step table: 3 pointers and 3 ints for each of nhist = T_max + 1
 // steps (at most kHistSteps).
@@ -81,23 +84,36 @@ constexpr int kMaxW = 1024;         // widest beam set the kernel serves
 struct Layout {
   uint32_t x;     // X [NK][64 rows][128 B]: k rows, then q rows
   uint32_t v;     // v [NV][32 rows][128 B]: this CTA's d_v columns
-  uint32_t a;     // region A: the S0 image; then D1^T; then the deltas
+  uint32_t a;     // region A: the S0 image (or its ring); then D1^T
   uint32_t d1;    // D1^T [64 vectors][this CTA's d_v rows] fp32
-  uint32_t dst;   // ancestor deltas [kDRows][this CTA's d_v rows] fp32
+  uint32_t dst;   // ancestor deltas [rows][this CTA's d_v rows] fp32
   uint32_t book;  // barriers and bookkeeping
   uint32_t total;
 };
 
 // nk: 64-element K atoms of a key row; nv: 64-row atoms of this CTA's d_v rows.
-__host__ __device__ inline Layout layout(int nk, int nv, int planes, int TM, int W_max, int hist_cap) {
+// ring (d_k = 256): the image passes through kRing slots of region A, and
+// the deltas are staged over X and region A, both consumed by then; else the
+// whole image sits in region A, which then holds D1^T and the deltas.
+__host__ __device__ inline Layout layout(int nk, int nv, int planes, int TM, int W_max, int hist_cap,
+                                         bool ring = false) {
   Layout L;
-  L.x = 0;
-  L.v = (uint32_t)nk * 8192u;
-  L.a = L.v + (uint32_t)nv * 4096u;
-  L.d1 = L.a + (uint32_t)nv * 16384u;
-  L.dst = L.a;
-  const uint32_t s0 = (uint32_t)planes * nk * 16384u, ops = (uint32_t)nv * 32768u;
-  L.book = L.a + (s0 > ops ? s0 : ops);
+  if (ring) {
+    L.v = 0;
+    L.x = (uint32_t)nv * 4096u;
+    L.a = L.x + (uint32_t)nk * 8192u;
+    L.d1 = L.a;
+    L.dst = L.x;
+    L.book = L.a + (uint32_t)kRing * 16384u;
+  } else {
+    L.x = 0;
+    L.v = (uint32_t)nk * 8192u;
+    L.a = L.v + (uint32_t)nv * 4096u;
+    L.d1 = L.a + (uint32_t)nv * 16384u;
+    L.dst = L.a;
+    const uint32_t s0 = (uint32_t)planes * nk * 16384u, ops = (uint32_t)nv * 32768u;
+    L.book = L.a + (s0 > ops ? s0 : ops);
+  }
   // 128 B of barriers and counters; 4 per-beam scalars; per (beam, depth)
   // the replay coefficients (float4), the chain, slot-list ints and gates
   // (the slot list 4 TM longer); a beam-index scratch [W_max]; the parents
@@ -112,13 +128,16 @@ __host__ __device__ inline Layout layout(int nk, int nv, int planes, int TM, int
 // handles -- all of them for d <= 128, one half of them for d = 256 (the two
 // halves of a beam tile are two CTAs; both form the full key products).
 template <int DK, int DV>
-__global__ void __launch_bounds__(kThreads, DK <= 128 ? 2 : 1) step_tc_kernel(const __grid_constant__ StepParams p) {
+__global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_constant__ StepParams p) {
+  constexpr bool RING = DK > 128;    // the image streamed through kRing slots (two CTAs per SM)
   constexpr int NK = DK / 64;        // 128-byte K atoms per key row
   constexpr int NV = DV / 64;        // 64-column atoms of this CTA's part of v
   constexpr uint32_t XA = kN * 128;  // bytes of one K atom of X (64 rows)
   constexpr uint32_t VA = kBT * 128; // bytes of one atom of v (32 rows)
   constexpr int NU = DV / 32;        // 4-element groups per thread of a value row, beam-major phase
   constexpr int NUK = DK / 32;       // the same for a key row
+  // Ancestor delta rows per staging round after the wait.
+  constexpr int DR = RING ? (NK * 8192 + kRing * 16384) / (DV * 4) : kDRows;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = ptx::smem_u32(smem_raw);
   uint8_t *base = smem_raw + ((1024u - (raw_u32 & 1023u)) & 1023u);
@@ -135,15 +154,17 @@ __global__ void __launch_bounds__(kThreads, DK <= 128 ? 2 : 1) step_tc_kernel(co
   const int hb = p.hbase;       // step of the history table's entry 0
   const uint64_t hmask = p.hist_inputs;  // bit i: history entry i from the callers' arrays
 
-  const Layout L = layout(NK, NV, P, TM, p.W_max, p.hist_cap);
+  const Layout L = layout(NK, NV, P, TM, p.W_max, p.hist_cap, RING);
   uint8_t *s_x = base + L.x;
   const uint8_t *s_v = base + L.v;
   float *s_d1 = reinterpret_cast<float *>(base + L.d1);
   const float *s_dst = reinterpret_cast<const float *>(base + L.dst);
   uint64_t *bars = reinterpret_cast<uint64_t *>(base + L.book);
-  uint64_t *bar_s0 = bars + 0;     // S0 image, X and v landed
+  uint64_t *bar_s0 = bars + 0;     // X and v (and the S0 image unless RING) landed
   uint64_t *bar1 = bars + 1;       // D1 complete
   uint64_t *bar_chain = bars + 2;  // ancestry warp: every beam's chain in s_chain
+  uint64_t *bar_full = bars + 10;  // RING: slot holds its image chunk (bytes 80..103)
+  uint64_t *bar_empty = bars + 13; // RING: the products reading the slot are done (bytes 104..127)
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(base + L.book + 64);
   int *s_U = reinterpret_cast<int *>(s_tmem + 1);
   int *s_mode = s_U + 1;  // the CTA's root: [0] its folded depth, [1] how it was chosen
@@ -180,6 +201,11 @@ __global__ void __launch_bounds__(kThreads, DK <= 128 ? 2 : 1) step_tc_kernel(co
     ptx::mbar_init(bar_s0, 1);
     ptx::mbar_init(bar1, 1);
     ptx::mbar_init(bar_chain, 32 + (p.stall ? 1 : 0));  // stall (tests): an arrival that never comes
+    if (RING)
+      for (int i = 0; i < kRing; ++i) {
+        ptx::mbar_init(bar_full + i, 1);
+        ptx::mbar_init(bar_empty + i, 1);
+      }
     ptx::mbar_fence_init();
     // The root this step replays from: the current folded state, or, while
     // the last fold is not complete, the one before it (where its depths fit
@@ -197,12 +223,20 @@ __global__ void __launch_bounds__(kThreads, DK <= 128 ? 2 : 1) step_tc_kernel(co
     // A new decode: its folds count from zero (no fold of an earlier decode
     // runs any more: step 1 is an ordinary launch).
     if (t == 1 && p.fold_reset && tile == 0 && h == 0 && mt == 0) p.fold_reset[r] = 0;
-    // S0 image (bulk copy); k, q, v tiles by TMA, beams past W read as zeros.
-    ptx::mbar_arrive_expect_tx(bar_s0, s0_bytes + NK * XA + NV * VA);
+    // S0 image (bulk copy; RING: its first chunks, one per slot); k, q, v
+    // tiles by TMA, beams past W read as zeros.
+    ptx::mbar_arrive_expect_tx(bar_s0, (RING ? 0u : s0_bytes) + NK * XA + NV * VA);
     const uint8_t *src =
         static_cast<const uint8_t *>(mode == 1 ? p.S0img_old : p.S0img) + ((size_t)(r * H + h) * nmt + mt) * s0_bytes;
-    for (uint32_t off = 0; off < s0_bytes; off += 16384u)
-      ptx::bulk_g2s(base + L.a + off, src + off, 16384u, bar_s0);
+    if (RING) {
+      for (int c = 0; c < kRing && c < P * NK; ++c) {
+        ptx::mbar_arrive_expect_tx(bar_full + c, 16384u);
+        ptx::bulk_g2s(base + L.a + c * 16384u, src + c * 16384u, 16384u, bar_full + c);
+      }
+    } else {
+      for (uint32_t off = 0; off < s0_bytes; off += 16384u)
+        ptx::bulk_g2s(base + L.a + off, src + off, 16384u, bar_s0);
+    }
 #pragma unroll
     for (int ka = 0; ka < NK; ++ka) {
       ptx::tma_load_4d(s_x + ka * XA, &p.tm_k, ka * 64, h, b0, r, bar_s0);
@@ -274,7 +308,14 @@ __global__ void __launch_bounds__(kThreads, DK <= 128 ? 2 : 1) step_tc_kernel(co
   // reading rows at the same step cover all 32 banks.
   const int bb = tid >> 3, l = tid & 7, sx = bb & 1;
   const bool bval = bb < nb;  // false in the ancestry warp (bb >= 32)
-  uint2 kb2[NUK], qb2[NUK];  // this thread's elements of k_b and q_b, bf16
+  // This thread's elements of k_b and q_b, bf16: in registers, or (RING,
+  // where the registers hold more key pieces in flight) read from X again.
+  uint2 kb2[RING ? 1 : NUK], qb2[RING ? 1 : NUK];
+  auto xpiece = [&](int u, int row) -> uint2 {
+    const int uu = u ^ sx;
+    const uint32_t off = (uint32_t)(uu >> 1) * XA + (uint32_t)(l & 1) * 8u;
+    return *reinterpret_cast<const uint2 *>(s_x + off + ptx::swz128(row, 4 * (uu & 1) + (l >> 1)));
+  };
   float kq = 0.f;
 
   if (warp == kAncWarp) {
@@ -353,7 +394,45 @@ __global__ void __launch_bounds__(kThreads, DK <= 128 ? 2 : 1) step_tc_kernel(co
     // ------------------------------------------------ the MMA warp
     // D1 = S0 . X^T on the tensor cores, issued by lane 0 once the image is
     // here.
-    if (lane == 0) {
+    if (lane == 0 && RING) {
+      // The image chunk by chunk (plane-major, then K atom) through the
+      // ring: a slot is refilled with the chunk kRing further on once the
+      // products reading it are done.  A wait that runs out stops the issue.
+      ok = ptx::mbar_wait(bar_s0, 0, p.wait_limit_ns);
+      ptx::tc_fence_after();
+      constexpr uint32_t idesc1 = ptx::idesc_bf16_f32(kM, kN);
+      const uint8_t *src = static_cast<const uint8_t *>(s_mode[1] == 1 ? p.S0img_old : p.S0img) +
+                           ((size_t)(r * H + h) * nmt + mt) * s0_bytes;
+      const int nch = P * NK;
+      int acc = 0;
+      for (int c = 0; c < nch && ok; ++c) {
+        const int sl = c % kRing;
+        const uint32_t ph = (uint32_t)(c / kRing) & 1u;
+        if (!ptx::mbar_wait(bar_full + sl, ph, p.wait_limit_ns)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        const int ka = c % NK;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t ad = ptx::desc_k128(a_u32 + sl * 16384 + kk * 32);
+          const uint64_t bd = ptx::desc_k128(x_u32 + ka * XA + kk * 32);
+          ptx::mma_bf16(tmem, ad, bd, idesc1, acc);
+          acc = 1;
+        }
+        if (c + kRing < nch) {
+          ptx::mma_commit(bar_empty + sl);
+          if (!ptx::mbar_wait(bar_empty + sl, ph, p.wait_limit_ns)) {
+            ok = false;
+            break;
+          }
+          ptx::mbar_arrive_expect_tx(bar_full + sl, 16384u);
+          ptx::bulk_g2s(base + L.a + sl * 16384u, src + (size_t)(c + kRing) * 16384u, 16384u, bar_full + sl);
+        }
+      }
+      ptx::mma_commit(bar1);
+    } else if (lane == 0) {
       ok = ptx::mbar_wait(bar_s0, 0, p.wait_limit_ns);
       ptx::tc_fence_after();
       constexpr uint32_t idesc1 = ptx::idesc_bf16_f32(kM, kN);
@@ -376,12 +455,9 @@ __global__ void __launch_bounds__(kThreads, DK <= 128 ? 2 : 1) step_tc_kernel(co
     // This thread's elements of k_b and q_b, and k_b . q_b.
 #pragma unroll
     for (int u = 0; u < NUK; ++u) {
-      const int uu = u ^ sx;
-      const uint32_t off = (uint32_t)(uu >> 1) * XA + (uint32_t)(l & 1) * 8u;
-      const int c = 4 * (uu & 1) + (l >> 1);
-      kb2[u] = *reinterpret_cast<const uint2 *>(s_x + off + ptx::swz128(bb, c));
-      qb2[u] = *reinterpret_cast<const uint2 *>(s_x + off + ptx::swz128(kBT + bb, c));
-      const float4 kf = bf16x4(kb2[u]), qf = bf16x4(qb2[u]);
+      const uint2 kx = xpiece(u, bb), qx = xpiece(u, kBT + bb);
+      if constexpr (!RING) kb2[u] = kx, qb2[u] = qx;
+      const float4 kf = bf16x4(kx), qf = bf16x4(qx);
       kq = fmaf(kf.x, qf.x, kq);
       kq = fmaf(kf.y, qf.y, kq);
       kq = fmaf(kf.z, qf.z, kq);
@@ -420,7 +496,11 @@ __global__ void __launch_bounds__(kThreads, DK <= 128 ? 2 : 1) step_tc_kernel(co
       for (int e = 0; e < 2; ++e) dk[e] = 0.f, dq[e] = 0.f;
 #pragma unroll
       for (int u = 0; u < NUK; ++u) {
-        const float4 kbu = bf16x4(kb2[u]), qbu = bf16x4(qb2[u]);
+        float4 kbu, qbu;
+        if constexpr (RING)
+          kbu = bf16x4(xpiece(u, bb)), qbu = bf16x4(xpiece(u, kBT + bb));
+        else
+          kbu = bf16x4(kb2[u]), qbu = bf16x4(qb2[u]);
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const float4 kf = bf16x4(buf[e][u]);
@@ -530,8 +610,8 @@ __global__ void __launch_bounds__(kThreads, DK <= 128 ? 2 : 1) step_tc_kernel(co
   // ------------------------------- after the wait: the ancestors' deltas
   ptx::pdl_wait();
   constexpr int PD = DV / 4;  // 16-byte pieces of a delta row
-  for (int lo = 0; lo < U; lo += kDRows) {
-    const int hi = min(U, lo + kDRows);
+  for (int lo = 0; lo < U; lo += DR) {
+    const int hi = min(U, lo + DR);
     const int nrows = hi - lo;
     if (lo > 0) __syncthreads();  // the previous round's deltas are consumed
     // The rows of slots lo .. hi - 1 in 16-byte pieces (a warp copies whole
@@ -677,7 +757,7 @@ cudaError_t launch_dk(const StepParams &p_in, bool pdl, cudaStream_t s) {
       !encode_rows(&p.tm_v, p.v, DK, p.H, p.W, p.R))
     return cudaErrorInvalidValue;
 
-  const Layout L = layout(DK / 64, DV / 64, p.s0_planes, p.T_max, p.W_max, p.hist_cap);
+  const Layout L = layout(DK / 64, DV / 64, p.s0_planes, p.T_max, p.W_max, p.hist_cap, DK > 128);
   const size_t smem = L.total + 1024;
   cudaError_t e = ensure_smem_limit((const void *)step_tc_kernel<DK, DV>, smem);
   if (e != cudaSuccess) return e;
@@ -697,10 +777,10 @@ cudaError_t launch_dk(const StepParams &p_in, bool pdl, cudaStream_t s) {
 }  // namespace
 
 bool tc_supports(int dk, int dv, int qkv_bf16, int T_max, int W_max, int planes) {
-  // d = 256: one CTA per half of the rows of S keeps a 128 KB image (two
-  // bf16 terms at most).
-  return qkv_bf16 && dk == dv && (dk == 64 || dk == 128 || (dk == 256 && planes <= 2)) && T_max <= kMaxT &&
-         W_max <= kMaxW;
+  // d = 256: one CTA per half of the rows of S, its image streamed through
+  // a ring of shared-memory slots (any number of terms).
+  return qkv_bf16 && dk == dv && (dk == 64 || dk == 128 || dk == 256) && planes >= 1 && planes <= 3 &&
+         T_max <= kMaxT && W_max <= kMaxW;
 }
 
 size_t s0_image_bytes(int R, int H, int dk, int dv, int planes) {
@@ -722,7 +802,7 @@ cudaError_t launch_step_tc(const StepParams &p, int pdl, cudaStream_t s) {
     return cudaErrorNotSupported;
   if (p.dk == 64 && p.dv == 64) return launch_dk<64, 64>(p, pdl != 0, s);
   if (p.dk == 128 && p.dv == 128) return launch_dk<128, 128>(p, pdl != 0, s);
-  if (p.dk == 256 && p.dv == 256 && p.s0_planes <= 2) return launch_dk<256, 128>(p, pdl != 0, s);
+  if (p.dk == 256 && p.dv == 256) return launch_dk<256, 128>(p, pdl != 0, s);
   return cudaErrorNotSupported;
 }
 

@@ -348,13 +348,17 @@ def test_tc_d256(s0_dtype, W, T, R, H):
     P.compare(gpu, P.oracle(S0c, steps), steps, s0_dtype)
 
 
-def test_tc_d256_three_terms_are_refused():
-    """A three-term split of an fp32 S0 does not fit one CTA at d = 256: the
-    tensor-core kernel refuses it and AUTO picks the general kernel."""
+@pytest.mark.parametrize("W,T,R,H", [(129, 4, 2, 3), (256, 6, 1, 2)])
+def test_tc_d256_three_terms(W, T, R, H):
+    """A three-term split of an fp32 S0 at d = 256: the image (192 KB per CTA)
+    streams through the kernel's ring of shared-memory slots, so AUTO keeps
+    the tensor-core kernel; whole decodes against the fp64 oracle."""
     import linear_attention_beam_shared_b200 as L
-    with pytest.raises(L.OnelaError) as e:
-        L.onela_create(1, 2, 256, 256, 32, 3, "f32", "bf16", L.ONELA_KERNEL_TC, s0_split=3)
-    assert e.value.code == L.ONELA_ERR_UNSUPPORTED
     h = L.onela_create(1, 2, 256, 256, 32, 3, "f32", "bf16", L.ONELA_KERNEL_AUTO, s0_split=3)
-    assert L.onela_kernel_kind(h) == L.ONELA_KERNEL_SIMT
+    assert L.onela_kernel_kind(h) == L.ONELA_KERNEL_TC
     L.onela_destroy(h)
+    wl, S0, steps = P.custom_steps(70 + W + T, R, H, 256, 256, (W,) * T, parents="mixed" if R > 1 else "zipf")
+    S0c = synth.cast_state(S0, "f32")
+    gpu, kind = P.run_gpu(S0c, steps, "bf16", L.ONELA_KERNEL_TC, s0_split=3)
+    assert kind == L.ONELA_KERNEL_TC
+    P.compare(gpu, P.oracle(S0c, steps), steps, "f32")
