@@ -80,6 +80,7 @@ constexpr int kTmemCols = 64;       // D1
 __host__ __device__ inline uint32_t tab_bytes(int nhist) { return (3u * 8u + 3u * 4u) * (uint32_t)nhist; }
 constexpr int kMaxT = 32;           // deepest decode the kernel serves
 constexpr int kMaxW = 1024;         // widest beam set the kernel serves
+constexpr int kSMs = 148;           // SMs of a B200
 
 struct Layout {
   uint32_t x;     // X [NK][64 rows][128 B]: k rows, then q rows
@@ -127,8 +128,9 @@ __host__ __device__ inline Layout layout(int nk, int nv, int planes, int TM, int
 // DK: d_k; DV: the d_v rows of S (and columns of v, o, delta) one CTA
 // handles -- all of them for d <= 128, one half of them for d = 256 (the two
 // halves of a beam tile are two CTAs; both form the full key products).
-template <int DK, int DV>
-__global__ void __launch_bounds__(kThreads, 2) step_tc_kernel(const __grid_constant__ StepParams p) {
+// MINB: CTAs per SM the registers must allow (3 only at d = 64).
+template <int DK, int DV, int MINB>
+__global__ void __launch_bounds__(kThreads, MINB) step_tc_kernel(const __grid_constant__ StepParams p) {
   constexpr bool RING = DK > 128;    // the image streamed through kRing slots (two CTAs per SM)
   constexpr int NK = DK / 64;        // 128-byte K atoms per key row
   constexpr int NV = DV / 64;        // 64-column atoms of this CTA's part of v
@@ -750,7 +752,7 @@ bool encode_rows(CUtensorMap *m, const void *base, int d, int H, int W, int R, i
 
 namespace {
 
-template <int DK, int DV>
+template <int DK, int DV, int MINB = 2>
 cudaError_t launch_dk(const StepParams &p_in, bool pdl, cudaStream_t s) {
   StepParams p = p_in;
   if (!encode_rows(&p.tm_k, p.k, DK, p.H, p.W, p.R) || !encode_rows(&p.tm_q, p.q, DK, p.H, p.W, p.R) ||
@@ -758,11 +760,12 @@ cudaError_t launch_dk(const StepParams &p_in, bool pdl, cudaStream_t s) {
     return cudaErrorInvalidValue;
 
   const Layout L = layout(DK / 64, DV / 64, p.s0_planes, p.T_max, p.W_max, p.hist_cap, DK > 128);
+  const dim3 grid((p.W + kBT - 1) / kBT, p.H, p.R * (p.dv / DV));
   const size_t smem = L.total + 1024;
-  cudaError_t e = ensure_smem_limit((const void *)step_tc_kernel<DK, DV>, smem);
+  cudaError_t e = ensure_smem_limit((const void *)step_tc_kernel<DK, DV, MINB>, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((p.W + kBT - 1) / kBT, p.H, p.R * (p.dv / DV));
+  cfg.gridDim = grid;
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
@@ -771,7 +774,7 @@ cudaError_t launch_dk(const StepParams &p_in, bool pdl, cudaStream_t s) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, step_tc_kernel<DK, DV>, p);
+  return cudaLaunchKernelEx(&cfg, step_tc_kernel<DK, DV, MINB>, p);
 }
 
 }  // namespace
@@ -800,7 +803,13 @@ cudaError_t launch_s0_image(const void *S0, void *img, int R, int H, int dk, int
 cudaError_t launch_step_tc(const StepParams &p, int pdl, cudaStream_t s) {
   if (p.T_max > kMaxT || p.W_max > kMaxW || p.s0_planes < 1 || p.s0_planes > 3 || p.hist_cap > kHistMaxInts)
     return cudaErrorNotSupported;
-  if (p.dk == 64 && p.dv == 64) return launch_dk<64, 64>(p, pdl != 0, s);
+  if (p.dk == 64 && p.dv == 64) {
+    // At d = 64 the kernel also builds with 64 registers, three CTAs per SM:
+    // faster once a step has more CTAs than two per SM hold, slower below
+    // (the 80-register build keeps more loads in flight).
+    if ((long)((p.W + kBT - 1) / kBT) * p.H * p.R > 2L * kSMs) return launch_dk<64, 64, 3>(p, pdl != 0, s);
+    return launch_dk<64, 64, 2>(p, pdl != 0, s);
+  }
   if (p.dk == 128 && p.dv == 128) return launch_dk<128, 128>(p, pdl != 0, s);
   if (p.dk == 256 && p.dv == 256) return launch_dk<256, 128>(p, pdl != 0, s);
   return cudaErrorNotSupported;

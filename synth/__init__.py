@@ -105,6 +105,10 @@ def shape_sweep_workload(R: int, H: int, d: int, W: int, T: int) -> Workload:
                     parents="mixed" if R > 1 else "zipf", seed_id=4)
 
 
+# The d = 256 point of the operator-shape sweep by name (profiling runs).
+WORKLOADS["sweep_R1_H16_d256_W256_T7"] = shape_sweep_workload(1, 16, 256, 256, 7)
+
+
 def workload(name: str) -> Workload:
     return WORKLOADS[name]
 
