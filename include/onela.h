@@ -106,7 +106,7 @@ enum { ONELA_FLAG_NVTX = 4 };
 
 /* Which decode kernel runs.  AUTO picks the tensor-core kernel when the
  * shape allows it (bf16 q/k/v, d_k = d_v in {64, 128, 256}; T_max <= 32,
- * W_max <= 1024) and the SIMT kernel otherwise. */
+ * W_max <= 4096) and the SIMT kernel otherwise. */
 enum { ONELA_KERNEL_AUTO = 0, ONELA_KERNEL_SIMT = 1, ONELA_KERNEL_TC = 2 };
 
 /* Handle configuration.

@@ -79,7 +79,7 @@ constexpr int kTmemCols = 64;       // D1
 // steps (at most kHistSteps).
 __host__ __device__ inline uint32_t tab_bytes(int nhist) { return (3u * 8u + 3u * 4u) * (uint32_t)nhist; }
 constexpr int kMaxT = 32;           // deepest decode the kernel serves
-constexpr int kMaxW = 1024;         // widest beam set the kernel serves
+constexpr int kMaxW = 4096;         // widest beam set the kernel serves (its beam-index scratch: 4 B per beam)
 constexpr int kSMs = 148;           // SMs of a B200
 
 struct Layout {

@@ -161,6 +161,23 @@ def test_tc_store_deeper_than_16(T, W, d, R, H):
         P.compare(gpu, ref, steps, "f32")
 
 
+@pytest.mark.parametrize("Ws,d,H", [((64, 2048, 1500, 4096), 64, 2), ((2048, 2048, 1111), 128, 1)])
+def test_tc_wide_beam_sets(Ws, d, H):
+    """Beam sets past 1024 on the tensor-core kernel (up to 4096: 128 beam
+    tiles per head, the parents of earlier steps read from global memory once
+    they no longer fit the kernel's shared copy), through the callers' arrays
+    and through the record store, against the fp64 oracle."""
+    import linear_attention_beam_shared_b200 as L
+    _skip_unavailable(2, d, d, "bf16")
+    wl, S0, steps = P.custom_steps(80 + d, 1, H, d, d, Ws, parents="zipf")
+    S0c = synth.cast_state(S0, "f32")
+    ref = P.oracle(S0c, steps)
+    for chunks in (None, [len(Ws)]):
+        gpu, used = P.run_gpu(S0c, steps, "bf16", L.ONELA_KERNEL_TC, chunks=chunks)
+        assert used == L.ONELA_KERNEL_TC
+        P.compare(gpu, ref, steps, "f32")
+
+
 @pytest.mark.parametrize("kernel", [1, 2])
 def test_identity_gate_keeps_s0(kernel):
     """alpha = 1 (g = 0), beta = 0: delta is exactly zero and o = S0 q."""
