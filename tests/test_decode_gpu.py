@@ -144,10 +144,12 @@ def test_deep_decode(kernel):
     P.compare(gpu, P.oracle(S0c, steps), steps, "f32")
 
 
-@pytest.mark.parametrize("T,W,d,R,H", [(24, 40, 64, 2, 3), (32, 256, 128, 1, 4), (20, 33, 128, 1, 2)])
+@pytest.mark.parametrize("T,W,d,R,H", [(24, 40, 64, 2, 3), (32, 256, 128, 1, 4), (20, 33, 128, 1, 2),
+                                        (20, 72, 256, 1, 2)])
 def test_tc_store_deeper_than_16(T, W, d, R, H):
     """A record store of up to 32 depths on the tensor-core kernel (one CTA
-    per SM past 16 depths at d = 128): every step replays up to T - 1
+    per SM past 16 depths at d = 128; at d = 256 the image ring and the
+    delta staging over it): every step replays up to T - 1
     ancestors, through both the callers' arrays (one onela_decode_steps
     call) and the record store (one call per step)."""
     import linear_attention_beam_shared_b200 as L
