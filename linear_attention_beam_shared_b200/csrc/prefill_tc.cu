@@ -216,6 +216,7 @@ __global__ void __launch_bounds__(kPrepThreads, 3) prefill_prep_kernel(const __g
 #pragma unroll
     for (int ka = 0; ka < NK; ++ka) ptx::tma_load_4d(base + PL::kt + ka * 16384, &p.tm_k, ka * 64, h, tok0, r, bar_k);
     ok = ptx::mbar_wait(bar_k, 0, p.wait_limit_ns);
+    if (!ok) ptx::mbar_wait(bar_k, 0, p.wait_limit_ns);  // the keys still in flight land first (bounded)
     if (ok) {
       ptx::tc_fence_after();
       constexpr uint32_t id = ptx::idesc_bf16_f32(128, 128);

@@ -406,6 +406,7 @@ __global__ void __launch_bounds__(kThreads, MINB) step_tc_kernel(const __grid_co
       const uint8_t *src = static_cast<const uint8_t *>(s_mode[1] == 1 ? p.S0img_old : p.S0img) +
                            ((size_t)(r * H + h) * nmt + mt) * s0_bytes;
       const int nch = P * NK;
+      int issued = nch < kRing ? nch : kRing, landed = 0;  // chunks issued / waited for
       int acc = 0;
       for (int c = 0; c < nch && ok; ++c) {
         const int sl = c % kRing;
@@ -414,6 +415,7 @@ __global__ void __launch_bounds__(kThreads, MINB) step_tc_kernel(const __grid_co
           ok = false;
           break;
         }
+        landed = c + 1;
         ptx::tc_fence_after();
         const int ka = c % NK;
 #pragma unroll
@@ -431,8 +433,13 @@ __global__ void __launch_bounds__(kThreads, MINB) step_tc_kernel(const __grid_co
           }
           ptx::mbar_arrive_expect_tx(bar_full + sl, 16384u);
           ptx::bulk_g2s(base + L.a + sl * 16384u, src + (size_t)(c + kRing) * 16384u, 16384u, bar_full + sl);
+          ++issued;
         }
       }
+      // After a wait that ran out, the chunks still in flight land before
+      // the CTA goes on (each wait bounded again).
+      for (int c = landed; !ok && c < issued; ++c)
+        ptx::mbar_wait(bar_full + c % kRing, (uint32_t)(c / kRing) & 1u, p.wait_limit_ns);
       ptx::mma_commit(bar1);
     } else if (lane == 0) {
       ok = ptx::mbar_wait(bar_s0, 0, p.wait_limit_ns);
@@ -453,7 +460,11 @@ __global__ void __launch_bounds__(kThreads, MINB) step_tc_kernel(const __grid_co
     }
   } else {
     // ------------------------------------------------ the beam warps
-    if (!ptx::mbar_wait(bar_s0, 0, p.wait_limit_ns)) ok = false;  // X and v visible to this thread
+    if (!ptx::mbar_wait(bar_s0, 0, p.wait_limit_ns)) {  // X and v visible to this thread
+      ok = false;
+      // The copies still in flight land before the CTA can exit (bounded again).
+      if (tid == 0) ptx::mbar_wait(bar_s0, 0, p.wait_limit_ns);
+    }
     // This thread's elements of k_b and q_b, and k_b . q_b.
 #pragma unroll
     for (int u = 0; u < NUK; ++u) {
